@@ -1,0 +1,70 @@
+"""Second, independent CPU statement of paged decode attention (numpy, fp64).
+
+TEST INFRASTRUCTURE ONLY.  Written separately from ``pa_oracle.c`` so that the two
+pin each other on small inputs.  It follows the same passages of the vLLM
+paged-attention pages: the "IO-5 vLLM Paged Attention" note, section 3 (each
+sequence owns a list of page indices) and section 4 (K = the pages concatenated in
+table order, then softmax(q K^T / sqrt(d_k)) V unchanged).
+
+Here the gather is done with numpy fancy indexing over whole pages, and the softmax
+with numpy reductions, instead of the C code's per-token loops.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+
+def widen(bits: np.ndarray, dtype: str) -> np.ndarray:
+    bits = np.asarray(bits, dtype=np.uint16)
+    if dtype == "fp16":
+        return bits.view(np.float16).astype(np.float64)
+    if dtype == "bf16":
+        return (bits.astype(np.uint32) << np.uint32(16)).view(np.float32).astype(np.float64)
+    raise ValueError(dtype)
+
+
+def gather(cache_f64: np.ndarray, table_row: np.ndarray, L: int, kv_head: int) -> np.ndarray:
+    """Contiguous [L, d] K (or V) of one sequence and kv head: pages in table order."""
+    bs = cache_f64.shape[2]
+    npages = -(-L // bs)
+    pages = cache_f64[np.asarray(table_row[:npages], dtype=np.int64), kv_head]  # [npages, bs, d]
+    return pages.reshape(npages * bs, -1)[:L]
+
+
+def decode(q, k_cache, v_cache, block_tables, context_lens, scale, dtype) -> np.ndarray:
+    qf = widen(q, dtype)
+    kf = widen(k_cache, dtype)
+    vf = widen(v_cache, dtype)
+    B, hq, d = qf.shape
+    hkv = kf.shape[1]
+    G = hq // hkv
+    out = np.zeros((B, hq, d), np.float64)
+    for s in range(B):
+        L = int(context_lens[s])
+        if L == 0:
+            continue
+        for g in range(hkv):
+            K = gather(kf, block_tables[s], L, g)
+            V = gather(vf, block_tables[s], L, g)
+            Q = qf[s, g * G:(g + 1) * G]  # [G, d]
+            z = scale * (Q @ K.T)  # [G, L]
+            z = z - z.max(axis=1, keepdims=True)
+            w = np.exp(z)
+            out[s, g * G:(g + 1) * G] = (w @ V) / w.sum(axis=1, keepdims=True)
+    return out
+
+
+def kv_write(key, value, slot_mapping, k_cache, v_cache) -> None:
+    bs = k_cache.shape[2]
+    for t, slot in enumerate(np.asarray(slot_mapping, dtype=np.int64)):
+        if slot < 0:
+            continue
+        blk, off = divmod(int(slot), bs)
+        k_cache[blk, :, off, :] = key[t]
+        v_cache[blk, :, off, :] = value[t]
+
+
+def copy_blocks(k_cache, v_cache, pairs) -> None:
+    for src, dst in np.asarray(pairs, dtype=np.int64).reshape(-1, 2):
+        k_cache[dst] = k_cache[src]
+        v_cache[dst] = v_cache[src]

@@ -1,0 +1,66 @@
+"""Structure of the seeded synthetic workloads (no GPU)."""
+import numpy as np
+
+from workloads import NAN_BITS, make_config
+from workloads.gen import make_prefix_cow
+
+
+def _check_tables(c):
+    bs = c.block_size
+    need = (c.context_lens.astype(np.int64) + bs - 1) // bs
+    used = []
+    for s in range(c.num_seqs):
+        row = c.block_tables[s]
+        assert np.all(row[: need[s]] >= 0) and np.all(row[: need[s]] < c.num_blocks)
+        assert np.all(row[need[s]:] == -1)
+        used.extend(row[: need[s]].tolist())
+    return used, need
+
+
+def test_tiny_matches_spec():
+    c = make_config("tiny")
+    assert (c.num_seqs, c.num_q_heads, c.num_kv_heads, c.head_dim, c.block_size) == (4, 4, 4, 64, 16)
+    assert c.dtype == "fp16" and c.scale == 1.0 / 8 and c.num_blocks == 64
+    assert c.context_lens.tolist() == [1, 17, 33, 100]
+    used, need = _check_tables(c)
+    assert need.tolist() == [1, 2, 3, 7]
+    assert len(set(used)) == len(used) == 13  # distinct ids carved from one permutation
+    # the new token lands at position L-1: L = 17, 33 start a block, L = 100 -> block 6, offset 3
+    for s, L in enumerate(c.context_lens):
+        blk, off = divmod(int(c.slot_mapping[s]), 16)
+        assert blk == c.block_tables[s, (L - 1) // 16] and off == (L - 1) % 16
+    assert [int(x) % 16 for x in c.slot_mapping] == [0, 0, 0, 3]
+
+
+def test_poison_marks_everything_not_read():
+    c = make_config("tiny")
+    nan = NAN_BITS["fp16"]
+    kept = 0
+    for s, L in enumerate(c.context_lens):
+        for t in range(int(L) - 1):
+            blk = c.block_tables[s, t // 16]
+            assert np.all(c.k_cache[blk, :, t % 16] != nan)
+            kept += 1
+    n_nan_rows = int(np.all(c.k_cache == nan, axis=-1).sum())
+    assert n_nan_rows == 64 * 4 * 16 - kept * 4
+
+
+def test_deterministic():
+    a, b = make_config("tiny"), make_config("tiny")
+    for f in ("q", "k_cache", "v_cache", "key", "value", "block_tables", "slot_mapping"):
+        assert np.array_equal(getattr(a, f), getattr(b, f))
+
+
+def test_prefix_cow_structure():
+    c = make_prefix_cow(groups=3, samples=8, max_suffix=40)
+    assert c.copy_pairs.shape == (3 * 7, 2)
+    assert np.all((c.context_lens >= 1001) & (c.context_lens <= 1041))
+    for g in range(3):
+        rows = c.block_tables[g * 8:(g + 1) * 8]
+        assert np.all(rows[:, :62] == rows[0, :62])  # shared full prefix blocks
+        partial = rows[:, 62]
+        assert partial[7] == c.copy_pairs[g * 7, 0]  # last sample keeps the original
+        assert len(set(partial.tolist())) == 8  # the rest own private copies
+    dst = c.copy_pairs[:, 1]
+    assert len(set(dst.tolist())) == len(dst) and not set(dst) & set(c.copy_pairs[:, 0])
+    assert len(set(c.slot_mapping.tolist())) == len(c.slot_mapping)
