@@ -1,0 +1,162 @@
+/*
+ * libpa -- paged KV-cache decode attention for NVIDIA B200 (sm_100a).
+ *
+ * C ABI.  Every pointer argument is DEVICE memory owned by the caller unless the
+ * comment says otherwise; the library allocates nothing on these paths.  Every
+ * call is asynchronous on `stream` (a cudaStream_t passed as void*, NULL = the
+ * legacy default stream) and never synchronises the device, except
+ * pa_get_device_error, which says so.
+ *
+ * Data layout (both caches, the same for every call):
+ *   k_cache, v_cache : [num_blocks][num_kv_heads][block_size][head_dim], 16-bit
+ *                      elements (pa_dtype); one (block, kv head) is one contiguous run.
+ *   block_tables     : int32 [num_seqs][max_blocks_per_seq]; entry j of row s is the
+ *                      physical block that holds logical tokens [j*bs, (j+1)*bs) of
+ *                      sequence s.  Entries at or past ceil(context_lens[s] / bs) are
+ *                      never read.
+ *   slot             : block * block_size + offset inside the block.
+ *
+ * Errors.  A problem the host can see (null or misaligned pointer, unsupported
+ * shape, too small a workspace) returns a status before anything is launched.  A
+ * problem in device data (a block id or slot outside the pool, a context longer
+ * than its table or than the partition grid, a bounded wait that expired) sets a
+ * bit in a sticky per-device error word (PA_DEVERR_*) and the offending item is
+ * skipped; its output is then unspecified.  No call traps, aborts or throws.
+ *
+ * Source of each operation: the vLLM paged-attention pages -- "IO-5 vLLM Paged
+ * Attention" note (sections 2-4: page table, K = concat of pages, attention
+ * unchanged) and the "PagedAttention and dynamic memory management" blog (KV of
+ * every generated token is stored in the cache; pages are shared between requests).
+ */
+#ifndef PA_H
+#define PA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    PA_OK = 0,
+    PA_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad size, workspace too small */
+    PA_ERR_UNSUPPORTED = 2, /* head_dim, block size or group size not built */
+    PA_ERR_CUDA = 3,        /* a CUDA runtime call failed (launch, attribute, ...) */
+    PA_ERR_OUT_OF_RANGE = 4,
+    PA_ERR_TIMEOUT = 5
+} pa_status;
+
+typedef enum { PA_FP16 = 0, PA_BF16 = 1 } pa_dtype;
+
+/* Bits of the sticky per-device error word. */
+#define PA_DEVERR_BLOCK_ID 0x1u /* a block table entry outside [0, num_blocks) */
+#define PA_DEVERR_SLOT 0x2u     /* a slot >= num_blocks * block_size */
+#define PA_DEVERR_PAIR 0x4u     /* a copy pair id outside [0, num_blocks) */
+#define PA_DEVERR_CONTEXT 0x8u  /* context longer than its table or the partition grid */
+#define PA_DEVERR_TIMEOUT 0x10u /* a bounded wait on a copy expired */
+
+/*
+ * Cache write ("PagedAttention and dynamic memory management" blog, first section:
+ * each generated token's K and V are stored in the KV cache; in a paged cache the
+ * store goes to the token's slot).
+ *
+ * For each token t < num_tokens with slot = slot_mapping[t] >= 0 and every kv head h:
+ *   k_cache[slot / block_size][h][slot % block_size][:] = key[t*key_token_stride + h*head_dim + :]
+ *   v_cache[...] likewise from value.   A negative slot is skipped.
+ * key, value      : [num_tokens][...] rows of num_kv_heads*head_dim elements, heads
+ *                   contiguous; token strides in ELEMENTS (multiple of 8).
+ * slot_mapping    : int64 [num_tokens].
+ * Alignment       : key, value, k_cache, v_cache 16-byte aligned.
+ * Duplicate slots within one call give an unspecified winner.
+ * Bit-exact copy of the 16-bit patterns.  head_dim multiple of 8, block_size >= 1.
+ */
+pa_status pa_kv_write(const void *key, const void *value, const int64_t *slot_mapping,
+                      int num_tokens, int num_kv_heads, int head_dim, int64_t key_token_stride,
+                      int64_t value_token_stride, void *k_cache, void *v_cache, int num_blocks,
+                      int block_size, pa_dtype dtype, void *stream);
+
+/*
+ * Block copy for copy-on-write of shared blocks (the pages let several requests
+ * share KV blocks -- "PagedAttention" summary, features 2; a sequence that appends
+ * into a shared, partially filled block first needs a private copy).
+ *
+ * For each pair p < num_pairs: block pairs[2p+1] := block pairs[2p] in both caches
+ * (all kv heads, all block_size slots).  src_dst_pairs: int64 [num_pairs][2], device.
+ * Destinations must be distinct and no destination may be a source of the same call.
+ * Bit-exact.  Caches 16-byte aligned; num_kv_heads*block_size*head_dim multiple of 8.
+ */
+pa_status pa_copy_blocks(void *k_cache, void *v_cache, const int64_t *src_dst_pairs,
+                         int num_pairs, int num_kv_heads, int block_size, int head_dim,
+                         int num_blocks, pa_dtype dtype, void *stream);
+
+/*
+ * Decode attention over the paged cache ("IO-5 vLLM Paged Attention" note, section 4:
+ * Attention(Q, K, V) = softmax(Q K^T / sqrt(d_k)) V with K, V loaded page by page,
+ * K = concat(K_page_a, K_page_b, ...) in table order; section 3: Sequence -> [page
+ * indices]).  For every sequence s and query head h, with G = num_q_heads /
+ * num_kv_heads and g = h / G:
+ *   out[s][h][:] = sum_{t < L} softmax_t(scale * <q[s][h], K_s[t]>) V_s[t]
+ *   K_s[t] = k_cache[block_tables[s][t / bs]][g][t % bs][:],   L = context_lens[s].
+ * L == 0 gives zeros.  Math in fp32 (online softmax), output rounded to nearest even.
+ *
+ * q, out          : [num_seqs][num_q_heads][head_dim], contiguous, 16-byte aligned.
+ * context_lens    : int32 [num_seqs].
+ * head_dim        : 64 or 128.  block_size: power of two in [8, 512].
+ * G               : 1, 2, 4 or 8.
+ * max_context_len : host-side upper bound of context_lens (0 = unknown: the table
+ *                   width max_blocks_per_seq * block_size is used).  A context longer
+ *                   than the bound sets PA_DEVERR_CONTEXT.
+ * partition_size  : tokens per context partition for the split-K path (a multiple of
+ *                   64), or 0 to let the library choose.  Contexts longer than one
+ *                   partition are processed in partitions whose fp32 partial results
+ *                   (running max, sum, normalised output) are merged by log-sum-exp.
+ * workspace       : fp32 scratch for those partial results, at least
+ *                   pa_decode_workspace_bytes(...) bytes, 256-byte aligned; may be
+ *                   NULL when no context needs more than one partition.  Its contents
+ *                   need no initialisation and are overwritten.  Calls that share a
+ *                   workspace must not overlap on the GPU.
+ * Launches 1 kernel (one partition per sequence) or 2 (partition pass + merge).
+ */
+pa_status pa_decode(void *out, const void *q, const void *k_cache, const void *v_cache,
+                    const int32_t *block_tables, const int32_t *context_lens, int num_seqs,
+                    int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                    int num_blocks, int max_blocks_per_seq, float scale, int max_context_len,
+                    int partition_size, void *workspace, size_t workspace_bytes, pa_dtype dtype,
+                    void *stream);
+
+/*
+ * Bytes of workspace pa_decode needs for these sizes and this partition_size
+ * (0 = the library's choice).  Host-only, no CUDA call.  Returns 0 when every
+ * context fits one partition.
+ */
+size_t pa_decode_workspace_bytes(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                                 int block_size, int max_blocks_per_seq, int max_context_len,
+                                 int partition_size);
+
+/*
+ * The partition size (tokens) pa_decode uses for these arguments when its
+ * partition_size argument is `partition_size` (0 = the library's choice); returns
+ * the whole context bound when one partition per sequence is used.  Host-only.
+ */
+int pa_decode_partition_tokens(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                               int block_size, int max_blocks_per_seq, int max_context_len,
+                               int partition_size);
+
+/*
+ * Reads (and with clear != 0 resets) the sticky error word of `device`.
+ * SYNCHRONISES that device first.  *bits_out receives PA_DEVERR_* bits (0 = none).
+ */
+pa_status pa_get_device_error(int device, uint32_t *bits_out, int clear);
+
+/* Static description of a status code.  Never NULL. */
+const char *pa_status_str(pa_status status);
+
+/* Library ABI version (major * 100 + minor). */
+int pa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PA_H */

@@ -1,0 +1,26 @@
+"""Paged KV-cache decode attention for B200 (sm_100a).
+
+The compute lives in ``libpa.so`` (CUDA kernels behind the C ABI in
+``include/pa.h``); this package is its Python binding.  Public calls:
+
+* ``kv_write(key, value, slot_mapping, k_cache, v_cache)`` -- scatter new tokens
+  into their cache slots;
+* ``copy_blocks(k_cache, v_cache, pairs)`` -- copy-on-write block copies;
+* ``decode(out, q, k_cache, v_cache, block_tables, context_lens, scale, ...)`` --
+  single-query attention through the block tables (single pass or split-K with a
+  log-sum-exp merge; GQA served from one page read per kv head).
+"""
+from ._lib import (  # noqa: F401
+    DEVERR,
+    EXPORTS,
+    LIB_PATH,
+    PAError,
+    copy_blocks,
+    decode,
+    decode_partition_tokens,
+    decode_workspace_bytes,
+    device_error,
+    kv_write,
+    load,
+    version,
+)

@@ -1,0 +1,147 @@
+"""ctypes binding of libpa (include/pa.h).  Argument marshalling only.
+
+Every function takes torch CUDA tensors, reads their pointers, shapes and the
+current CUDA stream, and calls the C entry point of the same name.  There is no
+fallback: if ``libpa.so`` is missing or a call fails, an exception is raised.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libpa.so")
+
+PA_FP16, PA_BF16 = 0, 1
+DEVERR = {"block_id": 0x1, "slot": 0x2, "pair": 0x4, "context": 0x8, "timeout": 0x10}
+EXPORTS = ("pa_kv_write", "pa_copy_blocks", "pa_decode", "pa_decode_workspace_bytes",
+           "pa_decode_partition_tokens", "pa_get_device_error", "pa_status_str", "pa_version")
+
+_lib = None
+
+
+class PAError(RuntimeError):
+    pass
+
+
+def load(path: str = LIB_PATH):
+    """Load libpa.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise PAError(f"libpa.so not found at {path}; build it with "
+                      "`python -m paged_kv_cache_441_b200.build`")
+    lib = ctypes.CDLL(path)
+    P, i32, i64, sz, f32 = (ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t,
+                            ctypes.c_float)
+    lib.pa_kv_write.argtypes = [P, P, P, i32, i32, i32, i64, i64, P, P, i32, i32, i32, P]
+    lib.pa_kv_write.restype = i32
+    lib.pa_copy_blocks.argtypes = [P, P, P, i32, i32, i32, i32, i32, i32, P]
+    lib.pa_copy_blocks.restype = i32
+    lib.pa_decode.argtypes = [P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, i32, f32, i32, i32,
+                              P, sz, i32, P]
+    lib.pa_decode.restype = i32
+    lib.pa_decode_workspace_bytes.argtypes = [i32] * 8
+    lib.pa_decode_workspace_bytes.restype = sz
+    lib.pa_decode_partition_tokens.argtypes = [i32] * 8
+    lib.pa_decode_partition_tokens.restype = i32
+    lib.pa_get_device_error.argtypes = [i32, ctypes.POINTER(ctypes.c_uint32), i32]
+    lib.pa_get_device_error.restype = i32
+    lib.pa_status_str.argtypes = [i32]
+    lib.pa_status_str.restype = ctypes.c_char_p
+    lib.pa_version.argtypes = []
+    lib.pa_version.restype = i32
+    _lib = lib
+    return lib
+
+
+def _check(status: int, what: str):
+    if status != 0:
+        msg = load().pa_status_str(status).decode()
+        raise PAError(f"{what} failed: status {status} ({msg})")
+
+
+def _dtype(t) -> int:
+    import torch
+    if t.dtype == torch.bfloat16:
+        return PA_BF16
+    if t.dtype == torch.float16:
+        return PA_FP16
+    raise PAError(f"unsupported dtype {t.dtype}")
+
+
+def _stream(stream):
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else None
+
+
+def kv_write(key, value, slot_mapping, k_cache, v_cache, stream=None) -> None:
+    """key/value [T, Hkv, d] (token stride may exceed Hkv*d), slot_mapping int64 [T]."""
+    T, hkv, d = key.shape
+    assert key.stride(2) == 1 and key.stride(1) == d and value.stride(1) == d
+    nb, _, bs, _ = k_cache.shape
+    _check(load().pa_kv_write(_ptr(key), _ptr(value), _ptr(slot_mapping), T, hkv, d,
+                              key.stride(0), value.stride(0), _ptr(k_cache), _ptr(v_cache), nb, bs,
+                              _dtype(k_cache), _stream(stream)), "pa_kv_write")
+
+
+def copy_blocks(k_cache, v_cache, pairs, stream=None) -> None:
+    """pairs int64 [P, 2] (src, dst) on the device."""
+    nb, hkv, bs, d = k_cache.shape
+    _check(load().pa_copy_blocks(_ptr(k_cache), _ptr(v_cache), _ptr(pairs), pairs.shape[0], hkv,
+                                 bs, d, nb, _dtype(k_cache), _stream(stream)), "pa_copy_blocks")
+
+
+def decode_workspace_bytes(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
+                           max_blocks_per_seq, max_context_len=0, partition_size=0) -> int:
+    return int(load().pa_decode_workspace_bytes(num_seqs, num_q_heads, num_kv_heads, head_dim,
+                                                block_size, max_blocks_per_seq, max_context_len,
+                                                partition_size))
+
+
+def decode_partition_tokens(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
+                            max_blocks_per_seq, max_context_len=0, partition_size=0) -> int:
+    return int(load().pa_decode_partition_tokens(num_seqs, num_q_heads, num_kv_heads, head_dim,
+                                                 block_size, max_blocks_per_seq, max_context_len,
+                                                 partition_size))
+
+
+def decode(out, q, k_cache, v_cache, block_tables, context_lens, scale, block_size=None,
+           max_context_len=0, partition_size=0, workspace=None, stream=None) -> None:
+    """out, q [B, Hq, d]; caches [NB, Hkv, bs, d]; block_tables int32 [B, W];
+    context_lens int32 [B].  ``workspace`` (a uint8 CUDA tensor) is allocated here
+    with torch when the plan needs one and none is given."""
+    import torch
+    B, hq, d = q.shape
+    nb, hkv, bs, _ = k_cache.shape
+    if block_size is not None and block_size != bs:
+        raise PAError(f"block_size {block_size} != cache block size {bs}")
+    W = block_tables.shape[1]
+    need = decode_workspace_bytes(B, hq, hkv, d, bs, W, max_context_len, partition_size)
+    if need and workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    wptr = _ptr(workspace) if workspace is not None else None
+    wbytes = workspace.numel() if workspace is not None else 0
+    _check(load().pa_decode(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
+                            _ptr(context_lens), B, hq, hkv, d, bs, nb, W, float(scale),
+                            int(max_context_len), int(partition_size), wptr, wbytes,
+                            _dtype(q), _stream(stream)), "pa_decode")
+
+
+def device_error(device: int = 0, clear: bool = True) -> int:
+    """Synchronises `device` and returns (and by default clears) its error bits."""
+    bits = ctypes.c_uint32(0)
+    _check(load().pa_get_device_error(device, ctypes.byref(bits), 1 if clear else 0),
+           "pa_get_device_error")
+    return int(bits.value)
+
+
+def version() -> int:
+    return int(load().pa_version())

@@ -1,0 +1,92 @@
+// Cache write (slot-mapped scatter of new tokens) and block copy (copy-on-write).
+//
+// Both are pure data movement at HBM bandwidth: 16-byte vector loads and stores,
+// several independent 16-byte transfers in flight per thread, bit-exact.
+#pragma once
+
+#include "pa_common.cuh"
+
+namespace pa {
+
+struct KvWriteParams {
+    const uint8_t *key;
+    const uint8_t *value;
+    const int64_t *slot_mapping;
+    uint8_t *k_cache;
+    uint8_t *v_cache;
+    long long key_stride_b;    // bytes between tokens of key
+    long long value_stride_b;  // bytes between tokens of value
+    long long num_slots;       // num_blocks * block_size
+    int num_tokens;
+    int num_kv_heads;
+    int row_chunks;            // head_dim / 8 (16-byte chunks per head row)
+    int block_size;
+};
+
+// One thread per 16-byte chunk of one (token, kv head) row, for K and V together.
+// "Every generated token's K and V are stored in the KV cache" (PagedAttention and
+// dynamic memory blog): the store goes to k_cache[slot / bs][h][slot % bs][:].
+__global__ void __launch_bounds__(256) pa_kv_write_kernel(const __grid_constant__ KvWriteParams p) {
+    const long long per_tok = (long long)p.num_kv_heads * p.row_chunks;
+    const long long total = per_tok * p.num_tokens;
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
+         i += (long long)gridDim.x * blockDim.x) {
+        const int t = (int)(i / per_tok);
+        const int rem = (int)(i % per_tok);
+        const int h = rem / p.row_chunks, c = rem % p.row_chunks;
+        const long long slot = p.slot_mapping[t];
+        if (slot < 0) continue;
+        if (slot >= p.num_slots) {
+            if (rem == 0) raise_error(PA_DEVERR_SLOT);
+            continue;
+        }
+        const long long blk = slot / p.block_size, off = slot % p.block_size;
+        const long long row = ((blk * p.num_kv_heads + h) * p.block_size + off) * p.row_chunks + c;
+        const long long src_off = (long long)(h * p.row_chunks + c) * 16;
+        const uint4 kv = ld_global_nc_v4(p.key + t * p.key_stride_b + src_off);
+        const uint4 vv = ld_global_nc_v4(p.value + t * p.value_stride_b + src_off);
+        reinterpret_cast<uint4 *>(p.k_cache)[row] = kv;
+        reinterpret_cast<uint4 *>(p.v_cache)[row] = vv;
+    }
+}
+
+struct CopyBlocksParams {
+    uint8_t *k_cache;
+    uint8_t *v_cache;
+    const int64_t *pairs;
+    long long block_chunks;  // 16-byte chunks per block per cache
+    int num_blocks;
+    int num_pairs;
+};
+
+constexpr int kCopyThreads = 256;
+constexpr int kCopyUnroll = 4;
+
+// grid = (chunks_of_a_block / (256 * 4) rounded up, num_pairs, 2 caches).
+// Each thread keeps kCopyUnroll 16-byte loads in flight before storing.
+__global__ void __launch_bounds__(kCopyThreads)
+    pa_copy_blocks_kernel(const __grid_constant__ CopyBlocksParams p) {
+    const int pair = blockIdx.y;
+    const long long src = p.pairs[2 * pair], dst = p.pairs[2 * pair + 1];
+    if (src < 0 || src >= p.num_blocks || dst < 0 || dst >= p.num_blocks) {
+        if (blockIdx.x == 0 && blockIdx.z == 0 && threadIdx.x == 0) raise_error(PA_DEVERR_PAIR);
+        return;
+    }
+    uint4 *cache = reinterpret_cast<uint4 *>(blockIdx.z == 0 ? p.k_cache : p.v_cache);
+    const uint4 *from = cache + src * p.block_chunks;
+    uint4 *to = cache + dst * p.block_chunks;
+    const long long c0 = (long long)blockIdx.x * kCopyThreads * kCopyUnroll + threadIdx.x;
+    uint4 buf[kCopyUnroll];
+#pragma unroll
+    for (int u = 0; u < kCopyUnroll; ++u) {
+        const long long c = c0 + (long long)u * kCopyThreads;
+        if (c < p.block_chunks) buf[u] = ld_global_nc_v4(from + c);
+    }
+#pragma unroll
+    for (int u = 0; u < kCopyUnroll; ++u) {
+        const long long c = c0 + (long long)u * kCopyThreads;
+        if (c < p.block_chunks) to[c] = buf[u];
+    }
+}
+
+}  // namespace pa

@@ -1,0 +1,624 @@
+// Paged decode attention kernels (sm_100a).
+//
+// What is computed ("IO-5 vLLM Paged Attention" note, sections 3-4): for sequence s
+// and query head h (kv head g = h / G),
+//     out[s][h] = softmax_t(scale * q[s][h] . K_s[t]) V_s[t],  t < L_s,
+// where K_s is the sequence's pages concatenated in block-table order.  The
+// arithmetic is the textbook one evaluated as an online softmax in fp32 (running
+// max m, running sum l, rescaled accumulator), so the pages' statement that paging
+// leaves the attention unchanged holds up to fp32 rounding.
+//
+// Work decomposition.  One CTA owns one item (sequence s, kv head g, context
+// partition p of `partition_tokens` tokens).  Its kWarps warps split the item's
+// 16-token tiles into contiguous runs.  Each warp streams its tiles through its own
+// kStages-deep ring in shared memory: lane 0 issues 2-D TMA loads (128-byte
+// swizzled boxes of 64 columns x min(bs, 16) rows) for the K and V rows of a tile
+// into a stage, completion is tracked by one mbarrier per stage, and the whole warp
+// consumes the stage once the barrier flips.  The block-table row is read 32
+// entries at a time with one coalesced load and broadcast by shuffles, so the table
+// lookup for tile j+kStages is done while tile j is being consumed.
+//
+// Compute per tile:
+//  * G <= 2 (SIMT): 16 (or 8) lanes cover one 128-wide (64-wide) row with 16-byte
+//    shared loads; q.k partial sums are reduced with a transposing butterfly
+//    (one shuffle per row and head), p.V with one broadcast shuffle per row and head.
+//  * G >= 4 (tensor cores): S^T[16 tokens x 8 heads] = K_tile . Q^T with
+//    mma.m16n8k16 (K from ldmatrix, Q^T kept in registers), then
+//    O^T[d x 8 heads] += V_tile^T . P^T with the probabilities P split into a
+//    high and a low 16-bit part (two mma per tile), so P keeps ~16 significant bits
+//    (fp32-grade accuracy for the weights) while the one page read serves all G heads.
+//
+// The warps' (m, l, O) are merged in shared memory.  A sequence that fits one
+// partition is written to `out` directly; otherwise the partition writes its fp32
+// (m, l, O/l) to the workspace and pa_merge_kernel combines the partitions by
+// log-sum-exp:  M = max m_p,  w_p = l_p 2^(m_p - M),  out = sum w_p o_p / sum w_p
+// (m is kept in the log2 domain: scores are pre-multiplied by scale * log2(e)).
+#pragma once
+
+#include "pa_common.cuh"
+
+namespace pa {
+
+constexpr int kTile = 16;   // tokens per tile (one mma M/K extent)
+constexpr int kWarps = 4;   // warps per CTA
+constexpr int kStages = 3;  // ring depth per warp
+constexpr unsigned kFull = 0xffffffffu;
+
+struct DecodeParams {
+    CUtensorMap kmap;  // [rows = num_blocks*Hkv*bs][D] 16-bit, box 64 x min(bs,16), swizzle 128B
+    CUtensorMap vmap;
+    void *out;
+    const void *q;
+    const int32_t *block_tables;
+    const int32_t *context_lens;
+    float *ws_o;  // [B][Hq][num_parts][D]
+    float *ws_m;  // [B][Hq][num_parts]
+    float *ws_l;  // [B][Hq][num_parts]
+    int num_q_heads;
+    int num_kv_heads;
+    int block_size;
+    int bs_shift;
+    int num_blocks;
+    int max_blocks_per_seq;
+    int partition_tokens;
+    int num_parts;
+    float scale_log2;
+};
+
+template <int D>
+struct Geom {
+    static constexpr int kHalves = D / 64;             // 128-byte column blocks per row
+    static constexpr int kRegion = kTile * 128;        // one column block of a tile
+    static constexpr int kMat = kHalves * kRegion;     // a 16 x D tile
+    static constexpr int kStage = 2 * kMat;            // K tile + V tile
+    static constexpr int kRing = kWarps * kStages * kStage;
+    static constexpr int kSmem = kRing + kWarps * kStages * 8 + 1024;  // + barriers + align
+};
+
+// Byte offset of 16-byte chunk `chunk` of row `row` in a tile as the TMA stores it:
+// column block chunk/8, then the 128-byte swizzle (chunk%8) ^ (row%8).
+__device__ __forceinline__ uint32_t tile_off(int row, int chunk) {
+    return (chunk >> 3) * (kTile * 128) + row * 128 + (((chunk & 7) ^ (row & 7)) << 4);
+}
+
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+    uint4 r;
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+                 : "r"(addr));
+    return r;
+}
+
+__device__ __forceinline__ void sts128_zero(uint32_t addr) {
+    asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(addr), "r"(0) : "memory");
+}
+
+// Transposing butterfly sum over the lanes that differ in bits MASK, MASK/2, ..., 1:
+// N values per lane in, the full sum of value index (lane bits from MASK down) out
+// in v[0].  N/2 + N/4 + ... shuffles instead of N * log2(lanes).
+template <int N, int MASK>
+struct Butterfly {
+    __device__ __forceinline__ static void run(float *v, int lane) {
+        if constexpr (MASK == 0) {
+            return;
+        } else if constexpr (N > 1) {
+            const bool upper = (lane & MASK) != 0;
+#pragma unroll
+            for (int k = 0; k < N / 2; ++k) {
+                const float send = upper ? v[k] : v[k + N / 2];
+                const float keep = upper ? v[k + N / 2] : v[k];
+                v[k] = keep + __shfl_xor_sync(kFull, send, MASK);
+            }
+            Butterfly<N / 2, MASK / 2>::run(v, lane);
+        } else {
+            v[0] += __shfl_xor_sync(kFull, v[0], MASK);
+            Butterfly<1, MASK / 2>::run(v, lane);
+        }
+    }
+};
+
+constexpr int ilog2(int x) { return x <= 1 ? 0 : 1 + ilog2(x / 2); }
+
+// --------------------------------------------------------------------------- SIMT path
+
+template <typename T, int D, int G>
+struct SimtWarp {
+    static constexpr int kCpr = D / 8;               // 16-byte chunks per row
+    static constexpr int kRps = 32 / kCpr;           // rows per warp step
+    static constexpr int kSteps = kTile / kRps;      // steps per tile
+    static constexpr int kN = kSteps * G;            // partial sums per lane per tile
+    static constexpr int kShift = ilog2(kCpr) - ilog2(kN);  // replicated low lane bits
+    static_assert(kN <= kCpr, "SIMT path needs steps*G <= chunks per row");
+
+    float qf[G][8];
+    float acc[G][8];
+    float m;  // running max (log2 domain) of this lane's head
+    float l;  // this lane's share of the running sum of its head
+    int lig, rr, c, my_v, my_i, my_h, my_row;
+    bool owner;
+
+    __device__ __forceinline__ void init(const T *q_item, int lane) {
+        lig = lane & (kCpr - 1);
+        rr = lane / kCpr;
+        c = lig;
+        my_v = lig >> kShift;
+        my_i = my_v / G;
+        my_h = my_v % G;
+        my_row = my_i * kRps + rr;
+        owner = (lig & ((1 << kShift) - 1)) == 0;
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+            const uint4 w = *reinterpret_cast<const uint4 *>(q_item + h * D + 8 * c);
+            const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 f = Fmt<T>::unpack(ws[e]);
+                qf[h][2 * e] = f.x;
+                qf[h][2 * e + 1] = f.y;
+            }
+#pragma unroll
+            for (int e = 0; e < 8; ++e) acc[h][e] = 0.f;
+        }
+        m = -INFINITY;
+        l = 0.f;
+    }
+
+    __device__ __forceinline__ void tile(uint32_t kd, uint32_t vd, int nrows, float sl2,
+                                         int lane) {
+        float v[kN];
+#pragma unroll
+        for (int i = 0; i < kSteps; ++i) {
+            const int r = i * kRps + rr;
+            const uint4 w = lds128(kd + tile_off(r, c));
+            const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+            float kf[8];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 f = Fmt<T>::unpack(ws[e]);
+                kf[2 * e] = f.x;
+                kf[2 * e + 1] = f.y;
+            }
+#pragma unroll
+            for (int h = 0; h < G; ++h) {
+                float a = 0.f;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) a = fmaf(qf[h][e], kf[e], a);
+                v[i * G + h] = a;
+            }
+        }
+        Butterfly<kN, kCpr / 2>::run(v, lane);
+        const bool valid = my_row < nrows;
+        const float sc = valid ? v[0] * sl2 : -INFINITY;
+        // tile max of this lane's head: all lane bits except the head bits
+        float mx = sc;
+#pragma unroll
+        for (int mask = 1; mask < 32; mask <<= 1) {
+            if (G > 1 && mask >= (1 << kShift) && mask < ((1 << kShift) * G)) continue;
+            mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, mask));
+        }
+        const float mn = fmaxf(m, mx);
+        const float alpha = (mn == -INFINITY) ? 1.f : fast_exp2(m - mn);
+        const float pr = valid ? fast_exp2(sc - mn) : 0.f;
+        m = mn;
+        l = l * alpha + (owner ? pr : 0.f);
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+            const float ah = (G == 1) ? alpha : __shfl_sync(kFull, alpha, h << kShift);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) acc[h][e] *= ah;
+        }
+        const int grp = lane & ~(kCpr - 1);
+#pragma unroll
+        for (int i = 0; i < kSteps; ++i) {
+            float ph[G];
+#pragma unroll
+            for (int h = 0; h < G; ++h) ph[h] = __shfl_sync(kFull, pr, grp | ((i * G + h) << kShift));
+            const int r = i * kRps + rr;
+            if (r < nrows) {
+                const uint4 w = lds128(vd + tile_off(r, c));
+                const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 f = Fmt<T>::unpack(ws[e]);
+#pragma unroll
+                    for (int h = 0; h < G; ++h) {
+                        acc[h][2 * e] = fmaf(ph[h], f.x, acc[h][2 * e]);
+                        acc[h][2 * e + 1] = fmaf(ph[h], f.y, acc[h][2 * e + 1]);
+                    }
+                }
+            }
+        }
+    }
+
+    // Writes this warp's O[G][D], m[G], l[G] (fp32) at `dst`.
+    __device__ __forceinline__ void finish(float *dst, int lane) {
+#pragma unroll
+        for (int mask = kCpr; mask < 32; mask <<= 1)
+#pragma unroll
+            for (int h = 0; h < G; ++h)
+#pragma unroll
+                for (int e = 0; e < 8; ++e) acc[h][e] += __shfl_xor_sync(kFull, acc[h][e], mask);
+        float lt = l;
+#pragma unroll
+        for (int mask = 1; mask < 32; mask <<= 1) {
+            if (G > 1 && mask >= (1 << kShift) && mask < ((1 << kShift) * G)) continue;
+            lt += __shfl_xor_sync(kFull, lt, mask);
+        }
+        if (lane < kCpr) {
+#pragma unroll
+            for (int h = 0; h < G; ++h)
+#pragma unroll
+                for (int e = 0; e < 8; ++e) dst[h * D + 8 * c + e] = acc[h][e];
+        }
+        if (lane < (G << kShift) && (lane & ((1 << kShift) - 1)) == 0) {
+            dst[G * D + my_h] = m;
+            dst[G * D + G + my_h] = lt;
+        }
+    }
+};
+
+// ---------------------------------------------------------------- tensor-core path
+
+template <typename T, int D, int G>
+struct MmaWarp {
+    static constexpr int kK = D / 16;  // k-steps of QK^T, m-tiles of PV
+    static_assert(G <= 8, "one mma N extent holds at most 8 heads");
+
+    uint32_t qb[kK][2];  // Q^T B-fragments (heads >= G are zero)
+    float o[kK][4];      // O^T accumulators: (d = 16mt + gq (+8), heads 2tq, 2tq+1)
+    float m0, m1, l0, l1;
+    int gq, tq;
+
+    __device__ __forceinline__ void init(const T *q_item, int lane) {
+        gq = lane >> 2;
+        tq = lane & 3;
+#pragma unroll
+        for (int kk = 0; kk < kK; ++kk) {
+            if (gq < G) {
+                const T *qh = q_item + gq * D + 16 * kk + 2 * tq;
+                qb[kk][0] = *reinterpret_cast<const uint32_t *>(qh);
+                qb[kk][1] = *reinterpret_cast<const uint32_t *>(qh + 8);
+            } else {
+                qb[kk][0] = 0u;
+                qb[kk][1] = 0u;
+            }
+#pragma unroll
+            for (int e = 0; e < 4; ++e) o[kk][e] = 0.f;
+        }
+        m0 = m1 = -INFINITY;
+        l0 = l1 = 0.f;
+    }
+
+    __device__ __forceinline__ void tile(uint32_t kd, uint32_t vd, int nrows, float sl2,
+                                         int lane) {
+        const int j = lane >> 3, r8 = lane & 7;
+        // S^T = K . Q^T  (A = K rows from ldmatrix: matrix j -> rows +8*(j&1), k +8*(j>>1))
+        float sc[4] = {0.f, 0.f, 0.f, 0.f};
+        {
+            const int row = r8 + ((j & 1) << 3);
+#pragma unroll
+            for (int kk = 0; kk < kK; ++kk) {
+                uint32_t a[4];
+                ldsm_x4(kd + tile_off(row, 2 * kk + (j >> 1)), a[0], a[1], a[2], a[3]);
+                Mma<T>::run(sc, a, qb[kk][0], qb[kk][1]);
+            }
+        }
+        const bool v0 = gq < nrows, v1 = gq + 8 < nrows;
+        const float s0 = v0 ? sc[0] * sl2 : -INFINITY;
+        const float s1 = v0 ? sc[1] * sl2 : -INFINITY;
+        const float s2 = v1 ? sc[2] * sl2 : -INFINITY;
+        const float s3 = v1 ? sc[3] * sl2 : -INFINITY;
+        float mx0 = fmaxf(s0, s2), mx1 = fmaxf(s1, s3);
+#pragma unroll
+        for (int mask = 4; mask < 32; mask <<= 1) {
+            mx0 = fmaxf(mx0, __shfl_xor_sync(kFull, mx0, mask));
+            mx1 = fmaxf(mx1, __shfl_xor_sync(kFull, mx1, mask));
+        }
+        const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+        const float al0 = (mn0 == -INFINITY) ? 1.f : fast_exp2(m0 - mn0);
+        const float al1 = (mn1 == -INFINITY) ? 1.f : fast_exp2(m1 - mn1);
+        m0 = mn0;
+        m1 = mn1;
+        const float p0 = v0 ? fast_exp2(s0 - mn0) : 0.f;
+        const float p1 = v0 ? fast_exp2(s1 - mn1) : 0.f;
+        const float p2 = v1 ? fast_exp2(s2 - mn0) : 0.f;
+        const float p3 = v1 ? fast_exp2(s3 - mn1) : 0.f;
+        l0 = l0 * al0 + (p0 + p2);
+        l1 = l1 * al1 + (p1 + p3);
+#pragma unroll
+        for (int mt = 0; mt < kK; ++mt) {
+            o[mt][0] *= al0;
+            o[mt][1] *= al1;
+            o[mt][2] *= al0;
+            o[mt][3] *= al1;
+        }
+        // P^T as B fragments: hi = RN(p), lo = RN(p - hi); the 8x8 transposes turn the
+        // (token row, head pair) layout of S^T into the (token pair, head) layout of B.
+        const uint32_t x0 = Fmt<T>::pack_rn(p0, p1), x1 = Fmt<T>::pack_rn(p2, p3);
+        const float2 h0 = Fmt<T>::unpack(x0), h1 = Fmt<T>::unpack(x1);
+        const uint32_t y0 = Fmt<T>::pack_rn(p0 - h0.x, p1 - h0.y);
+        const uint32_t y1 = Fmt<T>::pack_rn(p2 - h1.x, p3 - h1.y);
+        const uint32_t bh0 = movmatrix_trans(x0), bh1 = movmatrix_trans(x1);
+        const uint32_t bl0 = movmatrix_trans(y0), bl1 = movmatrix_trans(y1);
+        // rows past the context may hold anything (NaN): zero them so 0 * V stays 0
+        if (nrows < kTile) {
+            constexpr int kChunks = Geom<D>::kHalves * 8;
+            for (int idx = lane; idx < (kTile - nrows) * kChunks; idx += 32) {
+                const int r = nrows + idx / kChunks;
+                const int ch = idx % kChunks;
+                sts128_zero(vd + (ch >> 3) * (kTile * 128) + r * 128 + ((ch & 7) << 4));
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+        }
+        // O^T += V^T . P^T  (A = V^T via ldmatrix.trans: matrix j -> tokens +8*(j>>1),
+        // dims +8*(j&1))
+        {
+            const int row = r8 + ((j >> 1) << 3);
+#pragma unroll
+            for (int mt = 0; mt < kK; ++mt) {
+                uint32_t a[4];
+                ldsm_x4_trans(vd + tile_off(row, 2 * mt + (j & 1)), a[0], a[1], a[2], a[3]);
+                Mma<T>::run(o[mt], a, bh0, bh1);
+                Mma<T>::run(o[mt], a, bl0, bl1);
+            }
+        }
+    }
+
+    __device__ __forceinline__ void finish(float *dst, int lane) {
+        float lt0 = l0, lt1 = l1;
+#pragma unroll
+        for (int mask = 4; mask < 32; mask <<= 1) {
+            lt0 += __shfl_xor_sync(kFull, lt0, mask);
+            lt1 += __shfl_xor_sync(kFull, lt1, mask);
+        }
+        const int h0 = 2 * tq, h1 = 2 * tq + 1;
+#pragma unroll
+        for (int mt = 0; mt < kK; ++mt) {
+            const int d = 16 * mt + gq;
+            if (h0 < G) {
+                dst[h0 * D + d] = o[mt][0];
+                dst[h0 * D + d + 8] = o[mt][2];
+            }
+            if (h1 < G) {
+                dst[h1 * D + d] = o[mt][1];
+                dst[h1 * D + d + 8] = o[mt][3];
+            }
+        }
+        if (gq == 0) {
+            if (h0 < G) {
+                dst[G * D + h0] = m0;
+                dst[G * D + G + h0] = lt0;
+            }
+            if (h1 < G) {
+                dst[G * D + h1] = m1;
+                dst[G * D + G + h1] = lt1;
+            }
+        }
+    }
+};
+
+template <typename T, int D, int G>
+using WarpCompute = typename std::conditional<(G >= 4), MmaWarp<T, D, G>, SimtWarp<T, D, G>>::type;
+
+// ------------------------------------------------------------------ partition kernel
+
+template <typename T, int D, int G, int BOXR>
+__global__ void __launch_bounds__(kWarps * 32)
+    pa_decode_partition_kernel(const __grid_constant__ DecodeParams p) {
+    using Gm = Geom<D>;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    uint8_t *base_ptr = smem_raw + (base - raw);
+
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5, lane = tid & 31;
+    const int part = blockIdx.x, g = blockIdx.y, s = blockIdx.z;
+    const int Hq = p.num_q_heads;
+
+    int L = p.context_lens[s];
+    const int cap = p.max_blocks_per_seq << p.bs_shift;
+    if (L < 0 || L > cap) {
+        if (tid == 0 && part == 0) raise_error(PA_DEVERR_CONTEXT);
+        L = L < 0 ? 0 : cap;
+    }
+    const int P = p.partition_tokens;
+    const int nparts = (L + P - 1) / P;
+    if (nparts > p.num_parts && tid == 0 && part == 0) raise_error(PA_DEVERR_CONTEXT);
+    T *out = reinterpret_cast<T *>(p.out) + ((size_t)s * Hq + (size_t)g * G) * D;
+    if (L == 0) {
+        if (part == 0)
+            for (int e = tid; e < G * D; e += kWarps * 32) out[e] = Fmt<T>::from_float(0.f);
+        return;
+    }
+    if (part >= nparts) return;
+
+    const int t0 = part * P, t1 = min(t0 + P, L);
+    const int ntiles = (t1 - t0 + kTile - 1) / kTile;
+    const int qd = ntiles / kWarps, rm = ntiles % kWarps;
+    const int wt0 = warp * qd + min(warp, rm);
+    const int nt = qd + (warp < rm ? 1 : 0);
+    const int tok_begin = t0 + wt0 * kTile;
+    const int tok_end = min(tok_begin + nt * kTile, t1);
+
+    const uint32_t bars_all = base + Gm::kRing;
+    const uint32_t ring = base + warp * kStages * Gm::kStage;
+    const uint32_t bars = bars_all + warp * kStages * 8;
+    if (tid == 0) {
+        tma_prefetch_desc(&p.kmap);
+        tma_prefetch_desc(&p.vmap);
+        for (int i = 0; i < kWarps * kStages; ++i) mbar_init(bars_all + 8 * i, 1);
+        fence_barrier_init();
+    }
+
+    const T *q_item = reinterpret_cast<const T *>(p.q) + ((size_t)s * Hq + (size_t)g * G) * D;
+    WarpCompute<T, D, G> wc;
+    wc.init(q_item, lane);
+
+    const int32_t *table = p.block_tables + (size_t)s * p.max_blocks_per_seq;
+    const int npages = (L + p.block_size - 1) >> p.bs_shift;
+    int tab_base = -(1 << 30), tab_reg = -1;
+    const uint64_t pol = l2_policy_evict_first();
+    unsigned okmask = 0;
+
+    __syncthreads();
+
+    auto lookup = [&](int pg) -> int {
+        if (pg < tab_base || pg >= tab_base + 32) {  // warp-uniform
+            tab_base = pg;
+            const int e = pg + lane;
+            tab_reg = e < npages ? __ldg(table + e) : -1;
+        }
+        return __shfl_sync(kFull, tab_reg, pg - tab_base);
+    };
+
+    auto produce = [&](int jt) {
+        const int stage = jt % kStages;
+        const int tok = tok_begin + jt * kTile;
+        const int nrows = min(kTile, tok_end - tok);
+        constexpr int kBoxes = kTile / BOXR;
+        int ys[kBoxes];
+        int nbox = 0;
+        bool ok = true;
+#pragma unroll
+        for (int b = 0; b < kBoxes; ++b) {
+            ys[b] = 0;
+            if (b * BOXR < nrows) {
+                const int tb = tok + b * BOXR;
+                const int blk = lookup(tb >> p.bs_shift);
+                if ((unsigned)blk < (unsigned)p.num_blocks)
+                    ys[b] = (blk * p.num_kv_heads + g) * p.block_size + (tb & (p.block_size - 1));
+                else
+                    ok = false;
+                nbox = b + 1;
+            }
+        }
+        const uint32_t bar = bars + 8 * stage;
+        const uint32_t kd = ring + stage * Gm::kStage, vd = kd + Gm::kMat;
+        if (lane == 0) {
+            if (ok) {
+                mbar_arrive_expect_tx(bar, (uint32_t)(nbox * Gm::kHalves * BOXR * 128 * 2));
+#pragma unroll
+                for (int b = 0; b < kBoxes; ++b) {
+                    if (b < nbox) {
+#pragma unroll
+                        for (int hf = 0; hf < Gm::kHalves; ++hf) {
+                            const uint32_t off = hf * Gm::kRegion + b * BOXR * 128;
+                            tma_load_2d(kd + off, &p.kmap, bar, 64 * hf, ys[b], pol);
+                            tma_load_2d(vd + off, &p.vmap, bar, 64 * hf, ys[b], pol);
+                        }
+                    }
+                }
+            } else {
+                raise_error(PA_DEVERR_BLOCK_ID);
+                mbar_arrive(bar);
+            }
+        }
+        okmask = ok ? (okmask | (1u << stage)) : (okmask & ~(1u << stage));
+    };
+
+    const int npre = min(kStages, nt);
+    for (int jt = 0; jt < npre; ++jt) produce(jt);
+
+    bool failed = false;
+    for (int jt = 0; jt < nt; ++jt) {
+        const int stage = jt % kStages;
+        const uint32_t parity = (uint32_t)((jt / kStages) & 1);
+        const bool got = mbar_wait_bounded(bars + 8 * stage, parity);
+        if (!__all_sync(kFull, got)) {
+            // give up on this item: record it, wait (bounded) for the copies in flight
+            if (lane == 0) raise_error(PA_DEVERR_TIMEOUT);
+            for (int k = jt + 1; k < min(jt + kStages, nt); ++k)
+                (void)mbar_wait_bounded(bars + 8 * (k % kStages), (uint32_t)((k / kStages) & 1));
+            failed = true;
+            break;
+        }
+        const int tok = tok_begin + jt * kTile;
+        const int nrows = ((okmask >> stage) & 1u) ? min(kTile, tok_end - tok) : 0;
+        const uint32_t kd = ring + stage * Gm::kStage, vd = kd + Gm::kMat;
+        wc.tile(kd, vd, nrows, p.scale_log2, lane);
+        __syncwarp();
+        if (jt + kStages < nt) produce(jt + kStages);
+    }
+    if (failed) wc.init(q_item, lane);  // contributes nothing (m = -inf, l = 0)
+
+    // ---- merge the warps' partial softmax states (each warp uses its own ring)
+    float *mine = reinterpret_cast<float *>(base_ptr + warp * kStages * Gm::kStage);
+    wc.finish(mine, lane);
+    __syncthreads();
+
+    const bool single = (nparts == 1);
+    const size_t item = ((size_t)s * Hq + (size_t)g * G) * p.num_parts + part;
+    for (int e = tid; e < G * D; e += kWarps * 32) {
+        const int h = e / D, d = e % D;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) {
+            const float *src = reinterpret_cast<const float *>(base_ptr + w * kStages * Gm::kStage);
+            M = fmaxf(M, src[G * D + h]);
+        }
+        float num = 0.f, den = 0.f;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) {
+            const float *src = reinterpret_cast<const float *>(base_ptr + w * kStages * Gm::kStage);
+            const float mw = src[G * D + h];
+            if (mw != -INFINITY) {
+                const float wt = fast_exp2(mw - M);
+                num = fmaf(src[h * D + d], wt, num);
+                den = fmaf(src[G * D + G + h], wt, den);
+            }
+        }
+        const float val = den > 0.f ? num / den : 0.f;
+        if (single) {
+            out[e] = Fmt<T>::from_float(val);
+        } else {
+            const size_t idx = item + (size_t)h * p.num_parts;
+            p.ws_o[idx * D + d] = val;
+            if (d == 0) {
+                p.ws_m[idx] = M;
+                p.ws_l[idx] = den;
+            }
+        }
+    }
+}
+
+// ------------------------------------------------------------------------ merge kernel
+
+struct MergeParams {
+    void *out;
+    const int32_t *context_lens;
+    const float *ws_o;
+    const float *ws_m;
+    const float *ws_l;
+    int num_q_heads;
+    int cap;  // max_blocks_per_seq * block_size
+    int partition_tokens;
+    int num_parts;
+};
+
+// One CTA per (q head, sequence), one thread per output element.
+template <typename T, int D>
+__global__ void __launch_bounds__(D) pa_merge_kernel(const __grid_constant__ MergeParams p) {
+    const int h = blockIdx.x, s = blockIdx.y, d = threadIdx.x;
+    int L = p.context_lens[s];
+    L = L < 0 ? 0 : (L > p.cap ? p.cap : L);
+    int n = (L + p.partition_tokens - 1) / p.partition_tokens;
+    if (n <= 1) return;
+    n = min(n, p.num_parts);
+    const size_t base = ((size_t)s * p.num_q_heads + h) * p.num_parts;
+    float M = -INFINITY;
+    for (int i = 0; i < n; ++i) M = fmaxf(M, p.ws_m[base + i]);
+    float num = 0.f, den = 0.f;
+    for (int i = 0; i < n; ++i) {
+        const float mi = p.ws_m[base + i];
+        if (mi == -INFINITY) continue;
+        const float w = p.ws_l[base + i] * fast_exp2(mi - M);
+        num = fmaf(w, p.ws_o[(base + i) * D + d], num);
+        den += w;
+    }
+    T *out = reinterpret_cast<T *>(p.out) + ((size_t)s * p.num_q_heads + h) * D;
+    out[d] = Fmt<T>::from_float(den > 0.f ? num / den : 0.f);
+}
+
+}  // namespace pa

@@ -1,0 +1,381 @@
+// libpa host side: argument checks, launch planning and the C entry points of
+// include/pa.h.  One translation unit, so the device error word has one definition.
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstring>
+#include <mutex>
+#include <type_traits>
+
+#include "pa_cache.cuh"
+#include "pa_common.cuh"
+#include "pa_decode.cuh"
+
+using namespace pa;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr int kAutoSplitTokens = 512;   // partition size of the split-K path
+constexpr int kAutoSingleMax = 1024;    // contexts up to this stay single-partition
+
+bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+bool pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
+int ilog2_host(int x) {
+    int r = 0;
+    while ((1 << r) < x) ++r;
+    return r;
+}
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000,
+                                             cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    });
+    return fn;
+}
+
+// 2-D map over a cache seen as [rows][D] 16-bit elements; box 64 columns x boxr rows,
+// 128-byte swizzle (the layout the decode kernel's shared-memory reads assume).
+bool make_cache_map(CUtensorMap *m, const void *base, unsigned long long rows, int D,
+                    pa_dtype dt, int boxr) {
+    auto enc = encode_fn();
+    if (!enc) return false;
+    const CUtensorMapDataType t =
+        dt == PA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)D * 2};
+    cuuint32_t box[2] = {64u, (cuuint32_t)boxr};
+    cuuint32_t estr[2] = {1u, 1u};
+    return enc(m, t, 2, const_cast<void *>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+struct Plan {
+    int partition_tokens = 0;
+    int num_parts = 1;
+    size_t ws_bytes = 0;
+    size_t off_m = 0, off_l = 0;
+};
+
+Plan make_plan(int num_seqs, int num_q_heads, int head_dim, int block_size,
+               int max_blocks_per_seq, int max_context_len, int partition_size) {
+    Plan pl;
+    const long long cap = (long long)max_blocks_per_seq * block_size;
+    long long bound = cap;
+    if (max_context_len > 0 && max_context_len < cap) bound = max_context_len;
+    if (bound < 1) bound = 1;
+    long long P;
+    if (partition_size > 0)
+        P = partition_size;
+    else if (bound <= kAutoSingleMax)
+        P = round_up((size_t)bound, 64);
+    else
+        P = kAutoSplitTokens;
+    if (P > (1LL << 30)) P = 1LL << 30;
+    pl.partition_tokens = (int)P;
+    pl.num_parts = (int)((bound + P - 1) / P);
+    if (pl.num_parts > 1) {
+        const size_t n = (size_t)num_seqs * num_q_heads * pl.num_parts;
+        const size_t o_bytes = round_up(n * head_dim * sizeof(float), 256);
+        const size_t v_bytes = round_up(n * sizeof(float), 256);
+        pl.off_m = o_bytes;
+        pl.off_l = o_bytes + v_bytes;
+        pl.ws_bytes = o_bytes + 2 * v_bytes;
+    }
+    return pl;
+}
+
+int current_device() {
+    int d = 0;
+    if (cudaGetDevice(&d) != cudaSuccess) return -1;
+    return d;
+}
+
+template <typename K>
+cudaError_t ensure_smem(K kernel, int bytes, std::atomic<bool> *flags, int dev) {
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    if (flags[dev].load(std::memory_order_acquire)) return cudaSuccess;
+    cudaError_t e =
+        cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess) flags[dev].store(true, std::memory_order_release);
+    return e;
+}
+
+template <typename T, int D, int G, int BOXR>
+cudaError_t launch_partition(const DecodeParams &p, dim3 grid, cudaStream_t st, int dev) {
+    static std::atomic<bool> flags[kMaxDevices];
+    auto kernel = pa_decode_partition_kernel<T, D, G, BOXR>;
+    cudaError_t e = ensure_smem(kernel, Geom<D>::kSmem, flags, dev);
+    if (e != cudaSuccess) return e;
+    kernel<<<grid, kWarps * 32, Geom<D>::kSmem, st>>>(p);
+    return cudaGetLastError();
+}
+
+template <typename T, int D>
+cudaError_t launch_merge(const MergeParams &p, dim3 grid, cudaStream_t st) {
+    pa_merge_kernel<T, D><<<grid, D, 0, st>>>(p);
+    return cudaGetLastError();
+}
+
+template <typename T, int D, int G>
+cudaError_t dispatch_boxr(const DecodeParams &p, dim3 grid, cudaStream_t st, int dev, int boxr) {
+    return boxr == 8 ? launch_partition<T, D, G, 8>(p, grid, st, dev)
+                     : launch_partition<T, D, G, 16>(p, grid, st, dev);
+}
+
+template <typename T, int D>
+cudaError_t dispatch_group(const DecodeParams &p, dim3 grid, cudaStream_t st, int dev, int G,
+                           int boxr) {
+    switch (G) {
+        case 1: return dispatch_boxr<T, D, 1>(p, grid, st, dev, boxr);
+        case 2: return dispatch_boxr<T, D, 2>(p, grid, st, dev, boxr);
+        case 4: return dispatch_boxr<T, D, 4>(p, grid, st, dev, boxr);
+        case 8: return dispatch_boxr<T, D, 8>(p, grid, st, dev, boxr);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+template <typename T>
+cudaError_t dispatch_dim(const DecodeParams &p, dim3 grid, cudaStream_t st, int dev, int D,
+                         int G, int boxr) {
+    return D == 64 ? dispatch_group<T, 64>(p, grid, st, dev, G, boxr)
+                   : dispatch_group<T, 128>(p, grid, st, dev, G, boxr);
+}
+
+pa_status check_decode_shape(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                             int block_size, int num_blocks, int max_blocks_per_seq,
+                             int max_context_len, int partition_size) {
+    if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || num_blocks <= 0 ||
+        max_blocks_per_seq <= 0 || max_context_len < 0 || partition_size < 0)
+        return PA_ERR_INVALID_ARG;
+    if (num_q_heads % num_kv_heads != 0) return PA_ERR_INVALID_ARG;
+    const int G = num_q_heads / num_kv_heads;
+    if (G != 1 && G != 2 && G != 4 && G != 8) return PA_ERR_UNSUPPORTED;
+    if (head_dim != 64 && head_dim != 128) return PA_ERR_UNSUPPORTED;
+    if (!pow2(block_size) || block_size < 8 || block_size > 512) return PA_ERR_UNSUPPORTED;
+    if (partition_size % 64 != 0) return PA_ERR_INVALID_ARG;
+    if ((unsigned long long)num_blocks * num_kv_heads * block_size >= (1ull << 31))
+        return PA_ERR_UNSUPPORTED;
+    if ((long long)max_blocks_per_seq * block_size >= (1ll << 31)) return PA_ERR_INVALID_ARG;
+    if (num_seqs > 65535 || num_kv_heads > 65535) return PA_ERR_UNSUPPORTED;
+    return PA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int pa_version(void) { return 100; }
+
+const char *pa_status_str(pa_status s) {
+    switch (s) {
+        case PA_OK: return "ok";
+        case PA_ERR_INVALID_ARG: return "invalid argument";
+        case PA_ERR_UNSUPPORTED: return "unsupported configuration";
+        case PA_ERR_CUDA: return "CUDA runtime error";
+        case PA_ERR_OUT_OF_RANGE: return "index out of range (device error word)";
+        case PA_ERR_TIMEOUT: return "bounded wait expired (device error word)";
+    }
+    return "unknown status";
+}
+
+pa_status pa_get_device_error(int device, uint32_t *bits_out, int clear) {
+    if (!bits_out) return PA_ERR_INVALID_ARG;
+    int prev = 0;
+    if (cudaGetDevice(&prev) != cudaSuccess) return PA_ERR_CUDA;
+    if (cudaSetDevice(device) != cudaSuccess) return PA_ERR_INVALID_ARG;
+    pa_status st = PA_OK;
+    unsigned int v = 0;
+    if (cudaDeviceSynchronize() != cudaSuccess ||
+        cudaMemcpyFromSymbol(&v, g_error_word, sizeof v) != cudaSuccess) {
+        st = PA_ERR_CUDA;
+    } else if (clear) {
+        const unsigned int zero = 0;
+        if (cudaMemcpyToSymbol(g_error_word, &zero, sizeof zero) != cudaSuccess) st = PA_ERR_CUDA;
+    }
+    *bits_out = v;
+    cudaSetDevice(prev);
+    return st;
+}
+
+pa_status pa_kv_write(const void *key, const void *value, const int64_t *slot_mapping,
+                      int num_tokens, int num_kv_heads, int head_dim, int64_t key_token_stride,
+                      int64_t value_token_stride, void *k_cache, void *v_cache, int num_blocks,
+                      int block_size, pa_dtype dtype, void *stream) {
+    if (dtype != PA_FP16 && dtype != PA_BF16) return PA_ERR_INVALID_ARG;
+    if (num_tokens < 0 || num_kv_heads <= 0 || head_dim <= 0 || head_dim % 8 != 0 ||
+        num_blocks <= 0 || block_size <= 0)
+        return PA_ERR_INVALID_ARG;
+    if (num_tokens == 0) return PA_OK;
+    if (!key || !value || !slot_mapping || !k_cache || !v_cache) return PA_ERR_INVALID_ARG;
+    if (!aligned(key, 16) || !aligned(value, 16) || !aligned(k_cache, 16) ||
+        !aligned(v_cache, 16) || !aligned(slot_mapping, 8))
+        return PA_ERR_INVALID_ARG;
+    if (key_token_stride % 8 != 0 || value_token_stride % 8 != 0 ||
+        key_token_stride < (int64_t)num_kv_heads * head_dim ||
+        value_token_stride < (int64_t)num_kv_heads * head_dim)
+        return PA_ERR_INVALID_ARG;
+    KvWriteParams p;
+    p.key = static_cast<const uint8_t *>(key);
+    p.value = static_cast<const uint8_t *>(value);
+    p.slot_mapping = slot_mapping;
+    p.k_cache = static_cast<uint8_t *>(k_cache);
+    p.v_cache = static_cast<uint8_t *>(v_cache);
+    p.key_stride_b = (long long)key_token_stride * 2;
+    p.value_stride_b = (long long)value_token_stride * 2;
+    p.num_slots = (long long)num_blocks * block_size;
+    p.num_tokens = num_tokens;
+    p.num_kv_heads = num_kv_heads;
+    p.row_chunks = head_dim / 8;
+    p.block_size = block_size;
+    const long long total = (long long)num_tokens * num_kv_heads * p.row_chunks;
+    const long long blocks = (total + 255) / 256;
+    const int grid = (int)(blocks < 148 * 32 ? blocks : 148 * 32);
+    pa_kv_write_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(p);
+    return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+pa_status pa_copy_blocks(void *k_cache, void *v_cache, const int64_t *src_dst_pairs,
+                         int num_pairs, int num_kv_heads, int block_size, int head_dim,
+                         int num_blocks, pa_dtype dtype, void *stream) {
+    if (dtype != PA_FP16 && dtype != PA_BF16) return PA_ERR_INVALID_ARG;
+    if (num_pairs < 0 || num_kv_heads <= 0 || block_size <= 0 || head_dim <= 0 || num_blocks <= 0)
+        return PA_ERR_INVALID_ARG;
+    if (num_pairs == 0) return PA_OK;
+    if (!k_cache || !v_cache || !src_dst_pairs) return PA_ERR_INVALID_ARG;
+    if (!aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(src_dst_pairs, 8))
+        return PA_ERR_INVALID_ARG;
+    const long long elems = (long long)num_kv_heads * block_size * head_dim;
+    if (elems % 8 != 0) return PA_ERR_INVALID_ARG;
+    CopyBlocksParams p;
+    p.k_cache = static_cast<uint8_t *>(k_cache);
+    p.v_cache = static_cast<uint8_t *>(v_cache);
+    p.pairs = src_dst_pairs;
+    p.block_chunks = elems / 8;
+    p.num_blocks = num_blocks;
+    p.num_pairs = num_pairs;
+    const long long per_cta = (long long)kCopyThreads * kCopyUnroll;
+    const long long chunks = (p.block_chunks + per_cta - 1) / per_cta;
+    if (chunks > 65535 || num_pairs > 65535) return PA_ERR_UNSUPPORTED;
+    dim3 grid((unsigned)chunks, (unsigned)num_pairs, 2);
+    pa_copy_blocks_kernel<<<grid, kCopyThreads, 0, static_cast<cudaStream_t>(stream)>>>(p);
+    return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+size_t pa_decode_workspace_bytes(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                                 int block_size, int max_blocks_per_seq, int max_context_len,
+                                 int partition_size) {
+    (void)num_kv_heads;
+    if (num_seqs <= 0 || num_q_heads <= 0 || head_dim <= 0 || block_size <= 0 ||
+        max_blocks_per_seq <= 0 || partition_size < 0 || max_context_len < 0)
+        return 0;
+    return make_plan(num_seqs, num_q_heads, head_dim, block_size, max_blocks_per_seq,
+                     max_context_len, partition_size)
+        .ws_bytes;
+}
+
+int pa_decode_partition_tokens(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                               int block_size, int max_blocks_per_seq, int max_context_len,
+                               int partition_size) {
+    (void)num_kv_heads;
+    if (block_size <= 0 || max_blocks_per_seq <= 0 || partition_size < 0 || max_context_len < 0)
+        return 0;
+    return make_plan(num_seqs, num_q_heads, head_dim, block_size, max_blocks_per_seq,
+                     max_context_len, partition_size)
+        .partition_tokens;
+}
+
+pa_status pa_decode(void *out, const void *q, const void *k_cache, const void *v_cache,
+                    const int32_t *block_tables, const int32_t *context_lens, int num_seqs,
+                    int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                    int num_blocks, int max_blocks_per_seq, float scale, int max_context_len,
+                    int partition_size, void *workspace, size_t workspace_bytes, pa_dtype dtype,
+                    void *stream) {
+    if (dtype != PA_FP16 && dtype != PA_BF16) return PA_ERR_INVALID_ARG;
+    pa_status st = check_decode_shape(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
+                                      num_blocks, max_blocks_per_seq, max_context_len,
+                                      partition_size);
+    if (st != PA_OK) return st;
+    if (!std::isfinite(scale)) return PA_ERR_INVALID_ARG;
+    if (num_seqs == 0) return PA_OK;
+    if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens)
+        return PA_ERR_INVALID_ARG;
+    if (!aligned(out, 16) || !aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
+        !aligned(block_tables, 4) || !aligned(context_lens, 4))
+        return PA_ERR_INVALID_ARG;
+    const Plan pl = make_plan(num_seqs, num_q_heads, head_dim, block_size, max_blocks_per_seq,
+                              max_context_len, partition_size);
+    if (pl.ws_bytes > 0 &&
+        (!workspace || !aligned(workspace, 256) || workspace_bytes < pl.ws_bytes))
+        return PA_ERR_INVALID_ARG;
+
+    const int G = num_q_heads / num_kv_heads;
+    const int boxr = block_size < 16 ? block_size : 16;
+    DecodeParams p;
+    std::memset(&p, 0, sizeof p);
+    const unsigned long long rows = (unsigned long long)num_blocks * num_kv_heads * block_size;
+    if (!make_cache_map(&p.kmap, k_cache, rows, head_dim, dtype, boxr) ||
+        !make_cache_map(&p.vmap, v_cache, rows, head_dim, dtype, boxr))
+        return PA_ERR_CUDA;
+    p.out = out;
+    p.q = q;
+    p.block_tables = block_tables;
+    p.context_lens = context_lens;
+    if (pl.ws_bytes > 0) {
+        uint8_t *ws = static_cast<uint8_t *>(workspace);
+        p.ws_o = reinterpret_cast<float *>(ws);
+        p.ws_m = reinterpret_cast<float *>(ws + pl.off_m);
+        p.ws_l = reinterpret_cast<float *>(ws + pl.off_l);
+    }
+    p.num_q_heads = num_q_heads;
+    p.num_kv_heads = num_kv_heads;
+    p.block_size = block_size;
+    p.bs_shift = ilog2_host(block_size);
+    p.num_blocks = num_blocks;
+    p.max_blocks_per_seq = max_blocks_per_seq;
+    p.partition_tokens = pl.partition_tokens;
+    p.num_parts = pl.num_parts;
+    p.scale_log2 = scale * 1.4426950408889634f;
+
+    const int dev = current_device();
+    cudaStream_t st_ = static_cast<cudaStream_t>(stream);
+    dim3 grid((unsigned)pl.num_parts, (unsigned)num_kv_heads, (unsigned)num_seqs);
+    cudaError_t e = dtype == PA_BF16
+                        ? dispatch_dim<__nv_bfloat16>(p, grid, st_, dev, head_dim, G, boxr)
+                        : dispatch_dim<__half>(p, grid, st_, dev, head_dim, G, boxr);
+    if (e != cudaSuccess) return PA_ERR_CUDA;
+    if (pl.num_parts > 1) {
+        MergeParams mp;
+        mp.out = out;
+        mp.context_lens = context_lens;
+        mp.ws_o = p.ws_o;
+        mp.ws_m = p.ws_m;
+        mp.ws_l = p.ws_l;
+        mp.num_q_heads = num_q_heads;
+        mp.cap = max_blocks_per_seq * block_size;
+        mp.partition_tokens = pl.partition_tokens;
+        mp.num_parts = pl.num_parts;
+        dim3 mgrid((unsigned)num_q_heads, (unsigned)num_seqs);
+        if (dtype == PA_BF16)
+            e = head_dim == 64 ? launch_merge<__nv_bfloat16, 64>(mp, mgrid, st_)
+                               : launch_merge<__nv_bfloat16, 128>(mp, mgrid, st_);
+        else
+            e = head_dim == 64 ? launch_merge<__half, 64>(mp, mgrid, st_)
+                               : launch_merge<__half, 128>(mp, mgrid, st_);
+        if (e != cudaSuccess) return PA_ERR_CUDA;
+    }
+    return PA_OK;
+}
+
+}  // extern "C"

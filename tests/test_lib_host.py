@@ -1,0 +1,103 @@
+"""The C-ABI library loads, exports every entry point its header declares, and its
+host-only entry points behave (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import paged_kv_cache_441_b200 as pa
+from paged_kv_cache_441_b200 import build as pa_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    pa_build.build()
+    return pa.load()
+
+
+def header_functions():
+    src = open(os.path.join(ROOT, "include", "pa.h")).read()
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[a-z_0-9]+\s*\*?\s*(pa_[a-z_0-9]+)\s*\(",
+                                 src, flags=re.M)))
+
+
+def test_header_declares_the_calls():
+    names = header_functions()
+    for n in ("pa_kv_write", "pa_decode", "pa_copy_blocks", "pa_get_device_error"):
+        assert n in names
+    assert set(names) == set(pa.EXPORTS)
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in header_functions():
+        assert hasattr(lib, name), name
+        assert isinstance(getattr(lib, name), ctypes._CFuncPtr)
+
+
+def test_status_strings_and_version(lib):
+    assert pa.version() == 100
+    for code in range(6):
+        assert lib.pa_status_str(code)
+    assert lib.pa_status_str(77) == b"unknown status"
+
+
+def test_workspace_plan(lib):
+    # Llama-2-7B-shaped step: max context 2011 -> split into 512-token partitions
+    B, hq, hkv, d, bs, W = 64, 32, 32, 128, 16, 126
+    P = pa.decode_partition_tokens(B, hq, hkv, d, bs, W, 2011)
+    assert P == 512
+    nparts = -(-2011 // 512)
+    need = pa.decode_workspace_bytes(B, hq, hkv, d, bs, W, 2011)
+    assert need >= B * hq * nparts * (d + 2) * 4
+    # short contexts: one partition, no workspace
+    assert pa.decode_workspace_bytes(B, hq, hkv, d, bs, W, 300) == 0
+    assert pa.decode_partition_tokens(B, hq, hkv, d, bs, W, 300) == 320
+    # explicit partition size and unknown max length (table width bound)
+    assert pa.decode_partition_tokens(B, hq, hkv, d, bs, W, 0, 128) == 128
+    assert pa.decode_workspace_bytes(B, hq, hkv, d, bs, W, 0, 128) >= B * hq * 16 * (d + 2) * 4
+
+
+def _decode_args(**over):
+    a = dict(out=16, q=16, kc=16, vc=16, bt=16, cl=16, B=2, hq=8, hkv=2, d=128, bs=16, nb=10,
+             W=4, scale=0.1, mcl=0, ps=0, ws=None, wsb=0, dt=1, stream=None)
+    a.update(over)
+    return a
+
+
+def _call_decode(lib, a):
+    P = ctypes.c_void_p
+    return lib.pa_decode(P(a["out"]), P(a["q"]), P(a["kc"]), P(a["vc"]), P(a["bt"]), P(a["cl"]),
+                         a["B"], a["hq"], a["hkv"], a["d"], a["bs"], a["nb"], a["W"], a["scale"],
+                         a["mcl"], a["ps"], a["ws"], a["wsb"], a["dt"], a["stream"])
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(d=96), 2), (dict(hq=6), 2), (dict(hq=7), 1), (dict(bs=24), 2), (dict(bs=4), 2),
+    (dict(bs=1024), 2), (dict(q=0), 1), (dict(q=24), 1), (dict(out=8), 1), (dict(ps=100), 1),
+    (dict(scale=float("inf")), 1), (dict(dt=5), 1), (dict(nb=0), 1), (dict(W=0), 1),
+    (dict(mcl=-1), 1), (dict(B=-1), 1), (dict(hkv=0), 1),
+    (dict(ps=64, W=100), 1),  # needs a workspace, none given
+])
+def test_decode_rejects_before_launch(lib, over, code):
+    # every case is refused by host checks, so no CUDA call is made
+    assert _call_decode(lib, _decode_args(**over)) == code
+
+
+def test_zero_sized_calls_are_noops(lib):
+    P = ctypes.c_void_p
+    assert _call_decode(lib, _decode_args(B=0, out=0, q=0)) == 0
+    assert lib.pa_kv_write(None, None, None, 0, 2, 128, 256, 256, None, None, 10, 16, 1, None) == 0
+    assert lib.pa_copy_blocks(None, None, None, 0, 2, 16, 128, 10, 1, None) == 0
+
+
+def test_kv_write_and_copy_reject(lib):
+    P = ctypes.c_void_p
+    # misaligned key, stride too small, odd head_dim
+    assert lib.pa_kv_write(P(8), P(16), P(16), 1, 2, 128, 256, 256, P(16), P(16), 10, 16, 1, None) == 1
+    assert lib.pa_kv_write(P(16), P(16), P(16), 1, 2, 128, 128, 256, P(16), P(16), 10, 16, 1, None) == 1
+    assert lib.pa_kv_write(P(16), P(16), P(16), 1, 2, 12, 24, 24, P(16), P(16), 10, 16, 1, None) == 1
+    assert lib.pa_copy_blocks(P(16), P(16), None, 3, 2, 16, 128, 10, 1, None) == 1
+    assert lib.pa_copy_blocks(P(16), P(16), P(8), 3, 2, 16, 128, 0, 1, None) == 1
