@@ -266,6 +266,9 @@ def run_ours(args):
     from workloads import make_config
 
     name, kw, desc = WORKLOADS[args.workload]
+    if args.seqs:
+        kw = dict(kw, num_seqs=args.seqs)
+        desc = f"{desc} [profiling subset: first {args.seqs} seqs' distribution]"
     case = make_config(name, poison=False, **kw)
     dt = case.dtype
 
@@ -478,6 +481,8 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="llama2_7b")
     ap.add_argument("--partition-size", type=int, default=0)
+    ap.add_argument("--seqs", type=int, default=0,
+                    help="profiling only: build the workload with this many sequences")
     ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=10.0)

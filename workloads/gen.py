@@ -269,19 +269,20 @@ CONFIGS = {
     "tiny": lambda **kw: make_case("tiny", kw.pop("seed", 0), 4, 4, 4, 64, 16,
                                    _lens_const([1, 17, 33, 100]), dtype="fp16", scale=1.0 / 8,
                                    num_blocks=64, **kw),
-    "llama2_7b": lambda **kw: make_case("llama2_7b", kw.pop("seed", 1), 64, 32, 32, 128,
-                                        kw.pop("block_size", 16), _lens_uniform(128, 2048, 64),
-                                        **kw),
-    "gqa_llama3_8b": lambda **kw: make_case("gqa_llama3_8b", kw.pop("seed", 2), 256, 32, 8, 128,
-                                            kw.pop("block_size", 16),
-                                            _lens_lognormal(1024, 1.0, 16, 8192, 256), **kw),
-    "long_8_1": lambda **kw: make_case("long_8_1", kw.pop("seed", 3), 8, 8, 1, 128,
-                                       kw.pop("block_size", 16),
-                                       _lens_uniform(32768, 131072, 8), **kw),
-    "long_32_8": lambda **kw: make_case("long_32_8", kw.pop("seed", 3), 8, 32, 8, 128,
-                                        kw.pop("block_size", 16),
-                                        _lens_uniform(32768, 131072, 8), **kw),
-    "prefix_cow": lambda **kw: make_prefix_cow(**kw),
+    "llama2_7b": lambda num_seqs=64, **kw: make_case(
+        "llama2_7b", kw.pop("seed", 1), num_seqs, 32, 32, 128, kw.pop("block_size", 16),
+        _lens_uniform(128, 2048, num_seqs), **kw),
+    "gqa_llama3_8b": lambda num_seqs=256, **kw: make_case(
+        "gqa_llama3_8b", kw.pop("seed", 2), num_seqs, 32, 8, 128, kw.pop("block_size", 16),
+        _lens_lognormal(1024, 1.0, 16, 8192, num_seqs), **kw),
+    "long_8_1": lambda num_seqs=8, **kw: make_case(
+        "long_8_1", kw.pop("seed", 3), num_seqs, 8, 1, 128, kw.pop("block_size", 16),
+        _lens_uniform(32768, 131072, num_seqs), **kw),
+    "long_32_8": lambda num_seqs=8, **kw: make_case(
+        "long_32_8", kw.pop("seed", 3), num_seqs, 32, 8, 128, kw.pop("block_size", 16),
+        _lens_uniform(32768, 131072, num_seqs), **kw),
+    "prefix_cow": lambda num_seqs=None, **kw: make_prefix_cow(
+        groups=(kw.pop("groups", 64) if num_seqs is None else max(1, num_seqs // 8)), **kw),
 }
 
 
