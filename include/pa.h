@@ -144,6 +144,40 @@ int pa_decode_partition_tokens(int num_seqs, int num_q_heads, int num_kv_heads, 
                                int partition_size);
 
 /*
+ * pa_decode for callers that cannot allocate device memory.  The paged-attention
+ * pages have no counterpart to this call; it exists for users of this library.
+ *
+ * Some callers have no way to hand pa_decode a workspace: an engine that gave all
+ * free HBM to its KV-cache pool and offers its plugins no allocator, or a caller
+ * that must not run cudaMalloc (and its device-wide synchronisation) inside its
+ * decode loop.  This entry point takes the same arguments as pa_decode without the
+ * workspace and keeps the split-K partial results in a scratch array that the
+ * library itself holds in device memory: a fixed PA_STATIC_SCRATCH_BYTES per GPU,
+ * reserved on every GPU that loads the library until the process exits.  Nothing
+ * is allocated by the call.
+ *
+ *  - Sizes whose partial results need more than PA_STATIC_SCRATCH_BYTES (see
+ *    pa_decode_workspace_bytes) are rejected with PA_ERR_INVALID_ARG before any
+ *    launch; use pa_decode with a caller workspace for those.
+ *  - The first call on a device looks up the array's device address on that device
+ *    (cudaGetSymbolAddress, with the device current); make that first call before
+ *    any stream capture.  Later calls reuse the address.
+ *  - Every call on a device shares the one array, and it keeps the last call's
+ *    contents.  No part of it needs clearing (each call writes every partial result
+ *    it reads), but calls that overlap on the GPU race on it: serialise them (one
+ *    stream, or events between streams).
+ */
+#define PA_STATIC_SCRATCH_BYTES ((size_t)16 << 20) /* 16 MiB per GPU */
+
+pa_status pa_decode_static_scratch(void *out, const void *q, const void *k_cache,
+                                   const void *v_cache, const int32_t *block_tables,
+                                   const int32_t *context_lens, int num_seqs, int num_q_heads,
+                                   int num_kv_heads, int head_dim, int block_size,
+                                   int num_blocks, int max_blocks_per_seq, float scale,
+                                   int max_context_len, int partition_size, pa_dtype dtype,
+                                   void *stream);
+
+/*
  * Reads (and with clear != 0 resets) the sticky error word of `device`.
  * SYNCHRONISES that device first.  *bits_out receives PA_DEVERR_* bits (0 = none).
  */

@@ -15,8 +15,10 @@ from ._lib import (  # noqa: F401
     EXPORTS,
     LIB_PATH,
     PAError,
+    STATIC_SCRATCH_BYTES,
     copy_blocks,
     decode,
+    decode_static_scratch,
     decode_partition_tokens,
     decode_workspace_bytes,
     device_error,

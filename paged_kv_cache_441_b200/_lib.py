@@ -15,7 +15,9 @@ LIB_PATH = os.path.join(_HERE, "libpa.so")
 PA_FP16, PA_BF16 = 0, 1
 DEVERR = {"block_id": 0x1, "slot": 0x2, "pair": 0x4, "context": 0x8, "timeout": 0x10}
 EXPORTS = ("pa_kv_write", "pa_copy_blocks", "pa_decode", "pa_decode_workspace_bytes",
-           "pa_decode_partition_tokens", "pa_get_device_error", "pa_status_str", "pa_version")
+           "pa_decode_partition_tokens", "pa_get_device_error", "pa_status_str", "pa_version",
+           "pa_decode_static_scratch")
+STATIC_SCRATCH_BYTES = 16 << 20  # PA_STATIC_SCRATCH_BYTES in include/pa.h
 
 _lib = None
 
@@ -46,6 +48,9 @@ def load(path: str = LIB_PATH):
     lib.pa_decode_workspace_bytes.restype = sz
     lib.pa_decode_partition_tokens.argtypes = [i32] * 8
     lib.pa_decode_partition_tokens.restype = i32
+    lib.pa_decode_static_scratch.argtypes = [P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, i32,
+                                             f32, i32, i32, i32, P]
+    lib.pa_decode_static_scratch.restype = i32
     lib.pa_get_device_error.argtypes = [i32, ctypes.POINTER(ctypes.c_uint32), i32]
     lib.pa_get_device_error.restype = i32
     lib.pa_status_str.argtypes = [i32]
@@ -133,6 +138,28 @@ def decode(out, q, k_cache, v_cache, block_tables, context_lens, scale, block_si
                             _ptr(context_lens), B, hq, hkv, d, bs, nb, W, float(scale),
                             int(max_context_len), int(partition_size), wptr, wbytes,
                             _dtype(q), _stream(stream)), "pa_decode")
+
+
+def decode_static_scratch(out, q, k_cache, v_cache, block_tables, context_lens, scale,
+                          block_size=None, max_context_len=0, partition_size=0,
+                          stream=None) -> None:
+    """``decode`` for callers that cannot allocate device memory: the split-K partial
+    results go to the library's own fixed scratch array (STATIC_SCRATCH_BYTES per
+    GPU) instead of a workspace.  Calls that overlap on the GPU race on that array."""
+    B, hq, d = q.shape
+    nb, hkv, bs, _ = k_cache.shape
+    if block_size is not None and block_size != bs:
+        raise PAError(f"block_size {block_size} != cache block size {bs}")
+    W = block_tables.shape[1]
+    need = decode_workspace_bytes(B, hq, hkv, d, bs, W, max_context_len, partition_size)
+    if need > STATIC_SCRATCH_BYTES:
+        raise PAError(f"pa_decode_static_scratch: these sizes need {need} bytes of scratch, "
+                      f"more than the library's fixed {STATIC_SCRATCH_BYTES}; use decode() "
+                      "with a workspace")
+    _check(load().pa_decode_static_scratch(
+        _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
+        _ptr(context_lens), B, hq, hkv, d, bs, nb, W, float(scale), int(max_context_len),
+        int(partition_size), _dtype(q), _stream(stream)), "pa_decode_static_scratch")
 
 
 def device_error(device: int = 0, clear: bool = True) -> int:

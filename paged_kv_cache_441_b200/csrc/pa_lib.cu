@@ -379,3 +379,58 @@ pa_status pa_decode(void *out, const void *q, const void *k_cache, const void *v
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------------------
+// Decode without any allocation: the split-K partials live in a scratch array the
+// library holds in device memory (one copy per GPU that loads the library, kept
+// until the process exits).  Host code cannot use the array's name as a device
+// address, so the address is looked up once per device with cudaGetSymbolAddress
+// while that device is current, and passed to the kernels as their workspace.
+
+static __device__ __align__(256) unsigned char pa_static_scratch[PA_STATIC_SCRATCH_BYTES];
+
+namespace {
+
+std::mutex g_static_scratch_mu;
+void *g_static_scratch_addr[kMaxDevices];
+
+pa_status static_scratch_address(int dev, void **addr) {
+    if (dev < 0 || dev >= kMaxDevices) return PA_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_static_scratch_mu);
+    if (g_static_scratch_addr[dev] == nullptr) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, pa_static_scratch) != cudaSuccess || p == nullptr)
+            return PA_ERR_CUDA;
+        g_static_scratch_addr[dev] = p;
+    }
+    *addr = g_static_scratch_addr[dev];
+    return PA_OK;
+}
+
+}  // namespace
+
+extern "C" pa_status pa_decode_static_scratch(
+    void *out, const void *q, const void *k_cache, const void *v_cache,
+    const int32_t *block_tables, const int32_t *context_lens, int num_seqs, int num_q_heads,
+    int num_kv_heads, int head_dim, int block_size, int num_blocks, int max_blocks_per_seq,
+    float scale, int max_context_len, int partition_size, pa_dtype dtype, void *stream) {
+    if (dtype != PA_FP16 && dtype != PA_BF16) return PA_ERR_INVALID_ARG;
+    pa_status st = check_decode_shape(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
+                                      num_blocks, max_blocks_per_seq, max_context_len,
+                                      partition_size);
+    if (st != PA_OK) return st;
+    if (num_seqs == 0) return PA_OK;
+    const Plan pl = make_plan(num_seqs, num_q_heads, head_dim, block_size, max_blocks_per_seq,
+                              max_context_len, partition_size);
+    if (pl.ws_bytes > PA_STATIC_SCRATCH_BYTES) return PA_ERR_INVALID_ARG;  // over the limit
+    void *scratch = nullptr;
+    if (pl.ws_bytes > 0) {
+        const int dev = current_device();
+        st = static_scratch_address(dev, &scratch);
+        if (st != PA_OK) return st;
+    }
+    return pa_decode(out, q, k_cache, v_cache, block_tables, context_lens, num_seqs, num_q_heads,
+                     num_kv_heads, head_dim, block_size, num_blocks, max_blocks_per_seq, scale,
+                     max_context_len, partition_size, scratch,
+                     pl.ws_bytes > 0 ? (size_t)PA_STATIC_SCRATCH_BYTES : 0, dtype, stream);
+}
