@@ -292,9 +292,10 @@ def run_ours(args):
     ptoks = pa.decode_partition_tokens(case.num_seqs, case.num_q_heads, case.num_kv_heads,
                                        case.head_dim, case.block_size, W, mcl,
                                        args.partition_size)
-    nparts = -(-min(mcl, W * case.block_size) // ptoks)
+    # partition_tokens 0: balanced split over persistent warps (decode + merge kernels)
+    nparts = 0 if ptoks == 0 else -(-min(mcl, W * case.block_size) // ptoks)
     has_pairs = case.copy_pairs.shape[0] > 0
-    launches_per_step = 1 + (2 if nparts > 1 else 1) + (1 if has_pairs else 0)
+    launches_per_step = 1 + (1 if nparts == 1 else 2) + (1 if has_pairs else 0)
     stream = torch.cuda.current_stream()
 
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
@@ -409,8 +410,10 @@ def run_ours(args):
                        "num_q_heads": case.num_q_heads, "num_kv_heads": case.num_kv_heads,
                        "head_dim": case.head_dim, "block_size": case.block_size,
                        "num_blocks": case.num_blocks, "kv_tokens": int(case.context_lens.sum()),
-                       "max_context_len": mcl, "partition_tokens": ptoks,
-                       "partitions_max": nparts, "parallelism": f"dp{ws} (independent replicas)",
+                       "max_context_len": mcl,
+                       "split": ("balanced over persistent warps (stream-K) + LSE merge"
+                                 if ptoks == 0 else f"fixed {ptoks}-token partitions, {nparts} max"),
+                       "parallelism": f"dp{ws} (independent replicas)",
                        "l2": f"inputs larger than L2: {decode_bytes(case) / 1e9:.2f} GB of K/V "
                              f"read per step vs 126 MB L2; no flush"},
             "seq_steps_per_s": round(case.num_seqs * ws / (ms_per_step * 1e-3), 1),

@@ -107,10 +107,18 @@ pa_status pa_copy_blocks(void *k_cache, void *v_cache, const int64_t *src_dst_pa
  * max_context_len : host-side upper bound of context_lens (0 = unknown: the table
  *                   width max_blocks_per_seq * block_size is used).  A context longer
  *                   than the bound sets PA_DEVERR_CONTEXT.
- * partition_size  : tokens per context partition for the split-K path (a multiple of
- *                   64), or 0 to let the library choose.  Contexts longer than one
- *                   partition are processed in partitions whose fp32 partial results
- *                   (running max, sum, normalised output) are merged by log-sum-exp.
+ * partition_size  : how contexts are split (split-K); partial results of the pieces
+ *                   of one context -- fp32 running max, sum and normalised output --
+ *                   are merged by log-sum-exp in a second kernel.
+ *                     > 0 (a multiple of 64): fixed partitions of that many tokens, one
+ *                         CTA each (a context of at most one partition is done in a
+ *                         single pass and needs no merge);
+ *                     PA_PARTITION_BALANCED (-1): balanced split -- persistent warps each
+ *                         take an equal share of all (sequence, kv head, 16-token tile)
+ *                         work, cutting contexts wherever the shares end (needs
+ *                         num_seqs <= 16383 for head_dim 128, 8191 for 64; otherwise
+ *                         fixed partitions are used);
+ *                     0: the library chooses.
  * workspace       : fp32 scratch for those partial results, at least
  *                   pa_decode_workspace_bytes(...) bytes, 256-byte aligned; may be
  *                   NULL when no context needs more than one partition.  Its contents
@@ -125,10 +133,13 @@ pa_status pa_decode(void *out, const void *q, const void *k_cache, const void *v
                     int partition_size, void *workspace, size_t workspace_bytes, pa_dtype dtype,
                     void *stream);
 
+#define PA_PARTITION_BALANCED (-1)
+
 /*
- * Bytes of workspace pa_decode needs for these sizes and this partition_size
- * (0 = the library's choice).  Host-only, no CUDA call.  Returns 0 when every
- * context fits one partition.
+ * Bytes of workspace pa_decode needs for these sizes and this partition_size.
+ * Host-side; it reads the current device's SM count (cudaDeviceGetAttribute, no
+ * synchronisation; 148 when no device is visible), because the balanced split keeps
+ * two partial records per resident warp.  Returns 0 when no merge is needed.
  */
 size_t pa_decode_workspace_bytes(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
                                  int block_size, int max_blocks_per_seq, int max_context_len,
@@ -136,8 +147,9 @@ size_t pa_decode_workspace_bytes(int num_seqs, int num_q_heads, int num_kv_heads
 
 /*
  * The partition size (tokens) pa_decode uses for these arguments when its
- * partition_size argument is `partition_size` (0 = the library's choice); returns
- * the whole context bound when one partition per sequence is used.  Host-only.
+ * partition_size argument is `partition_size`: 0 means the balanced split is used;
+ * a value >= the longest context means one pass per sequence.  Host-side, as
+ * pa_decode_workspace_bytes.
  */
 int pa_decode_partition_tokens(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
                                int block_size, int max_blocks_per_seq, int max_context_len,

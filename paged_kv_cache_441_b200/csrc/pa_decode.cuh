@@ -39,9 +39,16 @@
 
 namespace pa {
 
-constexpr int kTile = 16;   // tokens per tile (one mma M/K extent)
-constexpr int kWarps = 4;   // warps per CTA
-constexpr int kStages = 3;  // ring depth per warp
+#ifndef PA_DECODE_WARPS
+#define PA_DECODE_WARPS 4
+#endif
+#ifndef PA_DECODE_STAGES
+#define PA_DECODE_STAGES 2
+#endif
+
+constexpr int kTile = 16;                  // tokens per tile (one mma M/K extent)
+constexpr int kWarps = PA_DECODE_WARPS;    // warps per CTA
+constexpr int kStages = PA_DECODE_STAGES;  // ring depth per warp
 constexpr unsigned kFull = 0xffffffffu;
 
 struct DecodeParams {
@@ -255,6 +262,50 @@ struct SimtWarp {
             dst[G * D + G + my_h] = lt;
         }
     }
+
+    // Ends a segment straight from registers: `whole` -> out[h][:] = O/l rounded to T;
+    // otherwise the fp32 partial record ro[h][:] = O/l, rm[h] = m, rl[h] = l.
+    __device__ __forceinline__ void store(bool whole, T *out, float *ro, float *rm, float *rl,
+                                          int lane) {
+#pragma unroll
+        for (int mask = kCpr; mask < 32; mask <<= 1)
+#pragma unroll
+            for (int h = 0; h < G; ++h)
+#pragma unroll
+                for (int e = 0; e < 8; ++e) acc[h][e] += __shfl_xor_sync(kFull, acc[h][e], mask);
+        float lt = l;
+#pragma unroll
+        for (int mask = 1; mask < 32; mask <<= 1) {
+            if (G > 1 && mask >= (1 << kShift) && mask < ((1 << kShift) * G)) continue;
+            lt += __shfl_xor_sync(kFull, lt, mask);
+        }
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+            const float lh = __shfl_sync(kFull, lt, h << kShift);
+            const float mh = __shfl_sync(kFull, m, h << kShift);
+            if (lane < kCpr) {
+                float v[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) v[e] = lh > 0.f ? acc[h][e] / lh : 0.f;
+                if (whole) {
+                    uint4 w;
+                    w.x = Fmt<T>::pack_rn(v[0], v[1]);
+                    w.y = Fmt<T>::pack_rn(v[2], v[3]);
+                    w.z = Fmt<T>::pack_rn(v[4], v[5]);
+                    w.w = Fmt<T>::pack_rn(v[6], v[7]);
+                    *reinterpret_cast<uint4 *>(out + h * D + 8 * c) = w;
+                } else {
+                    float4 *dst = reinterpret_cast<float4 *>(ro + h * D + 8 * c);
+                    dst[0] = make_float4(v[0], v[1], v[2], v[3]);
+                    dst[1] = make_float4(v[4], v[5], v[6], v[7]);
+                }
+            }
+            if (!whole && lane == 0) {
+                rm[h] = mh;
+                rl[h] = lh;
+            }
+        }
+    }
 };
 
 // ---------------------------------------------------------------- tensor-core path
@@ -393,6 +444,48 @@ struct MmaWarp {
             if (h1 < G) {
                 dst[G * D + h1] = m1;
                 dst[G * D + G + h1] = lt1;
+            }
+        }
+    }
+
+    // Ends a segment straight from registers (see SimtWarp::store).
+    __device__ __forceinline__ void store(bool whole, T *out, float *ro, float *rm, float *rl,
+                                          int lane) {
+        float lt0 = l0, lt1 = l1;
+#pragma unroll
+        for (int mask = 4; mask < 32; mask <<= 1) {
+            lt0 += __shfl_xor_sync(kFull, lt0, mask);
+            lt1 += __shfl_xor_sync(kFull, lt1, mask);
+        }
+        const int h0 = 2 * tq, h1 = 2 * tq + 1;
+#pragma unroll
+        for (int mt = 0; mt < kK; ++mt) {
+            const int d = 16 * mt + gq;
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                const int h = half ? h1 : h0;
+                const float lh = half ? lt1 : lt0;
+                if (h < G) {
+                    const float a = lh > 0.f ? o[mt][half] / lh : 0.f;
+                    const float b = lh > 0.f ? o[mt][2 + half] / lh : 0.f;
+                    if (whole) {
+                        out[h * D + d] = Fmt<T>::from_float(a);
+                        out[h * D + d + 8] = Fmt<T>::from_float(b);
+                    } else {
+                        ro[h * D + d] = a;
+                        ro[h * D + d + 8] = b;
+                    }
+                }
+            }
+        }
+        if (!whole && gq == 0) {
+            if (h0 < G) {
+                rm[h0] = m0;
+                rl[h0] = lt0;
+            }
+            if (h1 < G) {
+                rm[h1] = m1;
+                rl[h1] = lt1;
             }
         }
     }
@@ -585,6 +678,74 @@ __global__ void __launch_bounds__(kWarps * 32)
 
 // ------------------------------------------------------------------------ merge kernel
 
+// Log-sum-exp merge of n partial results of one (sequence, q head):
+//     M = max_i m_i,  w_i = l_i 2^(m_i - M),  out[:] = sum_i w_i o_i[:] / sum_i w_i.
+// rec(i) gives the record index of partial i, or -1 for "no record"; m at rm[rec],
+// l at rl[rec], o at ro[rec * D].  Block of kMergeThreads threads: all threads reduce
+// the max, then each warp takes every 8th record with one vector load of o per lane
+// (D/32 floats), and the warps' sums are added in shared memory.  The result for
+// element e is returned by thread e (e < D).
+constexpr int kMergeThreads = 256;
+
+template <int D, typename RecFn>
+__device__ __forceinline__ float lse_merge_block(int n, RecFn rec, const float *rm,
+                                                 const float *rl, const float *ro) {
+    constexpr int kW = kMergeThreads / 32;
+    constexpr int kV = D / 32;  // floats per lane
+    __shared__ float red[kW];
+    __shared__ float part[kW][D];
+    __shared__ float dpart[kW];
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    float M = -INFINITY;
+    for (int i = tid; i < n; i += kMergeThreads) {
+        const long long r = rec(i);
+        if (r >= 0) M = fmaxf(M, rm[r]);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, o));
+    if (lane == 0) red[wid] = M;
+    __syncthreads();
+    M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kW; ++w) M = fmaxf(M, red[w]);
+    float acc[kV];
+#pragma unroll
+    for (int e = 0; e < kV; ++e) acc[e] = 0.f;
+    float den = 0.f;
+    for (int i = wid; i < n; i += kW) {
+        const long long r = rec(i);
+        if (r < 0) continue;
+        const float mi = rm[r];
+        if (mi == -INFINITY) continue;
+        const float w = rl[r] * fast_exp2(mi - M);
+        den += w;
+        const float *src = ro + r * D + lane * kV;
+        if constexpr (kV == 4) {
+            const float4 v = *reinterpret_cast<const float4 *>(src);
+            acc[0] = fmaf(w, v.x, acc[0]);
+            acc[1] = fmaf(w, v.y, acc[1]);
+            acc[2] = fmaf(w, v.z, acc[2]);
+            acc[3] = fmaf(w, v.w, acc[3]);
+        } else {
+            const float2 v = *reinterpret_cast<const float2 *>(src);
+            acc[0] = fmaf(w, v.x, acc[0]);
+            acc[1] = fmaf(w, v.y, acc[1]);
+        }
+    }
+#pragma unroll
+    for (int e = 0; e < kV; ++e) part[wid][lane * kV + e] = acc[e];
+    if (lane == 0) dpart[wid] = den;
+    __syncthreads();
+    if (tid >= D) return 0.f;
+    float num = 0.f, dsum = 0.f;
+#pragma unroll
+    for (int w = 0; w < kW; ++w) {
+        num += part[w][tid];
+        dsum += dpart[w];
+    }
+    return dsum > 0.f ? num / dsum : 0.f;
+}
+
 struct MergeParams {
     void *out;
     const int32_t *context_lens;
@@ -597,28 +758,20 @@ struct MergeParams {
     int num_parts;
 };
 
-// One CTA per (q head, sequence), one thread per output element.
+// One CTA per (q head, sequence) with more than one partition.
 template <typename T, int D>
-__global__ void __launch_bounds__(D) pa_merge_kernel(const __grid_constant__ MergeParams p) {
-    const int h = blockIdx.x, s = blockIdx.y, d = threadIdx.x;
+__global__ void __launch_bounds__(kMergeThreads) pa_merge_kernel(const __grid_constant__ MergeParams p) {
+    const int h = blockIdx.x, s = blockIdx.y;
     int L = p.context_lens[s];
     L = L < 0 ? 0 : (L > p.cap ? p.cap : L);
     int n = (L + p.partition_tokens - 1) / p.partition_tokens;
     if (n <= 1) return;
     n = min(n, p.num_parts);
-    const size_t base = ((size_t)s * p.num_q_heads + h) * p.num_parts;
-    float M = -INFINITY;
-    for (int i = 0; i < n; ++i) M = fmaxf(M, p.ws_m[base + i]);
-    float num = 0.f, den = 0.f;
-    for (int i = 0; i < n; ++i) {
-        const float mi = p.ws_m[base + i];
-        if (mi == -INFINITY) continue;
-        const float w = p.ws_l[base + i] * fast_exp2(mi - M);
-        num = fmaf(w, p.ws_o[(base + i) * D + d], num);
-        den += w;
-    }
+    const long long base = ((long long)s * p.num_q_heads + h) * p.num_parts;
+    const float v = lse_merge_block<D>(
+        n, [&](int i) -> long long { return base + i; }, p.ws_m, p.ws_l, p.ws_o);
     T *out = reinterpret_cast<T *>(p.out) + ((size_t)s * p.num_q_heads + h) * D;
-    out[d] = Fmt<T>::from_float(den > 0.f ? num / den : 0.f);
+    if (threadIdx.x < D) out[threadIdx.x] = Fmt<T>::from_float(v);
 }
 
 }  // namespace pa

@@ -11,14 +11,19 @@
 #include "pa_cache.cuh"
 #include "pa_common.cuh"
 #include "pa_decode.cuh"
+#include "pa_decode_streamk.cuh"
 
 using namespace pa;
 
 namespace {
 
 constexpr int kMaxDevices = 64;
-constexpr int kAutoSplitTokens = 512;   // partition size of the split-K path
-constexpr int kAutoSingleMax = 1024;    // contexts up to this stay single-partition
+// Default fixed split (measured on B200 over the decode workloads): one pass for
+// contexts up to kAutoSingleMax tokens, else 1024-token partitions when there are at
+// least as many (sequence, kv head) pairs as SMs, 2048-token partitions when fewer.
+constexpr int kAutoSplitTokens = 1024;
+constexpr int kAutoSplitTokensFew = 2048;
+constexpr int kAutoSingleMax = 1280;
 
 bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 bool pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
@@ -62,26 +67,80 @@ bool make_cache_map(CUtensorMap *m, const void *base, unsigned long long rows, i
 }
 
 struct Plan {
+    bool streamk = false;   // balanced split over persistent warps
+    int grid = 0;           // stream-K CTAs
     int partition_tokens = 0;
     int num_parts = 1;
     size_t ws_bytes = 0;
-    size_t off_m = 0, off_l = 0;
+    size_t off_m = 0, off_l = 0, off_pre = 0;
 };
 
-Plan make_plan(int num_seqs, int num_q_heads, int head_dim, int block_size,
-               int max_blocks_per_seq, int max_context_len, int partition_size) {
+constexpr int kSmPerSmBytes = 233472;  // shared memory per SM usable by CTAs (228 KiB)
+
+template <int D>
+int streamk_ctas_per_sm() {
+    const int per_cta = SkGeom<D>::kSmem + 16 + 1024;  // + static smem + per-CTA reserve
+    const int n = kSmPerSmBytes / per_cta;
+    return n < 1 ? 1 : (n > 16 ? 16 : n);
+}
+
+int device_sms(int dev) {
+    static std::atomic<int> cache[kMaxDevices];
+    if (dev < 0 || dev >= kMaxDevices) return 148;
+    int v = cache[dev].load(std::memory_order_relaxed);
+    if (v > 0) return v;
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+        cudaGetLastError();
+        return 148;  // no device visible: size for a B200
+    }
+    cache[dev].store(n, std::memory_order_relaxed);
+    return n;
+}
+
+int current_device_or_zero() {
+    int d = 0;
+    if (cudaGetDevice(&d) != cudaSuccess) {
+        cudaGetLastError();
+        return 0;
+    }
+    return d;
+}
+
+Plan make_plan(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+               int max_blocks_per_seq, int max_context_len, int partition_size, int sms) {
     Plan pl;
     const long long cap = (long long)max_blocks_per_seq * block_size;
     long long bound = cap;
     if (max_context_len > 0 && max_context_len < cap) bound = max_context_len;
     if (bound < 1) bound = 1;
+    const int G = num_kv_heads > 0 ? num_q_heads / num_kv_heads : 1;
+    const int max_seqs = head_dim == 64 ? SkGeom<64>::kMaxSeqs : SkGeom<128>::kMaxSeqs;
+    const bool fits32 = (long long)num_seqs * ((cap + kTile - 1) / kTile) < (1LL << 31);
+    const bool balanced_ok = num_seqs <= max_seqs && fits32;
+    const bool want_balanced = partition_size == PA_PARTITION_BALANCED;
+    if (want_balanced && balanced_ok) {
+        pl.streamk = true;
+        const int per_sm = head_dim == 64 ? streamk_ctas_per_sm<64>() : streamk_ctas_per_sm<128>();
+        pl.grid = sms * per_sm;
+        const size_t recs = (size_t)pl.grid * kSkWarps * 2 * G;
+        const size_t o_bytes = round_up(recs * head_dim * sizeof(float), 256);
+        const size_t v_bytes = round_up(recs * sizeof(float), 256);
+        pl.off_m = o_bytes;
+        pl.off_l = o_bytes + v_bytes;
+        pl.off_pre = o_bytes + 2 * v_bytes;
+        pl.ws_bytes = pl.off_pre + round_up(((size_t)num_seqs + 1) * sizeof(int32_t), 256);
+        pl.partition_tokens = 0;
+        pl.num_parts = 0;
+        return pl;
+    }
     long long P;
     if (partition_size > 0)
         P = partition_size;
     else if (bound <= kAutoSingleMax)
         P = round_up((size_t)bound, 64);
     else
-        P = kAutoSplitTokens;
+        P = (long long)num_seqs * num_kv_heads >= sms ? kAutoSplitTokens : kAutoSplitTokensFew;
     if (P > (1LL << 30)) P = 1LL << 30;
     pl.partition_tokens = (int)P;
     pl.num_parts = (int)((bound + P - 1) / P);
@@ -124,7 +183,7 @@ cudaError_t launch_partition(const DecodeParams &p, dim3 grid, cudaStream_t st, 
 
 template <typename T, int D>
 cudaError_t launch_merge(const MergeParams &p, dim3 grid, cudaStream_t st) {
-    pa_merge_kernel<T, D><<<grid, D, 0, st>>>(p);
+    pa_merge_kernel<T, D><<<grid, kMergeThreads, 0, st>>>(p);
     return cudaGetLastError();
 }
 
@@ -153,18 +212,76 @@ cudaError_t dispatch_dim(const DecodeParams &p, dim3 grid, cudaStream_t st, int 
                    : dispatch_group<T, 128>(p, grid, st, dev, G, boxr);
 }
 
+template <typename T, int D, int G, int BOXR>
+cudaError_t launch_streamk(const StreamKParams &p, int grid_max, cudaStream_t st, int dev,
+                           int *grid_used) {
+    static std::atomic<bool> flags[kMaxDevices];
+    static std::atomic<int> occ[kMaxDevices];
+    auto kernel = pa_decode_streamk_kernel<T, D, G, BOXR>;
+    cudaError_t e = ensure_smem(kernel, SkGeom<D>::kSmem, flags, dev);
+    if (e != cudaSuccess) return e;
+    int n = occ[dev].load(std::memory_order_relaxed);
+    if (n == 0) {
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, kSkWarps * 32,
+                                                          SkGeom<D>::kSmem);
+        if (e != cudaSuccess || n < 1) return e != cudaSuccess ? e : cudaErrorInvalidConfiguration;
+        occ[dev].store(n, std::memory_order_relaxed);
+    }
+    const int sms = device_sms(dev);
+    int grid = sms * n;
+    if (grid > grid_max) grid = grid_max;
+    *grid_used = grid;
+    kernel<<<grid, kSkWarps * 32, SkGeom<D>::kSmem, st>>>(p);
+    return cudaGetLastError();
+}
+
+template <typename T, int D, int G>
+cudaError_t sk_dispatch_boxr(const StreamKParams &p, int gmax, cudaStream_t st, int dev, int boxr,
+                             int *gu) {
+    return boxr == 8 ? launch_streamk<T, D, G, 8>(p, gmax, st, dev, gu)
+                     : launch_streamk<T, D, G, 16>(p, gmax, st, dev, gu);
+}
+
+template <typename T, int D>
+cudaError_t sk_dispatch_group(const StreamKParams &p, int gmax, cudaStream_t st, int dev, int G,
+                              int boxr, int *gu) {
+    switch (G) {
+        case 1: return sk_dispatch_boxr<T, D, 1>(p, gmax, st, dev, boxr, gu);
+        case 2: return sk_dispatch_boxr<T, D, 2>(p, gmax, st, dev, boxr, gu);
+        case 4: return sk_dispatch_boxr<T, D, 4>(p, gmax, st, dev, boxr, gu);
+        case 8: return sk_dispatch_boxr<T, D, 8>(p, gmax, st, dev, boxr, gu);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+template <typename T>
+cudaError_t sk_dispatch(const StreamKParams &p, int gmax, cudaStream_t st, int dev, int D, int G,
+                        int boxr, int *gu) {
+    return D == 64 ? sk_dispatch_group<T, 64>(p, gmax, st, dev, G, boxr, gu)
+                   : sk_dispatch_group<T, 128>(p, gmax, st, dev, G, boxr, gu);
+}
+
+template <typename T>
+cudaError_t sk_merge(const SkMergeParams &p, dim3 grid, int D, cudaStream_t st) {
+    if (D == 64)
+        pa_merge_streamk_kernel<T, 64><<<grid, kMergeThreads, 0, st>>>(p);
+    else
+        pa_merge_streamk_kernel<T, 128><<<grid, kMergeThreads, 0, st>>>(p);
+    return cudaGetLastError();
+}
+
 pa_status check_decode_shape(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
                              int block_size, int num_blocks, int max_blocks_per_seq,
                              int max_context_len, int partition_size) {
     if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || num_blocks <= 0 ||
-        max_blocks_per_seq <= 0 || max_context_len < 0 || partition_size < 0)
+        max_blocks_per_seq <= 0 || max_context_len < 0 || partition_size < PA_PARTITION_BALANCED)
         return PA_ERR_INVALID_ARG;
     if (num_q_heads % num_kv_heads != 0) return PA_ERR_INVALID_ARG;
     const int G = num_q_heads / num_kv_heads;
     if (G != 1 && G != 2 && G != 4 && G != 8) return PA_ERR_UNSUPPORTED;
     if (head_dim != 64 && head_dim != 128) return PA_ERR_UNSUPPORTED;
     if (!pow2(block_size) || block_size < 8 || block_size > 512) return PA_ERR_UNSUPPORTED;
-    if (partition_size % 64 != 0) return PA_ERR_INVALID_ARG;
+    if (partition_size > 0 && partition_size % 64 != 0) return PA_ERR_INVALID_ARG;
     if ((unsigned long long)num_blocks * num_kv_heads * block_size >= (1ull << 31))
         return PA_ERR_UNSUPPORTED;
     if ((long long)max_blocks_per_seq * block_size >= (1ll << 31)) return PA_ERR_INVALID_ARG;
@@ -276,23 +393,25 @@ pa_status pa_copy_blocks(void *k_cache, void *v_cache, const int64_t *src_dst_pa
 size_t pa_decode_workspace_bytes(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
                                  int block_size, int max_blocks_per_seq, int max_context_len,
                                  int partition_size) {
-    (void)num_kv_heads;
-    if (num_seqs <= 0 || num_q_heads <= 0 || head_dim <= 0 || block_size <= 0 ||
-        max_blocks_per_seq <= 0 || partition_size < 0 || max_context_len < 0)
+    if (num_seqs <= 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 ||
+        block_size <= 0 || max_blocks_per_seq <= 0 || partition_size < PA_PARTITION_BALANCED ||
+        max_context_len < 0)
         return 0;
-    return make_plan(num_seqs, num_q_heads, head_dim, block_size, max_blocks_per_seq,
-                     max_context_len, partition_size)
+    return make_plan(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
+                     max_blocks_per_seq, max_context_len, partition_size,
+                     device_sms(current_device_or_zero()))
         .ws_bytes;
 }
 
 int pa_decode_partition_tokens(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
                                int block_size, int max_blocks_per_seq, int max_context_len,
                                int partition_size) {
-    (void)num_kv_heads;
-    if (block_size <= 0 || max_blocks_per_seq <= 0 || partition_size < 0 || max_context_len < 0)
+    if (num_kv_heads <= 0 || block_size <= 0 || max_blocks_per_seq <= 0 ||
+        partition_size < PA_PARTITION_BALANCED || max_context_len < 0)
         return 0;
-    return make_plan(num_seqs, num_q_heads, head_dim, block_size, max_blocks_per_seq,
-                     max_context_len, partition_size)
+    return make_plan(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
+                     max_blocks_per_seq, max_context_len, partition_size,
+                     device_sms(current_device_or_zero()))
         .partition_tokens;
 }
 
@@ -314,17 +433,66 @@ pa_status pa_decode(void *out, const void *q, const void *k_cache, const void *v
     if (!aligned(out, 16) || !aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
         !aligned(block_tables, 4) || !aligned(context_lens, 4))
         return PA_ERR_INVALID_ARG;
-    const Plan pl = make_plan(num_seqs, num_q_heads, head_dim, block_size, max_blocks_per_seq,
-                              max_context_len, partition_size);
+    const int dev = current_device();
+    const Plan pl = make_plan(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
+                              max_blocks_per_seq, max_context_len, partition_size,
+                              device_sms(dev));
     if (pl.ws_bytes > 0 &&
         (!workspace || !aligned(workspace, 256) || workspace_bytes < pl.ws_bytes))
         return PA_ERR_INVALID_ARG;
 
     const int G = num_q_heads / num_kv_heads;
     const int boxr = block_size < 16 ? block_size : 16;
+    cudaStream_t st_ = static_cast<cudaStream_t>(stream);
+    const unsigned long long rows = (unsigned long long)num_blocks * num_kv_heads * block_size;
+    if (pl.streamk) {
+        StreamKParams sp;
+        std::memset(&sp, 0, sizeof sp);
+        if (!make_cache_map(&sp.kmap, k_cache, rows, head_dim, dtype, boxr) ||
+            !make_cache_map(&sp.vmap, v_cache, rows, head_dim, dtype, boxr))
+            return PA_ERR_CUDA;
+        uint8_t *ws = static_cast<uint8_t *>(workspace);
+        sp.out = out;
+        sp.q = q;
+        sp.block_tables = block_tables;
+        sp.context_lens = context_lens;
+        sp.rec_o = reinterpret_cast<float *>(ws);
+        sp.rec_m = reinterpret_cast<float *>(ws + pl.off_m);
+        sp.rec_l = reinterpret_cast<float *>(ws + pl.off_l);
+        sp.ws_pre = reinterpret_cast<int32_t *>(ws + pl.off_pre);
+        sp.num_seqs = num_seqs;
+        sp.num_q_heads = num_q_heads;
+        sp.num_kv_heads = num_kv_heads;
+        sp.block_size = block_size;
+        sp.bs_shift = ilog2_host(block_size);
+        sp.num_blocks = num_blocks;
+        sp.max_blocks_per_seq = max_blocks_per_seq;
+        sp.scale_log2 = scale * 1.4426950408889634f;
+        int grid_used = 0;
+        cudaError_t e = dtype == PA_BF16
+                            ? sk_dispatch<__nv_bfloat16>(sp, pl.grid, st_, dev, head_dim, G, boxr,
+                                                         &grid_used)
+                            : sk_dispatch<__half>(sp, pl.grid, st_, dev, head_dim, G, boxr,
+                                                  &grid_used);
+        if (e != cudaSuccess) return PA_ERR_CUDA;
+        SkMergeParams mp;
+        mp.out = out;
+        mp.ws_pre = sp.ws_pre;
+        mp.rec_o = sp.rec_o;
+        mp.rec_m = sp.rec_m;
+        mp.rec_l = sp.rec_l;
+        mp.num_seqs = num_seqs;
+        mp.num_q_heads = num_q_heads;
+        mp.num_kv_heads = num_kv_heads;
+        mp.num_workers = grid_used * kSkWarps;
+        dim3 mgrid((unsigned)num_q_heads, (unsigned)num_seqs);
+        e = dtype == PA_BF16 ? sk_merge<__nv_bfloat16>(mp, mgrid, head_dim, st_)
+                             : sk_merge<__half>(mp, mgrid, head_dim, st_);
+        return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+    }
+
     DecodeParams p;
     std::memset(&p, 0, sizeof p);
-    const unsigned long long rows = (unsigned long long)num_blocks * num_kv_heads * block_size;
     if (!make_cache_map(&p.kmap, k_cache, rows, head_dim, dtype, boxr) ||
         !make_cache_map(&p.vmap, v_cache, rows, head_dim, dtype, boxr))
         return PA_ERR_CUDA;
@@ -348,8 +516,6 @@ pa_status pa_decode(void *out, const void *q, const void *k_cache, const void *v
     p.num_parts = pl.num_parts;
     p.scale_log2 = scale * 1.4426950408889634f;
 
-    const int dev = current_device();
-    cudaStream_t st_ = static_cast<cudaStream_t>(stream);
     dim3 grid((unsigned)pl.num_parts, (unsigned)num_kv_heads, (unsigned)num_seqs);
     cudaError_t e = dtype == PA_BF16
                         ? dispatch_dim<__nv_bfloat16>(p, grid, st_, dev, head_dim, G, boxr)
@@ -420,8 +586,9 @@ extern "C" pa_status pa_decode_static_scratch(
                                       partition_size);
     if (st != PA_OK) return st;
     if (num_seqs == 0) return PA_OK;
-    const Plan pl = make_plan(num_seqs, num_q_heads, head_dim, block_size, max_blocks_per_seq,
-                              max_context_len, partition_size);
+    const Plan pl = make_plan(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
+                              max_blocks_per_seq, max_context_len, partition_size,
+                              device_sms(current_device_or_zero()));
     if (pl.ws_bytes > PA_STATIC_SCRATCH_BYTES) return PA_ERR_INVALID_ARG;  // over the limit
     void *scratch = nullptr;
     if (pl.ws_bytes > 0) {

@@ -80,7 +80,7 @@ def test_every_kernel_variant(dtype, d, G, bs):
     rng = np.random.default_rng([d, G, bs, 1 if dtype == "bf16" else 2])
     lens = [1, 15, 16, 17, 63, 64, 65, 130, 333, int(rng.integers(1, 700))]
     case = _rand_case(7, dtype, len(lens), hkv * G, hkv, d, bs, lens)
-    for ps in (0, 64, 192):
+    for ps in (-1, 0, 64, 192):
         _check_step(case, partition_size=ps, full=True)
 
 
@@ -110,7 +110,7 @@ def test_permutation_bit_identical():
         nb = sum(-(-L // bs) for L in lens) + 7 * (trial + 1)
         tabs = _tables_for(rng, lens, bs, nb)
         kc, vc, bt = build_pool(Ks, Vs, tabs, nb, bs)
-        for ps in (0, 128):
+        for ps in (-1, 128):
             out = torch.empty_like(q)
             pa.decode(out, q, dev16(kc, "bf16"), dev16(vc, "bf16"), dev(bt),
                       dev(np.array(lens, np.int32)), 1 / math.sqrt(d), partition_size=ps)
@@ -187,6 +187,25 @@ def test_zero_length_and_unread_table_entries():
     case.slot_mapping[0] = -1  # nothing to write for the empty sequence
     err, dc = _check_step(case, full=True)
     assert np.all(to_f64(dc.out)[0] == 0.0)
+
+
+@pytest.mark.parametrize("seed", [31, 32, 33])
+def test_balanced_split_ragged_and_empty(seed):
+    """Default (balanced) split on ragged lengths with empty sequences in between and
+    segments cut at arbitrary tiles; fewer tiles than warps; one long sequence."""
+    rng = np.random.default_rng(seed)
+    lens = rng.integers(0, 400, size=40)
+    lens[rng.integers(0, 40, size=8)] = 0
+    lens[5] = 1
+    for hq, hkv, d, bs in ((8, 8, 128, 16), (32, 4, 128, 8), (16, 2, 64, 32)):
+        case = _rand_case(seed, "bf16", len(lens), hq, hkv, d, bs, lens)
+        case.slot_mapping[case.context_lens == 0] = -1
+        _check_step(case, partition_size=-1, full=True)
+    few = _rand_case(seed, "bf16", 3, 8, 2, 128, 16, [0, 3, 20])
+    few.slot_mapping[0] = -1
+    _check_step(few, partition_size=-1, full=True)
+    one = _rand_case(seed, "bf16", 2, 8, 1, 128, 16, [70001, 5])
+    _check_step(one, partition_size=-1, full=True)
 
 
 def test_table_width_bound():

@@ -45,18 +45,26 @@ def test_status_strings_and_version(lib):
 
 
 def test_workspace_plan(lib):
-    # Llama-2-7B-shaped step: max context 2011 -> split into 512-token partitions
+    warps = 148 * 3 * 4  # no device here: sized for 148 SMs x 3 CTAs x 4 warps
+    # Llama-2-7B-shaped step (2048 sequence x kv-head pairs): fixed 1024-token partitions
     B, hq, hkv, d, bs, W = 64, 32, 32, 128, 16, 126
-    P = pa.decode_partition_tokens(B, hq, hkv, d, bs, W, 2011)
-    assert P == 512
-    nparts = -(-2011 // 512)
-    need = pa.decode_workspace_bytes(B, hq, hkv, d, bs, W, 2011)
-    assert need >= B * hq * nparts * (d + 2) * 4
-    # short contexts: one partition, no workspace
-    assert pa.decode_workspace_bytes(B, hq, hkv, d, bs, W, 300) == 0
+    assert pa.decode_partition_tokens(B, hq, hkv, d, bs, W, 2011) == 1024
+    assert pa.decode_workspace_bytes(B, hq, hkv, d, bs, W, 2011) >= B * hq * 2 * (d + 2) * 4
+    # short contexts: one pass, no workspace
     assert pa.decode_partition_tokens(B, hq, hkv, d, bs, W, 300) == 320
-    # explicit partition size and unknown max length (table width bound)
-    assert pa.decode_partition_tokens(B, hq, hkv, d, bs, W, 0, 128) == 128
+    assert pa.decode_workspace_bytes(B, hq, hkv, d, bs, W, 300) == 0
+    assert pa.decode_partition_tokens(B, hq, hkv, d, bs, W, 1257) == 1280
+    # few sequence x kv-head pairs (8 x 1): 2048-token partitions
+    assert pa.decode_partition_tokens(8, 8, 1, d, bs, 8192, 131072) == 2048
+    assert pa.decode_workspace_bytes(8, 8, 1, d, bs, 8192, 131072) >= 8 * 8 * 64 * (d + 2) * 4
+    # forced balanced split: two records per warp, independent of the lengths
+    need = pa.decode_workspace_bytes(8, 8, 1, d, bs, 8192, 131072, -1)
+    assert need >= 2 * warps * 8 * (d + 2) * 4 + 9 * 4
+    assert need == pa.decode_workspace_bytes(8, 8, 1, d, bs, 8192, 0, -1)
+    # forced balanced split for the large batch, forced fixed split for the small one
+    assert pa.decode_partition_tokens(B, hq, hkv, d, bs, W, 2011, -1) == 0
+    assert pa.decode_workspace_bytes(B, hq, hkv, d, bs, W, 2011, -1) >= 2 * warps * (d + 2) * 4
+    assert pa.decode_partition_tokens(8, 8, 1, d, bs, 8192, 131072, 512) == 512
     assert pa.decode_workspace_bytes(B, hq, hkv, d, bs, W, 0, 128) >= B * hq * 16 * (d + 2) * 4
 
 
@@ -78,6 +86,7 @@ def _call_decode(lib, a):
     (dict(d=96), 2), (dict(hq=6), 2), (dict(hq=7), 1), (dict(bs=24), 2), (dict(bs=4), 2),
     (dict(bs=1024), 2), (dict(q=0), 1), (dict(q=24), 1), (dict(out=8), 1), (dict(ps=100), 1),
     (dict(scale=float("inf")), 1), (dict(dt=5), 1), (dict(nb=0), 1), (dict(W=0), 1),
+    (dict(ps=-2), 1), (dict(ps=-1), 1),  # balanced split needs a workspace
     (dict(mcl=-1), 1), (dict(B=-1), 1), (dict(hkv=0), 1),
     (dict(ps=64, W=100), 1),  # needs a workspace, none given
 ])

@@ -48,7 +48,8 @@ def _c_static(case, t, out, partition_size):
 
 
 def test_static_scratch_matches_workspace_path_twice():
-    runs = [(21, [3000, 17, 1290, 640, 2048], 128), (22, [700, 2500, 64, 1999], 256)]
+    runs = [(21, [3000, 17, 1290, 640, 2048], 128), (22, [700, 2500, 64, 1999], 256),
+            (24, [900, 0, 4100, 33], -1)]
     for seed, lens, ps in runs:
         case, t = _inputs(seed, lens)
         need = pa.decode_workspace_bytes(case.num_seqs, case.num_q_heads, case.num_kv_heads,
