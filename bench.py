@@ -88,13 +88,14 @@ def peaks():
 
 
 def kernel_sources_sha() -> str:
+    """Identity of the decode partition kernel's sources (the kernel the ncu traffic
+    figure was taken from)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "paged_kv_cache_441_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".cuh")):
-            with open(os.path.join(csrc, name), "rb") as f:
-                h.update(name.encode())
-                h.update(f.read())
+    for name in ("pa_common.cuh", "pa_decode.cuh"):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode())
+            h.update(f.read())
     return h.hexdigest()[:16]
 
 

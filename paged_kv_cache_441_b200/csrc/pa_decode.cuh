@@ -676,102 +676,4 @@ __global__ void __launch_bounds__(kWarps * 32)
     }
 }
 
-// ------------------------------------------------------------------------ merge kernel
-
-// Log-sum-exp merge of n partial results of one (sequence, q head):
-//     M = max_i m_i,  w_i = l_i 2^(m_i - M),  out[:] = sum_i w_i o_i[:] / sum_i w_i.
-// rec(i) gives the record index of partial i, or -1 for "no record"; m at rm[rec],
-// l at rl[rec], o at ro[rec * D].  Block of kMergeThreads threads: all threads reduce
-// the max, then each warp takes every 8th record with one vector load of o per lane
-// (D/32 floats), and the warps' sums are added in shared memory.  The result for
-// element e is returned by thread e (e < D).
-constexpr int kMergeThreads = 256;
-
-template <int D, typename RecFn>
-__device__ __forceinline__ float lse_merge_block(int n, RecFn rec, const float *rm,
-                                                 const float *rl, const float *ro) {
-    constexpr int kW = kMergeThreads / 32;
-    constexpr int kV = D / 32;  // floats per lane
-    __shared__ float red[kW];
-    __shared__ float part[kW][D];
-    __shared__ float dpart[kW];
-    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
-    float M = -INFINITY;
-    for (int i = tid; i < n; i += kMergeThreads) {
-        const long long r = rec(i);
-        if (r >= 0) M = fmaxf(M, rm[r]);
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, o));
-    if (lane == 0) red[wid] = M;
-    __syncthreads();
-    M = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < kW; ++w) M = fmaxf(M, red[w]);
-    float acc[kV];
-#pragma unroll
-    for (int e = 0; e < kV; ++e) acc[e] = 0.f;
-    float den = 0.f;
-    for (int i = wid; i < n; i += kW) {
-        const long long r = rec(i);
-        if (r < 0) continue;
-        const float mi = rm[r];
-        if (mi == -INFINITY) continue;
-        const float w = rl[r] * fast_exp2(mi - M);
-        den += w;
-        const float *src = ro + r * D + lane * kV;
-        if constexpr (kV == 4) {
-            const float4 v = *reinterpret_cast<const float4 *>(src);
-            acc[0] = fmaf(w, v.x, acc[0]);
-            acc[1] = fmaf(w, v.y, acc[1]);
-            acc[2] = fmaf(w, v.z, acc[2]);
-            acc[3] = fmaf(w, v.w, acc[3]);
-        } else {
-            const float2 v = *reinterpret_cast<const float2 *>(src);
-            acc[0] = fmaf(w, v.x, acc[0]);
-            acc[1] = fmaf(w, v.y, acc[1]);
-        }
-    }
-#pragma unroll
-    for (int e = 0; e < kV; ++e) part[wid][lane * kV + e] = acc[e];
-    if (lane == 0) dpart[wid] = den;
-    __syncthreads();
-    if (tid >= D) return 0.f;
-    float num = 0.f, dsum = 0.f;
-#pragma unroll
-    for (int w = 0; w < kW; ++w) {
-        num += part[w][tid];
-        dsum += dpart[w];
-    }
-    return dsum > 0.f ? num / dsum : 0.f;
-}
-
-struct MergeParams {
-    void *out;
-    const int32_t *context_lens;
-    const float *ws_o;
-    const float *ws_m;
-    const float *ws_l;
-    int num_q_heads;
-    int cap;  // max_blocks_per_seq * block_size
-    int partition_tokens;
-    int num_parts;
-};
-
-// One CTA per (q head, sequence) with more than one partition.
-template <typename T, int D>
-__global__ void __launch_bounds__(kMergeThreads) pa_merge_kernel(const __grid_constant__ MergeParams p) {
-    const int h = blockIdx.x, s = blockIdx.y;
-    int L = p.context_lens[s];
-    L = L < 0 ? 0 : (L > p.cap ? p.cap : L);
-    int n = (L + p.partition_tokens - 1) / p.partition_tokens;
-    if (n <= 1) return;
-    n = min(n, p.num_parts);
-    const long long base = ((long long)s * p.num_q_heads + h) * p.num_parts;
-    const float v = lse_merge_block<D>(
-        n, [&](int i) -> long long { return base + i; }, p.ws_m, p.ws_l, p.ws_o);
-    T *out = reinterpret_cast<T *>(p.out) + ((size_t)s * p.num_q_heads + h) * D;
-    if (threadIdx.x < D) out[threadIdx.x] = Fmt<T>::from_float(v);
-}
-
 }  // namespace pa

@@ -24,6 +24,7 @@
 #pragma once
 
 #include "pa_decode.cuh"
+#include "pa_merge.cuh"
 
 namespace pa {
 

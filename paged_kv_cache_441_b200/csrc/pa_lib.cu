@@ -11,6 +11,7 @@
 #include "pa_cache.cuh"
 #include "pa_common.cuh"
 #include "pa_decode.cuh"
+#include "pa_merge.cuh"
 #include "pa_decode_streamk.cuh"
 
 using namespace pa;
