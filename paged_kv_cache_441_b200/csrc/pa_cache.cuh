@@ -27,6 +27,7 @@ struct KvWriteParams {
 // "Every generated token's K and V are stored in the KV cache" (PagedAttention and
 // dynamic memory blog): the store goes to k_cache[slot / bs][h][slot % bs][:].
 __global__ void __launch_bounds__(256) pa_kv_write_kernel(const __grid_constant__ KvWriteParams p) {
+    pdl_wait_and_release();
     const long long per_tok = (long long)p.num_kv_heads * p.row_chunks;
     const long long total = per_tok * p.num_tokens;
     for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
@@ -66,6 +67,7 @@ constexpr int kCopyUnroll = 4;
 // Each thread keeps kCopyUnroll 16-byte loads in flight before storing.
 __global__ void __launch_bounds__(kCopyThreads)
     pa_copy_blocks_kernel(const __grid_constant__ CopyBlocksParams p) {
+    pdl_wait_and_release();
     const int pair = blockIdx.y;
     const long long src = p.pairs[2 * pair], dst = p.pairs[2 * pair + 1];
     if (src < 0 || src >= p.num_blocks || dst < 0 || dst >= p.num_blocks) {

@@ -33,6 +33,18 @@ __device__ __forceinline__ unsigned long long globaltimer_ns() {
     return t;
 }
 
+// ---------------------------------------------------------------- dependent launch
+//
+// Every libpa kernel is launched with programmatic stream serialisation: it may be
+// scheduled while the previous kernel on the stream is still finishing.  It waits for
+// that kernel's completion (and memory) with griddepcontrol.wait before touching
+// global memory, then lets its own dependents start launching.  Without the launch
+// attribute both instructions are no-ops.
+__device__ __forceinline__ void pdl_wait_and_release() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- mbarrier
 
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {

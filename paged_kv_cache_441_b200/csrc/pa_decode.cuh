@@ -47,6 +47,7 @@ namespace pa {
 #endif
 
 constexpr int kTile = 16;                  // tokens per tile (one mma M/K extent)
+constexpr int kTabSmem = 256;              // block-table entries of a partition kept in smem
 constexpr int kWarps = PA_DECODE_WARPS;    // warps per CTA
 constexpr int kStages = PA_DECODE_STAGES;  // ring depth per warp
 constexpr unsigned kFull = 0xffffffffu;
@@ -499,6 +500,7 @@ using WarpCompute = typename std::conditional<(G >= 4), MmaWarp<T, D, G>, SimtWa
 template <typename T, int D, int G, int BOXR>
 __global__ void __launch_bounds__(kWarps * 32)
     pa_decode_partition_kernel(const __grid_constant__ DecodeParams p) {
+    pdl_wait_and_release();
     using Gm = Geom<D>;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
@@ -510,13 +512,26 @@ __global__ void __launch_bounds__(kWarps * 32)
     const int part = blockIdx.x, g = blockIdx.y, s = blockIdx.z;
     const int Hq = p.num_q_heads;
 
-    int L = p.context_lens[s];
+    // Start the three independent loads of this item at once: its context length, the
+    // block-table entries of its partition (the page range does not depend on L) and q.
+    const int P = p.partition_tokens;
+    const int32_t *table = p.block_tables + (size_t)s * p.max_blocks_per_seq;
+    const int pg_first = (int)(((long long)part * P) >> p.bs_shift);
+    const int pg_count = min((int)((((long long)part * P + P - 1) >> p.bs_shift) - pg_first + 1),
+                             p.max_blocks_per_seq - pg_first);
+    const bool tab_in_smem = pg_count <= kTabSmem;
+    __shared__ int tab_smem[kTabSmem];
+    if (tab_in_smem)
+        for (int i = tid; i < pg_count; i += kWarps * 32) tab_smem[i] = __ldg(table + pg_first + i);
+    const T *q_item = reinterpret_cast<const T *>(p.q) + ((size_t)s * Hq + (size_t)g * G) * D;
+    WarpCompute<T, D, G> wc;
+    wc.init(q_item, lane);
+    int L = __ldg(p.context_lens + s);
     const int cap = p.max_blocks_per_seq << p.bs_shift;
     if (L < 0 || L > cap) {
         if (tid == 0 && part == 0) raise_error(PA_DEVERR_CONTEXT);
         L = L < 0 ? 0 : cap;
     }
-    const int P = p.partition_tokens;
     const int nparts = (L + P - 1) / P;
     if (nparts > p.num_parts && tid == 0 && part == 0) raise_error(PA_DEVERR_CONTEXT);
     T *out = reinterpret_cast<T *>(p.out) + ((size_t)s * Hq + (size_t)g * G) * D;
@@ -545,11 +560,6 @@ __global__ void __launch_bounds__(kWarps * 32)
         fence_barrier_init();
     }
 
-    const T *q_item = reinterpret_cast<const T *>(p.q) + ((size_t)s * Hq + (size_t)g * G) * D;
-    WarpCompute<T, D, G> wc;
-    wc.init(q_item, lane);
-
-    const int32_t *table = p.block_tables + (size_t)s * p.max_blocks_per_seq;
     const int npages = (L + p.block_size - 1) >> p.bs_shift;
     int tab_base = -(1 << 30), tab_reg = -1;
     const uint64_t pol = l2_policy_evict_first();
@@ -558,6 +568,7 @@ __global__ void __launch_bounds__(kWarps * 32)
     __syncthreads();
 
     auto lookup = [&](int pg) -> int {
+        if (tab_in_smem) return tab_smem[pg - pg_first];  // CTA-uniform
         if (pg < tab_base || pg >= tab_base + 32) {  // warp-uniform
             tab_base = pg;
             const int e = pg + lane;

@@ -74,6 +74,7 @@ struct Plan {
     int num_parts = 1;
     size_t ws_bytes = 0;
     size_t off_m = 0, off_l = 0, off_pre = 0;
+    size_t off_co = 0, off_cm = 0, off_cl = 0;  // balanced split: CTA-level records
 };
 
 constexpr int kSmPerSmBytes = 233472;  // shared memory per SM usable by CTAs (228 KiB)
@@ -124,12 +125,18 @@ Plan make_plan(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, in
         pl.streamk = true;
         const int per_sm = head_dim == 64 ? streamk_ctas_per_sm<64>() : streamk_ctas_per_sm<128>();
         pl.grid = sms * per_sm;
-        const size_t recs = (size_t)pl.grid * kSkWarps * 2 * G;
+        const size_t recs = (size_t)pl.grid * kSkWarps * 2 * G;  // warp pieces
+        const size_t crecs = (size_t)pl.grid * 2 * G;            // CTA records
         const size_t o_bytes = round_up(recs * head_dim * sizeof(float), 256);
         const size_t v_bytes = round_up(recs * sizeof(float), 256);
+        const size_t co_bytes = round_up(crecs * head_dim * sizeof(float), 256);
+        const size_t cv_bytes = round_up(crecs * sizeof(float), 256);
         pl.off_m = o_bytes;
         pl.off_l = o_bytes + v_bytes;
-        pl.off_pre = o_bytes + 2 * v_bytes;
+        pl.off_co = o_bytes + 2 * v_bytes;
+        pl.off_cm = pl.off_co + co_bytes;
+        pl.off_cl = pl.off_cm + cv_bytes;
+        pl.off_pre = pl.off_cl + cv_bytes;
         pl.ws_bytes = pl.off_pre + round_up(((size_t)num_seqs + 1) * sizeof(int32_t), 256);
         pl.partition_tokens = 0;
         pl.num_parts = 0;
@@ -156,6 +163,24 @@ Plan make_plan(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, in
     return pl;
 }
 
+// Launch with programmatic stream serialisation (see pdl_wait_and_release).
+template <typename Kern, typename P>
+cudaError_t launch_pdl(Kern kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       const P &p) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, p);
+    return e != cudaSuccess ? e : cudaGetLastError();
+}
+
 int current_device() {
     int d = 0;
     if (cudaGetDevice(&d) != cudaSuccess) return -1;
@@ -178,14 +203,12 @@ cudaError_t launch_partition(const DecodeParams &p, dim3 grid, cudaStream_t st, 
     auto kernel = pa_decode_partition_kernel<T, D, G, BOXR>;
     cudaError_t e = ensure_smem(kernel, Geom<D>::kSmem, flags, dev);
     if (e != cudaSuccess) return e;
-    kernel<<<grid, kWarps * 32, Geom<D>::kSmem, st>>>(p);
-    return cudaGetLastError();
+    return launch_pdl(kernel, grid, dim3(kWarps * 32), Geom<D>::kSmem, st, p);
 }
 
 template <typename T, int D>
 cudaError_t launch_merge(const MergeParams &p, dim3 grid, cudaStream_t st) {
-    pa_merge_kernel<T, D><<<grid, kMergeThreads, 0, st>>>(p);
-    return cudaGetLastError();
+    return launch_pdl(pa_merge_kernel<T, D>, grid, dim3(kMergeThreads), 0, st, p);
 }
 
 template <typename T, int D, int G>
@@ -232,8 +255,7 @@ cudaError_t launch_streamk(const StreamKParams &p, int grid_max, cudaStream_t st
     int grid = sms * n;
     if (grid > grid_max) grid = grid_max;
     *grid_used = grid;
-    kernel<<<grid, kSkWarps * 32, SkGeom<D>::kSmem, st>>>(p);
-    return cudaGetLastError();
+    return launch_pdl(kernel, dim3(grid), dim3(kSkWarps * 32), SkGeom<D>::kSmem, st, p);
 }
 
 template <typename T, int D, int G>
@@ -264,11 +286,9 @@ cudaError_t sk_dispatch(const StreamKParams &p, int gmax, cudaStream_t st, int d
 
 template <typename T>
 cudaError_t sk_merge(const SkMergeParams &p, dim3 grid, int D, cudaStream_t st) {
-    if (D == 64)
-        pa_merge_streamk_kernel<T, 64><<<grid, kMergeThreads, 0, st>>>(p);
-    else
-        pa_merge_streamk_kernel<T, 128><<<grid, kMergeThreads, 0, st>>>(p);
-    return cudaGetLastError();
+    return D == 64 ? launch_pdl(pa_merge_streamk_kernel<T, 64>, grid, dim3(kMergeThreads), 0, st, p)
+                   : launch_pdl(pa_merge_streamk_kernel<T, 128>, grid, dim3(kMergeThreads), 0, st,
+                                p);
 }
 
 pa_status check_decode_shape(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
@@ -360,8 +380,10 @@ pa_status pa_kv_write(const void *key, const void *value, const int64_t *slot_ma
     const long long total = (long long)num_tokens * num_kv_heads * p.row_chunks;
     const long long blocks = (total + 255) / 256;
     const int grid = (int)(blocks < 148 * 32 ? blocks : 148 * 32);
-    pa_kv_write_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(p);
-    return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+    return launch_pdl(pa_kv_write_kernel, dim3(grid), dim3(256), 0,
+                      static_cast<cudaStream_t>(stream), p) == cudaSuccess
+               ? PA_OK
+               : PA_ERR_CUDA;
 }
 
 pa_status pa_copy_blocks(void *k_cache, void *v_cache, const int64_t *src_dst_pairs,
@@ -387,8 +409,10 @@ pa_status pa_copy_blocks(void *k_cache, void *v_cache, const int64_t *src_dst_pa
     const long long chunks = (p.block_chunks + per_cta - 1) / per_cta;
     if (chunks > 65535 || num_pairs > 65535) return PA_ERR_UNSUPPORTED;
     dim3 grid((unsigned)chunks, (unsigned)num_pairs, 2);
-    pa_copy_blocks_kernel<<<grid, kCopyThreads, 0, static_cast<cudaStream_t>(stream)>>>(p);
-    return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+    return launch_pdl(pa_copy_blocks_kernel, grid, dim3(kCopyThreads), 0,
+                      static_cast<cudaStream_t>(stream), p) == cudaSuccess
+               ? PA_OK
+               : PA_ERR_CUDA;
 }
 
 size_t pa_decode_workspace_bytes(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
@@ -460,6 +484,9 @@ pa_status pa_decode(void *out, const void *q, const void *k_cache, const void *v
         sp.rec_o = reinterpret_cast<float *>(ws);
         sp.rec_m = reinterpret_cast<float *>(ws + pl.off_m);
         sp.rec_l = reinterpret_cast<float *>(ws + pl.off_l);
+        sp.crec_o = reinterpret_cast<float *>(ws + pl.off_co);
+        sp.crec_m = reinterpret_cast<float *>(ws + pl.off_cm);
+        sp.crec_l = reinterpret_cast<float *>(ws + pl.off_cl);
         sp.ws_pre = reinterpret_cast<int32_t *>(ws + pl.off_pre);
         sp.num_seqs = num_seqs;
         sp.num_q_heads = num_q_heads;
@@ -479,13 +506,13 @@ pa_status pa_decode(void *out, const void *q, const void *k_cache, const void *v
         SkMergeParams mp;
         mp.out = out;
         mp.ws_pre = sp.ws_pre;
-        mp.rec_o = sp.rec_o;
-        mp.rec_m = sp.rec_m;
-        mp.rec_l = sp.rec_l;
+        mp.rec_o = sp.crec_o;
+        mp.rec_m = sp.crec_m;
+        mp.rec_l = sp.crec_l;
         mp.num_seqs = num_seqs;
         mp.num_q_heads = num_q_heads;
         mp.num_kv_heads = num_kv_heads;
-        mp.num_workers = grid_used * kSkWarps;
+        mp.num_workers = grid_used;  // records are per CTA
         dim3 mgrid((unsigned)num_q_heads, (unsigned)num_seqs);
         e = dtype == PA_BF16 ? sk_merge<__nv_bfloat16>(mp, mgrid, head_dim, st_)
                              : sk_merge<__half>(mp, mgrid, head_dim, st_);

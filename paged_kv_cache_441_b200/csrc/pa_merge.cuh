@@ -75,8 +75,11 @@ __device__ __forceinline__ float lse_merge_block(int n, RecFn rec, const float *
                 wv[u] = w_s[j + u * kW];
                 src[u] = ro + (long long)r_s[j + u * kW] * D + lane * kV;
             }
+            // a zero weight marks a partial without a record: its slot may hold
+            // anything (even NaN), so it is not read at all
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
+                if (wv[u] == 0.f) continue;
                 if constexpr (kV == 4) {
                     const float4 v = *reinterpret_cast<const float4 *>(src[u]);
                     acc[0] = fmaf(wv[u], v.x, acc[0]);
@@ -92,6 +95,7 @@ __device__ __forceinline__ float lse_merge_block(int n, RecFn rec, const float *
         }
         for (; j < cnt; j += kW) {
             const float wv = w_s[j];
+            if (wv == 0.f) continue;
             const float *src = ro + (long long)r_s[j] * D + lane * kV;
 #pragma unroll
             for (int e = 0; e < kV; ++e) acc[e] = fmaf(wv, src[e], acc[e]);
@@ -129,6 +133,7 @@ struct MergeParams {
 // One CTA per (q head, sequence) with more than one partition.
 template <typename T, int D>
 __global__ void __launch_bounds__(kMergeThreads) pa_merge_kernel(const __grid_constant__ MergeParams p) {
+    pdl_wait_and_release();
     const int h = blockIdx.x, s = blockIdx.y;
     int L = p.context_lens[s];
     L = L < 0 ? 0 : (L > p.cap ? p.cap : L);

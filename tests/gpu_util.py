@@ -60,9 +60,16 @@ class DeviceCase:
         return self.out
 
     def decode(self, partition_size=0, max_context_len=None, workspace=None):
+        import torch
         import paged_kv_cache_441_b200 as pa
         c = self.case
         mcl = c.max_context_len if max_context_len is None else max_context_len
+        if workspace is None:
+            # all-ones bytes = NaN floats: nothing may be read that this call did not write
+            need = pa.decode_workspace_bytes(c.num_seqs, c.num_q_heads, c.num_kv_heads,
+                                             c.head_dim, c.block_size, c.max_blocks_per_seq,
+                                             mcl, partition_size)
+            workspace = torch.full((max(need, 256),), 255, dtype=torch.uint8, device=self.q.device)
         pa.decode(self.out, self.q, self.k_cache, self.v_cache, self.block_tables,
                   self.context_lens, c.scale, max_context_len=mcl,
                   partition_size=partition_size, workspace=workspace)
