@@ -288,17 +288,23 @@ def test_host_rejects_bad_arguments():
 
 # ------------------------------------------------------------------- full-size workloads
 
-FULL = [("llama2_7b", {}), ("gqa_llama3_8b", {"block_size": 16}),
-        ("gqa_llama3_8b", {"block_size": 32}), ("long_8_1", {"block_size": 16}),
-        ("long_8_1", {"block_size": 512}), ("long_32_8", {"block_size": 16}),
-        ("long_32_8", {"block_size": 512}), ("prefix_cow", {})]
+# (workload, builder overrides, partition_size): 0 is the library's choice (the launch
+# configuration the benchmark times); 512 is the long-context workload's literal
+# "context partitions of 512 tokens"; -1 the balanced split.
+FULL = [("llama2_7b", {}, 0), ("gqa_llama3_8b", {"block_size": 16}, 0),
+        ("gqa_llama3_8b", {"block_size": 32}, 0), ("long_8_1", {"block_size": 16}, 0),
+        ("long_8_1", {"block_size": 512}, 0), ("long_32_8", {"block_size": 16}, 0),
+        ("long_32_8", {"block_size": 512}, 0), ("prefix_cow", {}, 0),
+        ("long_8_1", {"block_size": 16}, 512), ("long_32_8", {"block_size": 512}, 512),
+        ("gqa_llama3_8b", {"block_size": 16}, -1)]
 
 
-@pytest.mark.parametrize("name,kw", FULL, ids=[f"{n}-{kw.get('block_size', 16)}" for n, kw in FULL])
-def test_full_size_sampled(name, kw):
+@pytest.mark.parametrize("name,kw,ps", FULL,
+                         ids=[f"{n}-bs{kw.get('block_size', 16)}-ps{ps}" for n, kw, ps in FULL])
+def test_full_size_sampled(name, kw, ps):
     case = make_config(name, **kw)
     sel = sample_pairs(case)
-    err, dc = _check_step(case, sel=sel)
+    err, dc = _check_step(case, partition_size=ps, sel=sel)
     out = dc.out
     assert torch.isfinite(out.float()).all(), "non-finite output somewhere"
     if name == "prefix_cow":
