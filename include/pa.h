@@ -136,6 +136,32 @@ pa_status pa_decode(void *out, const void *q, const void *k_cache, const void *v
 #define PA_PARTITION_BALANCED (-1)
 
 /*
+ * One decode step with its cache write fused in: the cache write of each sequence's
+ * new token followed by pa_decode, in one launch (plus the merge when contexts are
+ * split).  For every sequence s with L = context_lens[s] > 0 and every kv head h:
+ *   k_cache[block_tables[s][(L-1) / bs]][h][(L-1) % bs][:] = key[s*key_token_stride + h*head_dim + :]
+ *   v_cache[...] likewise from value,
+ * then the attention of pa_decode over [0, L) -- which therefore includes the new token.
+ * The write is done by the CTA that owns the last partition of (s, h) before it reads
+ * that position, so the result equals pa_kv_write (with slot = the slot of position L-1)
+ * followed by pa_decode, bit for bit.
+ * key, value : [num_seqs][...] rows, heads contiguous, token strides in elements
+ *              (multiples of 8), 16-byte aligned.
+ * Sequences must not share the block that holds their position L-1 (copy a shared
+ * block first with pa_copy_blocks).  partition_size as pa_decode; the balanced split
+ * (PA_PARTITION_BALANCED) is not supported here (PA_ERR_UNSUPPORTED).  Other
+ * arguments, errors and the workspace as pa_decode.
+ */
+pa_status pa_decode_append(void *out, const void *q, const void *key, const void *value,
+                           int64_t key_token_stride, int64_t value_token_stride, void *k_cache,
+                           void *v_cache, const int32_t *block_tables,
+                           const int32_t *context_lens, int num_seqs, int num_q_heads,
+                           int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                           int max_blocks_per_seq, float scale, int max_context_len,
+                           int partition_size, void *workspace, size_t workspace_bytes,
+                           pa_dtype dtype, void *stream);
+
+/*
  * Bytes of workspace pa_decode needs for these sizes and this partition_size.
  * Host-side; it reads the current device's SM count (cudaDeviceGetAttribute, no
  * synchronisation; 148 when no device is visible), because the balanced split keeps

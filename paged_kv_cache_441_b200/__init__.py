@@ -8,7 +8,9 @@ The compute lives in ``libpa.so`` (CUDA kernels behind the C ABI in
 * ``copy_blocks(k_cache, v_cache, pairs)`` -- copy-on-write block copies;
 * ``decode(out, q, k_cache, v_cache, block_tables, context_lens, scale, ...)`` --
   single-query attention through the block tables (single pass or split-K with a
-  log-sum-exp merge; GQA served from one page read per kv head).
+  log-sum-exp merge; GQA served from one page read per kv head);
+* ``decode_append(out, q, key, value, k_cache, v_cache, ...)`` -- the step's cache
+  write fused into the decode.
 """
 from ._lib import (  # noqa: F401
     DEVERR,
@@ -18,6 +20,7 @@ from ._lib import (  # noqa: F401
     STATIC_SCRATCH_BYTES,
     copy_blocks,
     decode,
+    decode_append,
     decode_static_scratch,
     decode_partition_tokens,
     decode_workspace_bytes,

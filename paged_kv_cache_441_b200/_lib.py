@@ -16,7 +16,7 @@ PA_FP16, PA_BF16 = 0, 1
 DEVERR = {"block_id": 0x1, "slot": 0x2, "pair": 0x4, "context": 0x8, "timeout": 0x10}
 EXPORTS = ("pa_kv_write", "pa_copy_blocks", "pa_decode", "pa_decode_workspace_bytes",
            "pa_decode_partition_tokens", "pa_get_device_error", "pa_status_str", "pa_version",
-           "pa_decode_static_scratch")
+           "pa_decode_static_scratch", "pa_decode_append")
 STATIC_SCRATCH_BYTES = 16 << 20  # PA_STATIC_SCRATCH_BYTES in include/pa.h
 
 _lib = None
@@ -51,6 +51,9 @@ def load(path: str = LIB_PATH):
     lib.pa_decode_static_scratch.argtypes = [P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, i32,
                                              f32, i32, i32, i32, P]
     lib.pa_decode_static_scratch.restype = i32
+    lib.pa_decode_append.argtypes = [P, P, P, P, i64, i64, P, P, P, P, i32, i32, i32, i32, i32,
+                                     i32, i32, f32, i32, i32, P, sz, i32, P]
+    lib.pa_decode_append.restype = i32
     lib.pa_get_device_error.argtypes = [i32, ctypes.POINTER(ctypes.c_uint32), i32]
     lib.pa_get_device_error.restype = i32
     lib.pa_status_str.argtypes = [i32]
@@ -138,6 +141,28 @@ def decode(out, q, k_cache, v_cache, block_tables, context_lens, scale, block_si
                             _ptr(context_lens), B, hq, hkv, d, bs, nb, W, float(scale),
                             int(max_context_len), int(partition_size), wptr, wbytes,
                             _dtype(q), _stream(stream)), "pa_decode")
+
+
+def decode_append(out, q, key, value, k_cache, v_cache, block_tables, context_lens, scale,
+                  max_context_len=0, partition_size=0, workspace=None, stream=None) -> None:
+    """Cache write of each sequence's new token (key/value [B, Hkv, d], stored at
+    position context_lens[s]-1) fused with decode; same result as kv_write + decode."""
+    import torch
+    B, hq, d = q.shape
+    nb, hkv, bs, _ = k_cache.shape
+    assert key.shape[0] == B and key.stride(2) == 1 and key.stride(1) == d
+    assert value.stride(2) == 1 and value.stride(1) == d
+    W = block_tables.shape[1]
+    need = decode_workspace_bytes(B, hq, hkv, d, bs, W, max_context_len, partition_size)
+    if need and workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    wptr = _ptr(workspace) if workspace is not None else None
+    wbytes = workspace.numel() if workspace is not None else 0
+    _check(load().pa_decode_append(_ptr(out), _ptr(q), _ptr(key), _ptr(value), key.stride(0),
+                                   value.stride(0), _ptr(k_cache), _ptr(v_cache),
+                                   _ptr(block_tables), _ptr(context_lens), B, hq, hkv, d, bs, nb,
+                                   W, float(scale), int(max_context_len), int(partition_size),
+                                   wptr, wbytes, _dtype(q), _stream(stream)), "pa_decode_append")
 
 
 def decode_static_scratch(out, q, k_cache, v_cache, block_tables, context_lens, scale,

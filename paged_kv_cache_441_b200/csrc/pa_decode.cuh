@@ -9,7 +9,7 @@
 // leaves the attention unchanged holds up to fp32 rounding.
 //
 // Work decomposition.  One CTA owns one item (sequence s, kv head g, context
-// partition p of `partition_tokens` tokens).  Its kWarps warps split the item's
+// partition p of `partition_tokens` tokens); grid = (kv heads, sequences, partitions).  Its kWarps warps split the item's
 // 16-token tiles into contiguous runs.  Each warp streams its tiles through its own
 // kStages-deep ring in shared memory: lane 0 issues 2-D TMA loads (128-byte
 // swizzled boxes of 64 columns x min(bs, 16) rows) for the K and V rows of a tile
@@ -71,6 +71,15 @@ struct DecodeParams {
     int partition_tokens;
     int num_parts;
     float scale_log2;
+    // Cache write fused into the decode (pa_decode_append): the new token of sequence s
+    // (key/value rows new_k + s * new_k_stride, heads contiguous) is stored at position
+    // L-1 by the CTA of the last partition before its first copy.  nullptr = no write.
+    const void *new_k;
+    const void *new_v;
+    long long new_k_stride;  // elements between tokens
+    long long new_v_stride;
+    void *k_cache;
+    void *v_cache;
 };
 
 template <int D>
@@ -509,7 +518,10 @@ __global__ void __launch_bounds__(kWarps * 32)
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
-    const int part = blockIdx.x, g = blockIdx.y, s = blockIdx.z;
+    // grid (kv head, sequence, partition): every first partition is scheduled before any
+    // second one, so the smaller remainder partitions run last and shorten the tail, and
+    // CTAs scheduled together read neighbouring heads of the same physical blocks.
+    const int g = blockIdx.x, s = blockIdx.y, part = blockIdx.z;
     const int Hq = p.num_q_heads;
 
     // Start the three independent loads of this item at once: its context length, the
@@ -541,6 +553,29 @@ __global__ void __launch_bounds__(kWarps * 32)
         return;
     }
     if (part >= nparts) return;
+
+    // Fused cache write of this step's token (position L-1, always in the last partition).
+    if (p.new_k != nullptr && part == nparts - 1) {
+        const int pos = L - 1;
+        const int blk = __ldg(table + (pos >> p.bs_shift));
+        if ((unsigned)blk < (unsigned)p.num_blocks) {
+            const size_t row =
+                ((size_t)blk * p.num_kv_heads + g) * p.block_size + (pos & (p.block_size - 1));
+            constexpr int kChunks = D / 8;  // 16-byte chunks of a head row
+            for (int c = tid; c < 2 * kChunks; c += kWarps * 32) {
+                const bool isv = c >= kChunks;
+                const int cc = isv ? c - kChunks : c;
+                const T *src = reinterpret_cast<const T *>(isv ? p.new_v : p.new_k) +
+                               (size_t)s * (isv ? p.new_v_stride : p.new_k_stride) +
+                               (size_t)g * D + 8 * cc;
+                T *dst = reinterpret_cast<T *>(isv ? p.v_cache : p.k_cache) + row * D + 8 * cc;
+                *reinterpret_cast<uint4 *>(dst) = ld_global_nc_v4(src);
+            }
+            fence_proxy_async_global();  // the TMA of the last tile reads this row
+        } else if (tid == 0) {
+            raise_error(PA_DEVERR_BLOCK_ID);
+        }
+    }
 
     const int t0 = part * P, t1 = min(t0 + P, L);
     const int ntiles = (t1 - t0 + kTile - 1) / kTile;

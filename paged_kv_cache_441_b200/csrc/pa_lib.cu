@@ -440,12 +440,18 @@ int pa_decode_partition_tokens(int num_seqs, int num_q_heads, int num_kv_heads, 
         .partition_tokens;
 }
 
-pa_status pa_decode(void *out, const void *q, const void *k_cache, const void *v_cache,
-                    const int32_t *block_tables, const int32_t *context_lens, int num_seqs,
-                    int num_q_heads, int num_kv_heads, int head_dim, int block_size,
-                    int num_blocks, int max_blocks_per_seq, float scale, int max_context_len,
-                    int partition_size, void *workspace, size_t workspace_bytes, pa_dtype dtype,
-                    void *stream) {
+}  // extern "C"
+
+namespace {
+
+// pa_decode, optionally with the step's cache write fused in (new_k != nullptr).
+pa_status decode_impl(void *out, const void *q, const void *k_cache, const void *v_cache,
+                      const int32_t *block_tables, const int32_t *context_lens, int num_seqs,
+                      int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                      int num_blocks, int max_blocks_per_seq, float scale, int max_context_len,
+                      int partition_size, void *workspace, size_t workspace_bytes,
+                      pa_dtype dtype, void *stream, const void *new_k, const void *new_v,
+                      long long new_k_stride, long long new_v_stride) {
     if (dtype != PA_FP16 && dtype != PA_BF16) return PA_ERR_INVALID_ARG;
     pa_status st = check_decode_shape(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
                                       num_blocks, max_blocks_per_seq, max_context_len,
@@ -470,6 +476,7 @@ pa_status pa_decode(void *out, const void *q, const void *k_cache, const void *v
     const int boxr = block_size < 16 ? block_size : 16;
     cudaStream_t st_ = static_cast<cudaStream_t>(stream);
     const unsigned long long rows = (unsigned long long)num_blocks * num_kv_heads * block_size;
+    if (pl.streamk && new_k != nullptr) return PA_ERR_UNSUPPORTED;  // fixed split only
     if (pl.streamk) {
         StreamKParams sp;
         std::memset(&sp, 0, sizeof sp);
@@ -543,8 +550,15 @@ pa_status pa_decode(void *out, const void *q, const void *k_cache, const void *v
     p.partition_tokens = pl.partition_tokens;
     p.num_parts = pl.num_parts;
     p.scale_log2 = scale * 1.4426950408889634f;
+    p.new_k = new_k;
+    p.new_v = new_v;
+    p.new_k_stride = new_k_stride;
+    p.new_v_stride = new_v_stride;
+    p.k_cache = const_cast<void *>(k_cache);
+    p.v_cache = const_cast<void *>(v_cache);
 
-    dim3 grid((unsigned)pl.num_parts, (unsigned)num_kv_heads, (unsigned)num_seqs);
+    if (pl.num_parts > 65535) return PA_ERR_UNSUPPORTED;  // use a larger partition_size
+    dim3 grid((unsigned)num_kv_heads, (unsigned)num_seqs, (unsigned)pl.num_parts);
     cudaError_t e = dtype == PA_BF16
                         ? dispatch_dim<__nv_bfloat16>(p, grid, st_, dev, head_dim, G, boxr)
                         : dispatch_dim<__half>(p, grid, st_, dev, head_dim, G, boxr);
@@ -570,6 +584,44 @@ pa_status pa_decode(void *out, const void *q, const void *k_cache, const void *v
         if (e != cudaSuccess) return PA_ERR_CUDA;
     }
     return PA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+pa_status pa_decode(void *out, const void *q, const void *k_cache, const void *v_cache,
+                    const int32_t *block_tables, const int32_t *context_lens, int num_seqs,
+                    int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                    int num_blocks, int max_blocks_per_seq, float scale, int max_context_len,
+                    int partition_size, void *workspace, size_t workspace_bytes, pa_dtype dtype,
+                    void *stream) {
+    return decode_impl(out, q, k_cache, v_cache, block_tables, context_lens, num_seqs,
+                       num_q_heads, num_kv_heads, head_dim, block_size, num_blocks,
+                       max_blocks_per_seq, scale, max_context_len, partition_size, workspace,
+                       workspace_bytes, dtype, stream, nullptr, nullptr, 0, 0);
+}
+
+pa_status pa_decode_append(void *out, const void *q, const void *key, const void *value,
+                           int64_t key_token_stride, int64_t value_token_stride, void *k_cache,
+                           void *v_cache, const int32_t *block_tables,
+                           const int32_t *context_lens, int num_seqs, int num_q_heads,
+                           int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                           int max_blocks_per_seq, float scale, int max_context_len,
+                           int partition_size, void *workspace, size_t workspace_bytes,
+                           pa_dtype dtype, void *stream) {
+    if (num_seqs > 0) {
+        if (!key || !value || !aligned(key, 16) || !aligned(value, 16)) return PA_ERR_INVALID_ARG;
+        if (key_token_stride % 8 != 0 || value_token_stride % 8 != 0 ||
+            key_token_stride < (int64_t)num_kv_heads * head_dim ||
+            value_token_stride < (int64_t)num_kv_heads * head_dim)
+            return PA_ERR_INVALID_ARG;
+    }
+    return decode_impl(out, q, k_cache, v_cache, block_tables, context_lens, num_seqs,
+                       num_q_heads, num_kv_heads, head_dim, block_size, num_blocks,
+                       max_blocks_per_seq, scale, max_context_len, partition_size, workspace,
+                       workspace_bytes, dtype, stream, key, value, key_token_stride,
+                       value_token_stride);
 }
 
 }  // extern "C"

@@ -24,6 +24,7 @@ namespace pa {
 // Thread e (e < D) returns element e of the merged output.
 constexpr int kMergeThreads = 256;
 constexpr int kMergeChunk = 512;
+constexpr int kMergeFew = 8;  // up to this many partials: one load round per thread
 
 template <int D, typename RecFn>
 __device__ __forceinline__ float lse_merge_block(int n, RecFn rec, const float *rm,
@@ -141,6 +142,32 @@ __global__ void __launch_bounds__(kMergeThreads) pa_merge_kernel(const __grid_co
     if (n <= 1) return;
     n = min(n, p.num_parts);
     const long long base = ((long long)s * p.num_q_heads + h) * p.num_parts;
+    if (n <= kMergeFew) {
+        // few partitions: every load of this thread's element is issued at once
+        const int d = threadIdx.x;
+        if (d >= D) return;
+        float m[kMergeFew], l[kMergeFew], o[kMergeFew];
+#pragma unroll
+        for (int i = 0; i < kMergeFew; ++i) {
+            m[i] = i < n ? p.ws_m[base + i] : -INFINITY;
+            l[i] = i < n ? p.ws_l[base + i] : 0.f;
+            o[i] = i < n ? p.ws_o[(base + i) * D + d] : 0.f;
+        }
+        float M = -INFINITY;
+#pragma unroll
+        for (int i = 0; i < kMergeFew; ++i) M = fmaxf(M, m[i]);
+        float num = 0.f, den = 0.f;
+#pragma unroll
+        for (int i = 0; i < kMergeFew; ++i) {
+            if (m[i] == -INFINITY) continue;
+            const float w = l[i] * fast_exp2(m[i] - M);
+            num = fmaf(w, o[i], num);
+            den += w;
+        }
+        T *out = reinterpret_cast<T *>(p.out) + ((size_t)s * p.num_q_heads + h) * D;
+        out[d] = Fmt<T>::from_float(den > 0.f ? num / den : 0.f);
+        return;
+    }
     const float v = lse_merge_block<D>(
         n, [&](int i) -> long long { return base + i; }, p.ws_m, p.ws_l, p.ws_o);
     T *out = reinterpret_cast<T *>(p.out) + ((size_t)s * p.num_q_heads + h) * D;

@@ -247,6 +247,30 @@ def test_copy_blocks_bit_exact():
         assert np.array_equal(bits(kc), kr) and np.array_equal(bits(vc), vr)
 
 
+@pytest.mark.parametrize("dtype", ["bf16", "fp16"])
+@pytest.mark.parametrize("G,d,bs", [(1, 128, 16), (2, 64, 8), (4, 128, 32), (8, 128, 512),
+                                    (8, 64, 16)])
+def test_decode_append_equals_write_then_decode(dtype, G, d, bs):
+    """The fused step gives the same cache and, bit for bit, the same output as the
+    cache write followed by decode (and both match the oracle)."""
+    hkv = 2
+    lens = [1, 15, 16, 17, 200, 1030, 2100, 33]
+    case = _rand_case(40 + G, dtype, len(lens), hkv * G, hkv, d, bs, lens)
+    for ps in (0, 256):
+        ref = DeviceCase(case)
+        ref.step(partition_size=ps)
+        fused = DeviceCase(case)
+        pa.decode_append(fused.out, fused.q, fused.key, fused.value, fused.k_cache,
+                         fused.v_cache, fused.block_tables, fused.context_lens, case.scale,
+                         max_context_len=case.max_context_len, partition_size=ps)
+        torch.cuda.synchronize()
+        assert np.array_equal(bits(fused.out), bits(ref.out)), (ps, "output differs")
+        assert np.array_equal(bits(fused.k_cache), bits(ref.k_cache))
+        assert np.array_equal(bits(fused.v_cache), bits(ref.v_cache))
+    want, _, _ = oracle.step(case)
+    assert np.max(np.abs(to_f64(fused.out) - want)) <= TOL[dtype]
+
+
 # ------------------------------------------------------------------------ error handling
 
 def test_device_errors_are_flagged_not_fatal():
