@@ -44,7 +44,8 @@ typedef enum {
     PA_ERR_UNSUPPORTED = 2, /* head_dim, block size or group size not built */
     PA_ERR_CUDA = 3,        /* a CUDA runtime call failed (launch, attribute, ...) */
     PA_ERR_OUT_OF_RANGE = 4,
-    PA_ERR_TIMEOUT = 5
+    PA_ERR_TIMEOUT = 5,
+    PA_ERR_NO_FREE_BLOCK = 6 /* host block manager: the pool cannot satisfy the request */
 } pa_status;
 
 typedef enum { PA_FP16 = 0, PA_BF16 = 1 } pa_dtype;

@@ -1,0 +1,99 @@
+/*
+ * Host block manager for the paged KV cache (part of libpa; host-only, no CUDA call).
+ *
+ * It owns the mapping the decode kernels read: for every sequence, the list of
+ * physical blocks that hold its tokens in order (the page table: "Sequence -> [page
+ * indices]", "IO-5 vLLM Paged Attention" note, section 3).  It follows the pages'
+ * description of the block manager:
+ *   - blocks are handed out on demand and returned as soon as a sequence ends
+ *     ("PagedAttention" summary, features 1 and 4; "PagedAttention and dynamic memory
+ *     management" blog, BlockSpaceManager: pool initialisation, "can this request be
+ *     allocated?", blocks_needed = ceil(seq_len / block_size));
+ *   - several sequences may share blocks (features 2: parallel sampling over one
+ *     prompt) -- a block carries a reference count;
+ *   - appending into a shared, partially filled block first gives the writer a
+ *     private copy (copy-on-write), emitted as a (src, dst) pair for pa_copy_blocks;
+ *   - block_usage_ratio = used blocks / pool blocks (the blog's deployment tip).
+ *
+ * The decode step that uses it:  pa_bm_append_slots (one new token per sequence)
+ * -> pa_copy_blocks(pairs) -> pa_kv_write(slot_mapping) -> pa_decode(tables, lens);
+ * pa_bm_block_tables fills the table and length arrays for the listed sequences.
+ *
+ * Not thread-safe: one manager per engine thread.  Sequence ids are caller-chosen
+ * int64 values.  Errors: PA_ERR_INVALID_ARG (null pointer, unknown or duplicate
+ * sequence id, bad size), PA_ERR_NO_FREE_BLOCK (the pool cannot satisfy the request;
+ * nothing is changed).
+ */
+#ifndef PA_BLOCK_MANAGER_H
+#define PA_BLOCK_MANAGER_H
+
+#include <stdint.h>
+
+#include "pa.h"
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct pa_block_manager pa_block_manager;
+
+/* Pool of num_blocks blocks of block_size tokens; NULL on bad arguments. */
+pa_block_manager *pa_bm_create(int num_blocks, int block_size);
+void pa_bm_destroy(pa_block_manager *bm);
+
+/* ceil(num_tokens / block_size) (the blog's blocks_needed); -1 on bad arguments. */
+int pa_bm_blocks_needed(int num_tokens, int block_size);
+
+int pa_bm_num_free_blocks(const pa_block_manager *bm);
+
+/* used blocks / pool blocks. */
+double pa_bm_usage_ratio(const pa_block_manager *bm);
+
+/* 1 if a new sequence of num_tokens tokens fits in the free blocks, else 0. */
+int pa_bm_can_allocate(const pa_block_manager *bm, int num_tokens);
+
+/* New sequence holding num_tokens tokens (a prompt): ceil(num_tokens / bs) fresh
+ * blocks, reference count 1.  The caller writes those tokens with pa_kv_write at
+ * slots pa_bm_slot(seq_id, 0 .. num_tokens-1). */
+pa_status pa_bm_allocate(pa_block_manager *bm, int64_t seq_id, int num_tokens);
+
+/* child := a sequence that shares all of parent's blocks and length (each block's
+ * reference count + 1). */
+pa_status pa_bm_fork(pa_block_manager *bm, int64_t parent_id, int64_t child_id);
+
+/* Ends a sequence: reference counts - 1; blocks that reach 0 return to the pool. */
+pa_status pa_bm_free(pa_block_manager *bm, int64_t seq_id);
+
+/*
+ * Reserves the slot of one new token for each of the n listed sequences (distinct
+ * ids), in order: a fresh block when the token starts a block; a private copy of the
+ * last block when it is shared and partially filled (pair (old, new) appended to
+ * copy_pairs, int64 [max_pairs][2]); otherwise the next free slot of the last block.
+ * slot_mapping[i] receives the slot (block * bs + offset); *num_pairs the number of
+ * pairs.  All or nothing: if the pool cannot cover the whole batch (or max_pairs is
+ * too small) nothing changes and PA_ERR_NO_FREE_BLOCK / PA_ERR_INVALID_ARG returns.
+ */
+pa_status pa_bm_append_slots(pa_block_manager *bm, const int64_t *seq_ids, int n,
+                             int64_t *slot_mapping, int64_t *copy_pairs, int max_pairs,
+                             int *num_pairs);
+
+/* Slot of token position pos of a sequence (block * bs + offset), -1 if out of range. */
+int64_t pa_bm_slot(const pa_block_manager *bm, int64_t seq_id, int pos);
+
+/* Context length of a sequence, -1 if unknown. */
+int pa_bm_seq_len(const pa_block_manager *bm, int64_t seq_id);
+
+/* Reference count of a physical block (0 = free), -1 if out of range. */
+int pa_bm_block_refcount(const pa_block_manager *bm, int block);
+
+/* For the n listed sequences: block_tables [n][width] (unused entries -1) and
+ * context_lens [n], host arrays ready to copy to the device for pa_decode.
+ * PA_ERR_INVALID_ARG if a table does not fit in width. */
+pa_status pa_bm_block_tables(const pa_block_manager *bm, const int64_t *seq_ids, int n,
+                             int32_t *block_tables, int width, int32_t *context_lens);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PA_BLOCK_MANAGER_H */

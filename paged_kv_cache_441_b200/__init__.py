@@ -10,7 +10,9 @@ The compute lives in ``libpa.so`` (CUDA kernels behind the C ABI in
   single-query attention through the block tables (single pass or split-K with a
   log-sum-exp merge; GQA served from one page read per kv head);
 * ``decode_append(out, q, key, value, k_cache, v_cache, ...)`` -- the step's cache
-  write fused into the decode.
+  write fused into the decode;
+* ``BlockManager`` -- the host owner of the page tables: on-demand allocation,
+  fork (shared blocks), copy-on-write pairs, free, usage ratio.
 """
 from ._lib import (  # noqa: F401
     DEVERR,
@@ -29,3 +31,4 @@ from ._lib import (  # noqa: F401
     load,
     version,
 )
+from .block_manager import BlockManager, blocks_needed  # noqa: F401

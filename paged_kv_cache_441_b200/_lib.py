@@ -16,7 +16,12 @@ PA_FP16, PA_BF16 = 0, 1
 DEVERR = {"block_id": 0x1, "slot": 0x2, "pair": 0x4, "context": 0x8, "timeout": 0x10}
 EXPORTS = ("pa_kv_write", "pa_copy_blocks", "pa_decode", "pa_decode_workspace_bytes",
            "pa_decode_partition_tokens", "pa_get_device_error", "pa_status_str", "pa_version",
-           "pa_decode_static_scratch", "pa_decode_append")
+           "pa_decode_static_scratch", "pa_decode_append",
+           # host block manager (include/pa_block_manager.h)
+           "pa_bm_create", "pa_bm_destroy", "pa_bm_blocks_needed", "pa_bm_num_free_blocks",
+           "pa_bm_usage_ratio", "pa_bm_can_allocate", "pa_bm_allocate", "pa_bm_fork",
+           "pa_bm_free", "pa_bm_append_slots", "pa_bm_slot", "pa_bm_seq_len",
+           "pa_bm_block_refcount", "pa_bm_block_tables")
 STATIC_SCRATCH_BYTES = 16 << 20  # PA_STATIC_SCRATCH_BYTES in include/pa.h
 
 _lib = None

@@ -1,0 +1,218 @@
+// Host block manager of the paged KV cache (include/pa_block_manager.h).
+//
+// A pool of reference-counted blocks, a LIFO free list and, per sequence, its page
+// table (physical block ids in token order) and length.  Allocation is on demand;
+// a sequence that appends into a shared, partially filled last block gets a private
+// copy first (copy-on-write), reported as a (src, dst) pair for pa_copy_blocks.
+#include <cstdint>
+#include <new>
+#include <unordered_map>
+#include <vector>
+
+#include "pa_block_manager.h"
+
+struct pa_block_manager {
+    int num_blocks = 0;
+    int block_size = 0;
+    std::vector<int> refcount;   // per physical block, 0 = free
+    std::vector<int> free_list;  // LIFO of free block ids
+    struct Seq {
+        std::vector<int> blocks;
+        int len = 0;
+        unsigned stamp = 0;  // last append batch that listed this sequence
+    };
+    std::unordered_map<int64_t, Seq> seqs;
+    // scratch of pa_bm_append_slots: references to a block given up earlier in the
+    // current batch, valid where released_stamp[block] == batch
+    std::vector<int> released;
+    std::vector<unsigned> released_stamp;
+    std::vector<Seq *> batch_seqs;
+    unsigned batch = 0;
+
+    int take() {  // caller checked that the free list is not empty
+        const int b = free_list.back();
+        free_list.pop_back();
+        refcount[b] = 1;
+        return b;
+    }
+    void drop(int b) {
+        if (--refcount[b] == 0) free_list.push_back(b);
+    }
+};
+
+extern "C" {
+
+pa_block_manager *pa_bm_create(int num_blocks, int block_size) {
+    if (num_blocks <= 0 || block_size <= 0) return nullptr;
+    pa_block_manager *bm = new (std::nothrow) pa_block_manager();
+    if (!bm) return nullptr;
+    bm->num_blocks = num_blocks;
+    bm->block_size = block_size;
+    bm->refcount.assign(num_blocks, 0);
+    bm->released.assign(num_blocks, 0);
+    bm->released_stamp.assign(num_blocks, 0);
+    bm->free_list.reserve(num_blocks);
+    for (int b = num_blocks - 1; b >= 0; --b) bm->free_list.push_back(b);  // hands out 0, 1, ...
+    return bm;
+}
+
+void pa_bm_destroy(pa_block_manager *bm) { delete bm; }
+
+int pa_bm_blocks_needed(int num_tokens, int block_size) {
+    if (num_tokens < 0 || block_size <= 0) return -1;
+    return (int)(((long long)num_tokens + block_size - 1) / block_size);
+}
+
+int pa_bm_num_free_blocks(const pa_block_manager *bm) {
+    return bm ? (int)bm->free_list.size() : 0;
+}
+
+double pa_bm_usage_ratio(const pa_block_manager *bm) {
+    if (!bm || bm->num_blocks == 0) return 0.0;
+    return (double)(bm->num_blocks - (int)bm->free_list.size()) / bm->num_blocks;
+}
+
+int pa_bm_can_allocate(const pa_block_manager *bm, int num_tokens) {
+    if (!bm) return 0;
+    const int need = pa_bm_blocks_needed(num_tokens, bm->block_size);
+    return need >= 0 && need <= (int)bm->free_list.size();
+}
+
+pa_status pa_bm_allocate(pa_block_manager *bm, int64_t seq_id, int num_tokens) {
+    if (!bm || num_tokens < 0 || bm->seqs.count(seq_id)) return PA_ERR_INVALID_ARG;
+    const int need = pa_bm_blocks_needed(num_tokens, bm->block_size);
+    if (need > (int)bm->free_list.size()) return PA_ERR_NO_FREE_BLOCK;
+    pa_block_manager::Seq s;
+    s.blocks.reserve(need);
+    for (int i = 0; i < need; ++i) s.blocks.push_back(bm->take());
+    s.len = num_tokens;
+    bm->seqs.emplace(seq_id, std::move(s));
+    return PA_OK;
+}
+
+pa_status pa_bm_fork(pa_block_manager *bm, int64_t parent_id, int64_t child_id) {
+    if (!bm || parent_id == child_id) return PA_ERR_INVALID_ARG;
+    auto it = bm->seqs.find(parent_id);
+    if (it == bm->seqs.end() || bm->seqs.count(child_id)) return PA_ERR_INVALID_ARG;
+    pa_block_manager::Seq child = it->second;
+    for (int b : child.blocks) ++bm->refcount[b];
+    bm->seqs.emplace(child_id, std::move(child));
+    return PA_OK;
+}
+
+pa_status pa_bm_free(pa_block_manager *bm, int64_t seq_id) {
+    if (!bm) return PA_ERR_INVALID_ARG;
+    auto it = bm->seqs.find(seq_id);
+    if (it == bm->seqs.end()) return PA_ERR_INVALID_ARG;
+    // return blocks back to front, so the next allocation reuses them in order
+    for (auto b = it->second.blocks.rbegin(); b != it->second.blocks.rend(); ++b) bm->drop(*b);
+    bm->seqs.erase(it);
+    return PA_OK;
+}
+
+pa_status pa_bm_append_slots(pa_block_manager *bm, const int64_t *seq_ids, int n,
+                             int64_t *slot_mapping, int64_t *copy_pairs, int max_pairs,
+                             int *num_pairs) {
+    if (!bm || n < 0 || (n > 0 && (!seq_ids || !slot_mapping)) || !num_pairs || max_pairs < 0 ||
+        (max_pairs > 0 && !copy_pairs))
+        return PA_ERR_INVALID_ARG;
+    const int bs = bm->block_size;
+    // pass 1: validate and count the fresh blocks the batch needs (without changing
+    // anything), following the reference counts as earlier entries of the batch
+    // would change them
+    const unsigned stamp = ++bm->batch;
+    bm->batch_seqs.resize(n);
+    int fresh = 0, pairs = 0;
+    for (int i = 0; i < n; ++i) {
+        auto it = bm->seqs.find(seq_ids[i]);
+        if (it == bm->seqs.end() || it->second.stamp == stamp) {  // unknown or listed twice
+            for (int j = 0; j < i; ++j) bm->batch_seqs[j]->stamp = 0;
+            return PA_ERR_INVALID_ARG;
+        }
+        pa_block_manager::Seq &s = it->second;
+        s.stamp = stamp;
+        bm->batch_seqs[i] = &s;
+        if (s.len % bs == 0) {
+            ++fresh;
+        } else {
+            const int last = s.blocks.back();
+            int &rel = bm->released[last];
+            if (bm->released_stamp[last] != stamp) {
+                bm->released_stamp[last] = stamp;
+                rel = 0;
+            }
+            if (bm->refcount[last] - rel > 1) {
+                ++fresh;
+                ++pairs;
+                ++rel;
+            }
+        }
+    }
+    if (fresh > (int)bm->free_list.size() || pairs > max_pairs) {
+        for (int i = 0; i < n; ++i) bm->batch_seqs[i]->stamp = 0;
+        return fresh > (int)bm->free_list.size() ? PA_ERR_NO_FREE_BLOCK : PA_ERR_INVALID_ARG;
+    }
+    // pass 2: apply
+    int np = 0;
+    for (int i = 0; i < n; ++i) {
+        pa_block_manager::Seq &s = *bm->batch_seqs[i];
+        const int off = s.len % bs;
+        int blk;
+        if (off == 0) {
+            blk = bm->take();
+            s.blocks.push_back(blk);
+        } else {
+            blk = s.blocks.back();
+            if (bm->refcount[blk] > 1) {
+                const int copy = bm->take();
+                copy_pairs[2 * np] = blk;
+                copy_pairs[2 * np + 1] = copy;
+                ++np;
+                bm->drop(blk);
+                s.blocks.back() = copy;
+                blk = copy;
+            }
+        }
+        slot_mapping[i] = (int64_t)blk * bs + off;
+        ++s.len;
+    }
+    *num_pairs = np;
+    return PA_OK;
+}
+
+int64_t pa_bm_slot(const pa_block_manager *bm, int64_t seq_id, int pos) {
+    if (!bm) return -1;
+    auto it = bm->seqs.find(seq_id);
+    if (it == bm->seqs.end() || pos < 0 || pos >= it->second.len) return -1;
+    return (int64_t)it->second.blocks[pos / bm->block_size] * bm->block_size +
+           pos % bm->block_size;
+}
+
+int pa_bm_seq_len(const pa_block_manager *bm, int64_t seq_id) {
+    if (!bm) return -1;
+    auto it = bm->seqs.find(seq_id);
+    return it == bm->seqs.end() ? -1 : it->second.len;
+}
+
+int pa_bm_block_refcount(const pa_block_manager *bm, int block) {
+    if (!bm || block < 0 || block >= bm->num_blocks) return -1;
+    return bm->refcount[block];
+}
+
+pa_status pa_bm_block_tables(const pa_block_manager *bm, const int64_t *seq_ids, int n,
+                             int32_t *block_tables, int width, int32_t *context_lens) {
+    if (!bm || n < 0 || width <= 0 || (n > 0 && (!seq_ids || !block_tables || !context_lens)))
+        return PA_ERR_INVALID_ARG;
+    for (int i = 0; i < n; ++i) {
+        auto it = bm->seqs.find(seq_ids[i]);
+        if (it == bm->seqs.end() || (int)it->second.blocks.size() > width)
+            return PA_ERR_INVALID_ARG;
+        const std::vector<int> &b = it->second.blocks;
+        for (int j = 0; j < width; ++j)
+            block_tables[(size_t)i * width + j] = j < (int)b.size() ? b[j] : -1;
+        context_lens[i] = it->second.len;
+    }
+    return PA_OK;
+}
+
+}  // extern "C"

@@ -324,6 +324,7 @@ const char *pa_status_str(pa_status s) {
         case PA_ERR_CUDA: return "CUDA runtime error";
         case PA_ERR_OUT_OF_RANGE: return "index out of range (device error word)";
         case PA_ERR_TIMEOUT: return "bounded wait expired (device error word)";
+        case PA_ERR_NO_FREE_BLOCK: return "no free block in the pool";
     }
     return "unknown status";
 }

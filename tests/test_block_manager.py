@@ -1,0 +1,185 @@
+"""Host block manager (C++ in libpa) against a separate Python model, invariants, the
+pages' worked examples, and the logical token streams it produces through the oracle's
+cache operations (no GPU)."""
+import numpy as np
+import pytest
+
+import oracle
+import paged_kv_cache_441_b200 as pa
+from oracle import oracle_np
+from tests.bm_model import Model, NoBlocks
+from tests.pins import read_golden
+
+
+def _invariants(bm, model):
+    assert bm.num_free_blocks == len(model.free_ids)
+    refs = [0] * len(model.ref)
+    for blocks, n in model.seqs.values():
+        assert len(blocks) == -(-n // model.bs)
+        for b in blocks:
+            refs[b] += 1
+    assert refs == model.ref
+    for b, r in enumerate(model.ref):
+        assert bm.refcount(b) == r
+    assert abs(bm.usage_ratio - (1 - len(model.free_ids) / len(model.ref))) < 1e-12
+
+
+def test_pages_worked_examples():
+    g = {k: kv for k, kv in read_golden() if k in ("blocks_needed", "pool_tokens")}
+    ex = g["blocks_needed"]
+    assert pa.blocks_needed(int(ex["seq_len"]), int(ex["block_size"])) == int(ex["expect"])
+    pool = g["pool_tokens"]
+    nb, bs, cap = int(pool["num_blocks"]), int(pool["block_size"]), int(pool["expect"])
+    bm = pa.BlockManager(nb, bs)
+    assert bm.can_allocate(cap) and not bm.can_allocate(cap + 1)
+    bm.allocate(1, 3200)
+    assert bm.num_free_blocks == nb - 7
+    bm.allocate(2, cap - 7 * bs)  # the rest of the pool, exactly
+    assert bm.num_free_blocks == 0 and bm.usage_ratio == 1.0
+    with pytest.raises(pa.PAError):
+        bm.allocate(3, 1)
+    bm.free(1)
+    assert bm.num_free_blocks == 7
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_random_operations_match_model(seed):
+    rng = np.random.default_rng(seed)
+    nb, bs = int(rng.integers(8, 64)), int(rng.choice([1, 2, 4, 16]))
+    bm, model = pa.BlockManager(nb, bs), Model(nb, bs)
+    next_id = 0
+    for step in range(300):
+        op = rng.choice(["alloc", "fork", "free", "append"], p=[0.25, 0.2, 0.15, 0.4])
+        live = list(model.seqs)
+        if op == "alloc":
+            n = int(rng.integers(0, 3 * bs + 2))
+            try:
+                model.allocate(next_id, n)
+                bm.allocate(next_id, n)
+            except NoBlocks:
+                with pytest.raises(pa.PAError):
+                    bm.allocate(next_id, n)
+            next_id += 1
+        elif op == "fork" and live:
+            p = int(rng.choice(live))
+            model.fork(p, next_id)
+            bm.fork(p, next_id)
+            next_id += 1
+        elif op == "free" and live:
+            s = int(rng.choice(live))
+            model.free(s)
+            bm.free(s)
+        elif op == "append" and live:
+            ids = [int(x) for x in rng.permutation(live)[: int(rng.integers(1, len(live) + 1))]]
+            try:
+                slots, pairs = model.append(ids)
+                s2, p2 = bm.append_slots(ids)
+                assert s2.tolist() == slots and [tuple(x) for x in p2.tolist()] == pairs
+                assert len(set(slots)) == len(slots)  # no two writers share a slot
+            except NoBlocks:
+                with pytest.raises(pa.PAError):
+                    bm.append_slots(ids)
+        _invariants(bm, model)
+        for sid, (blocks, n) in model.seqs.items():
+            assert bm.seq_len(sid) == n
+            bt, cl = bm.block_tables([sid], max(len(blocks), 1))
+            assert bt[0, : len(blocks)].tolist() == blocks and cl[0] == n
+
+
+def test_errors_change_nothing():
+    bm = pa.BlockManager(4, 4)
+    bm.allocate(7, 6)  # 2 blocks
+    bm.fork(7, 8)
+    for bad in (lambda: bm.allocate(7, 1), lambda: bm.fork(7, 8), lambda: bm.fork(99, 1),
+                lambda: bm.free(99), lambda: bm.append_slots([7, 7]),
+                lambda: bm.append_slots([42]), lambda: bm.block_tables([7], 1)):
+        with pytest.raises(pa.PAError):
+            bad()
+    # 2 free blocks; 7 and 8 share a partial block: 8 appends need a copy each -> 2 blocks
+    # for the pair, then every further block boundary needs more: exhaust, state unchanged
+    before = (bm.num_free_blocks, bm.seq_len(7), bm.seq_len(8))
+    bm.allocate(9, 8)  # takes the last 2 blocks
+    with pytest.raises(pa.PAError):
+        bm.append_slots([7, 8])  # 7 needs a private copy of the shared block: none left
+    assert (bm.seq_len(7), bm.seq_len(8)) == before[1:]
+    bm.free(9)
+    slots, pairs = bm.append_slots([7, 8])
+    assert len(pairs) == 1 and pairs[0, 0] == bm.block_tables([8], 2)[0][0, 1]
+
+
+def test_parallel_sampling_copy_on_write_counts():
+    """64 prompts of 1000 tokens, 8 samples each: the first append copies the shared
+    partial block for 7 samples of every group (448 pairs); the 8th writes in place."""
+    bs = 16
+    bm = pa.BlockManager(64 * (63 + 7) + 10, bs)
+    ids = []
+    for g in range(64):
+        bm.allocate(g * 8, 1000)
+        for j in range(1, 8):
+            bm.fork(g * 8, g * 8 + j)
+        ids += list(range(g * 8, g * 8 + 8))
+    assert bm.refcount(bm.block_tables([0], 63)[0][0, 62]) == 8
+    slots, pairs = bm.append_slots(ids)
+    assert pairs.shape == (448, 2)
+    assert len(set(slots.tolist())) == 512 and all(int(s) % bs == 1000 % bs for s in slots)
+    slots2, pairs2 = bm.append_slots(ids)
+    assert pairs2.shape == (0, 2)
+
+
+def test_logical_token_streams_through_tables():
+    """Drive the oracle's cache write / block copy with the manager through prompts,
+    forks, appends and frees: every live sequence's K, gathered through its table,
+    must equal the tokens it logically holds."""
+    rng = np.random.default_rng(3)
+    nb, hkv, bs, d = 96, 2, 4, 8
+    bm = pa.BlockManager(nb, bs)
+    kc = np.zeros((nb, hkv, bs, d), np.uint16)
+    vc = np.zeros_like(kc)
+    logical = {}
+    next_id, counter = 0, 1
+
+    def tok():
+        nonlocal counter
+        counter += 1
+        return np.full((1, hkv, d), counter % 60000, np.uint16)
+
+    for step in range(120):
+        live = list(logical)
+        r = rng.random()
+        if r < 0.15 or not live:
+            n = int(rng.integers(1, 11))
+            if bm.can_allocate(n):
+                bm.allocate(next_id, n)
+                toks = [tok() for _ in range(n)]
+                sm = np.array([bm.slot(next_id, i) for i in range(n)], np.int64)
+                oracle.kv_write(np.concatenate(toks), np.concatenate(toks), sm, kc, vc)
+                logical[next_id] = toks
+                next_id += 1
+        elif r < 0.3:
+            p = int(rng.choice(live))
+            bm.fork(p, next_id)
+            logical[next_id] = list(logical[p])
+            next_id += 1
+        elif r < 0.4:
+            s = int(rng.choice(live))
+            bm.free(s)
+            del logical[s]
+        else:
+            ids = [int(x) for x in rng.permutation(live)]
+            try:
+                slots, pairs = bm.append_slots(ids)
+            except pa.PAError:
+                continue
+            oracle.copy_blocks(kc, vc, pairs)  # copies first, then the new tokens
+            toks = [tok() for _ in ids]
+            oracle.kv_write(np.concatenate(toks), np.concatenate(toks), slots, kc, vc)
+            for s, t in zip(ids, toks):
+                logical[s].append(t)
+        for s, toks in logical.items():
+            L = len(toks)
+            bt, cl = bm.block_tables([s], max(-(-L // bs), 1))
+            assert cl[0] == L
+            for g in range(hkv):
+                got = oracle_np.gather(kc, bt[0], L, g)
+                want = np.concatenate([t[:, g] for t in toks])
+                assert np.array_equal(got, want), (step, s)
