@@ -92,6 +92,27 @@ pa_status pa_copy_blocks(void *k_cache, void *v_cache, const int64_t *src_dst_pa
                          int num_blocks, pa_dtype dtype, void *stream);
 
 /*
+ * Block swap between two pools -- the GPU cache and a host pool in pinned memory --
+ * for preemption ("PagedAttention" summary, section 5 and conclusion: block-level
+ * memory management with preemptive request scheduling; "PagedAttention and dynamic
+ * memory management" blog, BlockSpaceManager(num_cpu_blocks=...)): a preempted
+ * sequence's blocks are copied out to host blocks and later back in.
+ *
+ * For each pair p < num_pairs: dst block pairs[2p+1] := src block pairs[2p] in both
+ * caches (all kv heads and slots).  src/dst caches have the cache layout with
+ * src_num_blocks / dst_num_blocks blocks; each may be device memory or pinned host
+ * memory mapped for the device (cudaHostAlloc / cudaHostRegister, reached through
+ * unified addressing).  src_dst_pairs: int64 [num_pairs][2] in device memory (or
+ * mapped pinned memory).  Destination blocks must be distinct and the two pools must
+ * not overlap.  One launch; bit-exact.  A pair id outside its pool sets
+ * PA_DEVERR_PAIR and that pair is skipped.  Pointers 16-byte aligned.
+ */
+pa_status pa_swap_blocks(void *dst_k_cache, void *dst_v_cache, const void *src_k_cache,
+                         const void *src_v_cache, const int64_t *src_dst_pairs, int num_pairs,
+                         int num_kv_heads, int block_size, int head_dim, int src_num_blocks,
+                         int dst_num_blocks, pa_dtype dtype, void *stream);
+
+/*
  * Decode attention over the paged cache ("IO-5 vLLM Paged Attention" note, section 4:
  * Attention(Q, K, V) = softmax(Q K^T / sqrt(d_k)) V with K, V loaded page by page,
  * K = concat(K_page_a, K_page_b, ...) in table order; section 3: Sequence -> [page

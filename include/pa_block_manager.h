@@ -19,7 +19,8 @@
  * -> pa_copy_blocks(pairs) -> pa_kv_write(slot_mapping) -> pa_decode(tables, lens);
  * pa_bm_block_tables fills the table and length arrays for the listed sequences.
  *
- * Not thread-safe: one manager per engine thread.  Sequence ids are caller-chosen
+ * Not thread-safe: one manager per engine thread.  Operations other than swap-in and
+ * free on a swapped-out sequence return PA_ERR_INVALID_ARG.  Sequence ids are caller-chosen
  * int64 values.  Errors: PA_ERR_INVALID_ARG (null pointer, unknown or duplicate
  * sequence id, bad size), PA_ERR_NO_FREE_BLOCK (the pool cannot satisfy the request;
  * nothing is changed).
@@ -85,6 +86,34 @@ int pa_bm_seq_len(const pa_block_manager *bm, int64_t seq_id);
 
 /* Reference count of a physical block (0 = free), -1 if out of range. */
 int pa_bm_block_refcount(const pa_block_manager *bm, int block);
+
+/*
+ * Host pool for preemption (the blog's num_cpu_blocks; the summary's preemptive
+ * scheduling): a preempted group of sequences is swapped out to host blocks and later
+ * back in, with pa_swap_blocks moving the data.  A swapped-out sequence can only be
+ * swapped in or freed.
+ */
+pa_status pa_bm_set_cpu_pool(pa_block_manager *bm, int num_cpu_blocks); /* once */
+int pa_bm_num_free_cpu_blocks(const pa_block_manager *bm);
+
+/* 1 if the sequence's blocks are in the host pool, 0 if on the GPU, -1 if unknown. */
+int pa_bm_is_swapped(const pa_block_manager *bm, int64_t seq_id);
+
+/*
+ * Swap out the n listed GPU-resident sequences: every distinct GPU block they use gets
+ * one host block (so blocks shared inside the group stay shared), pairs (gpu block,
+ * host block) go to pairs [max_pairs][2] for pa_swap_blocks(host pool <- GPU cache),
+ * and the GPU blocks return to the GPU pool.  The group must hold every reference to
+ * its blocks (a block also used by an unlisted sequence: PA_ERR_INVALID_ARG).  All or
+ * nothing (PA_ERR_NO_FREE_BLOCK when the host pool is short).
+ */
+pa_status pa_bm_swap_out(pa_block_manager *bm, const int64_t *seq_ids, int n, int64_t *pairs,
+                         int max_pairs, int *num_pairs);
+
+/* The reverse: host blocks -> fresh GPU blocks, pairs (host block, gpu block) for
+ * pa_swap_blocks(GPU cache <- host pool).  All or nothing. */
+pa_status pa_bm_swap_in(pa_block_manager *bm, const int64_t *seq_ids, int n, int64_t *pairs,
+                        int max_pairs, int *num_pairs);
 
 /* For the n listed sequences: block_tables [n][width] (unused entries -1) and
  * context_lens [n], host arrays ready to copy to the device for pa_decode.

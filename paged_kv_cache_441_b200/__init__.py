@@ -29,6 +29,7 @@ from ._lib import (  # noqa: F401
     device_error,
     kv_write,
     load,
+    swap_blocks,
     version,
 )
 from .block_manager import BlockManager, blocks_needed  # noqa: F401

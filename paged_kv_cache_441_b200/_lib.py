@@ -16,12 +16,13 @@ PA_FP16, PA_BF16 = 0, 1
 DEVERR = {"block_id": 0x1, "slot": 0x2, "pair": 0x4, "context": 0x8, "timeout": 0x10}
 EXPORTS = ("pa_kv_write", "pa_copy_blocks", "pa_decode", "pa_decode_workspace_bytes",
            "pa_decode_partition_tokens", "pa_get_device_error", "pa_status_str", "pa_version",
-           "pa_decode_static_scratch", "pa_decode_append",
+           "pa_decode_static_scratch", "pa_decode_append", "pa_swap_blocks",
            # host block manager (include/pa_block_manager.h)
            "pa_bm_create", "pa_bm_destroy", "pa_bm_blocks_needed", "pa_bm_num_free_blocks",
            "pa_bm_usage_ratio", "pa_bm_can_allocate", "pa_bm_allocate", "pa_bm_fork",
            "pa_bm_free", "pa_bm_append_slots", "pa_bm_slot", "pa_bm_seq_len",
-           "pa_bm_block_refcount", "pa_bm_block_tables")
+           "pa_bm_block_refcount", "pa_bm_block_tables", "pa_bm_set_cpu_pool",
+           "pa_bm_num_free_cpu_blocks", "pa_bm_is_swapped", "pa_bm_swap_out", "pa_bm_swap_in")
 STATIC_SCRATCH_BYTES = 16 << 20  # PA_STATIC_SCRATCH_BYTES in include/pa.h
 
 _lib = None
@@ -46,6 +47,8 @@ def load(path: str = LIB_PATH):
     lib.pa_kv_write.restype = i32
     lib.pa_copy_blocks.argtypes = [P, P, P, i32, i32, i32, i32, i32, i32, P]
     lib.pa_copy_blocks.restype = i32
+    lib.pa_swap_blocks.argtypes = [P, P, P, P, P, i32, i32, i32, i32, i32, i32, i32, P]
+    lib.pa_swap_blocks.restype = i32
     lib.pa_decode.argtypes = [P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, i32, f32, i32, i32,
                               P, sz, i32, P]
     lib.pa_decode.restype = i32
@@ -110,6 +113,16 @@ def copy_blocks(k_cache, v_cache, pairs, stream=None) -> None:
     nb, hkv, bs, d = k_cache.shape
     _check(load().pa_copy_blocks(_ptr(k_cache), _ptr(v_cache), _ptr(pairs), pairs.shape[0], hkv,
                                  bs, d, nb, _dtype(k_cache), _stream(stream)), "pa_copy_blocks")
+
+
+def swap_blocks(dst_k_cache, dst_v_cache, src_k_cache, src_v_cache, pairs, stream=None) -> None:
+    """Copy blocks pairs[:, 0] of the source pool to blocks pairs[:, 1] of the destination
+    pool; either pool may be a pinned host tensor.  pairs: int64 [P, 2] (device or pinned)."""
+    snb, hkv, bs, d = src_k_cache.shape
+    dnb = dst_k_cache.shape[0]
+    _check(load().pa_swap_blocks(_ptr(dst_k_cache), _ptr(dst_v_cache), _ptr(src_k_cache),
+                                 _ptr(src_v_cache), _ptr(pairs), pairs.shape[0], hkv, bs, d, snb,
+                                 dnb, _dtype(src_k_cache), _stream(stream)), "pa_swap_blocks")
 
 
 def decode_workspace_bytes(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,

@@ -46,6 +46,15 @@ def _lib():
         lib.pa_bm_block_refcount.restype = i32
         lib.pa_bm_block_tables.argtypes = [P, P, i32, P, i32, P]
         lib.pa_bm_block_tables.restype = i32
+        lib.pa_bm_set_cpu_pool.argtypes = [P, i32]
+        lib.pa_bm_set_cpu_pool.restype = i32
+        lib.pa_bm_num_free_cpu_blocks.argtypes = [P]
+        lib.pa_bm_num_free_cpu_blocks.restype = i32
+        lib.pa_bm_is_swapped.argtypes = [P, i64]
+        lib.pa_bm_is_swapped.restype = i32
+        for f in (lib.pa_bm_swap_out, lib.pa_bm_swap_in):
+            f.argtypes = [P, P, i32, P, i32, ctypes.POINTER(i32)]
+            f.restype = i32
         _declared = True
     return lib
 
@@ -116,6 +125,32 @@ class BlockManager:
 
     def refcount(self, block: int) -> int:
         return int(self._lib.pa_bm_block_refcount(self._h, block))
+
+    def set_cpu_pool(self, num_cpu_blocks: int) -> None:
+        _check(self._lib.pa_bm_set_cpu_pool(self._h, num_cpu_blocks), "pa_bm_set_cpu_pool")
+
+    @property
+    def num_free_cpu_blocks(self) -> int:
+        return int(self._lib.pa_bm_num_free_cpu_blocks(self._h))
+
+    def is_swapped(self, seq_id: int) -> bool:
+        return self._lib.pa_bm_is_swapped(self._h, seq_id) == 1
+
+    def _move(self, fn, seq_ids, what):
+        ids = np.ascontiguousarray(seq_ids, np.int64)
+        cap = max(1, int(self.num_blocks))
+        pairs = np.empty((cap, 2), np.int64)
+        npairs = ctypes.c_int(0)
+        _check(fn(self._h, _p(ids), ids.shape[0], _p(pairs), cap, ctypes.byref(npairs)), what)
+        return pairs[:npairs.value].copy()
+
+    def swap_out(self, seq_ids):
+        """Move a group of sequences to the host pool -> pairs (gpu block, host block)."""
+        return self._move(self._lib.pa_bm_swap_out, seq_ids, "pa_bm_swap_out")
+
+    def swap_in(self, seq_ids):
+        """Move a swapped-out group back to the GPU -> pairs (host block, gpu block)."""
+        return self._move(self._lib.pa_bm_swap_in, seq_ids, "pa_bm_swap_in")
 
     def block_tables(self, seq_ids, width: int):
         """(block_tables int32 [n, width], context_lens int32 [n]) for the decode call."""

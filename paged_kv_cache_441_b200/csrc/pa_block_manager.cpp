@@ -17,10 +17,15 @@ struct pa_block_manager {
     std::vector<int> refcount;   // per physical block, 0 = free
     std::vector<int> free_list;  // LIFO of free block ids
     struct Seq {
-        std::vector<int> blocks;
+        std::vector<int> blocks;  // GPU block ids, or host block ids when on_cpu
         int len = 0;
         unsigned stamp = 0;  // last append batch that listed this sequence
+        bool on_cpu = false;
     };
+    // host pool (preemption)
+    int num_cpu_blocks = 0;
+    std::vector<int> cpu_refcount;
+    std::vector<int> cpu_free_list;
     std::unordered_map<int64_t, Seq> seqs;
     // scratch of pa_bm_append_slots: references to a block given up earlier in the
     // current batch, valid where released_stamp[block] == batch
@@ -40,7 +45,86 @@ struct pa_block_manager {
     }
 };
 
+namespace {
+
+// Moves the listed sequences between the pools: `from` (refcounts, free list) -> `to`.
+pa_status move_group(pa_block_manager *bm, const int64_t *seq_ids, int n, int64_t *pairs,
+                     int max_pairs, int *num_pairs, bool out) {
+    if (!bm || n < 0 || (n > 0 && !seq_ids) || !num_pairs || max_pairs < 0 ||
+        (max_pairs > 0 && !pairs))
+        return PA_ERR_INVALID_ARG;
+    if (out && bm->num_cpu_blocks == 0) return PA_ERR_INVALID_ARG;
+    std::vector<int> &from_ref = out ? bm->refcount : bm->cpu_refcount;
+    std::vector<int> &to_ref = out ? bm->cpu_refcount : bm->refcount;
+    std::vector<int> &from_free = out ? bm->free_list : bm->cpu_free_list;
+    std::vector<int> &to_free = out ? bm->cpu_free_list : bm->free_list;
+    std::vector<pa_block_manager::Seq *> group;
+    std::unordered_map<int, int> uses;  // block -> references held by the group
+    std::vector<int> order;             // distinct blocks, first-use order
+    for (int i = 0; i < n; ++i) {
+        auto it = bm->seqs.find(seq_ids[i]);
+        if (it == bm->seqs.end() || it->second.on_cpu != !out) return PA_ERR_INVALID_ARG;
+        for (pa_block_manager::Seq *g : group)
+            if (g == &it->second) return PA_ERR_INVALID_ARG;  // listed twice
+        group.push_back(&it->second);
+        for (int b : it->second.blocks)
+            if (uses[b]++ == 0) order.push_back(b);
+    }
+    for (int b : order)
+        if (uses[b] != from_ref[b]) return PA_ERR_INVALID_ARG;  // shared outside the group
+    if ((int)order.size() > (int)to_free.size()) return PA_ERR_NO_FREE_BLOCK;
+    if ((int)order.size() > max_pairs) return PA_ERR_INVALID_ARG;
+    std::unordered_map<int, int> moved;
+    for (size_t i = 0; i < order.size(); ++i) {
+        const int b = order[i];
+        const int nb = to_free.back();
+        to_free.pop_back();
+        to_ref[nb] = from_ref[b];
+        from_ref[b] = 0;
+        from_free.push_back(b);
+        moved[b] = nb;
+        pairs[2 * i] = b;
+        pairs[2 * i + 1] = nb;
+    }
+    for (pa_block_manager::Seq *g : group) {
+        for (int &b : g->blocks) b = moved[b];
+        g->on_cpu = out;
+    }
+    *num_pairs = (int)order.size();
+    return PA_OK;
+}
+
+}  // namespace
+
 extern "C" {
+
+pa_status pa_bm_set_cpu_pool(pa_block_manager *bm, int num_cpu_blocks) {
+    if (!bm || num_cpu_blocks <= 0 || bm->num_cpu_blocks != 0) return PA_ERR_INVALID_ARG;
+    bm->num_cpu_blocks = num_cpu_blocks;
+    bm->cpu_refcount.assign(num_cpu_blocks, 0);
+    for (int b = num_cpu_blocks - 1; b >= 0; --b) bm->cpu_free_list.push_back(b);
+    return PA_OK;
+}
+
+int pa_bm_num_free_cpu_blocks(const pa_block_manager *bm) {
+    return bm ? (int)bm->cpu_free_list.size() : 0;
+}
+
+int pa_bm_is_swapped(const pa_block_manager *bm, int64_t seq_id) {
+    if (!bm) return -1;
+    auto it = bm->seqs.find(seq_id);
+    return it == bm->seqs.end() ? -1 : (it->second.on_cpu ? 1 : 0);
+}
+
+pa_status pa_bm_swap_out(pa_block_manager *bm, const int64_t *seq_ids, int n, int64_t *pairs,
+                         int max_pairs, int *num_pairs) {
+    return move_group(bm, seq_ids, n, pairs, max_pairs, num_pairs, true);
+}
+
+pa_status pa_bm_swap_in(pa_block_manager *bm, const int64_t *seq_ids, int n, int64_t *pairs,
+                        int max_pairs, int *num_pairs) {
+    return move_group(bm, seq_ids, n, pairs, max_pairs, num_pairs, false);
+}
 
 pa_block_manager *pa_bm_create(int num_blocks, int block_size) {
     if (num_blocks <= 0 || block_size <= 0) return nullptr;
@@ -93,7 +177,8 @@ pa_status pa_bm_allocate(pa_block_manager *bm, int64_t seq_id, int num_tokens) {
 pa_status pa_bm_fork(pa_block_manager *bm, int64_t parent_id, int64_t child_id) {
     if (!bm || parent_id == child_id) return PA_ERR_INVALID_ARG;
     auto it = bm->seqs.find(parent_id);
-    if (it == bm->seqs.end() || bm->seqs.count(child_id)) return PA_ERR_INVALID_ARG;
+    if (it == bm->seqs.end() || it->second.on_cpu || bm->seqs.count(child_id))
+        return PA_ERR_INVALID_ARG;
     pa_block_manager::Seq child = it->second;
     for (int b : child.blocks) ++bm->refcount[b];
     bm->seqs.emplace(child_id, std::move(child));
@@ -105,7 +190,13 @@ pa_status pa_bm_free(pa_block_manager *bm, int64_t seq_id) {
     auto it = bm->seqs.find(seq_id);
     if (it == bm->seqs.end()) return PA_ERR_INVALID_ARG;
     // return blocks back to front, so the next allocation reuses them in order
-    for (auto b = it->second.blocks.rbegin(); b != it->second.blocks.rend(); ++b) bm->drop(*b);
+    for (auto b = it->second.blocks.rbegin(); b != it->second.blocks.rend(); ++b) {
+        if (it->second.on_cpu) {
+            if (--bm->cpu_refcount[*b] == 0) bm->cpu_free_list.push_back(*b);
+        } else {
+            bm->drop(*b);
+        }
+    }
     bm->seqs.erase(it);
     return PA_OK;
 }
@@ -125,7 +216,7 @@ pa_status pa_bm_append_slots(pa_block_manager *bm, const int64_t *seq_ids, int n
     int fresh = 0, pairs = 0;
     for (int i = 0; i < n; ++i) {
         auto it = bm->seqs.find(seq_ids[i]);
-        if (it == bm->seqs.end() || it->second.stamp == stamp) {  // unknown or listed twice
+        if (it == bm->seqs.end() || it->second.stamp == stamp || it->second.on_cpu) {
             for (int j = 0; j < i; ++j) bm->batch_seqs[j]->stamp = 0;
             return PA_ERR_INVALID_ARG;
         }
@@ -183,7 +274,7 @@ pa_status pa_bm_append_slots(pa_block_manager *bm, const int64_t *seq_ids, int n
 int64_t pa_bm_slot(const pa_block_manager *bm, int64_t seq_id, int pos) {
     if (!bm) return -1;
     auto it = bm->seqs.find(seq_id);
-    if (it == bm->seqs.end() || pos < 0 || pos >= it->second.len) return -1;
+    if (it == bm->seqs.end() || it->second.on_cpu || pos < 0 || pos >= it->second.len) return -1;
     return (int64_t)it->second.blocks[pos / bm->block_size] * bm->block_size +
            pos % bm->block_size;
 }
@@ -205,7 +296,8 @@ pa_status pa_bm_block_tables(const pa_block_manager *bm, const int64_t *seq_ids,
         return PA_ERR_INVALID_ARG;
     for (int i = 0; i < n; ++i) {
         auto it = bm->seqs.find(seq_ids[i]);
-        if (it == bm->seqs.end() || (int)it->second.blocks.size() > width)
+        if (it == bm->seqs.end() || it->second.on_cpu ||
+            (int)it->second.blocks.size() > width)
             return PA_ERR_INVALID_ARG;
         const std::vector<int> &b = it->second.blocks;
         for (int j = 0; j < width; ++j)

@@ -91,4 +91,46 @@ __global__ void __launch_bounds__(kCopyThreads)
     }
 }
 
+struct SwapBlocksParams {
+    uint8_t *dst_k;
+    uint8_t *dst_v;
+    const uint8_t *src_k;
+    const uint8_t *src_v;
+    const int64_t *pairs;     // [n][2]: block in the source pool, block in the destination pool
+    long long block_chunks;   // 16-byte chunks per block per cache
+    int src_blocks;
+    int dst_blocks;
+};
+
+// Block copy between two pools, one of which may be pinned host memory reached
+// through unified addressing (swap out: device -> host, swap in: host -> device).
+// grid = (pairs, chunks of a block, 2 caches); kCopyUnroll 16-byte loads in flight
+// per thread, which is what keeps the host link busy.
+__global__ void __launch_bounds__(kCopyThreads)
+    pa_swap_blocks_kernel(const __grid_constant__ SwapBlocksParams p) {
+    pdl_wait_and_release();
+    const int pair = blockIdx.x;
+    const long long src = p.pairs[2 * pair], dst = p.pairs[2 * pair + 1];
+    if (src < 0 || src >= p.src_blocks || dst < 0 || dst >= p.dst_blocks) {
+        if (blockIdx.y == 0 && blockIdx.z == 0 && threadIdx.x == 0) raise_error(PA_DEVERR_PAIR);
+        return;
+    }
+    const uint4 *from = reinterpret_cast<const uint4 *>(blockIdx.z == 0 ? p.src_k : p.src_v) +
+                        src * p.block_chunks;
+    uint4 *to = reinterpret_cast<uint4 *>(blockIdx.z == 0 ? p.dst_k : p.dst_v) +
+                dst * p.block_chunks;
+    const long long c0 = (long long)blockIdx.y * kCopyThreads * kCopyUnroll + threadIdx.x;
+    uint4 buf[kCopyUnroll];
+#pragma unroll
+    for (int u = 0; u < kCopyUnroll; ++u) {
+        const long long c = c0 + (long long)u * kCopyThreads;
+        if (c < p.block_chunks) buf[u] = from[c];
+    }
+#pragma unroll
+    for (int u = 0; u < kCopyUnroll; ++u) {
+        const long long c = c0 + (long long)u * kCopyThreads;
+        if (c < p.block_chunks) to[c] = buf[u];
+    }
+}
+
 }  // namespace pa

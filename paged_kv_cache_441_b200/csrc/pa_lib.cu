@@ -416,6 +416,56 @@ pa_status pa_copy_blocks(void *k_cache, void *v_cache, const int64_t *src_dst_pa
                : PA_ERR_CUDA;
 }
 
+pa_status pa_swap_blocks(void *dst_k_cache, void *dst_v_cache, const void *src_k_cache,
+                         const void *src_v_cache, const int64_t *src_dst_pairs, int num_pairs,
+                         int num_kv_heads, int block_size, int head_dim, int src_num_blocks,
+                         int dst_num_blocks, pa_dtype dtype, void *stream) {
+    if (dtype != PA_FP16 && dtype != PA_BF16) return PA_ERR_INVALID_ARG;
+    if (num_pairs < 0 || num_kv_heads <= 0 || block_size <= 0 || head_dim <= 0 ||
+        src_num_blocks <= 0 || dst_num_blocks <= 0)
+        return PA_ERR_INVALID_ARG;
+    if (num_pairs == 0) return PA_OK;
+    if (!dst_k_cache || !dst_v_cache || !src_k_cache || !src_v_cache || !src_dst_pairs)
+        return PA_ERR_INVALID_ARG;
+    if (!aligned(dst_k_cache, 16) || !aligned(dst_v_cache, 16) || !aligned(src_k_cache, 16) ||
+        !aligned(src_v_cache, 16) || !aligned(src_dst_pairs, 8))
+        return PA_ERR_INVALID_ARG;
+    const long long elems = (long long)num_kv_heads * block_size * head_dim;
+    if (elems % 8 != 0) return PA_ERR_INVALID_ARG;
+    // Every pointer must be reachable by the kernel at that address: device memory,
+    // managed memory, or pinned host memory mapped into the unified address space.
+    // Anything else (pageable host memory) is refused here, before any launch.
+    for (const void *ptr : {static_cast<const void *>(dst_k_cache),
+                            static_cast<const void *>(dst_v_cache), src_k_cache, src_v_cache,
+                            static_cast<const void *>(src_dst_pairs)}) {
+        cudaPointerAttributes a;
+        if (cudaPointerGetAttributes(&a, ptr) != cudaSuccess) {
+            cudaGetLastError();
+            return PA_ERR_INVALID_ARG;
+        }
+        const bool ok = a.type == cudaMemoryTypeDevice || a.type == cudaMemoryTypeManaged ||
+                        (a.type == cudaMemoryTypeHost && a.devicePointer == ptr);
+        if (!ok) return PA_ERR_INVALID_ARG;
+    }
+    SwapBlocksParams p;
+    p.dst_k = static_cast<uint8_t *>(dst_k_cache);
+    p.dst_v = static_cast<uint8_t *>(dst_v_cache);
+    p.src_k = static_cast<const uint8_t *>(src_k_cache);
+    p.src_v = static_cast<const uint8_t *>(src_v_cache);
+    p.pairs = src_dst_pairs;
+    p.block_chunks = elems / 8;
+    p.src_blocks = src_num_blocks;
+    p.dst_blocks = dst_num_blocks;
+    const long long per_cta = (long long)kCopyThreads * kCopyUnroll;
+    const long long chunks = (p.block_chunks + per_cta - 1) / per_cta;
+    if (chunks > 65535) return PA_ERR_UNSUPPORTED;
+    dim3 grid((unsigned)num_pairs, (unsigned)chunks, 2);
+    return launch_pdl(pa_swap_blocks_kernel, grid, dim3(kCopyThreads), 0,
+                      static_cast<cudaStream_t>(stream), p) == cudaSuccess
+               ? PA_OK
+               : PA_ERR_CUDA;
+}
+
 size_t pa_decode_workspace_bytes(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
                                  int block_size, int max_blocks_per_seq, int max_context_len,
                                  int partition_size) {

@@ -13,11 +13,14 @@ class NoBlocks(Exception):
 
 
 class Model:
-    def __init__(self, num_blocks, block_size):
+    def __init__(self, num_blocks, block_size, num_cpu_blocks=0):
         self.bs = block_size
         self.ref = [0] * num_blocks
         self.free_ids = list(range(num_blocks))[::-1]
         self.seqs = {}  # id -> (blocks list, length)
+        self.cpu_ref = [0] * num_cpu_blocks
+        self.cpu_free = list(range(num_cpu_blocks))[::-1]
+        self.on_cpu = set()
 
     def _take(self):
         b = self.free_ids.pop()
@@ -47,8 +50,49 @@ class Model:
 
     def free(self, sid):
         blocks, _ = self.seqs.pop(sid)
+        if sid in self.on_cpu:
+            self.on_cpu.discard(sid)
+            for b in reversed(blocks):
+                self.cpu_ref[b] -= 1
+                if self.cpu_ref[b] == 0:
+                    self.cpu_free.append(b)
+            return
         for b in reversed(blocks):
             self._drop(b)
+
+    def move(self, ids, out):
+        """Swap a group out (to the host pool) or in; returns the (from, to) pairs."""
+        src_ref, dst_ref = (self.ref, self.cpu_ref) if out else (self.cpu_ref, self.ref)
+        src_free, dst_free = (self.free_ids, self.cpu_free) if out else (self.cpu_free,
+                                                                          self.free_ids)
+        if len(set(ids)) != len(ids) or any((s in self.on_cpu) == out for s in ids):
+            raise KeyError(ids)
+        uses, order = {}, []
+        for s in ids:
+            for b in self.seqs[s][0]:
+                if b not in uses:
+                    order.append(b)
+                uses[b] = uses.get(b, 0) + 1
+        if any(uses[b] != src_ref[b] for b in order):
+            raise KeyError("shared outside the group")
+        if len(order) > len(dst_free):
+            raise NoBlocks()
+        moved, pairs = {}, []
+        for b in order:
+            nb = dst_free.pop()
+            dst_ref[nb] = src_ref[b]
+            src_ref[b] = 0
+            src_free.append(b)
+            moved[b] = nb
+            pairs.append((b, nb))
+        for s in ids:
+            blocks, n = self.seqs[s]
+            self.seqs[s] = ([moved[b] for b in blocks], n)
+            if out:
+                self.on_cpu.add(s)
+            else:
+                self.on_cpu.discard(s)
+        return pairs
 
     def append(self, ids):
         # count first: all or nothing

@@ -13,12 +13,18 @@ from tests.pins import read_golden
 
 def _invariants(bm, model):
     assert bm.num_free_blocks == len(model.free_ids)
+    assert bm.num_free_cpu_blocks == len(model.cpu_free)
     refs = [0] * len(model.ref)
-    for blocks, n in model.seqs.values():
+    cpu_refs = [0] * len(model.cpu_ref)
+    for sid, (blocks, n) in model.seqs.items():
         assert len(blocks) == -(-n // model.bs)
+        assert bm.is_swapped(sid) == (sid in model.on_cpu)
         for b in blocks:
-            refs[b] += 1
-    assert refs == model.ref
+            if sid in model.on_cpu:
+                cpu_refs[b] += 1
+            else:
+                refs[b] += 1
+    assert refs == model.ref and cpu_refs == model.cpu_ref
     for b, r in enumerate(model.ref):
         assert bm.refcount(b) == r
     assert abs(bm.usage_ratio - (1 - len(model.free_ids) / len(model.ref))) < 1e-12
@@ -42,15 +48,46 @@ def test_pages_worked_examples():
     assert bm.num_free_blocks == 7
 
 
+def _sharing_group(model, sid):
+    """sid and every sequence that shares a block with it (transitively), same pool."""
+    cpu = sid in model.on_cpu
+    group, todo = {sid}, [sid]
+    while todo:
+        blocks = set(model.seqs[todo.pop()][0])
+        for other, (ob, _) in model.seqs.items():
+            if other not in group and (other in model.on_cpu) == cpu and blocks & set(ob):
+                group.add(other)
+                todo.append(other)
+    return sorted(group)
+
+
 @pytest.mark.parametrize("seed", range(6))
 def test_random_operations_match_model(seed):
     rng = np.random.default_rng(seed)
     nb, bs = int(rng.integers(8, 64)), int(rng.choice([1, 2, 4, 16]))
-    bm, model = pa.BlockManager(nb, bs), Model(nb, bs)
+    ncpu = int(rng.integers(4, 40))
+    bm, model = pa.BlockManager(nb, bs), Model(nb, bs, ncpu)
+    bm.set_cpu_pool(ncpu)
     next_id = 0
     for step in range(300):
-        op = rng.choice(["alloc", "fork", "free", "append"], p=[0.25, 0.2, 0.15, 0.4])
-        live = list(model.seqs)
+        op = rng.choice(["alloc", "fork", "free", "append", "swap_out", "swap_in"],
+                        p=[0.22, 0.18, 0.13, 0.35, 0.06, 0.06])
+        on_gpu = [s for s in model.seqs if s not in model.on_cpu]
+        on_cpu = [s for s in model.seqs if s in model.on_cpu]
+        if op in ("swap_out", "swap_in"):
+            pool = on_gpu if op == "swap_out" else on_cpu
+            if pool:
+                group = _sharing_group(model, int(rng.choice(pool)))
+                try:
+                    want = model.move(group, op == "swap_out")
+                    got = (bm.swap_out if op == "swap_out" else bm.swap_in)(group)
+                    assert [tuple(x) for x in got.tolist()] == want
+                except NoBlocks:
+                    with pytest.raises(pa.PAError):
+                        (bm.swap_out if op == "swap_out" else bm.swap_in)(group)
+            _invariants(bm, model)
+            continue
+        live = on_gpu if op in ("fork", "append") else list(model.seqs)
         if op == "alloc":
             n = int(rng.integers(0, 3 * bs + 2))
             try:
@@ -82,6 +119,10 @@ def test_random_operations_match_model(seed):
         _invariants(bm, model)
         for sid, (blocks, n) in model.seqs.items():
             assert bm.seq_len(sid) == n
+            if sid in model.on_cpu:
+                with pytest.raises(pa.PAError):
+                    bm.block_tables([sid], max(len(blocks), 1))
+                continue
             bt, cl = bm.block_tables([sid], max(len(blocks), 1))
             assert bt[0, : len(blocks)].tolist() == blocks and cl[0] == n
 
@@ -133,8 +174,13 @@ def test_logical_token_streams_through_tables():
     rng = np.random.default_rng(3)
     nb, hkv, bs, d = 96, 2, 4, 8
     bm = pa.BlockManager(nb, bs)
+    bm.set_cpu_pool(40)
+    model = None
     kc = np.zeros((nb, hkv, bs, d), np.uint16)
     vc = np.zeros_like(kc)
+    kh = np.zeros((40, hkv, bs, d), np.uint16)  # host pool
+    vh = np.zeros_like(kh)
+    swapped = set()
     logical = {}
     next_id, counter = 0, 1
 
@@ -143,10 +189,41 @@ def test_logical_token_streams_through_tables():
         counter += 1
         return np.full((1, hkv, d), counter % 60000, np.uint16)
 
-    for step in range(120):
-        live = list(logical)
+    for step in range(160):
+        live = [s for s in logical if s not in swapped]
         r = rng.random()
-        if r < 0.15 or not live:
+        if r > 0.9 and (live or swapped):
+            # swap a whole sharing group out, or a swapped group back in
+            out = (not swapped) or (live and rng.random() < 0.5)
+            pool = live if out else sorted(swapped)
+            seed_id = int(rng.choice(pool))
+            group = {seed_id}
+            tabs = {}
+            for sid in pool:
+                L = len(logical[sid])
+                if out:
+                    tabs[sid] = set(bm.block_tables([sid], max(-(-L // bs), 1))[0][0].tolist()) - {-1}
+            if out:
+                changed = True
+                while changed:
+                    changed = False
+                    for sid in pool:
+                        if sid not in group and any(tabs[sid] & tabs[g] for g in group):
+                            group.add(sid)
+                            changed = True
+            else:
+                group = set(swapped)  # bring back everything that is out
+            try:
+                pairs = (bm.swap_out if out else bm.swap_in)(sorted(group))
+            except pa.PAError:
+                continue
+            for a, b in pairs:
+                if out:
+                    kh[b], vh[b] = kc[a], vc[a]
+                else:
+                    kc[b], vc[b] = kh[a], vh[a]
+            swapped = (swapped | group) if out else (swapped - group)
+        elif r < 0.15 or not live:
             n = int(rng.integers(1, 11))
             if bm.can_allocate(n):
                 bm.allocate(next_id, n)
@@ -161,9 +238,10 @@ def test_logical_token_streams_through_tables():
             logical[next_id] = list(logical[p])
             next_id += 1
         elif r < 0.4:
-            s = int(rng.choice(live))
+            s = int(rng.choice(list(logical)))
             bm.free(s)
             del logical[s]
+            swapped.discard(s)
         else:
             ids = [int(x) for x in rng.permutation(live)]
             try:
@@ -176,6 +254,8 @@ def test_logical_token_streams_through_tables():
             for s, t in zip(ids, toks):
                 logical[s].append(t)
         for s, toks in logical.items():
+            if s in swapped:
+                continue
             L = len(toks)
             bt, cl = bm.block_tables([s], max(-(-L // bs), 1))
             assert cl[0] == L

@@ -17,17 +17,51 @@ pytestmark = [pytest.mark.gpu,
               pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")]
 
 
-@pytest.mark.parametrize("hq,hkv,bs,fused", [(16, 4, 16, False), (8, 8, 32, True),
-                                             (32, 4, 16, True)])
-def test_block_manager_serving_loop(hq, hkv, bs, fused):
+def test_swap_blocks_device_and_pinned_host():
+    rng = np.random.default_rng(60)
+    nb, ncpu, hkv, bs, d = 50, 30, 8, 16, 128
+    kd0 = _rand_bits(rng, (nb, hkv, bs, d))
+    vd0 = _rand_bits(rng, (nb, hkv, bs, d))
+    kd, vd = dev16(kd0, "bf16"), dev16(vd0, "bf16")
+    kh = torch.zeros(ncpu, hkv, bs, d, dtype=torch.bfloat16, pin_memory=True)
+    vh = torch.zeros_like(kh).pin_memory()
+    gpu = rng.permutation(nb)[:12]
+    cpu = rng.permutation(ncpu)[:12]
+    pa.swap_blocks(kh, vh, kd, vd, dev(np.stack([gpu, cpu], 1).astype(np.int64)))  # out
+    torch.cuda.synchronize()
+    assert np.array_equal(bits(kh)[cpu], kd0[gpu]) and np.array_equal(bits(vh)[cpu], vd0[gpu])
+    kd.zero_()
+    vd.zero_()
+    back = rng.permutation(nb)[:12]
+    pa.swap_blocks(kd, vd, kh, vh, dev(np.stack([cpu, back], 1).astype(np.int64)))  # in
+    torch.cuda.synchronize()
+    assert np.array_equal(bits(kd)[back], kd0[gpu]) and np.array_equal(bits(vd)[back], vd0[gpu])
+    assert pa.device_error(0) == 0
+    pageable = torch.zeros(ncpu, hkv, bs, d, dtype=torch.bfloat16)  # not mapped: refused
+    with pytest.raises(pa.PAError):
+        pa.swap_blocks(pageable, pageable, kd, vd, dev(np.array([[0, 0]], np.int64)))
+    pa.swap_blocks(kh, vh, kd, vd, dev(np.array([[0, ncpu]], np.int64)))  # bad host id
+    assert pa.device_error(0) == pa.DEVERR["pair"]
+
+
+@pytest.mark.parametrize("hq,hkv,bs,fused,preempt", [(16, 4, 16, False, False),
+                                                     (8, 8, 32, True, False),
+                                                     (32, 4, 16, True, False),
+                                                     (16, 2, 16, True, True)])
+def test_block_manager_serving_loop(hq, hkv, bs, fused, preempt):
     rng = np.random.default_rng(hq * 100 + bs)
-    nb, d, width = 700, 128, 64
+    nb, d, width, ncpu = 700, 128, 64, 300
     scale = 1 / math.sqrt(d)
     bm = pa.BlockManager(nb, bs)
+    bm.set_cpu_pool(ncpu)
     kc_h = np.full((nb, hkv, bs, d), 0x7FC0, np.uint16)  # NaN where nothing was written
     vc_h = kc_h.copy()
     kc, vc = dev16(kc_h, "bf16"), dev16(vc_h, "bf16")
-    live, next_id = [], 0
+    kh_h = np.zeros((ncpu, hkv, bs, d), np.uint16)  # host pool mirror and the pinned pool
+    vh_h = kh_h.copy()
+    kh = torch.zeros(ncpu, hkv, bs, d, dtype=torch.bfloat16, pin_memory=True)
+    vh = torch.zeros_like(kh).pin_memory()
+    live, next_id, parked = [], 0, []
 
     def write(ids_tokens_slots):
         key = np.concatenate([k for k, _, _ in ids_tokens_slots])
@@ -55,6 +89,22 @@ def test_block_manager_serving_loop(hq, hkv, bs, fused):
             next_id += 1
 
     for step in range(10):
+        if preempt and step == 2:  # preempt the first prompt and its samples
+            group = [s for s in live if bm.block_tables([s], width)[0][0, 0]
+                     == bm.block_tables([live[0]], width)[0][0, 0]]
+            pairs = bm.swap_out(group)
+            for g_blk, c_blk in pairs:
+                kh_h[c_blk], vh_h[c_blk] = kc_h[g_blk], vc_h[g_blk]
+            pa.swap_blocks(kh, vh, kc, vc, dev(pairs))
+            live = [s for s in live if s not in group]
+            parked = group
+        if preempt and step == 6:  # and bring it back into (other) GPU blocks
+            pairs = bm.swap_in(parked)
+            for c_blk, g_blk in pairs:
+                kc_h[g_blk], vc_h[g_blk] = kh_h[c_blk], vh_h[c_blk]
+            pa.swap_blocks(kc, vc, kh, vh, dev(pairs))
+            live += parked
+            parked = []
         if step % 4 == 3:  # one request ends, one arrives
             bm.free(live.pop(int(rng.integers(0, len(live)))))
             new_prompt()
