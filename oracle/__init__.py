@@ -52,6 +52,9 @@ def _declare(lib):
     lib.orc_decode.argtypes = [P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, i32, dbl, i32, P,
                                i32, i32]
     lib.orc_decode.restype = i32
+    lib.orc_decode_window.argtypes = [P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, i32, dbl,
+                                      i32, i32, P, i32, i32]
+    lib.orc_decode_window.restype = i32
     lib.orc_max_threads.argtypes = []
     lib.orc_max_threads.restype = i32
 
@@ -81,8 +84,9 @@ def copy_blocks(k_cache, v_cache, pairs, lib=None) -> int:
 
 
 def decode(q, k_cache, v_cache, block_tables, context_lens, scale, dtype, num_q_heads=None,
-           sel=None, nthreads=0, lib=None, return_bad=False):
-    """fp64 attention output, [B, Hq, d] (or [len(sel), d] for selected (s, h) pairs)."""
+           sel=None, nthreads=0, lib=None, return_bad=False, sliding_window=0):
+    """fp64 attention output, [B, Hq, d] (or [len(sel), d] for selected (s, h) pairs).
+    ``sliding_window`` > 0: each query attends to the last that many tokens only."""
     lib = lib or load()
     q = np.ascontiguousarray(q, np.uint16)
     kc = np.ascontiguousarray(k_cache, np.uint16)
@@ -94,13 +98,14 @@ def decode(q, k_cache, v_cache, block_tables, context_lens, scale, dtype, num_q_
     if sel is not None:
         sel = np.ascontiguousarray(sel, np.int32).reshape(-1, 2)
         out = np.zeros((sel.shape[0], d), np.float64)
-        bad = lib.orc_decode(_p(out), _p(q), _p(kc), _p(vc), _p(bt), _p(cl), B, hq, hkv, d, bs,
-                             nb, bt.shape[1], float(scale), _dt(dtype), _p(sel), sel.shape[0],
-                             nthreads)
+        bad = lib.orc_decode_window(_p(out), _p(q), _p(kc), _p(vc), _p(bt), _p(cl), B, hq, hkv,
+                                    d, bs, nb, bt.shape[1], float(scale), _dt(dtype),
+                                    int(sliding_window), _p(sel), sel.shape[0], nthreads)
     else:
         out = np.zeros((B, hq, d), np.float64)
-        bad = lib.orc_decode(_p(out), _p(q), _p(kc), _p(vc), _p(bt), _p(cl), B, hq, hkv, d, bs,
-                             nb, bt.shape[1], float(scale), _dt(dtype), None, 0, nthreads)
+        bad = lib.orc_decode_window(_p(out), _p(q), _p(kc), _p(vc), _p(bt), _p(cl), B, hq, hkv,
+                                    d, bs, nb, bt.shape[1], float(scale), _dt(dtype),
+                                    int(sliding_window), None, 0, nthreads)
     return (out, bad) if return_bad else out
 
 

@@ -31,7 +31,18 @@ def gather(cache_f64: np.ndarray, table_row: np.ndarray, L: int, kv_head: int) -
     return pages.reshape(npages * bs, -1)[:L]
 
 
-def decode(q, k_cache, v_cache, block_tables, context_lens, scale, dtype) -> np.ndarray:
+def gather_positions(cache_f64: np.ndarray, table_row: np.ndarray, lo: int, L: int,
+                     kv_head: int) -> np.ndarray:
+    """[L - lo, d] rows of token positions lo .. L-1: page table_row[t // bs], row t % bs."""
+    bs = cache_f64.shape[2]
+    t = np.arange(lo, L)
+    pages = np.asarray(table_row, dtype=np.int64)[t // bs]
+    return cache_f64[pages, kv_head, t % bs]
+
+
+def decode(q, k_cache, v_cache, block_tables, context_lens, scale, dtype,
+           sliding_window: int = 0) -> np.ndarray:
+    """sliding_window > 0: each query attends to its last ``sliding_window`` tokens."""
     qf = widen(q, dtype)
     kf = widen(k_cache, dtype)
     vf = widen(v_cache, dtype)
@@ -43,9 +54,14 @@ def decode(q, k_cache, v_cache, block_tables, context_lens, scale, dtype) -> np.
         L = int(context_lens[s])
         if L == 0:
             continue
+        lo = L - sliding_window if 0 < sliding_window < L else 0
         for g in range(hkv):
-            K = gather(kf, block_tables[s], L, g)
-            V = gather(vf, block_tables[s], L, g)
+            if lo == 0:
+                K = gather(kf, block_tables[s], L, g)
+                V = gather(vf, block_tables[s], L, g)
+            else:
+                K = gather_positions(kf, block_tables[s], lo, L, g)
+                V = gather_positions(vf, block_tables[s], lo, L, g)
             Q = qf[s, g * G:(g + 1) * G]  # [G, d]
             z = scale * (Q @ K.T)  # [G, L]
             z = z - z.max(axis=1, keepdims=True)

@@ -23,7 +23,12 @@
  *  - cache layout [num_blocks][num_kv_heads][block_size][head_dim];
  *  - slot = block * block_size + offset, negative slot = no write;
  *  - q head h reads kv head h / (num_q_heads / num_kv_heads);
- *  - context length 0 gives an all-zero output.
+ *  - context length 0 gives an all-zero output;
+ *  - sliding window W > 0 (the block manager's sliding_window setting in the
+ *    dynamic-memory blog, BlockSpaceManager example): the query attends to the last
+ *    W tokens of its context, positions max(0, L - W) .. L - 1, and table entries
+ *    of pages wholly before that range are never read (their blocks may have been
+ *    returned to the pool).
  *
  * Values arrive as 16-bit patterns (bf16 or fp16) and are widened exactly to double.
  */
@@ -108,23 +113,27 @@ int orc_copy_blocks(uint16_t *k_cache, uint16_t *v_cache, const int64_t *pairs, 
 
 /* Attention for one (sequence, q head), written as the definition:
  *   K_s = concat of the sequence's pages in table order (first L rows),
- *   z_t = scale * <q, K_s[t]>,  out = sum_t softmax(z)_t V_s[t].
- * Returns 0, or -1 if a table entry needed for t < L is outside [0, num_blocks). */
+ *   z_t = scale * <q, K_s[t]>,  out = sum_t softmax(z)_t V_s[t],
+ * with t over [t_lo, L): t_lo = 0, or L - window under a sliding window shorter
+ * than the context.
+ * Returns 0, or -1 if a table entry needed for a token in range is outside
+ * [0, num_blocks). */
 static int orc_one(double *out, const uint16_t *q, const uint16_t *k_cache,
                    const uint16_t *v_cache, const int32_t *table, int L, int h, int num_q_heads,
                    int num_kv_heads, int head_dim, int block_size, int num_blocks, double scale,
-                   int dtype) {
+                   int dtype, int window) {
     int d = head_dim;
     int g = h / (num_q_heads / num_kv_heads);
     for (int i = 0; i < d; ++i) out[i] = 0.0;
     if (L <= 0) return 0;
+    int t_lo = (window > 0 && L > window) ? L - window : 0;
     double *Kc = (double *)malloc(sizeof(double) * (size_t)L * d);
     double *Vc = (double *)malloc(sizeof(double) * (size_t)L * d);
     double *z = (double *)malloc(sizeof(double) * (size_t)L);
     double *qd = (double *)malloc(sizeof(double) * (size_t)d);
     int rc = 0;
     /* gather: logical token t lives in page table[t / bs] at row t % bs */
-    for (int t = 0; t < L && rc == 0; ++t) {
+    for (int t = t_lo; t < L && rc == 0; ++t) {
         int blk = table[t / block_size];
         if (blk < 0 || blk >= num_blocks) { rc = -1; break; }
         size_t row = (((size_t)blk * num_kv_heads + g) * block_size + (t % block_size)) * d;
@@ -136,18 +145,18 @@ static int orc_one(double *out, const uint16_t *q, const uint16_t *k_cache,
     if (rc == 0) {
         for (int i = 0; i < d; ++i) qd[i] = orc_widen(q[i], dtype);
         double m = -INFINITY;
-        for (int t = 0; t < L; ++t) {
+        for (int t = t_lo; t < L; ++t) {
             double acc = 0.0;
             for (int i = 0; i < d; ++i) acc += qd[i] * Kc[(size_t)t * d + i];
             z[t] = scale * acc;
             if (z[t] > m) m = z[t];
         }
         double denom = 0.0;
-        for (int t = 0; t < L; ++t) {
+        for (int t = t_lo; t < L; ++t) {
             z[t] = exp(z[t] - m); /* softmax numerator, max-shifted */
             denom += z[t];
         }
-        for (int t = 0; t < L; ++t)
+        for (int t = t_lo; t < L; ++t)
             for (int i = 0; i < d; ++i) out[i] += z[t] * Vc[(size_t)t * d + i];
         for (int i = 0; i < d; ++i) out[i] /= denom;
     }
@@ -160,13 +169,15 @@ static int orc_one(double *out, const uint16_t *q, const uint16_t *k_cache,
 
 /* Decode attention for every (sequence, q head), or only for the n_sel pairs listed
  * in sel[2*i] = sequence, sel[2*i+1] = q head (out is then [n_sel][head_dim]).
- * out (fp64) is [num_seqs][num_q_heads][head_dim] when sel is NULL.
+ * out (fp64) is [num_seqs][num_q_heads][head_dim] when sel is NULL.  window > 0
+ * restricts every query to the last `window` tokens of its context (0 = whole context).
  * Returns the number of (s, h) whose table referenced an out-of-range block. */
-int orc_decode(double *out, const uint16_t *q, const uint16_t *k_cache, const uint16_t *v_cache,
-               const int32_t *block_tables, const int32_t *context_lens, int num_seqs,
-               int num_q_heads, int num_kv_heads, int head_dim, int block_size, int num_blocks,
-               int max_blocks_per_seq, double scale, int dtype, const int32_t *sel, int n_sel,
-               int nthreads) {
+int orc_decode_window(double *out, const uint16_t *q, const uint16_t *k_cache,
+                      const uint16_t *v_cache, const int32_t *block_tables,
+                      const int32_t *context_lens, int num_seqs, int num_q_heads,
+                      int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                      int max_blocks_per_seq, double scale, int dtype, int window,
+                      const int32_t *sel, int n_sel, int nthreads) {
     int n = sel ? n_sel : num_seqs * num_q_heads;
     int bad = 0;
 #ifdef _OPENMP
@@ -181,11 +192,22 @@ int orc_decode(double *out, const uint16_t *q, const uint16_t *k_cache, const ui
         if (L > max_blocks_per_seq * block_size) { ++bad; continue; }
         const uint16_t *qs = q + ((size_t)s * num_q_heads + h) * head_dim;
         if (orc_one(out + (size_t)i * head_dim, qs, k_cache, v_cache, table, L, h, num_q_heads,
-                    num_kv_heads, head_dim, block_size, num_blocks, scale, dtype) != 0)
+                    num_kv_heads, head_dim, block_size, num_blocks, scale, dtype, window) != 0)
             ++bad;
     }
     (void)nthreads;
     return bad;
+}
+
+/* The whole context (no sliding window). */
+int orc_decode(double *out, const uint16_t *q, const uint16_t *k_cache, const uint16_t *v_cache,
+               const int32_t *block_tables, const int32_t *context_lens, int num_seqs,
+               int num_q_heads, int num_kv_heads, int head_dim, int block_size, int num_blocks,
+               int max_blocks_per_seq, double scale, int dtype, const int32_t *sel, int n_sel,
+               int nthreads) {
+    return orc_decode_window(out, q, k_cache, v_cache, block_tables, context_lens, num_seqs,
+                             num_q_heads, num_kv_heads, head_dim, block_size, num_blocks,
+                             max_blocks_per_seq, scale, dtype, 0, sel, n_sel, nthreads);
 }
 
 /* Threads the OpenMP runtime would use (1 without OpenMP). */

@@ -11,7 +11,9 @@ Each ``pin_*`` takes a loaded oracle library (ctypes handle) and raises
   size, any physical permutation, shared prefix blocks);
 * the worked examples the pages print (``tests/golden/pages_examples.txt``);
 * exact library conversions of the 16-bit formats (numpy float16, torch bfloat16);
-* the independent numpy statement in ``oracle/oracle_np.py``.
+* the independent numpy statement in ``oracle/oracle_np.py``;
+* for the sliding window: the last token's V exactly at W = 1, and torch fp64
+  attention on the last W contiguous rows.
 
 The same functions run against deliberately broken copies of the oracle in
 ``test_oracle_mutants.py``, which checks that each plausible mistake trips a pin.
@@ -378,9 +380,88 @@ def pin_copy_blocks(lib):
         assert np.array_equal(kc_c[b], kc[b]) and np.array_equal(vc_c[b], vc[b])
 
 
+# ------------------------------------------------------------------ sliding window
+
+def _recycle_before(tables, lens, bs, window):
+    """Table entries of pages wholly before each sequence's window -> -1 (returned to the
+    pool): page j is unused once (j + 1) * bs <= L - window."""
+    out = []
+    for t, L in zip(tables, lens):
+        t = t.copy()
+        lo = L - window if 0 < window < L else 0
+        t[:lo // bs] = -1
+        out.append(t)
+    return out
+
+
+def pin_window_last_token(lib):
+    """A window of one token returns the last token's V exactly, whatever the length and
+    whatever the (recycled, -1) table entries before it hold."""
+    rng = np.random.default_rng(21)
+    for dtype in ("bf16", "fp16"):
+        hq, hkv, d, bs = 4, 2, 16, 8
+        lens = [1, 7, 8, 9, 16, 17, 37]
+        B = len(lens)
+        nb = sum(-(-L // bs) for L in lens) + 2
+        Ks = [_rand_bits(rng, (L, hkv, d), dtype) for L in lens]
+        Vs = [_rand_bits(rng, (L, hkv, d), dtype) for L in lens]
+        tabs = _tables_for(rng, lens, bs, nb)
+        kc, vc, _ = build_pool(Ks, Vs, tabs, nb, bs)
+        _, _, bt = build_pool(Ks, Vs, _recycle_before(tabs, lens, bs, 1), nb, bs)
+        q = _rand_bits(rng, (B, hq, d), dtype)
+        out, bad = oracle.decode(q, kc, vc, bt, np.array(lens, np.int32), 0.25, dtype, lib=lib,
+                                 return_bad=True, sliding_window=1)
+        assert bad == 0
+        G = hq // hkv
+        for s, L in enumerate(lens):
+            for h in range(hq):
+                want = bits_to_f32(Vs[s][L - 1, h // G], dtype).astype(np.float64)
+                assert np.array_equal(out[s, h], want), (dtype, s, h)
+
+
+def pin_window_vs_sdpa(lib):
+    """Windowed paged result == torch fp64 scaled-dot-product attention on the last W
+    rows of the contiguous K/V, with the pages before the window recycled (-1); a
+    window at least as long as the context is the plain result."""
+    import torch
+    import torch.nn.functional as F
+    rng = np.random.default_rng(22)
+    hq, hkv, d, bs = 4, 2, 16, 4
+    lens = [1, 5, 12, 13, 30, 41]
+    B = len(lens)
+    nb = sum(-(-L // bs) for L in lens) + 3
+    Ks = [_rand_bits(rng, (L, hkv, d)) for L in lens]
+    Vs = [_rand_bits(rng, (L, hkv, d)) for L in lens]
+    tabs = _tables_for(rng, lens, bs, nb)
+    kc, vc, bt_full = build_pool(Ks, Vs, tabs, nb, bs)
+    q = _rand_bits(rng, (B, hq, d))
+    cl = np.array(lens, np.int32)
+    G = hq // hkv
+    plain = oracle.decode(q, kc, vc, bt_full, cl, 0.3, "bf16", lib=lib)
+    for W in (2, 3, 4, 9, 12, 40, 41, 100):
+        _, _, bt = build_pool(Ks, Vs, _recycle_before(tabs, lens, bs, W), nb, bs)
+        out, bad = oracle.decode(q, kc, vc, bt, cl, 0.3, "bf16", lib=lib, return_bad=True,
+                                 sliding_window=W)
+        assert bad == 0, W
+        for s, L in enumerate(lens):
+            lo = max(0, L - W)
+            qt = torch.from_numpy(bits_to_f32(q[s], "bf16").astype(np.float64))[None, :, None, :]
+            kt = torch.from_numpy(bits_to_f32(Ks[s][lo:], "bf16").astype(np.float64))
+            vt = torch.from_numpy(bits_to_f32(Vs[s][lo:], "bf16").astype(np.float64))
+            kt = kt.permute(1, 0, 2).repeat_interleave(G, dim=0)[None]
+            vt = vt.permute(1, 0, 2).repeat_interleave(G, dim=0)[None]
+            ref = F.scaled_dot_product_attention(qt, kt, vt, scale=0.3)[0, :, 0, :].numpy()
+            assert np.max(np.abs(out[s] - ref)) < 1e-12, (W, s)
+            if W >= L:
+                assert np.array_equal(out[s], plain[s]), (W, s)
+        npv = oracle_np.decode(q, kc, vc, bt, cl, 0.3, "bf16", sliding_window=W)
+        assert np.max(np.abs(out - npv)) < 1e-12, W
+
+
 ALL_PINS = [pin_two_token, pin_len1_exact, pin_identical_keys, pin_zero_len, pin_paged_vs_sdpa,
             pin_block_size_and_permutation, pin_shared_prefix, pin_golden_examples,
-            pin_widening, pin_c_vs_numpy, pin_kv_write, pin_copy_blocks]
+            pin_widening, pin_c_vs_numpy, pin_kv_write, pin_copy_blocks, pin_window_last_token,
+            pin_window_vs_sdpa]
 
 
 def run_all(lib):

@@ -28,6 +28,11 @@ MUTANTS = [
     ("copy_reversed", "int64_t src = pairs[2 * p], dst = pairs[2 * p + 1];",
      "int64_t dst = pairs[2 * p], src = pairs[2 * p + 1];"),
     ("softmax_no_exp", "z[t] = exp(z[t] - m);", "z[t] = (z[t] - m) + 1000.0;"),
+    ("window_one_short", "int t_lo = (window > 0 && L > window) ? L - window : 0;",
+     "int t_lo = (window > 0 && L > window) ? L - window + 1 : 0;"),
+    ("window_one_long", "int t_lo = (window > 0 && L > window) ? L - window : 0;",
+     "int t_lo = (window > 0 && L > window) ? L - window - 1 : 0;"),
+    ("window_ignored", "int t_lo = (window > 0 && L > window) ? L - window : 0;", "int t_lo = 0;"),
 ]
 
 
