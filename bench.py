@@ -53,19 +53,25 @@ WORKLOADS = {
                         "32/8 heads, head_dim 128, bs 512, lens U[32768,131072]"),
     "prefix_cow": ("prefix_cow", {}, "prefix sharing + copy-on-write: 64 groups x 8 samples, "
                    "1000-token shared prefix, 32/8 heads, bs 16"),
+    "window_4096_gqa": ("window_4096_gqa", {}, "sliding-window decode (W = 4096): 64 seqs, 32/8 "
+                        "heads, head_dim 128, bs 16, lens U[8192,32768], only the pages of each "
+                        "window held (earlier table entries -1)"),
 }
 
 
 # ----------------------------------------------------------------------------- bytes
 
 def decode_bytes(case) -> int:
-    """Algorithmic bytes of one pa_decode: K and V of every (sequence, kv head, token)
-    once, q and out once, the block-table entries read, context lengths."""
+    """Algorithmic bytes of one pa_decode: K and V of every attended (sequence, kv head,
+    token) once -- all L tokens, or the last W under a sliding window -- q and out once,
+    the block-table entries of the attended pages, context lengths."""
     eb = 2
     L = case.context_lens.astype(np.int64)
-    kv = int(L.sum()) * 2 * case.num_kv_heads * case.head_dim * eb
+    lo = np.maximum(L - case.window, 0) if case.window > 0 else np.zeros_like(L)
+    kv = int((L - lo).sum()) * 2 * case.num_kv_heads * case.head_dim * eb
     qo = 2 * case.num_seqs * case.num_q_heads * case.head_dim * eb
-    tables = int(((L + case.block_size - 1) // case.block_size).sum()) * 4 * case.num_kv_heads
+    pages = (L + case.block_size - 1) // case.block_size - lo // case.block_size
+    tables = int(pages.sum()) * 4 * case.num_kv_heads
     return kv + qo + tables + 4 * case.num_seqs
 
 
@@ -208,7 +214,8 @@ def oracle_step_time(case, sel=None, nthreads=0):
     import oracle
     t = time.perf_counter()
     oracle.decode(case.q, case._kc_written, case._vc_written, case.block_tables,
-                  case.context_lens, case.scale, case.dtype, sel=sel, nthreads=nthreads)
+                  case.context_lens, case.scale, case.dtype, sel=sel, nthreads=nthreads,
+                  sliding_window=case.window)
     dt = time.perf_counter() - t
     return dt
 
@@ -228,7 +235,8 @@ def sel_bytes(case, sel) -> int:
     # the oracle reads K and V once per (s, q head); count the distinct kv rows like the
     # GPU metric does: per (s, kv head) covered by the sample
     kvh = {(int(s), int(h) // G) for s, h in sel}
-    kv = sum(int(L[s]) for s, _ in kvh) * 2 * case.head_dim * 2
+    span = np.minimum(L, case.window) if case.window > 0 else L
+    kv = sum(int(span[s]) for s, _ in kvh) * 2 * case.head_dim * 2
     return kv + 2 * len(sel) * case.head_dim * 2
 
 
@@ -291,14 +299,17 @@ def run_ours(args):
     out = torch.empty_like(q)
     W = case.max_blocks_per_seq
     mcl = case.max_context_len
+    win = case.window
     need = pa.decode_workspace_bytes(case.num_seqs, case.num_q_heads, case.num_kv_heads,
-                                     case.head_dim, case.block_size, W, mcl, args.partition_size)
+                                     case.head_dim, case.block_size, W, mcl, args.partition_size,
+                                     win)
     workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=device)
     ptoks = pa.decode_partition_tokens(case.num_seqs, case.num_q_heads, case.num_kv_heads,
                                        case.head_dim, case.block_size, W, mcl,
-                                       args.partition_size)
+                                       args.partition_size, win)
     # partition_tokens 0: balanced split over persistent warps (decode + merge kernels)
-    nparts = 0 if ptoks == 0 else -(-min(mcl, W * case.block_size) // ptoks)
+    span = min(mcl, W * case.block_size, win + 15 if win > 0 else mcl)
+    nparts = 0 if ptoks == 0 else -(-span // ptoks)
     has_pairs = case.copy_pairs.shape[0] > 0
     launches_per_step = 1 + (1 if nparts == 1 else 2) + (1 if has_pairs else 0)
     stream = torch.cuda.current_stream()
@@ -311,13 +322,15 @@ def run_ours(args):
     def step():
         if fused:
             pa.decode_append(out, q, key, val, kc, vc, bt, cl, case.scale, max_context_len=mcl,
-                             partition_size=args.partition_size, workspace=workspace)
+                             partition_size=args.partition_size, workspace=workspace,
+                             sliding_window=win)
             return
         if has_pairs:
             pa.copy_blocks(kc, vc, pairs)
         pa.kv_write(key, val, sm, kc, vc)
         pa.decode(out, q, kc, vc, bt, cl, case.scale, max_context_len=mcl,
-                  partition_size=args.partition_size, workspace=workspace)
+                  partition_size=args.partition_size, workspace=workspace,
+                  sliding_window=win)
 
     for _ in range(args.warmup):
         step()
@@ -355,7 +368,7 @@ def run_ours(args):
             for _ in range(group):
                 pa.decode_append(out, q, key, val, kc, vc, bt, cl, case.scale,
                                  max_context_len=mcl, partition_size=args.partition_size,
-                                 workspace=workspace)
+                                 workspace=workspace, sliding_window=win)
             ev[i][1].record(stream)
         else:
             if has_pairs:
@@ -363,7 +376,8 @@ def run_ours(args):
             pa.kv_write(key, val, sm, kc, vc)
             ev[i][0].record(stream)
             pa.decode(out, q, kc, vc, bt, cl, case.scale, max_context_len=mcl,
-                      partition_size=args.partition_size, workspace=workspace)
+                      partition_size=args.partition_size, workspace=workspace,
+                             sliding_window=win)
             ev[i][1].record(stream)
     torch.cuda.synchronize()
     clocks = sampler.stop()
@@ -422,14 +436,15 @@ def run_ours(args):
         if fused:
             pa.decode_append(b["out"], b["q"], b["key"], b["val"], kc, vc, b["bt"], b["cl"],
                              case.scale, max_context_len=mcl,
-                             partition_size=args.partition_size, workspace=workspace)
+                             partition_size=args.partition_size, workspace=workspace,
+                             sliding_window=win)
         else:
             if has_pairs:
                 pa.copy_blocks(kc, vc, b["pairs"])
             pa.kv_write(b["key"], b["val"], b["sm"], kc, vc)
             pa.decode(b["out"], b["q"], kc, vc, b["bt"], b["cl"], case.scale,
                       max_context_len=mcl, partition_size=args.partition_size,
-                      workspace=workspace)
+                      workspace=workspace, sliding_window=win)
         ev_done[i % 2].record(stream)
 
     def d2h(i):
@@ -494,7 +509,7 @@ def run_ours(args):
                        "num_q_heads": case.num_q_heads, "num_kv_heads": case.num_kv_heads,
                        "head_dim": case.head_dim, "block_size": case.block_size,
                        "num_blocks": case.num_blocks, "kv_tokens": int(case.context_lens.sum()),
-                       "max_context_len": mcl,
+                       "max_context_len": mcl, "sliding_window": win,
                        "split": ("balanced over persistent warps (stream-K) + LSE merge"
                                  if ptoks == 0 else f"fixed {ptoks}-token partitions, {nparts} max"),
                        "parallelism": f"dp{ws} (independent replicas)",
@@ -526,6 +541,120 @@ def run_ours(args):
                          "traffic": traffic_from_profile(args.workload)},
             "clocks": clocks,
             "cpu_baseline": cpu,
+        }
+    if ws > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return result
+
+
+def run_swap(args):
+    """Preemption swap of the benchmark workload: the block manager swaps a group of
+    sequences out to a pinned host pool and back in; pa_swap_blocks moves the blocks.
+    value = bytes that cross the host link per (swap out + swap in) / device time;
+    the ceiling is a contiguous pinned cudaMemcpyAsync of the same bytes, each way,
+    timed in the same process."""
+    import torch
+    ws, rank, local = dist_env()
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    device = torch.device("cuda", torch.cuda.current_device())
+    import paged_kv_cache_441_b200 as pa
+    from workloads import make_config
+
+    name, kw, desc = WORKLOADS[args.workload]
+    case = make_config(name, poison=False, **kw)
+    tdt = torch.bfloat16 if case.dtype == "bf16" else torch.float16
+    kc = torch.from_numpy(case.k_cache.view(np.int16)).to(device).view(tdt)
+    vc = torch.from_numpy(case.v_cache.view(np.int16)).to(device).view(tdt)
+    nb, hkv, bs, d = kc.shape
+    lens = case.context_lens.astype(np.int64)
+    bm = pa.BlockManager(nb, bs)
+    for s in range(case.num_seqs):
+        bm.allocate(s, int(lens[s]))
+    group = list(range(min(args.swap_seqs, case.num_seqs)))  # the preempted sequences
+    ncpu = sum(pa.blocks_needed(int(lens[s]), bs) for s in group)
+    bm.set_cpu_pool(ncpu)
+    kh = torch.empty((ncpu, hkv, bs, d), dtype=tdt).pin_memory()
+    vh = torch.empty((ncpu, hkv, bs, d), dtype=tdt).pin_memory()
+    stream = torch.cuda.current_stream()
+
+    def swap_cycle():
+        out_pairs = torch.from_numpy(bm.swap_out(group)).to(device)
+        pa.swap_blocks(kh, vh, kc, vc, out_pairs)
+        in_pairs = torch.from_numpy(bm.swap_in(group)).to(device)
+        pa.swap_blocks(kc, vc, kh, vh, in_pairs)
+
+    # kernel-only pass: fixed pair lists, resident on the device
+    out_pairs = torch.from_numpy(bm.swap_out(group)).to(device)
+    in_pairs = torch.from_numpy(bm.swap_in(group)).to(device)
+    moved = 2 * ncpu * hkv * bs * d * kc.element_size()  # K and V, one direction
+
+    def timed(fn, reps):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize()
+        if ws > 1:
+            dist.barrier()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(reps):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        return max_over_ranks(a.elapsed_time(b), ws, device) / reps
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    ms_out = timed(lambda: pa.swap_blocks(kh, vh, kc, vc, out_pairs), args.steps)
+    ms_in = timed(lambda: pa.swap_blocks(kc, vc, kh, vh, in_pairs), args.steps)
+    clocks = sampler.stop()
+    ms_e2e = timed(swap_cycle, args.steps)
+    flat_h = torch.empty(moved // 2, dtype=torch.int16).pin_memory()
+    flat_d = torch.empty(moved // 2, dtype=torch.int16, device=device)
+    ms_d2h = timed(lambda: flat_h.copy_(flat_d, non_blocking=True), args.steps)
+    ms_h2d = timed(lambda: flat_d.copy_(flat_h, non_blocking=True), args.steps)
+    err = pa.device_error(device.index)
+    bm.close()
+    result = None
+    if rank == 0:
+        step_ms = ms_out + ms_in
+        value = 2 * moved * ws / (step_ms * 1e-3) / 1e9
+        peak = 2 * moved / ((ms_d2h + ms_h2d) * 1e-3) / 1e9
+        result = {
+            "metric": "KV block swap GB/s (device <-> pinned host, out + in)",
+            "value": round(value, 2), "unit": "GB/s", "n_gpus": ws, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(step_ms, 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": case.dtype,
+            "data": "synthetic (the benchmark workload's seeded cache)",
+            "config": {"workload": f"swap out + swap in of {len(group)} of {case.num_seqs} "
+                                   f"sequences of: {desc}",
+                       "blocks_per_direction": ncpu, "bytes_per_direction": moved,
+                       "l2": "host memory is not cached in L2; no flush"},
+            "swap_out_gbs": round(moved / (ms_out * 1e-3) / 1e9, 2),
+            "swap_in_gbs": round(moved / (ms_in * 1e-3) / 1e9, 2),
+            "e2e": {"value": round(2 * moved * ws / (ms_e2e * 1e-3) / 1e9, 2), "unit": "GB/s",
+                    "h2d_bytes_per_step": 8 * 2 * ncpu * 2, "d2h_bytes_per_step": 0,
+                    "how": "BlockManager.swap_out / swap_in on the host, the pair lists "
+                           "copied to the device, then pa_swap_blocks each way"},
+            "gpu_launches": 2 * args.steps,
+            "roofline": {"bound": "host_link", "achieved": round(value / ws, 2),
+                         "peak": round(peak, 2), "unit": "GB/s",
+                         "frac": round(value / ws / peak, 4),
+                         "peak_kind": "measured in this run: contiguous pinned cudaMemcpyAsync "
+                                      "of the same bytes, device->host and host->device",
+                         "memcpy_d2h_gbs": round(moved / (ms_d2h * 1e-3) / 1e9, 2),
+                         "memcpy_h2d_gbs": round(moved / (ms_h2d * 1e-3) / 1e9, 2),
+                         "kernel": "pa_swap_blocks", "traffic": None},
+            "clocks": clocks,
+            "device_error": err,
         }
     if ws > 1:
         dist.barrier()
@@ -586,10 +715,17 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=10.0)
     ap.add_argument("--reference-budget", type=float, default=60.0)
+    ap.add_argument("--op", choices=["step", "swap"], default="step",
+                    help="swap: time the preemption swap of the workload instead of the step")
+    ap.add_argument("--swap-seqs", type=int, default=8,
+                    help="swap: number of sequences preempted and restored per step")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
-    res = run_reference(args) if args.impl == "reference" else run_ours(args)
+    if args.op == "swap":
+        res = run_swap(args) if args.impl == "ours" else None
+    else:
+        res = run_reference(args) if args.impl == "reference" else run_ours(args)
     if res is not None:
         print(json.dumps(res), flush=True)
 

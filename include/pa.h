@@ -129,6 +129,13 @@ pa_status pa_swap_blocks(void *dst_k_cache, void *dst_v_cache, const void *src_k
  * max_context_len : host-side upper bound of context_lens (0 = unknown: the table
  *                   width max_blocks_per_seq * block_size is used).  A context longer
  *                   than the bound sets PA_DEVERR_CONTEXT.
+ * sliding_window  : 0 = attend to the whole context.  W > 0 = attend to the last W
+ *                   tokens only, t in [max(0, L - W), L) (the block manager's
+ *                   sliding_window setting, "PagedAttention and dynamic memory
+ *                   management" blog, BlockSpaceManager example).  Table entries of
+ *                   pages wholly before that range are never read, so their blocks
+ *                   may have been returned to the pool (entry -1).  Negative:
+ *                   PA_ERR_INVALID_ARG.
  * partition_size  : how contexts are split (split-K); partial results of the pieces
  *                   of one context -- fp32 running max, sum and normalised output --
  *                   are merged by log-sum-exp in a second kernel.
@@ -152,8 +159,8 @@ pa_status pa_decode(void *out, const void *q, const void *k_cache, const void *v
                     const int32_t *block_tables, const int32_t *context_lens, int num_seqs,
                     int num_q_heads, int num_kv_heads, int head_dim, int block_size,
                     int num_blocks, int max_blocks_per_seq, float scale, int max_context_len,
-                    int partition_size, void *workspace, size_t workspace_bytes, pa_dtype dtype,
-                    void *stream);
+                    int sliding_window, int partition_size, void *workspace,
+                    size_t workspace_bytes, pa_dtype dtype, void *stream);
 
 #define PA_PARTITION_BALANCED (-1)
 
@@ -163,7 +170,8 @@ pa_status pa_decode(void *out, const void *q, const void *k_cache, const void *v
  * split).  For every sequence s with L = context_lens[s] > 0 and every kv head h:
  *   k_cache[block_tables[s][(L-1) / bs]][h][(L-1) % bs][:] = key[s*key_token_stride + h*head_dim + :]
  *   v_cache[...] likewise from value,
- * then the attention of pa_decode over [0, L) -- which therefore includes the new token.
+ * then the attention of pa_decode over [0, L) (or the last sliding_window tokens of
+ * it) -- which therefore includes the new token.
  * The write is done by the CTA that owns the last partition of (s, h) before it reads
  * that position, so the result equals pa_kv_write (with slot = the slot of position L-1)
  * followed by pa_decode, bit for bit.
@@ -180,8 +188,8 @@ pa_status pa_decode_append(void *out, const void *q, const void *key, const void
                            const int32_t *context_lens, int num_seqs, int num_q_heads,
                            int num_kv_heads, int head_dim, int block_size, int num_blocks,
                            int max_blocks_per_seq, float scale, int max_context_len,
-                           int partition_size, void *workspace, size_t workspace_bytes,
-                           pa_dtype dtype, void *stream);
+                           int sliding_window, int partition_size, void *workspace,
+                           size_t workspace_bytes, pa_dtype dtype, void *stream);
 
 /*
  * Bytes of workspace pa_decode needs for these sizes and this partition_size.
@@ -191,7 +199,7 @@ pa_status pa_decode_append(void *out, const void *q, const void *key, const void
  */
 size_t pa_decode_workspace_bytes(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
                                  int block_size, int max_blocks_per_seq, int max_context_len,
-                                 int partition_size);
+                                 int sliding_window, int partition_size);
 
 /*
  * The partition size (tokens) pa_decode uses for these arguments when its
@@ -201,7 +209,7 @@ size_t pa_decode_workspace_bytes(int num_seqs, int num_q_heads, int num_kv_heads
  */
 int pa_decode_partition_tokens(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
                                int block_size, int max_blocks_per_seq, int max_context_len,
-                               int partition_size);
+                               int sliding_window, int partition_size);
 
 /*
  * pa_decode for callers that cannot allocate device memory.  The paged-attention
@@ -234,8 +242,8 @@ pa_status pa_decode_static_scratch(void *out, const void *q, const void *k_cache
                                    const int32_t *context_lens, int num_seqs, int num_q_heads,
                                    int num_kv_heads, int head_dim, int block_size,
                                    int num_blocks, int max_blocks_per_seq, float scale,
-                                   int max_context_len, int partition_size, pa_dtype dtype,
-                                   void *stream);
+                                   int max_context_len, int sliding_window,
+                                   int partition_size, pa_dtype dtype, void *stream);
 
 /*
  * Reads (and with clear != 0 resets) the sticky error word of `device`.

@@ -22,7 +22,8 @@ EXPORTS = ("pa_kv_write", "pa_copy_blocks", "pa_decode", "pa_decode_workspace_by
            "pa_bm_usage_ratio", "pa_bm_can_allocate", "pa_bm_allocate", "pa_bm_fork",
            "pa_bm_free", "pa_bm_append_slots", "pa_bm_slot", "pa_bm_seq_len",
            "pa_bm_block_refcount", "pa_bm_block_tables", "pa_bm_set_cpu_pool",
-           "pa_bm_num_free_cpu_blocks", "pa_bm_is_swapped", "pa_bm_swap_out", "pa_bm_swap_in")
+           "pa_bm_num_free_cpu_blocks", "pa_bm_is_swapped", "pa_bm_swap_out", "pa_bm_swap_in",
+           "pa_bm_set_sliding_window")
 STATIC_SCRATCH_BYTES = 16 << 20  # PA_STATIC_SCRATCH_BYTES in include/pa.h
 
 _lib = None
@@ -50,17 +51,17 @@ def load(path: str = LIB_PATH):
     lib.pa_swap_blocks.argtypes = [P, P, P, P, P, i32, i32, i32, i32, i32, i32, i32, P]
     lib.pa_swap_blocks.restype = i32
     lib.pa_decode.argtypes = [P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, i32, f32, i32, i32,
-                              P, sz, i32, P]
+                              i32, P, sz, i32, P]
     lib.pa_decode.restype = i32
-    lib.pa_decode_workspace_bytes.argtypes = [i32] * 8
+    lib.pa_decode_workspace_bytes.argtypes = [i32] * 9
     lib.pa_decode_workspace_bytes.restype = sz
-    lib.pa_decode_partition_tokens.argtypes = [i32] * 8
+    lib.pa_decode_partition_tokens.argtypes = [i32] * 9
     lib.pa_decode_partition_tokens.restype = i32
     lib.pa_decode_static_scratch.argtypes = [P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, i32,
-                                             f32, i32, i32, i32, P]
+                                             f32, i32, i32, i32, i32, P]
     lib.pa_decode_static_scratch.restype = i32
     lib.pa_decode_append.argtypes = [P, P, P, P, i64, i64, P, P, P, P, i32, i32, i32, i32, i32,
-                                     i32, i32, f32, i32, i32, P, sz, i32, P]
+                                     i32, i32, f32, i32, i32, i32, P, sz, i32, P]
     lib.pa_decode_append.restype = i32
     lib.pa_get_device_error.argtypes = [i32, ctypes.POINTER(ctypes.c_uint32), i32]
     lib.pa_get_device_error.restype = i32
@@ -126,43 +127,49 @@ def swap_blocks(dst_k_cache, dst_v_cache, src_k_cache, src_v_cache, pairs, strea
 
 
 def decode_workspace_bytes(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
-                           max_blocks_per_seq, max_context_len=0, partition_size=0) -> int:
+                           max_blocks_per_seq, max_context_len=0, partition_size=0,
+                           sliding_window=0) -> int:
     return int(load().pa_decode_workspace_bytes(num_seqs, num_q_heads, num_kv_heads, head_dim,
                                                 block_size, max_blocks_per_seq, max_context_len,
-                                                partition_size))
+                                                sliding_window, partition_size))
 
 
 def decode_partition_tokens(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
-                            max_blocks_per_seq, max_context_len=0, partition_size=0) -> int:
+                            max_blocks_per_seq, max_context_len=0, partition_size=0,
+                            sliding_window=0) -> int:
     return int(load().pa_decode_partition_tokens(num_seqs, num_q_heads, num_kv_heads, head_dim,
                                                  block_size, max_blocks_per_seq, max_context_len,
-                                                 partition_size))
+                                                 sliding_window, partition_size))
 
 
 def decode(out, q, k_cache, v_cache, block_tables, context_lens, scale, block_size=None,
-           max_context_len=0, partition_size=0, workspace=None, stream=None) -> None:
+           max_context_len=0, partition_size=0, workspace=None, stream=None,
+           sliding_window=0) -> None:
     """out, q [B, Hq, d]; caches [NB, Hkv, bs, d]; block_tables int32 [B, W];
     context_lens int32 [B].  ``workspace`` (a uint8 CUDA tensor) is allocated here
-    with torch when the plan needs one and none is given."""
+    with torch when the plan needs one and none is given.  ``sliding_window`` > 0:
+    each query attends to the last that many tokens of its context."""
     import torch
     B, hq, d = q.shape
     nb, hkv, bs, _ = k_cache.shape
     if block_size is not None and block_size != bs:
         raise PAError(f"block_size {block_size} != cache block size {bs}")
     W = block_tables.shape[1]
-    need = decode_workspace_bytes(B, hq, hkv, d, bs, W, max_context_len, partition_size)
+    need = decode_workspace_bytes(B, hq, hkv, d, bs, W, max_context_len, partition_size,
+                                  sliding_window)
     if need and workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     wptr = _ptr(workspace) if workspace is not None else None
     wbytes = workspace.numel() if workspace is not None else 0
     _check(load().pa_decode(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
                             _ptr(context_lens), B, hq, hkv, d, bs, nb, W, float(scale),
-                            int(max_context_len), int(partition_size), wptr, wbytes,
-                            _dtype(q), _stream(stream)), "pa_decode")
+                            int(max_context_len), int(sliding_window), int(partition_size), wptr,
+                            wbytes, _dtype(q), _stream(stream)), "pa_decode")
 
 
 def decode_append(out, q, key, value, k_cache, v_cache, block_tables, context_lens, scale,
-                  max_context_len=0, partition_size=0, workspace=None, stream=None) -> None:
+                  max_context_len=0, partition_size=0, workspace=None, stream=None,
+                  sliding_window=0) -> None:
     """Cache write of each sequence's new token (key/value [B, Hkv, d], stored at
     position context_lens[s]-1) fused with decode; same result as kv_write + decode."""
     import torch
@@ -171,7 +178,8 @@ def decode_append(out, q, key, value, k_cache, v_cache, block_tables, context_le
     assert key.shape[0] == B and key.stride(2) == 1 and key.stride(1) == d
     assert value.stride(2) == 1 and value.stride(1) == d
     W = block_tables.shape[1]
-    need = decode_workspace_bytes(B, hq, hkv, d, bs, W, max_context_len, partition_size)
+    need = decode_workspace_bytes(B, hq, hkv, d, bs, W, max_context_len, partition_size,
+                                  sliding_window)
     if need and workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     wptr = _ptr(workspace) if workspace is not None else None
@@ -179,13 +187,14 @@ def decode_append(out, q, key, value, k_cache, v_cache, block_tables, context_le
     _check(load().pa_decode_append(_ptr(out), _ptr(q), _ptr(key), _ptr(value), key.stride(0),
                                    value.stride(0), _ptr(k_cache), _ptr(v_cache),
                                    _ptr(block_tables), _ptr(context_lens), B, hq, hkv, d, bs, nb,
-                                   W, float(scale), int(max_context_len), int(partition_size),
-                                   wptr, wbytes, _dtype(q), _stream(stream)), "pa_decode_append")
+                                   W, float(scale), int(max_context_len), int(sliding_window),
+                                   int(partition_size), wptr, wbytes, _dtype(q), _stream(stream)),
+           "pa_decode_append")
 
 
 def decode_static_scratch(out, q, k_cache, v_cache, block_tables, context_lens, scale,
                           block_size=None, max_context_len=0, partition_size=0,
-                          stream=None) -> None:
+                          stream=None, sliding_window=0) -> None:
     """``decode`` for callers that cannot allocate device memory: the split-K partial
     results go to the library's own fixed scratch array (STATIC_SCRATCH_BYTES per
     GPU) instead of a workspace.  Calls that overlap on the GPU race on that array."""
@@ -194,7 +203,8 @@ def decode_static_scratch(out, q, k_cache, v_cache, block_tables, context_lens, 
     if block_size is not None and block_size != bs:
         raise PAError(f"block_size {block_size} != cache block size {bs}")
     W = block_tables.shape[1]
-    need = decode_workspace_bytes(B, hq, hkv, d, bs, W, max_context_len, partition_size)
+    need = decode_workspace_bytes(B, hq, hkv, d, bs, W, max_context_len, partition_size,
+                                  sliding_window)
     if need > STATIC_SCRATCH_BYTES:
         raise PAError(f"pa_decode_static_scratch: these sizes need {need} bytes of scratch, "
                       f"more than the library's fixed {STATIC_SCRATCH_BYTES}; use decode() "
@@ -202,7 +212,8 @@ def decode_static_scratch(out, q, k_cache, v_cache, block_tables, context_lens, 
     _check(load().pa_decode_static_scratch(
         _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
         _ptr(context_lens), B, hq, hkv, d, bs, nb, W, float(scale), int(max_context_len),
-        int(partition_size), _dtype(q), _stream(stream)), "pa_decode_static_scratch")
+        int(sliding_window), int(partition_size), _dtype(q), _stream(stream)),
+        "pa_decode_static_scratch")
 
 
 def device_error(device: int = 0, clear: bool = True) -> int:

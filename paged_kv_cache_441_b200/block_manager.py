@@ -55,6 +55,8 @@ def _lib():
         for f in (lib.pa_bm_swap_out, lib.pa_bm_swap_in):
             f.argtypes = [P, P, i32, P, i32, ctypes.POINTER(i32)]
             f.restype = i32
+        lib.pa_bm_set_sliding_window.argtypes = [P, i32]
+        lib.pa_bm_set_sliding_window.restype = i32
         _declared = True
     return lib
 
@@ -125,6 +127,11 @@ class BlockManager:
 
     def refcount(self, block: int) -> int:
         return int(self._lib.pa_bm_block_refcount(self._h, block))
+
+    def set_sliding_window(self, window: int) -> None:
+        """Keep only each sequence's last ``window`` positions: blocks wholly before them
+        go back to the pool (table entry -1).  Only while no sequence exists."""
+        _check(self._lib.pa_bm_set_sliding_window(self._h, window), "pa_bm_set_sliding_window")
 
     def set_cpu_pool(self, num_cpu_blocks: int) -> None:
         _check(self._lib.pa_bm_set_cpu_pool(self._h, num_cpu_blocks), "pa_bm_set_cpu_pool")

@@ -4,6 +4,8 @@
 // table (physical block ids in token order) and length.  Allocation is on demand;
 // a sequence that appends into a shared, partially filled last block gets a private
 // copy first (copy-on-write), reported as a (src, dst) pair for pa_copy_blocks.
+// Under a sliding window of W tokens, a block that lies wholly before the last W
+// positions of its sequence is given back and its table entry becomes -1.
 #include <cstdint>
 #include <new>
 #include <unordered_map>
@@ -17,8 +19,9 @@ struct pa_block_manager {
     std::vector<int> refcount;   // per physical block, 0 = free
     std::vector<int> free_list;  // LIFO of free block ids
     struct Seq {
-        std::vector<int> blocks;  // GPU block ids, or host block ids when on_cpu
+        std::vector<int> blocks;  // GPU block ids, or host block ids when on_cpu; -1 = released
         int len = 0;
+        int first_live = 0;  // blocks[0 .. first_live) were released (sliding window)
         unsigned stamp = 0;  // last append batch that listed this sequence
         bool on_cpu = false;
     };
@@ -33,6 +36,24 @@ struct pa_block_manager {
     std::vector<unsigned> released_stamp;
     std::vector<Seq *> batch_seqs;
     unsigned batch = 0;
+    int window = 0;  // sliding window in tokens, 0 = whole contexts
+
+    // Blocks of a context of n tokens that lie wholly before its window.
+    int blocks_before_window(int n) const {
+        return (window > 0 && n > window) ? (n - window) / block_size : 0;
+    }
+    // Blocks a new sequence of n tokens holds.
+    int live_blocks(int n) const {
+        return (int)(((long long)n + block_size - 1) / block_size) - blocks_before_window(n);
+    }
+    void release_before_window(Seq &s) {
+        const int upto = blocks_before_window(s.len);
+        for (int j = s.first_live; j < upto; ++j) {
+            drop(s.blocks[j]);
+            s.blocks[j] = -1;
+        }
+        if (upto > s.first_live) s.first_live = upto;
+    }
 
     int take() {  // caller checked that the free list is not empty
         const int b = free_list.back();
@@ -68,7 +89,7 @@ pa_status move_group(pa_block_manager *bm, const int64_t *seq_ids, int n, int64_
             if (g == &it->second) return PA_ERR_INVALID_ARG;  // listed twice
         group.push_back(&it->second);
         for (int b : it->second.blocks)
-            if (uses[b]++ == 0) order.push_back(b);
+            if (b >= 0 && uses[b]++ == 0) order.push_back(b);
     }
     for (int b : order)
         if (uses[b] != from_ref[b]) return PA_ERR_INVALID_ARG;  // shared outside the group
@@ -87,7 +108,8 @@ pa_status move_group(pa_block_manager *bm, const int64_t *seq_ids, int n, int64_
         pairs[2 * i + 1] = nb;
     }
     for (pa_block_manager::Seq *g : group) {
-        for (int &b : g->blocks) b = moved[b];
+        for (int &b : g->blocks)
+            if (b >= 0) b = moved[b];
         g->on_cpu = out;
     }
     *num_pairs = (int)order.size();
@@ -126,6 +148,12 @@ pa_status pa_bm_swap_in(pa_block_manager *bm, const int64_t *seq_ids, int n, int
     return move_group(bm, seq_ids, n, pairs, max_pairs, num_pairs, false);
 }
 
+pa_status pa_bm_set_sliding_window(pa_block_manager *bm, int window) {
+    if (!bm || window < 0 || !bm->seqs.empty()) return PA_ERR_INVALID_ARG;
+    bm->window = window;
+    return PA_OK;
+}
+
 pa_block_manager *pa_bm_create(int num_blocks, int block_size) {
     if (num_blocks <= 0 || block_size <= 0) return nullptr;
     pa_block_manager *bm = new (std::nothrow) pa_block_manager();
@@ -158,18 +186,21 @@ double pa_bm_usage_ratio(const pa_block_manager *bm) {
 
 int pa_bm_can_allocate(const pa_block_manager *bm, int num_tokens) {
     if (!bm) return 0;
-    const int need = pa_bm_blocks_needed(num_tokens, bm->block_size);
-    return need >= 0 && need <= (int)bm->free_list.size();
+    if (num_tokens < 0) return 0;
+    return bm->live_blocks(num_tokens) <= (int)bm->free_list.size();
 }
 
 pa_status pa_bm_allocate(pa_block_manager *bm, int64_t seq_id, int num_tokens) {
     if (!bm || num_tokens < 0 || bm->seqs.count(seq_id)) return PA_ERR_INVALID_ARG;
-    const int need = pa_bm_blocks_needed(num_tokens, bm->block_size);
+    const int before = bm->blocks_before_window(num_tokens);
+    const int need = bm->live_blocks(num_tokens);
     if (need > (int)bm->free_list.size()) return PA_ERR_NO_FREE_BLOCK;
     pa_block_manager::Seq s;
-    s.blocks.reserve(need);
+    s.blocks.assign(before, -1);
+    s.blocks.reserve(before + need);
     for (int i = 0; i < need; ++i) s.blocks.push_back(bm->take());
     s.len = num_tokens;
+    s.first_live = before;
     bm->seqs.emplace(seq_id, std::move(s));
     return PA_OK;
 }
@@ -180,7 +211,9 @@ pa_status pa_bm_fork(pa_block_manager *bm, int64_t parent_id, int64_t child_id) 
     if (it == bm->seqs.end() || it->second.on_cpu || bm->seqs.count(child_id))
         return PA_ERR_INVALID_ARG;
     pa_block_manager::Seq child = it->second;
-    for (int b : child.blocks) ++bm->refcount[b];
+    child.stamp = 0;
+    for (int b : child.blocks)
+        if (b >= 0) ++bm->refcount[b];
     bm->seqs.emplace(child_id, std::move(child));
     return PA_OK;
 }
@@ -191,6 +224,7 @@ pa_status pa_bm_free(pa_block_manager *bm, int64_t seq_id) {
     if (it == bm->seqs.end()) return PA_ERR_INVALID_ARG;
     // return blocks back to front, so the next allocation reuses them in order
     for (auto b = it->second.blocks.rbegin(); b != it->second.blocks.rend(); ++b) {
+        if (*b < 0) continue;  // released (sliding window)
         if (it->second.on_cpu) {
             if (--bm->cpu_refcount[*b] == 0) bm->cpu_free_list.push_back(*b);
         } else {
@@ -267,6 +301,9 @@ pa_status pa_bm_append_slots(pa_block_manager *bm, const int64_t *seq_ids, int n
         slot_mapping[i] = (int64_t)blk * bs + off;
         ++s.len;
     }
+    // pass 3: blocks that fell out of the window of their sequence go back to the pool
+    if (bm->window > 0)
+        for (int i = 0; i < n; ++i) bm->release_before_window(*bm->batch_seqs[i]);
     *num_pairs = np;
     return PA_OK;
 }
@@ -275,8 +312,9 @@ int64_t pa_bm_slot(const pa_block_manager *bm, int64_t seq_id, int pos) {
     if (!bm) return -1;
     auto it = bm->seqs.find(seq_id);
     if (it == bm->seqs.end() || it->second.on_cpu || pos < 0 || pos >= it->second.len) return -1;
-    return (int64_t)it->second.blocks[pos / bm->block_size] * bm->block_size +
-           pos % bm->block_size;
+    const int blk = it->second.blocks[pos / bm->block_size];
+    if (blk < 0) return -1;  // released (sliding window)
+    return (int64_t)blk * bm->block_size + pos % bm->block_size;
 }
 
 int pa_bm_seq_len(const pa_block_manager *bm, int64_t seq_id) {

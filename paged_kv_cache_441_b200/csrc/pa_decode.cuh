@@ -70,6 +70,7 @@ struct DecodeParams {
     int max_blocks_per_seq;
     int partition_tokens;
     int num_parts;
+    int sliding_window;  // > 0: attend to the last sliding_window tokens only; 0: all
     float scale_log2;
     // Cache write fused into the decode (pa_decode_append): the new token of sequence s
     // (key/value rows new_k + s * new_k_stride, heads contiguous) is stored at position
@@ -96,6 +97,17 @@ struct Geom {
 // column block chunk/8, then the 128-byte swizzle (chunk%8) ^ (row%8).
 __device__ __forceinline__ uint32_t tile_off(int row, int chunk) {
     return (chunk >> 3) * (kTile * 128) + row * 128 + (((chunk & 7) ^ (row & 7)) << 4);
+}
+
+// Sliding window: the attended tokens of a context of L are [window_lo, L); the
+// tiles that cover them start at the 16-aligned position span_begin, so every tile
+// stays inside one page (block sizes are powers of two) and its rows below
+// window_lo are masked.  Without a window both are 0.
+__host__ __device__ __forceinline__ int window_lo(int L, int W) {
+    return (W > 0 && L > W) ? L - W : 0;
+}
+__host__ __device__ __forceinline__ int span_begin(int L, int W) {
+    return window_lo(L, W) & ~(kTile - 1);
 }
 
 __device__ __forceinline__ uint4 lds128(uint32_t addr) {
@@ -180,8 +192,9 @@ struct SimtWarp {
         l = 0.f;
     }
 
-    __device__ __forceinline__ void tile(uint32_t kd, uint32_t vd, int nrows, float sl2,
-                                         int lane) {
+    // Rows [row_lo, nrows) of the tile are context tokens; the others are masked.
+    __device__ __forceinline__ void tile(uint32_t kd, uint32_t vd, int row_lo, int nrows,
+                                         float sl2, int lane) {
         float v[kN];
 #pragma unroll
         for (int i = 0; i < kSteps; ++i) {
@@ -204,7 +217,7 @@ struct SimtWarp {
             }
         }
         Butterfly<kN, kCpr / 2>::run(v, lane);
-        const bool valid = my_row < nrows;
+        const bool valid = my_row >= row_lo && my_row < nrows;
         const float sc = valid ? v[0] * sl2 : -INFINITY;
         // tile max of this lane's head: all lane bits except the head bits
         float mx = sc;
@@ -231,7 +244,7 @@ struct SimtWarp {
 #pragma unroll
             for (int h = 0; h < G; ++h) ph[h] = __shfl_sync(kFull, pr, grp | ((i * G + h) << kShift));
             const int r = i * kRps + rr;
-            if (r < nrows) {
+            if (r >= row_lo && r < nrows) {
                 const uint4 w = lds128(vd + tile_off(r, c));
                 const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
@@ -350,8 +363,9 @@ struct MmaWarp {
         l0 = l1 = 0.f;
     }
 
-    __device__ __forceinline__ void tile(uint32_t kd, uint32_t vd, int nrows, float sl2,
-                                         int lane) {
+    // Rows [row_lo, nrows) of the tile are context tokens; the others are masked.
+    __device__ __forceinline__ void tile(uint32_t kd, uint32_t vd, int row_lo, int nrows,
+                                         float sl2, int lane) {
         const int j = lane >> 3, r8 = lane & 7;
         // S^T = K . Q^T  (A = K rows from ldmatrix: matrix j -> rows +8*(j&1), k +8*(j>>1))
         float sc[4] = {0.f, 0.f, 0.f, 0.f};
@@ -364,7 +378,7 @@ struct MmaWarp {
                 Mma<T>::run(sc, a, qb[kk][0], qb[kk][1]);
             }
         }
-        const bool v0 = gq < nrows, v1 = gq + 8 < nrows;
+        const bool v0 = gq >= row_lo && gq < nrows, v1 = gq + 8 >= row_lo && gq + 8 < nrows;
         const float s0 = v0 ? sc[0] * sl2 : -INFINITY;
         const float s1 = v0 ? sc[1] * sl2 : -INFINITY;
         const float s2 = v1 ? sc[2] * sl2 : -INFINITY;
@@ -401,7 +415,8 @@ struct MmaWarp {
         const uint32_t y1 = Fmt<T>::pack_rn(p2 - h1.x, p3 - h1.y);
         const uint32_t bh0 = movmatrix_trans(x0), bh1 = movmatrix_trans(x1);
         const uint32_t bl0 = movmatrix_trans(y0), bl1 = movmatrix_trans(y1);
-        // rows past the context may hold anything (NaN): zero them so 0 * V stays 0
+        // rows outside the context may hold anything (NaN, or rows that were never
+        // loaded): zero them so 0 * V stays 0
         if (nrows < kTile) {
             constexpr int kChunks = Geom<D>::kHalves * 8;
             for (int idx = lane; idx < (kTile - nrows) * kChunks; idx += 32) {
@@ -409,6 +424,17 @@ struct MmaWarp {
                 const int ch = idx % kChunks;
                 sts128_zero(vd + (ch >> 3) * (kTile * 128) + r * 128 + ((ch & 7) << 4));
             }
+        }
+        if (row_lo > 0) {
+            constexpr int kChunks = Geom<D>::kHalves * 8;
+            const int nlo = min(row_lo, kTile);
+            for (int idx = lane; idx < nlo * kChunks; idx += 32) {
+                const int r = idx / kChunks;
+                const int ch = idx % kChunks;
+                sts128_zero(vd + (ch >> 3) * (kTile * 128) + r * 128 + ((ch & 7) << 4));
+            }
+        }
+        if (nrows < kTile || row_lo > 0) {
             fence_proxy_async_smem();
             __syncwarp();
         }
@@ -506,7 +532,9 @@ using WarpCompute = typename std::conditional<(G >= 4), MmaWarp<T, D, G>, SimtWa
 
 // ------------------------------------------------------------------ partition kernel
 
-template <typename T, int D, int G, int BOXR>
+// WIN: compiled with sliding-window support (p.sliding_window > 0); the instances
+// without it keep the whole-context path free of the window's bookkeeping.
+template <typename T, int D, int G, int BOXR, bool WIN>
 __global__ void __launch_bounds__(kWarps * 32)
     pa_decode_partition_kernel(const __grid_constant__ DecodeParams p) {
     pdl_wait_and_release();
@@ -525,13 +553,16 @@ __global__ void __launch_bounds__(kWarps * 32)
     const int Hq = p.num_q_heads;
 
     // Start the three independent loads of this item at once: its context length, the
-    // block-table entries of its partition (the page range does not depend on L) and q.
+    // block-table entries of its partition (without a sliding window the page range
+    // does not depend on L) and q.  Under a window the table is read through the
+    // per-warp lookup below once L is known.
     const int P = p.partition_tokens;
+    const int W = WIN ? p.sliding_window : 0;
     const int32_t *table = p.block_tables + (size_t)s * p.max_blocks_per_seq;
     const int pg_first = (int)(((long long)part * P) >> p.bs_shift);
     const int pg_count = min((int)((((long long)part * P + P - 1) >> p.bs_shift) - pg_first + 1),
                              p.max_blocks_per_seq - pg_first);
-    const bool tab_in_smem = pg_count <= kTabSmem;
+    const bool tab_in_smem = W == 0 && pg_count <= kTabSmem;
     __shared__ int tab_smem[kTabSmem];
     if (tab_in_smem)
         for (int i = tid; i < pg_count; i += kWarps * 32) tab_smem[i] = __ldg(table + pg_first + i);
@@ -544,7 +575,8 @@ __global__ void __launch_bounds__(kWarps * 32)
         if (tid == 0 && part == 0) raise_error(PA_DEVERR_CONTEXT);
         L = L < 0 ? 0 : cap;
     }
-    const int nparts = (L + P - 1) / P;
+    const int wlo = WIN ? window_lo(L, W) : 0, span0 = WIN ? span_begin(L, W) : 0;
+    const int nparts = (L - span0 + P - 1) / P;
     if (nparts > p.num_parts && tid == 0 && part == 0) raise_error(PA_DEVERR_CONTEXT);
     T *out = reinterpret_cast<T *>(p.out) + ((size_t)s * Hq + (size_t)g * G) * D;
     if (L == 0) {
@@ -577,7 +609,7 @@ __global__ void __launch_bounds__(kWarps * 32)
         }
     }
 
-    const int t0 = part * P, t1 = min(t0 + P, L);
+    const int t0 = span0 + part * P, t1 = min(t0 + P, L);
     const int ntiles = (t1 - t0 + kTile - 1) / kTile;
     const int qd = ntiles / kWarps, rm = ntiles % kWarps;
     const int wt0 = warp * qd + min(warp, rm);
@@ -616,31 +648,33 @@ __global__ void __launch_bounds__(kWarps * 32)
         const int stage = jt % kStages;
         const int tok = tok_begin + jt * kTile;
         const int nrows = min(kTile, tok_end - tok);
+        const int row_lo = WIN ? max(0, wlo - tok) : 0;
         constexpr int kBoxes = kTile / BOXR;
         int ys[kBoxes];
-        int nbox = 0;
+        unsigned boxes = 0;  // boxes that hold context rows (a box below the window is skipped)
         bool ok = true;
 #pragma unroll
         for (int b = 0; b < kBoxes; ++b) {
             ys[b] = 0;
-            if (b * BOXR < nrows) {
+            if (b * BOXR < nrows && (b + 1) * BOXR > row_lo) {
                 const int tb = tok + b * BOXR;
                 const int blk = lookup(tb >> p.bs_shift);
                 if ((unsigned)blk < (unsigned)p.num_blocks)
                     ys[b] = (blk * p.num_kv_heads + g) * p.block_size + (tb & (p.block_size - 1));
                 else
                     ok = false;
-                nbox = b + 1;
+                boxes |= 1u << b;
             }
         }
         const uint32_t bar = bars + 8 * stage;
         const uint32_t kd = ring + stage * Gm::kStage, vd = kd + Gm::kMat;
         if (lane == 0) {
             if (ok) {
-                mbar_arrive_expect_tx(bar, (uint32_t)(nbox * Gm::kHalves * BOXR * 128 * 2));
+                mbar_arrive_expect_tx(bar,
+                                      (uint32_t)(__popc(boxes) * Gm::kHalves * BOXR * 128 * 2));
 #pragma unroll
                 for (int b = 0; b < kBoxes; ++b) {
-                    if (b < nbox) {
+                    if ((boxes >> b) & 1u) {
 #pragma unroll
                         for (int hf = 0; hf < Gm::kHalves; ++hf) {
                             const uint32_t off = hf * Gm::kRegion + b * BOXR * 128;
@@ -676,7 +710,7 @@ __global__ void __launch_bounds__(kWarps * 32)
         const int tok = tok_begin + jt * kTile;
         const int nrows = ((okmask >> stage) & 1u) ? min(kTile, tok_end - tok) : 0;
         const uint32_t kd = ring + stage * Gm::kStage, vd = kd + Gm::kMat;
-        wc.tile(kd, vd, nrows, p.scale_log2, lane);
+        wc.tile(kd, vd, WIN ? max(0, wlo - tok) : 0, nrows, p.scale_log2, lane);
         __syncwarp();
         if (jt + kStages < nt) produce(jt + kStages);
     }

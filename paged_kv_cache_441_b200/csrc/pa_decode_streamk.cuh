@@ -52,6 +52,7 @@ struct StreamKParams {
     int bs_shift;
     int num_blocks;
     int max_blocks_per_seq;
+    int sliding_window;  // > 0: each query attends to its last sliding_window tokens
     float scale_log2;
 };
 
@@ -76,6 +77,7 @@ constexpr int kSkFirstSeg = 8;  // the segment is the first of this warp's range
 constexpr int kSkOk = 16;       // block ids valid, data loaded
 constexpr int kSkStarts = 32;   // the segment starts (j = 0) inside this warp
 constexpr int kSkEnds = 64;     // the segment ends (last tile) inside this warp
+constexpr int kSkRowLoShift = 8;  // bits 8+: first context row of the tile (window start)
 
 __host__ __device__ __forceinline__ long long sk_range_begin(long long T, int k, int NW) {
     return T * k / NW;
@@ -87,6 +89,11 @@ __host__ __device__ __forceinline__ int sk_worker_of(long long x, long long T, i
 }
 
 __device__ __forceinline__ int clamp_len(int L, int cap) { return L < 0 ? 0 : (L > cap ? cap : L); }
+
+// 16-token tiles of a (sequence, kv head) segment: from span_begin(L, W) to L.
+__device__ __forceinline__ int seg_tiles(int L, int W) {
+    return (L - span_begin(L, W) + kTile - 1) / kTile;
+}
 
 // T k / NW without a 64-bit division per call: T = q NW + r, so T k / NW = q k + r k / NW
 // with r k < NW k < 2^32.
@@ -127,7 +134,7 @@ __global__ void __launch_bounds__(kSkWarps * 32)
     for (int s = s_lo; s < s_hi; ++s) {
         const int L = p.context_lens[s];
         if ((L < 0 || L > cap) && blockIdx.x == 0) raise_error(PA_DEVERR_CONTEXT);
-        local += (clamp_len(L, cap) + kTile - 1) / kTile;
+        local += seg_tiles(clamp_len(L, cap), p.sliding_window);
     }
     int incl = local;
 #pragma unroll
@@ -146,7 +153,7 @@ __global__ void __launch_bounds__(kSkWarps * 32)
     int run = woff + incl - local;
     for (int s = s_lo; s < s_hi; ++s) {
         pre[s] = run;
-        run += (clamp_len(p.context_lens[s], cap) + kTile - 1) / kTile;
+        run += seg_tiles(clamp_len(p.context_lens[s], cap), p.sliding_window);
     }
     if (tid == 0) pre[B] = total;
     __syncthreads();
@@ -221,24 +228,25 @@ __global__ void __launch_bounds__(kSkWarps * 32)
 
         auto produce = [&](int t) {
             const int stage = t % kSkStages;
-            const int tok = pj * kTile;
+            const int tok = span_begin(pL, p.sliding_window) + pj * kTile;
             const int nrows = min(kTile, pL - tok);
+            const int row_lo = max(0, window_lo(pL, p.sliding_window) - tok);
             const int npages = (pL + p.block_size - 1) >> p.bs_shift;
             constexpr int kBoxes = kTile / BOXR;
             int ys[kBoxes];
-            int nbox = 0;
+            unsigned boxes = 0;  // boxes holding context rows (below the window: skipped)
             bool ok = true;
     #pragma unroll
             for (int bx = 0; bx < kBoxes; ++bx) {
                 ys[bx] = 0;
-                if (bx * BOXR < nrows) {
+                if (bx * BOXR < nrows && (bx + 1) * BOXR > row_lo) {
                     const int tb = tok + bx * BOXR;
                     const int blk = lookup(ps, tb >> p.bs_shift, npages);
                     if ((unsigned)blk < (unsigned)p.num_blocks)
                         ys[bx] = (blk * Hkv + pg) * p.block_size + (tb & (p.block_size - 1));
                     else
                         ok = false;
-                    nbox = bx + 1;
+                    boxes |= 1u << bx;
                 }
             }
             int flags = 0;
@@ -249,15 +257,17 @@ __global__ void __launch_bounds__(kSkWarps * 32)
             if (pj == pn - 1) flags |= kSkEnds;
             if (p_segidx == 0) flags |= kSkFirstSeg;
             if (ok) flags |= kSkOk;
+            flags |= row_lo << kSkRowLoShift;
             const uint32_t bar = bars + 8 * stage;
             const uint32_t kd = ring + stage * Gm::kStage, vd = kd + Gm::kMat;
             if (lane == 0) {
                 meta[stage] = make_int4(ps, pg, nrows, flags);
                 if (ok) {
-                    mbar_arrive_expect_tx(bar, (uint32_t)(nbox * Gm::kHalves * BOXR * 128 * 2));
+                    mbar_arrive_expect_tx(
+                        bar, (uint32_t)(__popc(boxes) * Gm::kHalves * BOXR * 128 * 2));
     #pragma unroll
                     for (int bx = 0; bx < kBoxes; ++bx) {
-                        if (bx < nbox) {
+                        if ((boxes >> bx) & 1u) {
     #pragma unroll
                             for (int hf = 0; hf < Gm::kHalves; ++hf) {
                                 const uint32_t off = hf * Gm::kRegion + bx * BOXR * 128;
@@ -283,7 +293,7 @@ __global__ void __launch_bounds__(kSkWarps * 32)
                         ++ps;
                         pL = get_len(ps);
                     } while (pL == 0 && ps + 1 < B);
-                    pn = (pL + kTile - 1) / kTile;
+                    pn = seg_tiles(pL, p.sliding_window);
                 }
                 p_segfirst = true;
                 p_seg_j0 = 0;
@@ -312,7 +322,8 @@ __global__ void __launch_bounds__(kSkWarps * 32)
             if (flags & kSkFirst)
                 wc.init(reinterpret_cast<const T *>(p.q) + head0 * D, lane);
             const uint32_t kd = ring + stage * Gm::kStage, vd = kd + Gm::kMat;
-            wc.tile(kd, vd, (flags & kSkOk) ? md.z : 0, p.scale_log2, lane);
+            wc.tile(kd, vd, flags >> kSkRowLoShift, (flags & kSkOk) ? md.z : 0, p.scale_log2,
+                    lane);
             if (flags & kSkLast) {
                 const int slot = (flags & kSkFirstSeg) ? 0 : 1;
                 const size_t rec = (size_t)k * 2 + slot;

@@ -110,11 +110,16 @@ int current_device_or_zero() {
 }
 
 Plan make_plan(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int block_size,
-               int max_blocks_per_seq, int max_context_len, int partition_size, int sms) {
+               int max_blocks_per_seq, int max_context_len, int sliding_window,
+               int partition_size, int sms) {
     Plan pl;
     const long long cap = (long long)max_blocks_per_seq * block_size;
     long long bound = cap;
     if (max_context_len > 0 && max_context_len < cap) bound = max_context_len;
+    // under a window the tiles of a context span at most W + 15 tokens (span_begin
+    // rounds the window start down to a tile)
+    if (sliding_window > 0 && (long long)sliding_window + kTile - 1 < bound)
+        bound = (long long)sliding_window + kTile - 1;
     if (bound < 1) bound = 1;
     const int G = num_kv_heads > 0 ? num_q_heads / num_kv_heads : 1;
     const int max_seqs = head_dim == 64 ? SkGeom<64>::kMaxSeqs : SkGeom<128>::kMaxSeqs;
@@ -197,10 +202,10 @@ cudaError_t ensure_smem(K kernel, int bytes, std::atomic<bool> *flags, int dev) 
     return e;
 }
 
-template <typename T, int D, int G, int BOXR>
+template <typename T, int D, int G, int BOXR, bool WIN>
 cudaError_t launch_partition(const DecodeParams &p, dim3 grid, cudaStream_t st, int dev) {
     static std::atomic<bool> flags[kMaxDevices];
-    auto kernel = pa_decode_partition_kernel<T, D, G, BOXR>;
+    auto kernel = pa_decode_partition_kernel<T, D, G, BOXR, WIN>;
     cudaError_t e = ensure_smem(kernel, Geom<D>::kSmem, flags, dev);
     if (e != cudaSuccess) return e;
     return launch_pdl(kernel, grid, dim3(kWarps * 32), Geom<D>::kSmem, st, p);
@@ -213,8 +218,11 @@ cudaError_t launch_merge(const MergeParams &p, dim3 grid, cudaStream_t st) {
 
 template <typename T, int D, int G>
 cudaError_t dispatch_boxr(const DecodeParams &p, dim3 grid, cudaStream_t st, int dev, int boxr) {
-    return boxr == 8 ? launch_partition<T, D, G, 8>(p, grid, st, dev)
-                     : launch_partition<T, D, G, 16>(p, grid, st, dev);
+    if (p.sliding_window > 0)
+        return boxr == 8 ? launch_partition<T, D, G, 8, true>(p, grid, st, dev)
+                         : launch_partition<T, D, G, 16, true>(p, grid, st, dev);
+    return boxr == 8 ? launch_partition<T, D, G, 8, false>(p, grid, st, dev)
+                     : launch_partition<T, D, G, 16, false>(p, grid, st, dev);
 }
 
 template <typename T, int D>
@@ -293,9 +301,10 @@ cudaError_t sk_merge(const SkMergeParams &p, dim3 grid, int D, cudaStream_t st) 
 
 pa_status check_decode_shape(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
                              int block_size, int num_blocks, int max_blocks_per_seq,
-                             int max_context_len, int partition_size) {
+                             int max_context_len, int sliding_window, int partition_size) {
     if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || num_blocks <= 0 ||
-        max_blocks_per_seq <= 0 || max_context_len < 0 || partition_size < PA_PARTITION_BALANCED)
+        max_blocks_per_seq <= 0 || max_context_len < 0 || sliding_window < 0 ||
+        partition_size < PA_PARTITION_BALANCED)
         return PA_ERR_INVALID_ARG;
     if (num_q_heads % num_kv_heads != 0) return PA_ERR_INVALID_ARG;
     const int G = num_q_heads / num_kv_heads;
@@ -314,7 +323,7 @@ pa_status check_decode_shape(int num_seqs, int num_q_heads, int num_kv_heads, in
 
 extern "C" {
 
-int pa_version(void) { return 100; }
+int pa_version(void) { return 200; }
 
 const char *pa_status_str(pa_status s) {
     switch (s) {
@@ -468,25 +477,25 @@ pa_status pa_swap_blocks(void *dst_k_cache, void *dst_v_cache, const void *src_k
 
 size_t pa_decode_workspace_bytes(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
                                  int block_size, int max_blocks_per_seq, int max_context_len,
-                                 int partition_size) {
+                                 int sliding_window, int partition_size) {
     if (num_seqs <= 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 ||
         block_size <= 0 || max_blocks_per_seq <= 0 || partition_size < PA_PARTITION_BALANCED ||
-        max_context_len < 0)
+        max_context_len < 0 || sliding_window < 0)
         return 0;
     return make_plan(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
-                     max_blocks_per_seq, max_context_len, partition_size,
+                     max_blocks_per_seq, max_context_len, sliding_window, partition_size,
                      device_sms(current_device_or_zero()))
         .ws_bytes;
 }
 
 int pa_decode_partition_tokens(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
                                int block_size, int max_blocks_per_seq, int max_context_len,
-                               int partition_size) {
+                               int sliding_window, int partition_size) {
     if (num_kv_heads <= 0 || block_size <= 0 || max_blocks_per_seq <= 0 ||
-        partition_size < PA_PARTITION_BALANCED || max_context_len < 0)
+        partition_size < PA_PARTITION_BALANCED || max_context_len < 0 || sliding_window < 0)
         return 0;
     return make_plan(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
-                     max_blocks_per_seq, max_context_len, partition_size,
+                     max_blocks_per_seq, max_context_len, sliding_window, partition_size,
                      device_sms(current_device_or_zero()))
         .partition_tokens;
 }
@@ -500,13 +509,13 @@ pa_status decode_impl(void *out, const void *q, const void *k_cache, const void 
                       const int32_t *block_tables, const int32_t *context_lens, int num_seqs,
                       int num_q_heads, int num_kv_heads, int head_dim, int block_size,
                       int num_blocks, int max_blocks_per_seq, float scale, int max_context_len,
-                      int partition_size, void *workspace, size_t workspace_bytes,
-                      pa_dtype dtype, void *stream, const void *new_k, const void *new_v,
-                      long long new_k_stride, long long new_v_stride) {
+                      int sliding_window, int partition_size, void *workspace,
+                      size_t workspace_bytes, pa_dtype dtype, void *stream, const void *new_k,
+                      const void *new_v, long long new_k_stride, long long new_v_stride) {
     if (dtype != PA_FP16 && dtype != PA_BF16) return PA_ERR_INVALID_ARG;
     pa_status st = check_decode_shape(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
                                       num_blocks, max_blocks_per_seq, max_context_len,
-                                      partition_size);
+                                      sliding_window, partition_size);
     if (st != PA_OK) return st;
     if (!std::isfinite(scale)) return PA_ERR_INVALID_ARG;
     if (num_seqs == 0) return PA_OK;
@@ -517,8 +526,8 @@ pa_status decode_impl(void *out, const void *q, const void *k_cache, const void 
         return PA_ERR_INVALID_ARG;
     const int dev = current_device();
     const Plan pl = make_plan(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
-                              max_blocks_per_seq, max_context_len, partition_size,
-                              device_sms(dev));
+                              max_blocks_per_seq, max_context_len, sliding_window,
+                              partition_size, device_sms(dev));
     if (pl.ws_bytes > 0 &&
         (!workspace || !aligned(workspace, 256) || workspace_bytes < pl.ws_bytes))
         return PA_ERR_INVALID_ARG;
@@ -553,6 +562,7 @@ pa_status decode_impl(void *out, const void *q, const void *k_cache, const void 
         sp.bs_shift = ilog2_host(block_size);
         sp.num_blocks = num_blocks;
         sp.max_blocks_per_seq = max_blocks_per_seq;
+        sp.sliding_window = sliding_window;
         sp.scale_log2 = scale * 1.4426950408889634f;
         int grid_used = 0;
         cudaError_t e = dtype == PA_BF16
@@ -600,6 +610,7 @@ pa_status decode_impl(void *out, const void *q, const void *k_cache, const void 
     p.max_blocks_per_seq = max_blocks_per_seq;
     p.partition_tokens = pl.partition_tokens;
     p.num_parts = pl.num_parts;
+    p.sliding_window = sliding_window;
     p.scale_log2 = scale * 1.4426950408889634f;
     p.new_k = new_k;
     p.new_v = new_v;
@@ -625,6 +636,7 @@ pa_status decode_impl(void *out, const void *q, const void *k_cache, const void 
         mp.cap = max_blocks_per_seq * block_size;
         mp.partition_tokens = pl.partition_tokens;
         mp.num_parts = pl.num_parts;
+        mp.sliding_window = sliding_window;
         dim3 mgrid((unsigned)num_q_heads, (unsigned)num_seqs);
         if (dtype == PA_BF16)
             e = head_dim == 64 ? launch_merge<__nv_bfloat16, 64>(mp, mgrid, st_)
@@ -645,12 +657,13 @@ pa_status pa_decode(void *out, const void *q, const void *k_cache, const void *v
                     const int32_t *block_tables, const int32_t *context_lens, int num_seqs,
                     int num_q_heads, int num_kv_heads, int head_dim, int block_size,
                     int num_blocks, int max_blocks_per_seq, float scale, int max_context_len,
-                    int partition_size, void *workspace, size_t workspace_bytes, pa_dtype dtype,
-                    void *stream) {
+                    int sliding_window, int partition_size, void *workspace,
+                    size_t workspace_bytes, pa_dtype dtype, void *stream) {
     return decode_impl(out, q, k_cache, v_cache, block_tables, context_lens, num_seqs,
                        num_q_heads, num_kv_heads, head_dim, block_size, num_blocks,
-                       max_blocks_per_seq, scale, max_context_len, partition_size, workspace,
-                       workspace_bytes, dtype, stream, nullptr, nullptr, 0, 0);
+                       max_blocks_per_seq, scale, max_context_len, sliding_window,
+                       partition_size, workspace, workspace_bytes, dtype, stream, nullptr,
+                       nullptr, 0, 0);
 }
 
 pa_status pa_decode_append(void *out, const void *q, const void *key, const void *value,
@@ -659,8 +672,8 @@ pa_status pa_decode_append(void *out, const void *q, const void *key, const void
                            const int32_t *context_lens, int num_seqs, int num_q_heads,
                            int num_kv_heads, int head_dim, int block_size, int num_blocks,
                            int max_blocks_per_seq, float scale, int max_context_len,
-                           int partition_size, void *workspace, size_t workspace_bytes,
-                           pa_dtype dtype, void *stream) {
+                           int sliding_window, int partition_size, void *workspace,
+                           size_t workspace_bytes, pa_dtype dtype, void *stream) {
     if (num_seqs > 0) {
         if (!key || !value || !aligned(key, 16) || !aligned(value, 16)) return PA_ERR_INVALID_ARG;
         if (key_token_stride % 8 != 0 || value_token_stride % 8 != 0 ||
@@ -670,9 +683,9 @@ pa_status pa_decode_append(void *out, const void *q, const void *key, const void
     }
     return decode_impl(out, q, k_cache, v_cache, block_tables, context_lens, num_seqs,
                        num_q_heads, num_kv_heads, head_dim, block_size, num_blocks,
-                       max_blocks_per_seq, scale, max_context_len, partition_size, workspace,
-                       workspace_bytes, dtype, stream, key, value, key_token_stride,
-                       value_token_stride);
+                       max_blocks_per_seq, scale, max_context_len, sliding_window,
+                       partition_size, workspace, workspace_bytes, dtype, stream, key, value,
+                       key_token_stride, value_token_stride);
 }
 
 }  // extern "C"
@@ -710,16 +723,17 @@ extern "C" pa_status pa_decode_static_scratch(
     void *out, const void *q, const void *k_cache, const void *v_cache,
     const int32_t *block_tables, const int32_t *context_lens, int num_seqs, int num_q_heads,
     int num_kv_heads, int head_dim, int block_size, int num_blocks, int max_blocks_per_seq,
-    float scale, int max_context_len, int partition_size, pa_dtype dtype, void *stream) {
+    float scale, int max_context_len, int sliding_window, int partition_size, pa_dtype dtype,
+    void *stream) {
     if (dtype != PA_FP16 && dtype != PA_BF16) return PA_ERR_INVALID_ARG;
     pa_status st = check_decode_shape(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
                                       num_blocks, max_blocks_per_seq, max_context_len,
-                                      partition_size);
+                                      sliding_window, partition_size);
     if (st != PA_OK) return st;
     if (num_seqs == 0) return PA_OK;
     const Plan pl = make_plan(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
-                              max_blocks_per_seq, max_context_len, partition_size,
-                              device_sms(current_device_or_zero()));
+                              max_blocks_per_seq, max_context_len, sliding_window,
+                              partition_size, device_sms(current_device_or_zero()));
     if (pl.ws_bytes > PA_STATIC_SCRATCH_BYTES) return PA_ERR_INVALID_ARG;  // over the limit
     void *scratch = nullptr;
     if (pl.ws_bytes > 0) {
@@ -729,6 +743,6 @@ extern "C" pa_status pa_decode_static_scratch(
     }
     return pa_decode(out, q, k_cache, v_cache, block_tables, context_lens, num_seqs, num_q_heads,
                      num_kv_heads, head_dim, block_size, num_blocks, max_blocks_per_seq, scale,
-                     max_context_len, partition_size, scratch,
+                     max_context_len, sliding_window, partition_size, scratch,
                      pl.ws_bytes > 0 ? (size_t)PA_STATIC_SCRATCH_BYTES : 0, dtype, stream);
 }

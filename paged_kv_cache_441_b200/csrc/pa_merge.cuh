@@ -129,6 +129,7 @@ struct MergeParams {
     int cap;  // max_blocks_per_seq * block_size
     int partition_tokens;
     int num_parts;
+    int sliding_window;  // as in DecodeParams: partitions start at span_begin(L, W)
 };
 
 // One CTA per (q head, sequence) with more than one partition.
@@ -138,7 +139,7 @@ __global__ void __launch_bounds__(kMergeThreads) pa_merge_kernel(const __grid_co
     const int h = blockIdx.x, s = blockIdx.y;
     int L = p.context_lens[s];
     L = L < 0 ? 0 : (L > p.cap ? p.cap : L);
-    int n = (L + p.partition_tokens - 1) / p.partition_tokens;
+    int n = (L - span_begin(L, p.sliding_window) + p.partition_tokens - 1) / p.partition_tokens;
     if (n <= 1) return;
     n = min(n, p.num_parts);
     const long long base = ((long long)s * p.num_q_heads + h) * p.num_parts;

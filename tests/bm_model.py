@@ -5,6 +5,11 @@ a reference count, a private copy before writing into a shared partially filled
 block): allocate ceil(n / bs) blocks; fork shares every block; free returns blocks
 whose count reaches 0; append reserves position L of each sequence.  Free blocks are
 handed out last-returned-first, lowest id first at the start.
+
+Sliding window W (the blog's sliding_window setting, read as: a sequence of length L
+needs only positions L-W .. L-1): a block whose positions all lie before L-W is given
+back and its table entry becomes None; a new sequence never takes those blocks; after
+an append batch the sequences of the batch give back what fell out of their window.
 """
 
 
@@ -13,8 +18,9 @@ class NoBlocks(Exception):
 
 
 class Model:
-    def __init__(self, num_blocks, block_size, num_cpu_blocks=0):
+    def __init__(self, num_blocks, block_size, num_cpu_blocks=0, window=0):
         self.bs = block_size
+        self.window = window
         self.ref = [0] * num_blocks
         self.free_ids = list(range(num_blocks))[::-1]
         self.seqs = {}  # id -> (blocks list, length)
@@ -32,20 +38,35 @@ class Model:
         if self.ref[b] == 0:
             self.free_ids.append(b)
 
+    def _dead(self, n):
+        """Pages of a length-n context whose every position is before the window."""
+        if self.window <= 0 or n <= self.window:
+            return 0
+        return sum(1 for j in range(-(-n // self.bs)) if (j + 1) * self.bs <= n - self.window)
+
     def allocate(self, sid, n):
         if sid in self.seqs:
             raise KeyError(sid)
-        need = -(-n // self.bs)
+        dead = self._dead(n)
+        need = -(-n // self.bs) - dead
         if need > len(self.free_ids):
             raise NoBlocks()
-        self.seqs[sid] = ([self._take() for _ in range(need)], n)
+        self.seqs[sid] = ([None] * dead + [self._take() for _ in range(need)], n)
+
+    def _trim(self, sid):
+        blocks, n = self.seqs[sid]
+        for j in range(self._dead(n)):
+            if blocks[j] is not None:
+                self._drop(blocks[j])
+                blocks[j] = None
 
     def fork(self, parent, child):
         if child in self.seqs or parent not in self.seqs:
             raise KeyError(child)
         blocks, n = self.seqs[parent]
         for b in blocks:
-            self.ref[b] += 1
+            if b is not None:
+                self.ref[b] += 1
         self.seqs[child] = (list(blocks), n)
 
     def free(self, sid):
@@ -53,12 +74,15 @@ class Model:
         if sid in self.on_cpu:
             self.on_cpu.discard(sid)
             for b in reversed(blocks):
+                if b is None:
+                    continue
                 self.cpu_ref[b] -= 1
                 if self.cpu_ref[b] == 0:
                     self.cpu_free.append(b)
             return
         for b in reversed(blocks):
-            self._drop(b)
+            if b is not None:
+                self._drop(b)
 
     def move(self, ids, out):
         """Swap a group out (to the host pool) or in; returns the (from, to) pairs."""
@@ -70,6 +94,8 @@ class Model:
         uses, order = {}, []
         for s in ids:
             for b in self.seqs[s][0]:
+                if b is None:
+                    continue
                 if b not in uses:
                     order.append(b)
                 uses[b] = uses.get(b, 0) + 1
@@ -87,7 +113,7 @@ class Model:
             pairs.append((b, nb))
         for s in ids:
             blocks, n = self.seqs[s]
-            self.seqs[s] = ([moved[b] for b in blocks], n)
+            self.seqs[s] = ([None if b is None else moved[b] for b in blocks], n)
             if out:
                 self.on_cpu.add(s)
             else:
@@ -126,4 +152,6 @@ class Model:
                     b = c
             slots.append(b * self.bs + off)
             self.seqs[sid] = (blocks, n + 1)
+        for sid in ids:
+            self._trim(sid)
         return slots, pairs

@@ -50,16 +50,16 @@ class DeviceCase:
         self.pairs = dev(case.copy_pairs.astype(np.int64).reshape(-1, 2), device)
         self.out = torch.empty_like(self.q)
 
-    def step(self, partition_size=0, max_context_len=None, workspace=None):
+    def step(self, partition_size=0, max_context_len=None, workspace=None, sliding_window=0):
         import paged_kv_cache_441_b200 as pa
         c = self.case
         if self.pairs.shape[0]:
             pa.copy_blocks(self.k_cache, self.v_cache, self.pairs)
         pa.kv_write(self.key, self.value, self.slot_mapping, self.k_cache, self.v_cache)
-        self.decode(partition_size, max_context_len, workspace)
+        self.decode(partition_size, max_context_len, workspace, sliding_window)
         return self.out
 
-    def decode(self, partition_size=0, max_context_len=None, workspace=None):
+    def decode(self, partition_size=0, max_context_len=None, workspace=None, sliding_window=0):
         import torch
         import paged_kv_cache_441_b200 as pa
         c = self.case
@@ -68,11 +68,12 @@ class DeviceCase:
             # all-ones bytes = NaN floats: nothing may be read that this call did not write
             need = pa.decode_workspace_bytes(c.num_seqs, c.num_q_heads, c.num_kv_heads,
                                              c.head_dim, c.block_size, c.max_blocks_per_seq,
-                                             mcl, partition_size)
+                                             mcl, partition_size, sliding_window)
             workspace = torch.full((max(need, 256),), 255, dtype=torch.uint8, device=self.q.device)
         pa.decode(self.out, self.q, self.k_cache, self.v_cache, self.block_tables,
                   self.context_lens, c.scale, max_context_len=mcl,
-                  partition_size=partition_size, workspace=workspace)
+                  partition_size=partition_size, workspace=workspace,
+                  sliding_window=sliding_window)
         return self.out
 
 

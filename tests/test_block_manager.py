@@ -19,7 +19,11 @@ def _invariants(bm, model):
     for sid, (blocks, n) in model.seqs.items():
         assert len(blocks) == -(-n // model.bs)
         assert bm.is_swapped(sid) == (sid in model.on_cpu)
+        if model.window:  # a sequence holds the pages of its window only
+            assert sum(b is not None for b in blocks) <= -(-model.window // model.bs) + 1
         for b in blocks:
+            if b is None:
+                continue
             if sid in model.on_cpu:
                 cpu_refs[b] += 1
             else:
@@ -53,7 +57,7 @@ def _sharing_group(model, sid):
     cpu = sid in model.on_cpu
     group, todo = {sid}, [sid]
     while todo:
-        blocks = set(model.seqs[todo.pop()][0])
+        blocks = set(model.seqs[todo.pop()][0]) - {None}
         for other, (ob, _) in model.seqs.items():
             if other not in group and (other in model.on_cpu) == cpu and blocks & set(ob):
                 group.add(other)
@@ -61,13 +65,15 @@ def _sharing_group(model, sid):
     return sorted(group)
 
 
-@pytest.mark.parametrize("seed", range(6))
-def test_random_operations_match_model(seed):
+@pytest.mark.parametrize("seed,window", [(s, 0) for s in range(6)] +
+                         [(6, 1), (7, 5), (8, 16), (9, 33)])
+def test_random_operations_match_model(seed, window):
     rng = np.random.default_rng(seed)
     nb, bs = int(rng.integers(8, 64)), int(rng.choice([1, 2, 4, 16]))
     ncpu = int(rng.integers(4, 40))
-    bm, model = pa.BlockManager(nb, bs), Model(nb, bs, ncpu)
+    bm, model = pa.BlockManager(nb, bs), Model(nb, bs, ncpu, window)
     bm.set_cpu_pool(ncpu)
+    bm.set_sliding_window(window)
     next_id = 0
     for step in range(300):
         op = rng.choice(["alloc", "fork", "free", "append", "swap_out", "swap_in"],
@@ -124,7 +130,11 @@ def test_random_operations_match_model(seed):
                     bm.block_tables([sid], max(len(blocks), 1))
                 continue
             bt, cl = bm.block_tables([sid], max(len(blocks), 1))
-            assert bt[0, : len(blocks)].tolist() == blocks and cl[0] == n
+            assert bt[0, : len(blocks)].tolist() == [-1 if b is None else b for b in blocks]
+            assert cl[0] == n
+            for pos in range(n):
+                blk = blocks[pos // bs]
+                assert bm.slot(sid, pos) == (-1 if blk is None else blk * bs + pos % bs)
 
 
 def test_errors_change_nothing():
@@ -167,14 +177,17 @@ def test_parallel_sampling_copy_on_write_counts():
     assert pairs2.shape == (0, 2)
 
 
-def test_logical_token_streams_through_tables():
+@pytest.mark.parametrize("window", [0, 5, 8])
+def test_logical_token_streams_through_tables(window):
     """Drive the oracle's cache write / block copy with the manager through prompts,
-    forks, appends and frees: every live sequence's K, gathered through its table,
-    must equal the tokens it logically holds."""
+    forks, appends, swaps and frees: every live sequence's K, gathered through its
+    table, must equal the tokens it logically holds (under a sliding window: its last
+    `window` tokens, with the pages before them given back)."""
     rng = np.random.default_rng(3)
     nb, hkv, bs, d = 96, 2, 4, 8
     bm = pa.BlockManager(nb, bs)
     bm.set_cpu_pool(40)
+    bm.set_sliding_window(window)
     model = None
     kc = np.zeros((nb, hkv, bs, d), np.uint16)
     vc = np.zeros_like(kc)
@@ -228,7 +241,7 @@ def test_logical_token_streams_through_tables():
             if bm.can_allocate(n):
                 bm.allocate(next_id, n)
                 toks = [tok() for _ in range(n)]
-                sm = np.array([bm.slot(next_id, i) for i in range(n)], np.int64)
+                sm = np.array([bm.slot(next_id, i) for i in range(n)], np.int64)  # -1: skip
                 oracle.kv_write(np.concatenate(toks), np.concatenate(toks), sm, kc, vc)
                 logical[next_id] = toks
                 next_id += 1
@@ -259,7 +272,9 @@ def test_logical_token_streams_through_tables():
             L = len(toks)
             bt, cl = bm.block_tables([s], max(-(-L // bs), 1))
             assert cl[0] == L
+            lo = L - window if 0 < window < L else 0
+            assert np.all(bt[0, :lo // bs] == -1) and np.all(bt[0, lo // bs:-(-L // bs)] >= 0)
             for g in range(hkv):
-                got = oracle_np.gather(kc, bt[0], L, g)
-                want = np.concatenate([t[:, g] for t in toks])
+                got = oracle_np.gather_positions(kc, bt[0], lo, L, g)
+                want = np.concatenate([t[:, g] for t in toks[lo:]])
                 assert np.array_equal(got, want), (step, s)

@@ -44,16 +44,19 @@ def test_swap_blocks_device_and_pinned_host():
     assert pa.device_error(0) == pa.DEVERR["pair"]
 
 
-@pytest.mark.parametrize("hq,hkv,bs,fused,preempt", [(16, 4, 16, False, False),
-                                                     (8, 8, 32, True, False),
-                                                     (32, 4, 16, True, False),
-                                                     (16, 2, 16, True, True)])
-def test_block_manager_serving_loop(hq, hkv, bs, fused, preempt):
-    rng = np.random.default_rng(hq * 100 + bs)
+@pytest.mark.parametrize("hq,hkv,bs,fused,preempt,window", [(16, 4, 16, False, False, 0),
+                                                            (8, 8, 32, True, False, 0),
+                                                            (32, 4, 16, True, False, 0),
+                                                            (16, 2, 16, True, True, 0),
+                                                            (8, 8, 32, False, False, 37),
+                                                            (16, 4, 16, True, True, 100)])
+def test_block_manager_serving_loop(hq, hkv, bs, fused, preempt, window):
+    rng = np.random.default_rng(hq * 100 + bs + window)
     nb, d, width, ncpu = 700, 128, 64, 300
     scale = 1 / math.sqrt(d)
     bm = pa.BlockManager(nb, bs)
     bm.set_cpu_pool(ncpu)
+    bm.set_sliding_window(window)  # 0: whole contexts
     kc_h = np.full((nb, hkv, bs, d), 0x7FC0, np.uint16)  # NaN where nothing was written
     vc_h = kc_h.copy()
     kc, vc = dev16(kc_h, "bf16"), dev16(vc_h, "bf16")
@@ -120,12 +123,16 @@ def test_block_manager_serving_loop(hq, hkv, bs, fused, preempt):
         out = torch.empty(len(live), hq, d, dtype=torch.bfloat16, device="cuda")
         if fused:  # cache write fused into the decode
             pa.decode_append(out, dev16(q, "bf16"), dev16(key, "bf16"), dev16(val, "bf16"), kc,
-                             vc, dev(bt), dev(cl), scale, max_context_len=int(cl.max()))
+                             vc, dev(bt), dev(cl), scale, max_context_len=int(cl.max()),
+                             sliding_window=window)
         else:
             pa.kv_write(dev16(key, "bf16"), dev16(val, "bf16"), dev(slots), kc, vc)
             pa.decode(out, dev16(q, "bf16"), kc, vc, dev(bt), dev(cl), scale,
-                      max_context_len=int(cl.max()), partition_size=128)
-        want = oracle.decode(q, kc_h, vc_h, bt, cl, scale, "bf16")
+                      max_context_len=int(cl.max()), partition_size=128,
+                      sliding_window=window)
+        want, bad = oracle.decode(q, kc_h, vc_h, bt, cl, scale, "bf16", return_bad=True,
+                                  sliding_window=window)
+        assert bad == 0
         err = np.max(np.abs(to_f64(out) - want))
         assert np.isfinite(err) and err <= TOL["bf16"], (step, err)
     torch.cuda.synchronize()

@@ -42,7 +42,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_status_strings_and_version(lib):
-    assert pa.version() == 100
+    assert pa.version() == 200
     for code in range(7):
         assert lib.pa_status_str(code) != b"unknown status"
     assert lib.pa_status_str(77) == b"unknown status"
@@ -70,11 +70,18 @@ def test_workspace_plan(lib):
     assert pa.decode_workspace_bytes(B, hq, hkv, d, bs, W, 2011, -1) >= 2 * warps * (d + 2) * 4
     assert pa.decode_partition_tokens(8, 8, 1, d, bs, 8192, 131072, 512) == 512
     assert pa.decode_workspace_bytes(B, hq, hkv, d, bs, W, 0, 128) >= B * hq * 16 * (d + 2) * 4
+    # sliding window: the tiles of a context span at most W + 15 tokens, whatever L is
+    assert pa.decode_partition_tokens(8, 8, 1, d, bs, 8192, 131072, 0, 1000) == 1024
+    assert pa.decode_workspace_bytes(8, 8, 1, d, bs, 8192, 131072, 0, 1000) == 0
+    assert pa.decode_partition_tokens(8, 8, 1, d, bs, 8192, 131072, 0, 4096) == 2048
+    ws3 = pa.decode_workspace_bytes(8, 8, 1, d, bs, 8192, 131072, 0, 4096)
+    assert 8 * 8 * 3 * (d + 2) * 4 <= ws3 < 8 * 8 * 4 * (d + 2) * 4 + 1024  # 3 partitions
+    assert pa.decode_workspace_bytes(8, 8, 1, d, bs, 8192, 100, 0, 4096) == 0  # bound by L
 
 
 def _decode_args(**over):
     a = dict(out=16, q=16, kc=16, vc=16, bt=16, cl=16, B=2, hq=8, hkv=2, d=128, bs=16, nb=10,
-             W=4, scale=0.1, mcl=0, ps=0, ws=None, wsb=0, dt=1, stream=None)
+             W=4, scale=0.1, mcl=0, win=0, ps=0, ws=None, wsb=0, dt=1, stream=None)
     a.update(over)
     return a
 
@@ -83,7 +90,7 @@ def _call_decode(lib, a):
     P = ctypes.c_void_p
     return lib.pa_decode(P(a["out"]), P(a["q"]), P(a["kc"]), P(a["vc"]), P(a["bt"]), P(a["cl"]),
                          a["B"], a["hq"], a["hkv"], a["d"], a["bs"], a["nb"], a["W"], a["scale"],
-                         a["mcl"], a["ps"], a["ws"], a["wsb"], a["dt"], a["stream"])
+                         a["mcl"], a["win"], a["ps"], a["ws"], a["wsb"], a["dt"], a["stream"])
 
 
 @pytest.mark.parametrize("over,code", [
@@ -91,7 +98,7 @@ def _call_decode(lib, a):
     (dict(bs=1024), 2), (dict(q=0), 1), (dict(q=24), 1), (dict(out=8), 1), (dict(ps=100), 1),
     (dict(scale=float("inf")), 1), (dict(dt=5), 1), (dict(nb=0), 1), (dict(W=0), 1),
     (dict(ps=-2), 1), (dict(ps=-1), 1),  # balanced split needs a workspace
-    (dict(mcl=-1), 1), (dict(B=-1), 1), (dict(hkv=0), 1),
+    (dict(mcl=-1), 1), (dict(B=-1), 1), (dict(hkv=0), 1), (dict(win=-1), 1),
     (dict(ps=64, W=100), 1),  # needs a workspace, none given
 ])
 def test_decode_rejects_before_launch(lib, over, code):

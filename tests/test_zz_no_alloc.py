@@ -42,7 +42,7 @@ def _c_static(case, t, out, partition_size):
         P(out.data_ptr()), P(t["q"].data_ptr()), P(t["kc"].data_ptr()), P(t["vc"].data_ptr()),
         P(t["bt"].data_ptr()), P(t["cl"].data_ptr()), case.num_seqs, case.num_q_heads,
         case.num_kv_heads, case.head_dim, case.block_size, case.num_blocks,
-        case.max_blocks_per_seq, ctypes.c_float(case.scale), case.max_context_len,
+        case.max_blocks_per_seq, ctypes.c_float(case.scale), case.max_context_len, 0,
         partition_size, 1, P(torch.cuda.current_stream().cuda_stream))
     return st
 

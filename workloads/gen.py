@@ -84,6 +84,7 @@ class DecodeCase:
     slot_mapping: np.ndarray
     copy_pairs: np.ndarray = field(default_factory=lambda: np.zeros((0, 2), np.int64))
     seed: int = 0
+    window: int = 0  # sliding window the decode uses (0 = whole contexts)
 
     @property
     def max_blocks_per_seq(self) -> int:
@@ -104,7 +105,8 @@ def _blocks_needed(lens: np.ndarray, bs: int) -> np.ndarray:
 
 
 def _poison(k_cache, v_cache, tables, lens, bs, dtype):
-    """NaN in every slot except positions [0, L-1) of each sequence."""
+    """NaN in every slot except positions [0, L-1) of each sequence (in the pages it
+    holds: table entries of -1 have no block)."""
     nan = NAN_BITS[dtype]
     nb = k_cache.shape[0]
     keep = np.zeros((nb, bs), dtype=bool)
@@ -114,9 +116,11 @@ def _poison(k_cache, v_cache, tables, lens, bs, dtype):
             continue
         nblk = (n_keep + bs - 1) // bs
         ids = tables[s, :nblk]
-        keep[ids[:-1], :] = True
+        full = ids[:-1]
+        keep[full[full >= 0], :] = True
         last = n_keep - (nblk - 1) * bs
-        keep[ids[-1], :last] = True
+        if ids[-1] >= 0:
+            keep[ids[-1], :last] = True
     kill = ~keep
     k_cache.transpose(0, 2, 1, 3)[kill] = nan
     v_cache.transpose(0, 2, 1, 3)[kill] = nan
@@ -125,14 +129,20 @@ def _poison(k_cache, v_cache, tables, lens, bs, dtype):
 def make_case(name: str, seed: int, num_seqs: int, num_q_heads: int, num_kv_heads: int,
               head_dim: int, block_size: int, lens_fn, dtype: str = "bf16",
               scale: float | None = None, spare: float = 0.10, num_blocks: int | None = None,
-              poison: bool = True) -> DecodeCase:
-    """Generic decode-step case: one new token per sequence, written at L-1."""
+              poison: bool = True, window: int = 0) -> DecodeCase:
+    """Generic decode-step case: one new token per sequence, written at L-1.
+
+    window > 0: the sequences hold only the pages of their last `window` positions, as
+    the block manager leaves them under that sliding window; the table entries of the
+    pages before are -1 and the pool is sized for the held pages."""
     rng = np.random.default_rng(seed)
     lens = np.asarray(lens_fn(rng), dtype=np.int32)
     assert lens.shape == (num_seqs,)
     bs = block_size
     nblk = _blocks_needed(lens, bs)
-    total = int(nblk.sum())
+    dead = (np.maximum(lens.astype(np.int64) - window, 0) // bs if window > 0
+            else np.zeros_like(nblk))
+    total = int((nblk - dead).sum())
     nb = num_blocks if num_blocks is not None else max(int(math.ceil((1.0 + spare) * total)), 1)
     assert nb >= total
     perm = rng.permutation(nb).astype(np.int32)
@@ -140,9 +150,9 @@ def make_case(name: str, seed: int, num_seqs: int, num_q_heads: int, num_kv_head
     tables = np.full((num_seqs, width), -1, dtype=np.int32)
     pos = 0
     for s in range(num_seqs):
-        n = int(nblk[s])
-        tables[s, :n] = perm[pos:pos + n]
-        pos += n
+        n, d0 = int(nblk[s]), int(dead[s])
+        tables[s, d0:n] = perm[pos:pos + n - d0]
+        pos += n - d0
     q = _draw(rng, (num_seqs, num_q_heads, head_dim), dtype)
     k_cache = _draw(rng, (nb, num_kv_heads, bs, head_dim), dtype)
     v_cache = _draw(rng, (nb, num_kv_heads, bs, head_dim), dtype)
@@ -159,7 +169,7 @@ def make_case(name: str, seed: int, num_seqs: int, num_q_heads: int, num_kv_head
         scale = 1.0 / math.sqrt(head_dim)
     return DecodeCase(name, dtype, num_seqs, num_q_heads, num_kv_heads, head_dim, bs, nb,
                       float(scale), lens, tables, q, k_cache, v_cache, key, value, slots,
-                      seed=seed)
+                      seed=seed, window=window)
 
 
 def make_prefix_cow(seed: int = 5, groups: int = 64, samples: int = 8, prefix: int = 1000,
@@ -281,6 +291,10 @@ CONFIGS = {
     "long_32_8": lambda num_seqs=8, **kw: make_case(
         "long_32_8", kw.pop("seed", 3), num_seqs, 32, 8, 128, kw.pop("block_size", 16),
         _lens_uniform(32768, 131072, num_seqs), **kw),
+    # sliding-window decode over long contexts: only the last 4096 positions are held
+    "window_4096_gqa": lambda num_seqs=64, **kw: make_case(
+        "window_4096_gqa", kw.pop("seed", 6), num_seqs, 32, 8, 128, kw.pop("block_size", 16),
+        _lens_uniform(8192, 32768, num_seqs), window=kw.pop("window", 4096), **kw),
     "prefix_cow": lambda num_seqs=None, **kw: make_prefix_cow(
         groups=(kw.pop("groups", 64) if num_seqs is None else max(1, num_seqs // 8)), **kw),
 }
