@@ -46,12 +46,14 @@ void pa_bm_destroy(pa_block_manager *bm);
  * Sliding window (the blog's BlockSpaceManager(sliding_window=...)): with window W > 0
  * a sequence of length L only needs its last W positions, [max(0, L - W), L), so a
  * block that lies wholly before them ((j + 1) * bs <= L - W for table index j) is
- * returned to the pool as soon as the length passes that point (allocate,
- * append_slots) and its table entry becomes -1; pa_decode with the same
- * sliding_window never reads such an entry.  A new sequence takes only the blocks of
- * its window.  Blocks that fall out of the window during pa_bm_append_slots are given
- * back after the whole batch has its slots (so its all-or-nothing check counts only
- * blocks that were free before the call).  pa_bm_slot of a released position is -1.
+ * returned to the pool at the sequence's next pa_bm_append_slots and its table entry
+ * becomes -1; pa_decode with the same sliding_window never reads such an entry.  A
+ * new sequence takes the blocks of all its tokens (its prompt is written and
+ * attended in full, as pa_prefill with a window needs the W - 1 tokens before its
+ * first query).  Blocks that fall out of the window during pa_bm_append_slots are
+ * given back after the whole batch has its slots (so its all-or-nothing check counts
+ * only blocks that were free before the call).  pa_bm_slot of a released position is
+ * -1.
  * Only while the manager holds no sequence; 0 = whole contexts (the default).
  */
 pa_status pa_bm_set_sliding_window(pa_block_manager *bm, int window);
@@ -64,8 +66,7 @@ int pa_bm_num_free_blocks(const pa_block_manager *bm);
 /* used blocks / pool blocks. */
 double pa_bm_usage_ratio(const pa_block_manager *bm);
 
-/* 1 if a new sequence of num_tokens tokens fits in the free blocks, else 0 (under a
- * sliding window: the blocks of its window). */
+/* 1 if a new sequence of num_tokens tokens fits in the free blocks, else 0. */
 int pa_bm_can_allocate(const pa_block_manager *bm, int num_tokens);
 
 /* New sequence holding num_tokens tokens (a prompt): ceil(num_tokens / bs) fresh

@@ -42,10 +42,6 @@ struct pa_block_manager {
     int blocks_before_window(int n) const {
         return (window > 0 && n > window) ? (n - window) / block_size : 0;
     }
-    // Blocks a new sequence of n tokens holds.
-    int live_blocks(int n) const {
-        return (int)(((long long)n + block_size - 1) / block_size) - blocks_before_window(n);
-    }
     void release_before_window(Seq &s) {
         const int upto = blocks_before_window(s.len);
         for (int j = s.first_live; j < upto; ++j) {
@@ -186,21 +182,20 @@ double pa_bm_usage_ratio(const pa_block_manager *bm) {
 
 int pa_bm_can_allocate(const pa_block_manager *bm, int num_tokens) {
     if (!bm) return 0;
-    if (num_tokens < 0) return 0;
-    return bm->live_blocks(num_tokens) <= (int)bm->free_list.size();
+    const int need = pa_bm_blocks_needed(num_tokens, bm->block_size);
+    return need >= 0 && need <= (int)bm->free_list.size();
 }
 
 pa_status pa_bm_allocate(pa_block_manager *bm, int64_t seq_id, int num_tokens) {
     if (!bm || num_tokens < 0 || bm->seqs.count(seq_id)) return PA_ERR_INVALID_ARG;
-    const int before = bm->blocks_before_window(num_tokens);
-    const int need = bm->live_blocks(num_tokens);
+    // every token of a prompt is written and attended (prefill), so a new sequence
+    // takes all its blocks; those before the window go back at its next append
+    const int need = pa_bm_blocks_needed(num_tokens, bm->block_size);
     if (need > (int)bm->free_list.size()) return PA_ERR_NO_FREE_BLOCK;
     pa_block_manager::Seq s;
-    s.blocks.assign(before, -1);
-    s.blocks.reserve(before + need);
+    s.blocks.reserve(need);
     for (int i = 0; i < need; ++i) s.blocks.push_back(bm->take());
     s.len = num_tokens;
-    s.first_live = before;
     bm->seqs.emplace(seq_id, std::move(s));
     return PA_OK;
 }

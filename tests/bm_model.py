@@ -8,8 +8,9 @@ handed out last-returned-first, lowest id first at the start.
 
 Sliding window W (the blog's sliding_window setting, read as: a sequence of length L
 needs only positions L-W .. L-1): a block whose positions all lie before L-W is given
-back and its table entry becomes None; a new sequence never takes those blocks; after
-an append batch the sequences of the batch give back what fell out of their window.
+back and its table entry becomes None.  A new sequence takes the blocks of all its
+tokens (the prompt is attended in full); after an append batch the sequences of the
+batch give back what fell out of their window.
 """
 
 
@@ -47,11 +48,10 @@ class Model:
     def allocate(self, sid, n):
         if sid in self.seqs:
             raise KeyError(sid)
-        dead = self._dead(n)
-        need = -(-n // self.bs) - dead
+        need = -(-n // self.bs)
         if need > len(self.free_ids):
             raise NoBlocks()
-        self.seqs[sid] = ([None] * dead + [self._take() for _ in range(need)], n)
+        self.seqs[sid] = ([self._take() for _ in range(need)], n)
 
     def _trim(self, sid):
         blocks, n = self.seqs[sid]
