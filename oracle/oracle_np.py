@@ -70,6 +70,44 @@ def decode(q, k_cache, v_cache, block_tables, context_lens, scale, dtype,
     return out
 
 
+def prefill(q, k_cache, v_cache, block_tables, context_lens, query_start_loc, scale, dtype,
+            sliding_window: int = 0) -> np.ndarray:
+    """Causal multi-query attention: per sequence, the chunk Q [n, Hq, d] against the whole
+    gathered context K, V [L, d], with the score matrix masked where key t is after the
+    query's position L - n + i (or more than sliding_window - 1 before it)."""
+    qf = widen(q, dtype)
+    kf = widen(k_cache, dtype)
+    vf = widen(v_cache, dtype)
+    T, hq, d = qf.shape
+    hkv = kf.shape[1]
+    G = hq // hkv
+    out = np.zeros((T, hq, d), np.float64)
+    qsl = np.asarray(query_start_loc, dtype=np.int64)
+    for s in range(len(qsl) - 1):
+        a, b = int(qsl[s]), int(qsl[s + 1])
+        n, L = b - a, int(context_lens[s])
+        if n == 0:
+            continue
+        # the earliest position any query of the chunk attends (pages before it are
+        # never read: under a window they may have been given back)
+        lo = max(0, L - n - sliding_window + 1) if sliding_window > 0 else 0
+        pos = np.arange(L - n, L)[:, None]  # [n, 1]
+        t = np.arange(lo, L)[None, :]  # [1, L - lo]
+        allowed = t <= pos
+        if sliding_window > 0:
+            allowed &= t > pos - sliding_window
+        for g in range(hkv):
+            K = gather_positions(kf, block_tables[s], lo, L, g)
+            V = gather_positions(vf, block_tables[s], lo, L, g)
+            Q = qf[a:b, g * G:(g + 1) * G]  # [n, G, d]
+            z = scale * np.einsum("ngd,td->ngt", Q, K)
+            z = np.where(allowed[:, None, :], z, -np.inf)
+            z = z - z.max(axis=2, keepdims=True)
+            w = np.exp(z)
+            out[a:b, g * G:(g + 1) * G] = np.einsum("ngt,td->ngd", w, V) / w.sum(axis=2)[..., None]
+    return out
+
+
 def kv_write(key, value, slot_mapping, k_cache, v_cache) -> None:
     bs = k_cache.shape[2]
     for t, slot in enumerate(np.asarray(slot_mapping, dtype=np.int64)):

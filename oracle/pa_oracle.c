@@ -210,6 +210,51 @@ int orc_decode(double *out, const uint16_t *q, const uint16_t *k_cache, const ui
                              max_blocks_per_seq, scale, dtype, 0, sel, n_sel, nthreads);
 }
 
+/* Multi-query (prefill / chunked prefill) attention over the paged cache: section 4
+ * of the "IO-5 vLLM Paged Attention" note with a matrix Q (one row per new token of a
+ * request, as continuous batching -- section 6 -- brings new requests' prompts into
+ * the batch).  Reading where the pages are silent: causal, as in an autoregressive
+ * model -- the chunk's n tokens sit at positions L - n .. L - 1 of a context of L
+ * tokens already in the cache, and the token at position p attends to positions
+ * 0 .. p (the last `window` of them under a sliding window).  That is exactly the
+ * decode attention of a context of length p + 1, which is how it is evaluated here.
+ *
+ * q, out: [num_tokens][num_q_heads][head_dim] (out fp64); the tokens of sequence s are
+ * rows query_start_loc[s] .. query_start_loc[s+1]-1.  Returns the number of
+ * (token, head) outputs that could not be computed (chunk longer than its context,
+ * or an out-of-range table entry). */
+int orc_prefill(double *out, const uint16_t *q, const uint16_t *k_cache, const uint16_t *v_cache,
+                const int32_t *block_tables, const int32_t *context_lens,
+                const int32_t *query_start_loc, int num_seqs, int num_tokens, int num_q_heads,
+                int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                int max_blocks_per_seq, double scale, int dtype, int window, int nthreads) {
+    int n_items = num_tokens * num_q_heads;
+    int bad = 0;
+#ifdef _OPENMP
+    if (nthreads <= 0) nthreads = omp_get_max_threads();
+#pragma omp parallel for schedule(dynamic, 4) num_threads(nthreads) reduction(+ : bad)
+#endif
+    for (int i = 0; i < n_items; ++i) {
+        int tok = i / num_q_heads, h = i % num_q_heads;
+        double *o = out + (size_t)i * head_dim;
+        for (int e = 0; e < head_dim; ++e) o[e] = 0.0;
+        int s = 0;
+        while (s < num_seqs && !(query_start_loc[s] <= tok && tok < query_start_loc[s + 1])) ++s;
+        if (s == num_seqs) { ++bad; continue; }
+        int n = query_start_loc[s + 1] - query_start_loc[s];
+        int L = context_lens[s];
+        if (n > L || L > max_blocks_per_seq * block_size) { ++bad; continue; }
+        int pos = L - n + (tok - query_start_loc[s]);
+        const int32_t *table = block_tables + (size_t)s * max_blocks_per_seq;
+        if (orc_one(o, q + (size_t)i * head_dim, k_cache, v_cache, table, pos + 1, h,
+                    num_q_heads, num_kv_heads, head_dim, block_size, num_blocks, scale, dtype,
+                    window) != 0)
+            ++bad;
+    }
+    (void)nthreads;
+    return bad;
+}
+
 /* Threads the OpenMP runtime would use (1 without OpenMP). */
 int orc_max_threads(void) {
 #ifdef _OPENMP

@@ -13,7 +13,9 @@ Each ``pin_*`` takes a loaded oracle library (ctypes handle) and raises
 * exact library conversions of the 16-bit formats (numpy float16, torch bfloat16);
 * the independent numpy statement in ``oracle/oracle_np.py``;
 * for the sliding window: the last token's V exactly at W = 1, and torch fp64
-  attention on the last W contiguous rows.
+  attention on the last W contiguous rows;
+* for multi-query (prefill) attention: torch fp64 attention with its causal path or
+  a tril/triu mask on the contiguous K/V, and the one-token chunk equal to decode.
 
 The same functions run against deliberately broken copies of the oracle in
 ``test_oracle_mutants.py``, which checks that each plausible mistake trips a pin.
@@ -458,10 +460,80 @@ def pin_window_vs_sdpa(lib):
         assert np.max(np.abs(out - npv)) < 1e-12, W
 
 
+# ------------------------------------------------------------- multi-query (prefill)
+
+def _prefill_case(rng, specs, hq, hkv, d, bs, dtype="bf16"):
+    """specs: [(n, L)] per sequence -> contiguous K/V, pool, tables, q, qsl."""
+    lens = [L for _, L in specs]
+    nb = sum(-(-L // bs) for L in lens) + 3
+    Ks = [_rand_bits(rng, (L, hkv, d), dtype) for L in lens]
+    Vs = [_rand_bits(rng, (L, hkv, d), dtype) for L in lens]
+    tabs = _tables_for(rng, lens, bs, nb)
+    kc, vc, bt = build_pool(Ks, Vs, tabs, nb, bs)
+    qsl = np.concatenate([[0], np.cumsum([n for n, _ in specs])]).astype(np.int32)
+    q = _rand_bits(rng, (int(qsl[-1]), hq, d), dtype)
+    return Ks, Vs, tabs, kc, vc, bt, q, qsl, np.array(lens, np.int32)
+
+
+def pin_prefill_vs_sdpa(lib):
+    """Causal multi-query attention == torch fp64 scaled-dot-product attention on the
+    contiguous K/V: torch's own causal path when the chunk is the whole context, a
+    lower-triangular mask aligned to the last query (torch.tril) for a chunk that
+    follows earlier context, and that mask cut to the last W keys (torch.triu) under a
+    sliding window, with the pages before the first query's window given back (-1)."""
+    import torch
+    import torch.nn.functional as F
+    rng = np.random.default_rng(23)
+    hq, hkv, d, bs = 4, 2, 16, 4
+    specs = [(9, 9), (5, 13), (1, 7), (17, 17), (3, 30)]
+    Ks, Vs, tabs, kc, vc, bt_full, q, qsl, cl = _prefill_case(rng, specs, hq, hkv, d, bs)
+    G = hq // hkv
+    for W in (0, 1, 3, 7, 100):
+        bt = bt_full.copy()
+        if W:
+            for s, (n, L) in enumerate(specs):
+                lo = max(0, L - n - W + 1)
+                bt[s, :lo // bs] = -1
+        out, bad = oracle.prefill(q, kc, vc, bt, cl, qsl, 0.3, "bf16", sliding_window=W,
+                                  lib=lib, return_bad=True)
+        assert bad == 0, W
+        for s, (n, L) in enumerate(specs):
+            a = int(qsl[s])
+            qt = torch.from_numpy(bits_to_f32(q[a:a + n], "bf16").astype(np.float64))
+            qt = qt.permute(1, 0, 2)[None]  # [1, hq, n, d]
+            kt = torch.from_numpy(bits_to_f32(Ks[s], "bf16").astype(np.float64))
+            vt = torch.from_numpy(bits_to_f32(Vs[s], "bf16").astype(np.float64))
+            kt = kt.permute(1, 0, 2).repeat_interleave(G, dim=0)[None]
+            vt = vt.permute(1, 0, 2).repeat_interleave(G, dim=0)[None]
+            if W == 0 and n == L:
+                ref = F.scaled_dot_product_attention(qt, kt, vt, is_causal=True, scale=0.3)
+            else:
+                mask = torch.ones(n, L, dtype=torch.bool).tril(diagonal=L - n)
+                if W:
+                    mask &= torch.ones(n, L, dtype=torch.bool).triu(diagonal=L - n - W + 1)
+                ref = F.scaled_dot_product_attention(qt, kt, vt, attn_mask=mask, scale=0.3)
+            ref = ref[0].permute(1, 0, 2).numpy()  # [n, hq, d]
+            assert np.max(np.abs(out[a:a + n] - ref)) < 1e-12, (W, s)
+        npv = oracle_np.prefill(q, kc, vc, bt, cl, qsl, 0.3, "bf16", sliding_window=W)
+        assert np.max(np.abs(out - npv)) < 1e-12, W
+
+
+def pin_prefill_one_token_is_decode(lib):
+    """A chunk of one token at the end of its context is the decode step (whose oracle
+    the decode pins tie down), with and without a window."""
+    rng = np.random.default_rng(24)
+    specs = [(1, 1), (1, 8), (1, 9), (1, 40)]
+    _, _, _, kc, vc, bt, q, qsl, cl = _prefill_case(rng, specs, 8, 2, 16, 8)
+    for W in (0, 5):
+        a = oracle.prefill(q, kc, vc, bt, cl, qsl, 0.25, "bf16", sliding_window=W, lib=lib)
+        b = oracle.decode(q, kc, vc, bt, cl, 0.25, "bf16", sliding_window=W, lib=lib)
+        assert np.array_equal(a, b), W
+
+
 ALL_PINS = [pin_two_token, pin_len1_exact, pin_identical_keys, pin_zero_len, pin_paged_vs_sdpa,
             pin_block_size_and_permutation, pin_shared_prefix, pin_golden_examples,
             pin_widening, pin_c_vs_numpy, pin_kv_write, pin_copy_blocks, pin_window_last_token,
-            pin_window_vs_sdpa]
+            pin_window_vs_sdpa, pin_prefill_vs_sdpa, pin_prefill_one_token_is_decode]
 
 
 def run_all(lib):

@@ -33,6 +33,12 @@ MUTANTS = [
     ("window_one_long", "int t_lo = (window > 0 && L > window) ? L - window : 0;",
      "int t_lo = (window > 0 && L > window) ? L - window - 1 : 0;"),
     ("window_ignored", "int t_lo = (window > 0 && L > window) ? L - window : 0;", "int t_lo = 0;"),
+    ("prefill_pos_early", "int pos = L - n + (tok - query_start_loc[s]);",
+     "int pos = L - n + (tok - query_start_loc[s]) - 1;"),
+    ("prefill_pos_late", "int pos = L - n + (tok - query_start_loc[s]);",
+     "int pos = L - n + (tok - query_start_loc[s]) + (n < L);"),
+    ("prefill_wrong_seq", "query_start_loc[s] <= tok && tok < query_start_loc[s + 1]",
+     "query_start_loc[s] <= tok && tok <= query_start_loc[s + 1]"),
 ]
 
 
