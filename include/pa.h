@@ -246,6 +246,37 @@ pa_status pa_decode_static_scratch(void *out, const void *q, const void *k_cache
                                    int partition_size, pa_dtype dtype, void *stream);
 
 /*
+ * Multi-query attention over the paged cache: prefill and chunked prefill ("IO-5 vLLM
+ * Paged Attention" note, section 4, Attention(Q, K, V) = softmax(Q K^T / sqrt(d_k)) V
+ * with a matrix Q: the new tokens of requests that continuous batching -- section 6 --
+ * adds to the batch).  The tokens of sequence s are rows query_start_loc[s] ..
+ * query_start_loc[s+1]-1 of q (n_s of them); their K and V are already in the cache
+ * (pa_kv_write), which holds L_s = context_lens[s] >= n_s tokens of the sequence, so
+ * token i of the chunk is at position p = L_s - n_s + i.  It attends causally:
+ *   out[t][h][:] = sum_{u <= p} softmax_u(scale * <q[t][h], K_s[u]>) V_s[u],  g = h / G,
+ * over u in [max(0, p - W + 1), p] under a sliding window W > 0 (the table must then
+ * hold the pages from position L_s - n_s - W + 1 on; earlier entries are never read).
+ * Causality is the reading taken where the pages are silent (autoregressive models).
+ * A chunk of one token is a decode step; pa_decode is the faster call for those.
+ *
+ * q, out          : [num_tokens][num_q_heads][head_dim], contiguous, 16-byte aligned.
+ * query_start_loc : int32 [num_seqs + 1], non-decreasing, [0] = 0, [num_seqs] = num_tokens.
+ * Other arguments : as pa_decode (head_dim 64 or 128, G in {1, 2, 4, 8}, block_size a
+ *                   power of two in [8, 512]).
+ * Math: S = Q K^T and O = P V on the tcgen05 tensor cores (fp32 accumulation in tensor
+ * memory), softmax in fp32 with P rounded to the input type for the P V product.
+ * One launch, no workspace.  Errors: host-checkable problems as pa_decode; n_s > L_s
+ * or L_s beyond the table sets PA_DEVERR_CONTEXT (that sequence's rows are not
+ * written); an out-of-range table entry sets PA_DEVERR_BLOCK_ID.
+ */
+pa_status pa_prefill(void *out, const void *q, const void *k_cache, const void *v_cache,
+                     const int32_t *block_tables, const int32_t *context_lens,
+                     const int32_t *query_start_loc, int num_seqs, int num_tokens,
+                     int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                     int num_blocks, int max_blocks_per_seq, float scale, int sliding_window,
+                     pa_dtype dtype, void *stream);
+
+/*
  * Reads (and with clear != 0 resets) the sticky error word of `device`.
  * SYNCHRONISES that device first.  *bits_out receives PA_DEVERR_* bits (0 = none).
  */

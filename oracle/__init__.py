@@ -56,7 +56,7 @@ def _declare(lib):
                                       i32, i32, P, i32, i32]
     lib.orc_decode_window.restype = i32
     lib.orc_prefill.argtypes = [P, P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, i32, i32, dbl,
-                                i32, i32, i32]
+                                i32, i32, P, i32, i32]
     lib.orc_prefill.restype = i32
     lib.orc_max_threads.argtypes = []
     lib.orc_max_threads.restype = i32
@@ -113,9 +113,10 @@ def decode(q, k_cache, v_cache, block_tables, context_lens, scale, dtype, num_q_
 
 
 def prefill(q, k_cache, v_cache, block_tables, context_lens, query_start_loc, scale, dtype,
-            sliding_window=0, nthreads=0, lib=None, return_bad=False):
-    """fp64 causal multi-query attention, [num_tokens, Hq, d]: token i of sequence s sits
-    at position context_lens[s] - n_s + i and attends to positions up to its own."""
+            sliding_window=0, sel=None, nthreads=0, lib=None, return_bad=False):
+    """fp64 causal multi-query attention, [num_tokens, Hq, d] (or [len(sel), d] for the
+    selected (token, head) pairs): token i of sequence s sits at position
+    context_lens[s] - n_s + i and attends to positions up to its own."""
     lib = lib or load()
     q = np.ascontiguousarray(q, np.uint16)
     kc = np.ascontiguousarray(k_cache, np.uint16)
@@ -125,10 +126,17 @@ def prefill(q, k_cache, v_cache, block_tables, context_lens, query_start_loc, sc
     qsl = np.ascontiguousarray(query_start_loc, np.int32)
     T, hq, d = q.shape
     nb, hkv, bs, _ = kc.shape
-    out = np.zeros((T, hq, d), np.float64)
-    bad = lib.orc_prefill(_p(out), _p(q), _p(kc), _p(vc), _p(bt), _p(cl), _p(qsl),
-                          qsl.shape[0] - 1, T, hq, hkv, d, bs, nb, bt.shape[1], float(scale),
-                          _dt(dtype), int(sliding_window), nthreads)
+    if sel is not None:
+        sel = np.ascontiguousarray(sel, np.int32).reshape(-1, 2)
+        out = np.zeros((sel.shape[0], d), np.float64)
+        bad = lib.orc_prefill(_p(out), _p(q), _p(kc), _p(vc), _p(bt), _p(cl), _p(qsl),
+                              qsl.shape[0] - 1, T, hq, hkv, d, bs, nb, bt.shape[1], float(scale),
+                              _dt(dtype), int(sliding_window), _p(sel), sel.shape[0], nthreads)
+    else:
+        out = np.zeros((T, hq, d), np.float64)
+        bad = lib.orc_prefill(_p(out), _p(q), _p(kc), _p(vc), _p(bt), _p(cl), _p(qsl),
+                              qsl.shape[0] - 1, T, hq, hkv, d, bs, nb, bt.shape[1], float(scale),
+                              _dt(dtype), int(sliding_window), None, 0, nthreads)
     return (out, bad) if return_bad else out
 
 

@@ -220,22 +220,25 @@ int orc_decode(double *out, const uint16_t *q, const uint16_t *k_cache, const ui
  * decode attention of a context of length p + 1, which is how it is evaluated here.
  *
  * q, out: [num_tokens][num_q_heads][head_dim] (out fp64); the tokens of sequence s are
- * rows query_start_loc[s] .. query_start_loc[s+1]-1.  Returns the number of
- * (token, head) outputs that could not be computed (chunk longer than its context,
+ * rows query_start_loc[s] .. query_start_loc[s+1]-1.  With sel != NULL only the n_sel
+ * (token, head) pairs sel[2i], sel[2i+1] are computed, into out[i][head_dim].  Returns
+ * the number of outputs that could not be computed (chunk longer than its context,
  * or an out-of-range table entry). */
 int orc_prefill(double *out, const uint16_t *q, const uint16_t *k_cache, const uint16_t *v_cache,
                 const int32_t *block_tables, const int32_t *context_lens,
                 const int32_t *query_start_loc, int num_seqs, int num_tokens, int num_q_heads,
                 int num_kv_heads, int head_dim, int block_size, int num_blocks,
-                int max_blocks_per_seq, double scale, int dtype, int window, int nthreads) {
-    int n_items = num_tokens * num_q_heads;
+                int max_blocks_per_seq, double scale, int dtype, int window, const int32_t *sel,
+                int n_sel, int nthreads) {
+    int n_items = sel ? n_sel : num_tokens * num_q_heads;
     int bad = 0;
 #ifdef _OPENMP
     if (nthreads <= 0) nthreads = omp_get_max_threads();
 #pragma omp parallel for schedule(dynamic, 4) num_threads(nthreads) reduction(+ : bad)
 #endif
     for (int i = 0; i < n_items; ++i) {
-        int tok = i / num_q_heads, h = i % num_q_heads;
+        int tok = sel ? sel[2 * i] : i / num_q_heads;
+        int h = sel ? sel[2 * i + 1] : i % num_q_heads;
         double *o = out + (size_t)i * head_dim;
         for (int e = 0; e < head_dim; ++e) o[e] = 0.0;
         int s = 0;
@@ -246,7 +249,8 @@ int orc_prefill(double *out, const uint16_t *q, const uint16_t *k_cache, const u
         if (n > L || L > max_blocks_per_seq * block_size) { ++bad; continue; }
         int pos = L - n + (tok - query_start_loc[s]);
         const int32_t *table = block_tables + (size_t)s * max_blocks_per_seq;
-        if (orc_one(o, q + (size_t)i * head_dim, k_cache, v_cache, table, pos + 1, h,
+        if (orc_one(o, q + ((size_t)tok * num_q_heads + h) * head_dim, k_cache, v_cache, table,
+                    pos + 1, h,
                     num_q_heads, num_kv_heads, head_dim, block_size, num_blocks, scale, dtype,
                     window) != 0)
             ++bad;

@@ -11,8 +11,12 @@ The compute lives in ``libpa.so`` (CUDA kernels behind the C ABI in
   log-sum-exp merge; GQA served from one page read per kv head);
 * ``decode_append(out, q, key, value, k_cache, v_cache, ...)`` -- the step's cache
   write fused into the decode;
+* ``prefill(out, q, k_cache, v_cache, block_tables, context_lens, query_start_loc,
+  scale)`` -- causal multi-query attention for prompts and prompt chunks (tcgen05);
+* ``swap_blocks(...)`` -- block copies between the GPU cache and a pinned host pool;
 * ``BlockManager`` -- the host owner of the page tables: on-demand allocation,
-  fork (shared blocks), copy-on-write pairs, free, usage ratio.
+  fork (shared blocks), copy-on-write pairs, free, usage ratio, swap, sliding window.
+Every attention call takes ``sliding_window`` (0 = whole context).
 """
 from ._lib import (  # noqa: F401
     DEVERR,
@@ -29,6 +33,7 @@ from ._lib import (  # noqa: F401
     device_error,
     kv_write,
     load,
+    prefill,
     swap_blocks,
     version,
 )

@@ -16,7 +16,7 @@ PA_FP16, PA_BF16 = 0, 1
 DEVERR = {"block_id": 0x1, "slot": 0x2, "pair": 0x4, "context": 0x8, "timeout": 0x10}
 EXPORTS = ("pa_kv_write", "pa_copy_blocks", "pa_decode", "pa_decode_workspace_bytes",
            "pa_decode_partition_tokens", "pa_get_device_error", "pa_status_str", "pa_version",
-           "pa_decode_static_scratch", "pa_decode_append", "pa_swap_blocks",
+           "pa_decode_static_scratch", "pa_decode_append", "pa_swap_blocks", "pa_prefill",
            # host block manager (include/pa_block_manager.h)
            "pa_bm_create", "pa_bm_destroy", "pa_bm_blocks_needed", "pa_bm_num_free_blocks",
            "pa_bm_usage_ratio", "pa_bm_can_allocate", "pa_bm_allocate", "pa_bm_fork",
@@ -63,6 +63,9 @@ def load(path: str = LIB_PATH):
     lib.pa_decode_append.argtypes = [P, P, P, P, i64, i64, P, P, P, P, i32, i32, i32, i32, i32,
                                      i32, i32, f32, i32, i32, i32, P, sz, i32, P]
     lib.pa_decode_append.restype = i32
+    lib.pa_prefill.argtypes = [P, P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, i32, i32, f32,
+                               i32, i32, P]
+    lib.pa_prefill.restype = i32
     lib.pa_get_device_error.argtypes = [i32, ctypes.POINTER(ctypes.c_uint32), i32]
     lib.pa_get_device_error.restype = i32
     lib.pa_status_str.argtypes = [i32]
@@ -214,6 +217,22 @@ def decode_static_scratch(out, q, k_cache, v_cache, block_tables, context_lens, 
         _ptr(context_lens), B, hq, hkv, d, bs, nb, W, float(scale), int(max_context_len),
         int(sliding_window), int(partition_size), _dtype(q), _stream(stream)),
         "pa_decode_static_scratch")
+
+
+def prefill(out, q, k_cache, v_cache, block_tables, context_lens, query_start_loc, scale,
+            sliding_window=0, stream=None) -> None:
+    """Causal multi-query attention: q, out [T, Hq, d] (the new tokens of every sequence,
+    sequence s in rows query_start_loc[s] .. [s+1]); caches [NB, Hkv, bs, d];
+    block_tables int32 [B, W]; context_lens int32 [B] (tokens in the cache, the chunk
+    included); query_start_loc int32 [B + 1]."""
+    T, hq, d = q.shape
+    nb, hkv, bs, _ = k_cache.shape
+    B = context_lens.shape[0]
+    assert query_start_loc.shape[0] == B + 1
+    _check(load().pa_prefill(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                             _ptr(block_tables), _ptr(context_lens), _ptr(query_start_loc), B, T,
+                             hq, hkv, d, bs, nb, block_tables.shape[1], float(scale),
+                             int(sliding_window), _dtype(q), _stream(stream)), "pa_prefill")
 
 
 def device_error(device: int = 0, clear: bool = True) -> int:

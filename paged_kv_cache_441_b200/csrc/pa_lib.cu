@@ -13,6 +13,7 @@
 #include "pa_decode.cuh"
 #include "pa_merge.cuh"
 #include "pa_decode_streamk.cuh"
+#include "pa_prefill.cuh"
 
 using namespace pa;
 
@@ -62,6 +63,24 @@ bool make_cache_map(CUtensorMap *m, const void *base, unsigned long long rows, i
     cuuint32_t box[2] = {64u, (cuuint32_t)boxr};
     cuuint32_t estr[2] = {1u, 1u};
     return enc(m, t, 2, const_cast<void *>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 3-D map over q [num_tokens][Hq][D]: box 64 columns x G heads x 128/G tokens (the
+// 128 query rows of one kv head's group), 128-byte swizzle.
+bool make_q_map(CUtensorMap *m, const void *base, int num_tokens, int Hq, int D, int G,
+                pa_dtype dt) {
+    auto enc = encode_fn();
+    if (!enc) return false;
+    const CUtensorMapDataType t =
+        dt == PA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)Hq, (cuuint64_t)num_tokens};
+    cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)Hq * D * 2};
+    cuuint32_t box[3] = {64u, (cuuint32_t)G, (cuuint32_t)(kPfRows / G)};
+    cuuint32_t estr[3] = {1u, 1u, 1u};
+    return enc(m, t, 3, const_cast<void *>(base), dims, strides, box, estr,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
@@ -297,6 +316,34 @@ cudaError_t sk_merge(const SkMergeParams &p, dim3 grid, int D, cudaStream_t st) 
     return D == 64 ? launch_pdl(pa_merge_streamk_kernel<T, 64>, grid, dim3(kMergeThreads), 0, st, p)
                    : launch_pdl(pa_merge_streamk_kernel<T, 128>, grid, dim3(kMergeThreads), 0, st,
                                 p);
+}
+
+template <typename T, int D, int G>
+cudaError_t launch_prefill(const PrefillParams &p, dim3 grid, cudaStream_t st, int dev) {
+    static std::atomic<bool> flags[kMaxDevices];
+    auto kernel = pa_prefill_kernel<T, D, G>;
+    cudaError_t e = ensure_smem(kernel, PfGeom<D>::kSmem, flags, dev);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(kernel, grid, dim3(kPfThreads), PfGeom<D>::kSmem, st, p);
+}
+
+template <typename T, int D>
+cudaError_t prefill_dispatch_group(const PrefillParams &p, dim3 grid, cudaStream_t st, int dev,
+                                   int G) {
+    switch (G) {
+        case 1: return launch_prefill<T, D, 1>(p, grid, st, dev);
+        case 2: return launch_prefill<T, D, 2>(p, grid, st, dev);
+        case 4: return launch_prefill<T, D, 4>(p, grid, st, dev);
+        case 8: return launch_prefill<T, D, 8>(p, grid, st, dev);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+template <typename T>
+cudaError_t prefill_dispatch(const PrefillParams &p, dim3 grid, cudaStream_t st, int dev, int D,
+                             int G) {
+    return D == 64 ? prefill_dispatch_group<T, 64>(p, grid, st, dev, G)
+                   : prefill_dispatch_group<T, 128>(p, grid, st, dev, G);
 }
 
 pa_status check_decode_shape(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
@@ -745,4 +792,70 @@ extern "C" pa_status pa_decode_static_scratch(
                      num_kv_heads, head_dim, block_size, num_blocks, max_blocks_per_seq, scale,
                      max_context_len, sliding_window, partition_size, scratch,
                      pl.ws_bytes > 0 ? (size_t)PA_STATIC_SCRATCH_BYTES : 0, dtype, stream);
+}
+
+// ------------------------------------------------------------------------------
+// Multi-query (prefill / chunked prefill) attention on the tcgen05 tensor cores.
+
+extern "C" pa_status pa_prefill(void *out, const void *q, const void *k_cache,
+                                const void *v_cache, const int32_t *block_tables,
+                                const int32_t *context_lens, const int32_t *query_start_loc,
+                                int num_seqs, int num_tokens, int num_q_heads, int num_kv_heads,
+                                int head_dim, int block_size, int num_blocks,
+                                int max_blocks_per_seq, float scale, int sliding_window,
+                                pa_dtype dtype, void *stream) {
+    if (dtype != PA_FP16 && dtype != PA_BF16) return PA_ERR_INVALID_ARG;
+    if (num_seqs < 0 || num_tokens < 0 || num_q_heads <= 0 || num_kv_heads <= 0 ||
+        num_blocks <= 0 || max_blocks_per_seq <= 0 || sliding_window < 0 ||
+        !std::isfinite(scale))
+        return PA_ERR_INVALID_ARG;
+    if (num_q_heads % num_kv_heads != 0) return PA_ERR_INVALID_ARG;
+    const int G = num_q_heads / num_kv_heads;
+    if (G != 1 && G != 2 && G != 4 && G != 8) return PA_ERR_UNSUPPORTED;
+    if (head_dim != 64 && head_dim != 128) return PA_ERR_UNSUPPORTED;
+    if (!pow2(block_size) || block_size < 8 || block_size > 512) return PA_ERR_UNSUPPORTED;
+    if ((unsigned long long)num_blocks * num_kv_heads * block_size >= (1ull << 31))
+        return PA_ERR_UNSUPPORTED;
+    if ((long long)max_blocks_per_seq * block_size >= (1ll << 31)) return PA_ERR_INVALID_ARG;
+    if (num_kv_heads > 65535) return PA_ERR_UNSUPPORTED;
+    if (num_seqs == 0 || num_tokens == 0) return PA_OK;
+    if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens || !query_start_loc)
+        return PA_ERR_INVALID_ARG;
+    if (!aligned(out, 16) || !aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
+        !aligned(block_tables, 4) || !aligned(context_lens, 4) || !aligned(query_start_loc, 4))
+        return PA_ERR_INVALID_ARG;
+    const int dev = current_device();
+    PrefillParams p;
+    std::memset(&p, 0, sizeof p);
+    const int boxr = block_size < kPfKeys ? block_size : kPfKeys;
+    const unsigned long long rows = (unsigned long long)num_blocks * num_kv_heads * block_size;
+    if (!make_q_map(&p.qmap, q, num_tokens, num_q_heads, head_dim, G, dtype) ||
+        !make_cache_map(&p.kmap, k_cache, rows, head_dim, dtype, boxr) ||
+        !make_cache_map(&p.vmap, v_cache, rows, head_dim, dtype, boxr))
+        return PA_ERR_CUDA;
+    p.out = out;
+    p.block_tables = block_tables;
+    p.context_lens = context_lens;
+    p.query_start_loc = query_start_loc;
+    p.num_seqs = num_seqs;
+    p.num_tokens = num_tokens;
+    p.num_q_heads = num_q_heads;
+    p.num_kv_heads = num_kv_heads;
+    p.block_size = block_size;
+    p.bs_shift = ilog2_host(block_size);
+    p.box_rows = boxr;
+    p.num_blocks = num_blocks;
+    p.max_blocks_per_seq = max_blocks_per_seq;
+    p.sliding_window = sliding_window;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    // sum over sequences of ceil(n_s / tpt) <= num_tokens / tpt + num_seqs
+    const long long tpt = kPfRows / G;
+    const long long tiles = (long long)num_tokens / tpt + num_seqs;
+    if (tiles >= (1ll << 31)) return PA_ERR_UNSUPPORTED;
+    const dim3 grid((unsigned)tiles, (unsigned)num_kv_heads);
+    cudaStream_t st_ = static_cast<cudaStream_t>(stream);
+    const cudaError_t e = dtype == PA_BF16
+                              ? prefill_dispatch<__nv_bfloat16>(p, grid, st_, dev, head_dim, G)
+                              : prefill_dispatch<__half>(p, grid, st_, dev, head_dim, G);
+    return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }

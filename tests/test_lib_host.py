@@ -121,3 +121,24 @@ def test_kv_write_and_copy_reject(lib):
     assert lib.pa_kv_write(P(16), P(16), P(16), 1, 2, 12, 24, 24, P(16), P(16), 10, 16, 1, None) == 1
     assert lib.pa_copy_blocks(P(16), P(16), None, 3, 2, 16, 128, 10, 1, None) == 1
     assert lib.pa_copy_blocks(P(16), P(16), P(8), 3, 2, 16, 128, 0, 1, None) == 1
+
+
+def _call_prefill(lib, **over):
+    a = dict(out=16, q=16, kc=16, vc=16, bt=16, cl=16, qsl=16, B=2, T=10, hq=8, hkv=2, d=128,
+             bs=16, nb=10, W=4, scale=0.1, win=0, dt=1, stream=None)
+    a.update(over)
+    P = ctypes.c_void_p
+    return lib.pa_prefill(P(a["out"]), P(a["q"]), P(a["kc"]), P(a["vc"]), P(a["bt"]), P(a["cl"]),
+                          P(a["qsl"]), a["B"], a["T"], a["hq"], a["hkv"], a["d"], a["bs"],
+                          a["nb"], a["W"], a["scale"], a["win"], a["dt"], a["stream"])
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(d=96), 2), (dict(hq=6), 2), (dict(hq=7), 1), (dict(hq=32), 2), (dict(bs=24), 2),
+    (dict(bs=1024), 2), (dict(q=0), 1), (dict(q=24), 1), (dict(qsl=0), 1), (dict(qsl=2), 1),
+    (dict(win=-1), 1), (dict(scale=float("nan")), 1), (dict(dt=7), 1), (dict(T=-1), 1),
+    (dict(B=0), 0), (dict(T=0), 0),
+])
+def test_prefill_rejects_before_launch(lib, over, code):
+    # every case is settled by host checks (or has nothing to do): no CUDA call is made
+    assert _call_prefill(lib, **over) == code

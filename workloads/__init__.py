@@ -14,4 +14,8 @@ from .gen import (  # noqa: F401
     round_to_bits,
     bits_to_f32,
     NAN_BITS,
+    PrefillCase,
+    PREFILL_CONFIGS,
+    make_prefill_case,
+    make_prefill_config,
 )

@@ -257,6 +257,110 @@ def make_prefix_cow(seed: int = 5, groups: int = 64, samples: int = 8, prefix: i
                       seed=seed)
 
 
+@dataclass
+class PrefillCase:
+    """A prefill / chunked-prefill step: sequence s has ``context_lens[s]`` tokens once
+    its ``n_s`` new tokens (q rows ``query_start_loc[s] .. [s+1]``) are written; the
+    step writes the new tokens' key/value at ``slot_mapping`` and attends causally."""
+    name: str
+    dtype: str
+    num_q_heads: int
+    num_kv_heads: int
+    head_dim: int
+    block_size: int
+    num_blocks: int
+    scale: float
+    context_lens: np.ndarray     # int32 [B]
+    query_start_loc: np.ndarray  # int32 [B + 1]
+    block_tables: np.ndarray     # int32 [B, W]
+    q: np.ndarray                # uint16 [T, Hq, d]
+    k_cache: np.ndarray
+    v_cache: np.ndarray
+    key: np.ndarray              # uint16 [T, Hkv, d]
+    value: np.ndarray
+    slot_mapping: np.ndarray     # int64 [T]
+    window: int = 0
+    seed: int = 0
+
+    @property
+    def num_seqs(self) -> int:
+        return int(self.context_lens.shape[0])
+
+    @property
+    def num_tokens(self) -> int:
+        return int(self.query_start_loc[-1])
+
+    @property
+    def max_blocks_per_seq(self) -> int:
+        return int(self.block_tables.shape[1])
+
+
+def make_prefill_case(name: str, seed: int, specs, num_q_heads: int, num_kv_heads: int,
+                      head_dim: int, block_size: int, dtype: str = "bf16",
+                      spare: float = 0.10, window: int = 0, poison: bool = True) -> PrefillCase:
+    """specs: [(n_s, L_s)] -- a chunk of n_s new tokens ending a context of L_s tokens
+    (n_s == L_s: the whole prompt).  Draw order: the pool permutation, q, K pool, V
+    pool, the new tokens' key, value.  With poison, every slot that is neither one of
+    the earlier L_s - n_s tokens nor written by the step holds NaN."""
+    bs = block_size
+    rng = np.random.default_rng(seed)
+    ns = np.array([n for n, _ in specs], np.int64)
+    lens = np.array([L for _, L in specs], np.int32)
+    assert np.all(ns <= lens) and np.all(ns >= 0)
+    nblk = _blocks_needed(lens, bs)
+    total = int(nblk.sum())
+    nb = max(int(math.ceil((1.0 + spare) * total)), 1)
+    perm = rng.permutation(nb).astype(np.int32)
+    B = len(specs)
+    tables = np.full((B, max(int(nblk.max()) if B else 1, 1)), -1, np.int32)
+    pos = 0
+    for s in range(B):
+        tables[s, :nblk[s]] = perm[pos:pos + nblk[s]]
+        pos += int(nblk[s])
+    qsl = np.concatenate([[0], np.cumsum(ns)]).astype(np.int32)
+    T = int(qsl[-1])
+    q = _draw(rng, (T, num_q_heads, head_dim), dtype)
+    k_cache = _draw(rng, (nb, num_kv_heads, bs, head_dim), dtype)
+    v_cache = _draw(rng, (nb, num_kv_heads, bs, head_dim), dtype)
+    key = _draw(rng, (T, num_kv_heads, head_dim), dtype)
+    value = _draw(rng, (T, num_kv_heads, head_dim), dtype)
+    slots = np.empty(T, np.int64)
+    for s in range(B):
+        L, n = int(lens[s]), int(ns[s])
+        for i in range(n):
+            p = L - n + i
+            slots[qsl[s] + i] = int(tables[s, p // bs]) * bs + p % bs
+    if poison:
+        nan = NAN_BITS[dtype]
+        keep = np.zeros((nb, bs), dtype=bool)
+        for s in range(B):
+            for p in range(int(lens[s]) - int(ns[s])):
+                keep[tables[s, p // bs], p % bs] = True
+        kill = ~keep
+        k_cache.transpose(0, 2, 1, 3)[kill] = nan
+        v_cache.transpose(0, 2, 1, 3)[kill] = nan
+    return PrefillCase(name, dtype, num_q_heads, num_kv_heads, head_dim, bs, nb,
+                       1.0 / math.sqrt(head_dim), lens, qsl, tables, q, k_cache, v_cache, key,
+                       value, slots, window=window, seed=seed)
+
+
+PREFILL_CONFIGS = {
+    # whole prompts: 8 sequences of 2048 tokens, Llama-3-8B-shaped GQA heads
+    "prefill_2k_gqa": lambda **kw: make_prefill_case(
+        "prefill_2k_gqa", kw.pop("seed", 7), [(2048, 2048)] * kw.pop("num_seqs", 8), 32, 8, 128,
+        kw.pop("block_size", 16), **kw),
+    # chunked prefill: 16 sequences each adding a 512-token chunk to 1536..3072 earlier tokens
+    "prefill_chunk512_gqa": lambda **kw: make_prefill_case(
+        "prefill_chunk512_gqa", kw.pop("seed", 8),
+        [(512, 2048 + 128 * (i % 13)) for i in range(kw.pop("num_seqs", 16))], 32, 8, 128,
+        kw.pop("block_size", 16), **kw),
+}
+
+
+def make_prefill_config(name: str, **kw) -> PrefillCase:
+    return PREFILL_CONFIGS[name](**kw)
+
+
 def _lens_const(vals):
     return lambda rng: np.asarray(vals, dtype=np.int32)
 
