@@ -662,6 +662,227 @@ def run_swap(args):
     return result
 
 
+PREFILL_WORKLOADS = {
+    "prefill_2k_gqa": "prefill of whole prompts: 8 sequences x 2048 tokens, 32/8 heads, "
+                      "head_dim 128, bs 16, bf16",
+    "prefill_chunk512_gqa": "chunked prefill: 16 sequences each adding 512 tokens to "
+                            "1536..3072 earlier ones, 32/8 heads, head_dim 128, bs 16, bf16",
+}
+
+
+def prefill_flops(case) -> int:
+    """Algorithmic FLOPs of one pa_prefill: for every (token, query head), q.K over the
+    keys it attends (2 d each) and P.V over the same keys (2 d each)."""
+    qsl = case.query_start_loc.astype(np.int64)
+    keys = 0
+    for s in range(case.num_seqs):
+        n, L = int(qsl[s + 1] - qsl[s]), int(case.context_lens[s])
+        pos = np.arange(L - n, L, dtype=np.int64)
+        att = pos + 1 if case.window <= 0 else np.minimum(pos + 1, case.window)
+        keys += int(att.sum())
+    return 4 * case.head_dim * case.num_q_heads * keys
+
+
+def prefill_sample_flops(case, sel) -> int:
+    qsl = case.query_start_loc.astype(np.int64)
+    tot = 0
+    for t, _ in sel:
+        s = int(np.searchsorted(qsl, t, side="right") - 1)
+        n, L = int(qsl[s + 1] - qsl[s]), int(case.context_lens[s])
+        p = L - n + (int(t) - int(qsl[s]))
+        tot += 4 * case.head_dim * (p + 1 if case.window <= 0 else min(p + 1, case.window))
+    return tot
+
+
+def prefill_oracle_sample(case, budget_s, rng):
+    """The fp64 oracle (after the chunk's cache write) on seeded (token, head) samples
+    until about budget_s seconds: (TFLOP/s, threads, sample text)."""
+    import oracle
+    kc, vc = case.k_cache.copy(), case.v_cache.copy()
+    oracle.kv_write(case.key, case.value, case.slot_mapping, kc, vc)
+    nthreads = oracle.max_threads()
+    n, t_all, fl = 256, 0.0, 0
+    while t_all < budget_s:
+        sel = np.stack([rng.integers(0, case.num_tokens, size=n),
+                        rng.integers(0, case.num_q_heads, size=n)], 1).astype(np.int32)
+        t = time.perf_counter()
+        oracle.prefill(case.q, kc, vc, case.block_tables, case.context_lens,
+                       case.query_start_loc, case.scale, case.dtype,
+                       sliding_window=case.window, sel=sel, nthreads=nthreads)
+        t_all += time.perf_counter() - t
+        fl += prefill_sample_flops(case, sel)
+    return fl / t_all / 1e12, nthreads, (f"{fl / prefill_flops(case):.4f} of the step's work as "
+                                        f"seeded (token, head) samples, {t_all:.1f} s")
+
+
+def run_prefill(args):
+    """Prefill / chunked-prefill step: the chunk's cache write + causal attention."""
+    import torch
+    ws, rank, local = dist_env()
+    if args.impl == "reference":
+        if rank != 0:
+            return None
+        from workloads import make_prefill_config
+        case = make_prefill_config(args.workload)
+        value, nthreads, sample = prefill_oracle_sample(case, args.reference_budget,
+                                                        np.random.default_rng(0))
+        return {"impl": "reference", "metric": "prefill attention TFLOP/s", "value": round(value, 6),
+                "unit": "TFLOP/s", "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": round(prefill_flops(case) / (value * 1e12) * 1e3, 3),
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                "data": "synthetic", "config": {"workload": PREFILL_WORKLOADS[args.workload]},
+                "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": nthreads,
+                                 "kind": "oracle", "sample": sample},
+                "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}}
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    device = torch.device("cuda", torch.cuda.current_device())
+    import paged_kv_cache_441_b200 as pa
+    from workloads import make_prefill_config
+    case = make_prefill_config(args.workload, poison=False)
+    tdt = torch.bfloat16 if case.dtype == "bf16" else torch.float16
+
+    def d16(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(device).view(tdt)
+
+    def di(a):
+        return torch.from_numpy(np.ascontiguousarray(a)).to(device)
+
+    q, kc, vc = d16(case.q), d16(case.k_cache), d16(case.v_cache)
+    key, val, sm = d16(case.key), d16(case.value), di(case.slot_mapping)
+    bt, cl, qsl = di(case.block_tables), di(case.context_lens), di(case.query_start_loc)
+    out = torch.empty_like(q)
+    win = case.window
+    stream = torch.cuda.current_stream()
+
+    def step():
+        pa.kv_write(key, val, sm, kc, vc)
+        pa.prefill(out, q, kc, vc, bt, cl, qsl, case.scale, sliding_window=win)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    pa.device_error(device.index)
+    sampler = ClockSampler(device.index)
+    sampler.start()
+    time.sleep(0.3)
+    if ws > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(args.steps):
+        step()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    elapsed = t0.elapsed_time(t1)
+    # roofline pass: pa_prefill alone, events around groups of 10 calls
+    group = 10
+    ngroups = max(1, args.steps // group)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(ngroups)]
+    for i in range(ngroups):
+        ev[i][0].record(stream)
+        for _ in range(group):
+            pa.prefill(out, q, kc, vc, bt, cl, qsl, case.scale, sliding_window=win)
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    call_ms = sum(a.elapsed_time(b) for a, b in ev) / (ngroups * group)
+    err = pa.device_error(device.index)
+    if err:
+        raise RuntimeError(f"device error word {err:#x} during the timed loop")
+
+    # end to end: q and the chunk's key/value/slots and metadata in from pinned memory,
+    # the output back, every step (serialised on one stream)
+    hq_ = torch.from_numpy(case.q.view(np.int16)).view(tdt).pin_memory()
+    hk_ = torch.from_numpy(case.key.view(np.int16)).view(tdt).pin_memory()
+    hv_ = torch.from_numpy(case.value.view(np.int16)).view(tdt).pin_memory()
+    hsm = torch.from_numpy(case.slot_mapping).pin_memory()
+    hmeta = [torch.from_numpy(a).pin_memory() for a in (case.block_tables, case.context_lens,
+                                                         case.query_start_loc)]
+    hout = torch.empty(out.shape, dtype=tdt).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in [hq_, hk_, hv_, hsm] + hmeta)
+    d2h = hout.numel() * hout.element_size()
+    e2e_steps = max(1, min(args.steps, args.e2e_steps))
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        q.copy_(hq_, non_blocking=True)
+        key.copy_(hk_, non_blocking=True)
+        val.copy_(hv_, non_blocking=True)
+        sm.copy_(hsm, non_blocking=True)
+        for d_, h_ in zip((bt, cl, qsl), hmeta):
+            d_.copy_(h_, non_blocking=True)
+        step()
+        hout.copy_(out, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+
+    flops = prefill_flops(case)
+    max_ms = max_over_ranks(elapsed, ws, device)
+    ms_step = max_ms / args.steps
+    value = flops * ws / (ms_step * 1e-3) / 1e12
+    e2e_val = flops * ws / (max_over_ranks(e2e_ms, ws, device) / e2e_steps * 1e-3) / 1e12
+    achieved = flops / (call_ms * 1e-3) / 1e12
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            peak, peak_kind = float(json.load(f)["bf16_tflops"]), "measured"
+    except Exception:
+        peak, peak_kind = 1590.0, "fallback"
+    result = None
+    if rank == 0:
+        cpu = None
+        if not args.no_cpu_baseline and ws == 1:
+            v, nthreads, sample = prefill_oracle_sample(case, args.cpu_budget,
+                                                        np.random.default_rng(1))
+            cpu = {"value": round(v, 6), "unit": "TFLOP/s", "cores": nthreads, "kind": "oracle",
+                   "sample": sample}
+        result = {
+            "metric": "prefill attention TFLOP/s", "value": round(value, 2), "unit": "TFLOP/s",
+            "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(ms_step, 5), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": case.dtype,
+            "data": "synthetic (seeded N(0,1) q/K/V rounded to bf16, shuffled block pool)",
+            "config": {"workload": PREFILL_WORKLOADS[args.workload],
+                       "num_seqs": case.num_seqs, "num_tokens": case.num_tokens,
+                       "num_q_heads": case.num_q_heads, "num_kv_heads": case.num_kv_heads,
+                       "head_dim": case.head_dim, "block_size": case.block_size,
+                       "sliding_window": win, "step": "pa_kv_write (chunk) + pa_prefill",
+                       "parallelism": f"dp{ws} (independent replicas)",
+                       "l2": "no flush: the K/V read per call is well under L2; the work is "
+                             "tensor-bound"},
+            "algorithmic_flops_per_step": flops,
+            "e2e": {"value": round(e2e_val, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+            "gpu_launches": 2 * args.steps,
+            "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak,
+                         "peak_kind": f"{peak_kind} cuBLAS bf16 TFLOP/s (burst)", "unit": "TFLOP/s",
+                         "frac": round(achieved / peak, 4), "kernel": "pa_prefill",
+                         "avg_call_us": round(call_ms * 1e3, 2),
+                         "achieved_how": "algorithmic FLOPs (both products once; the split "
+                                         "P's second product and masked tile work not "
+                                         "counted) / mean CUDA-event time per call, events "
+                                         "around groups of 10 calls",
+                         "traffic": None},
+            "clocks": clocks,
+            "cpu_baseline": cpu,
+        }
+    if ws > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return result
+
+
 def run_reference(args):
     ws, rank, _ = dist_env()
     if rank != 0:
@@ -707,7 +928,8 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="llama2_7b")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS) + sorted(PREFILL_WORKLOADS),
+                    default=None)
     ap.add_argument("--partition-size", type=int, default=0)
     ap.add_argument("--seqs", type=int, default=0,
                     help="profiling only: build the workload with this many sequences")
@@ -715,14 +937,21 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=10.0)
     ap.add_argument("--reference-budget", type=float, default=60.0)
-    ap.add_argument("--op", choices=["step", "swap"], default="step",
-                    help="swap: time the preemption swap of the workload instead of the step")
+    ap.add_argument("--op", choices=["step", "swap", "prefill"], default="step",
+                    help="swap: time the preemption swap of the workload instead of the step; "
+                         "prefill: the prefill / chunked-prefill step (--workload prefill_*)")
     ap.add_argument("--swap-seqs", type=int, default=8,
                     help="swap: number of sequences preempted and restored per step")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
-    if args.op == "swap":
+    if args.workload is None:
+        args.workload = "prefill_2k_gqa" if args.op == "prefill" else "llama2_7b"
+    if (args.op == "prefill") != (args.workload in PREFILL_WORKLOADS):
+        ap.error("prefill workloads go with --op prefill, the others with --op step/swap")
+    if args.op == "prefill":
+        res = run_prefill(args)
+    elif args.op == "swap":
         res = run_swap(args) if args.impl == "ours" else None
     else:
         res = run_reference(args) if args.impl == "reference" else run_ours(args)
