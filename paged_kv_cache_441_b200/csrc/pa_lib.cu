@@ -848,11 +848,12 @@ extern "C" pa_status pa_prefill(void *out, const void *q, const void *k_cache,
     p.max_blocks_per_seq = max_blocks_per_seq;
     p.sliding_window = sliding_window;
     p.scale_log2 = scale * 1.4426950408889634f;
-    // sum over sequences of ceil(n_s / tpt) <= num_tokens / tpt + num_seqs
+    // a CTA takes two query tiles of tpt tokens: sum over sequences of
+    // ceil(ceil(n_s / tpt) / 2) <= num_tokens / (2 tpt) + num_seqs
     const long long tpt = kPfRows / G;
-    const long long tiles = (long long)num_tokens / tpt + num_seqs;
-    if (tiles >= (1ll << 31)) return PA_ERR_UNSUPPORTED;
-    const dim3 grid((unsigned)tiles, (unsigned)num_kv_heads);
+    const long long pairs = (long long)num_tokens / (2 * tpt) + num_seqs;
+    if (pairs >= (1ll << 31)) return PA_ERR_UNSUPPORTED;
+    const dim3 grid((unsigned)pairs, (unsigned)num_kv_heads);
     cudaStream_t st_ = static_cast<cudaStream_t>(stream);
     const cudaError_t e = dtype == PA_BF16
                               ? prefill_dispatch<__nv_bfloat16>(p, grid, st_, dev, head_dim, G)

@@ -9,41 +9,47 @@
 // under a sliding window):
 //     out[t][h] = sum_{u <= p} softmax_u(scale * q[t][h] . K_s[u][g]) V_s[u][g],  g = h / G.
 //
-// Work decomposition.  One CTA owns 128 query rows of one (sequence, kv head): 128/G
-// consecutive tokens times the G query heads that share the kv head (row r = token
-// r / G, head r % G), so one K/V tile read serves all G heads.  It walks the keys the
-// rows need in tiles of 128:
-//   S     = Q K^T      tcgen05.mma (M 128, N 128, K head_dim), Q and K K-major in
-//                      128-byte swizzled shared memory, fp32 S in tensor memory;
-//   softmax            row r is thread r is tensor-memory lane r: the row is read back
-//                      with tcgen05.ld, masked (causal, window, context end), and its
-//                      online-softmax state (m, l) updated in fp32; the 16-bit
-//                      probabilities P go to shared memory in the K-major layout;
-//   O += P V           tcgen05.mma (M 128, N head_dim, K 128) with V as an MN-major
-//                      operand (the cache rows as TMA lays them down), accumulated in
-//                      tensor memory; before it, each warp rescales its rows of O in
-//                      tensor memory by 2^(m_old - m_new) (skipped when no row of the
-//                      warp changed its maximum).  P is split into a high and a low
-//                      16-bit part (two products) so the weights keep ~16 bits, as in
-//                      the decode kernels' tensor-core path.
-// K/V tiles stream through a two-stage TMA ring (one mbarrier per stage and operand);
-// the tile two ahead is loaded while the current one is used.  Scores are kept in the
-// log2 domain (scale * log2 e folded in), as in the decode kernels.
+// Work decomposition.  A query tile is 128 rows of one (sequence, kv head): 128/G
+// consecutive tokens times the G query heads that share the kv head (row r = token r / G,
+// head r % G), so one K/V tile read serves all G heads.  A CTA owns two consecutive
+// query tiles, A and B, and walks the keys they need in tiles of 128:
+//   S_X   = Q_X K^T     tcgen05.mma (M 128, N 128, K head_dim): Q_X and K K-major in
+//                       128-byte swizzled shared memory, fp32 S_X in tensor memory;
+//   softmax             a warpgroup per query tile; row r is thread r is tensor-memory
+//                       lane r.  The row is read once into registers (tcgen05.ld),
+//                       masked (causal, window, context end; tiles wholly inside every
+//                       row's range skip the masks), and the online-softmax state
+//                       (m, l) updated in fp32; the probabilities go back over S_X in
+//                       tensor memory as a high and a low 16-bit part (tcgen05.st);
+//   O_X  += P_X V       tcgen05.mma with P_X read from tensor memory and V as an MN-major
+//                       shared-memory operand (the cache rows as TMA lays them down), two
+//                       products (high and low part) so the weights keep ~16 bits; before
+//                       it the warpgroup rescales its rows of O_X by 2^(m_old - m_new)
+//                       (skipped in a warp where no row raised its maximum).
+// Roles (warp specialisation): warps 0-3 softmax A, warps 4-7 softmax B, warp 8 issues the
+// matrix products (and zeroes V rows outside the attended keys), warp 9 issues the TMA
+// loads of Q and of a two-stage K/V ring.  The products of one tile overlap the softmax
+// of the other: the tensor core runs P_A V and S_A for the next key tile while the B
+// warpgroup works, and the other way round.  Scores are kept in the log2 domain (scale *
+// log2 e folded in), as in the decode kernels.
 //
-// Every wait is bounded: on a timeout the CTA records PA_DEVERR_TIMEOUT, waits (again
-// bounded) for its copies and matrix operations in flight, frees its tensor memory and
-// returns.
+// Every wait is bounded: on a timeout a role records PA_DEVERR_TIMEOUT and stops, the
+// others see the shared failure flag (or time out themselves), the copies and products
+// in flight are waited for (bounded), and the tensor memory is freed.
 #pragma once
 
 #include "pa_common.cuh"
 
 namespace pa {
 
-constexpr int kPfRows = 128;     // query rows per CTA = UMMA M = tensor-memory lanes
-constexpr int kPfKeys = 128;     // keys per tile = UMMA N of S and K of P.V
-constexpr int kPfThreads = 128;  // row r <-> thread r
-constexpr int kPfStages = 2;     // K/V ring depth
-constexpr int kPfTmemCols = 256; // S: columns [0, 128), O tile: [128, 128 + D)
+constexpr int kPfRows = 128;        // query rows per tile = UMMA M = tensor-memory lanes
+constexpr int kPfKeys = 128;        // keys per tile = UMMA N of S and K of P.V
+constexpr int kPfSoftWarps = 8;     // two softmax warpgroups
+constexpr int kPfMmaWarp = 8;
+constexpr int kPfLoadWarp = 9;
+constexpr int kPfThreads = 320;
+constexpr int kPfStages = 2;        // K/V ring depth
+constexpr int kPfTmemCols = 512;    // tile X: S/P at [256X, 256X + 128), O at [256X + 128, ...)
 
 struct PrefillParams {
     CUtensorMap qmap;  // 3-D [num_tokens][Hq][D] 16-bit, box {64, G, 128/G}, swizzle 128B
@@ -70,15 +76,13 @@ template <int D>
 struct PfGeom {
     static constexpr int kHalves = D / 64;                // 128-byte column blocks of a row
     static constexpr int kRegion = 128 * 128;             // 128 rows of one column block
-    static constexpr int kQ = kHalves * kRegion;          // Q tile
+    static constexpr int kQ = kHalves * kRegion;          // one Q tile
     static constexpr int kKV = kHalves * kRegion;         // one K (or V) stage
-    static constexpr int kP = 2 * kRegion;                // P: 128 rows x 128 keys
-    static constexpr int kOffK = kQ;
+    static constexpr int kOffK = 2 * kQ;
     static constexpr int kOffV = kOffK + kPfStages * kKV;
-    static constexpr int kOffP = kOffV + kPfStages * kKV;  // high part of P
-    static constexpr int kOffPlo = kOffP + kP;             // low part of P
-    static constexpr int kOffBar = kOffPlo + kP;
-    static constexpr int kBars = 1 + 2 * kPfStages + 2;  // q, k[2], v[2], s, o
+    static constexpr int kOffBar = kOffV + kPfStages * kKV;
+    // q, k[2], v[2], empty[2], s[2], p[2], o[2]
+    static constexpr int kBars = 1 + 4 * kPfStages + 6;
     static constexpr int kSmem = kOffBar + 8 * kBars + 1024;  // + alignment slack
 };
 
@@ -157,6 +161,17 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
         : "memory");
 }
 
+// Stores 16 consecutive 32-bit columns of this thread's tensor-memory lane.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t *r) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,"
+        "%13,%14,%15,%16};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+        "r"(r[15])
+        : "memory");
+}
+
 __device__ __forceinline__ void tmem_wait_st() {
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
@@ -182,21 +197,52 @@ __device__ __forceinline__ void sts_v4(uint32_t addr, uint32_t a, uint32_t b, ui
                  : "memory");
 }
 
+// A from tensor memory (lane = row, a 32-bit column holds two consecutive 16-bit K
+// elements, the first in the low half), B from shared memory.
+__device__ __forceinline__ void umma_f16_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t b,
+                                            uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(tmem_d),
+        "r"(tmem_a), "l"(b), "r"(idesc), "r"(accumulate));
+}
+
 // ---------------------------------------------------------------- the kernel
 
-// grid = (an upper bound of the number of 128-row tiles, kv heads); CTAs past the last
-// tile return at once.
+// One query tile's place in its sequence.
+struct PfTile {
+    bool live;
+    int tok0, ntok;   // first token (within the chunk) and valid tokens
+    int pos0;         // position of its first token
+    int kv_begin;     // first key any row attends
+    int j0, j1;       // key tiles [j0, j1)
+};
+
+__device__ __forceinline__ PfTile pf_tile(int qt, int tpt, int n, int L, int W) {
+    PfTile t;
+    t.tok0 = qt * tpt;
+    t.live = t.tok0 < n;
+    t.ntok = t.live ? min(tpt, n - t.tok0) : 0;
+    t.pos0 = L - n + t.tok0;
+    t.kv_begin = W > 0 ? max(0, t.pos0 - W + 1) : 0;
+    t.j0 = t.kv_begin / kPfKeys;
+    t.j1 = t.live ? (t.pos0 + t.ntok - 1) / kPfKeys + 1 : t.j0;
+    return t;
+}
+
+// grid = (an upper bound of the number of tile pairs, kv heads); CTAs past the last pair
+// return at once.
 template <typename T, int D, int G>
 __global__ void __launch_bounds__(kPfThreads, 1)
     pa_prefill_kernel(const __grid_constant__ PrefillParams p) {
     pdl_wait_and_release();
     using Gm = PfGeom<D>;
-    constexpr int kTpt = kPfRows / G;  // tokens per tile
+    constexpr int kTpt = kPfRows / G;  // tokens per query tile
     extern __shared__ uint8_t smem_raw[];
-    __shared__ int sh_item[2];  // sequence, tile index within it
+    __shared__ int sh_item[2];  // sequence, pair index within it
     __shared__ int warp_tot[kPfThreads / 32];
     __shared__ uint32_t sh_tmem;
-    __shared__ int stage_ok[kPfStages];
+    __shared__ volatile int sh_fail;
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
 
@@ -204,19 +250,23 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     const int g = blockIdx.y;
     const int cta = blockIdx.x;
 
-    // ---- 1. this CTA's (sequence, q tile): block-wide prefix sum of tiles per sequence.
-    // Within a sequence the last (longest-context) tile comes first.
-    if (tid == 0) sh_item[0] = -1;
+    // ---- 1. this CTA's (sequence, tile pair): block-wide prefix sum of pairs per
+    // sequence; within a sequence the last (longest-context) pair comes first.
+    if (tid == 0) {
+        sh_item[0] = -1;
+        sh_fail = 0;
+    }
     __syncthreads();
     int run = 0;
     for (int s0 = 0; s0 < p.num_seqs; s0 += kPfThreads) {
         const int s = s0 + tid;
-        int nt = 0;
+        int np = 0;
         if (s < p.num_seqs) {
             const int n = __ldg(p.query_start_loc + s + 1) - __ldg(p.query_start_loc + s);
-            nt = n > 0 ? (n + kTpt - 1) / kTpt : 0;
+            const int nt = n > 0 ? (n + kTpt - 1) / kTpt : 0;
+            np = (nt + 1) / 2;
         }
-        int incl = nt;
+        int incl = np;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             const int v = __shfl_up_sync(0xffffffffu, incl, o);
@@ -230,10 +280,10 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             woff += (w < warp) ? warp_tot[w] : 0;
             total += warp_tot[w];
         }
-        const int excl = run + woff + incl - nt;
-        if (nt > 0 && cta >= excl && cta < excl + nt) {
+        const int excl = run + woff + incl - np;
+        if (np > 0 && cta >= excl && cta < excl + np) {
             sh_item[0] = s;
-            sh_item[1] = nt - 1 - (cta - excl);
+            sh_item[1] = np - 1 - (cta - excl);
         }
         run += total;
         __syncthreads();
@@ -241,42 +291,45 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     }
     const int s = sh_item[0];
     if (s < 0) return;
-    const int qt = sh_item[1];
     const int q0 = __ldg(p.query_start_loc + s);
     const int n = __ldg(p.query_start_loc + s + 1) - q0;
     const int L = __ldg(p.context_lens + s);
     if (q0 < 0 || q0 + n > p.num_tokens || n > L || L > (p.max_blocks_per_seq << p.bs_shift)) {
-        if (tid == 0 && qt == 0) raise_error(PA_DEVERR_CONTEXT);
+        if (tid == 0 && sh_item[1] == 0) raise_error(PA_DEVERR_CONTEXT);
         return;
     }
     const int W = p.sliding_window;
-    const int tok0 = qt * kTpt;               // first token of the tile within the chunk
-    const int ntok = min(kTpt, n - tok0);     // its valid tokens
-    const int pos0 = L - n + tok0;            // position of its first token
-    const int posN = pos0 + ntok - 1;         // position of its last valid token
-    const int kv_begin = W > 0 ? max(0, pos0 - W + 1) : 0;  // first key any row attends
-    const int j0 = kv_begin / kPfKeys, j1 = posN / kPfKeys + 1;
-
-    // this thread's row
-    const int rtok = tid / G, rh = tid % G;
-    const bool rvalid = rtok < ntok;
-    const int rpos = rvalid ? pos0 + rtok : -1;              // invalid rows attend nothing
-    const int rlo = (W > 0 && rvalid) ? rpos - W + 1 : 0;
+    const PfTile ta = pf_tile(2 * sh_item[1], kTpt, n, L, W);
+    const PfTile tb = pf_tile(2 * sh_item[1] + 1, kTpt, n, L, W);
+    const int j0 = ta.j0, j1 = max(ta.j1, tb.live ? tb.j1 : ta.j1);  // tb.j0 >= ta.j0
+    const int kv_begin = ta.kv_begin;  // first key either tile attends
 
     // ---- 2. barriers, tensor memory
-    const uint32_t sq = base, sk = base + Gm::kOffK, sv = base + Gm::kOffV, sp = base + Gm::kOffP;
-    const uint32_t splo = base + Gm::kOffPlo;
+    const uint32_t sq = base, sk = base + Gm::kOffK, sv = base + Gm::kOffV;
     const uint32_t bar_q = base + Gm::kOffBar;
     const uint32_t bar_k0 = bar_q + 8, bar_v0 = bar_k0 + 8 * kPfStages;
-    const uint32_t bar_s = bar_v0 + 8 * kPfStages, bar_o = bar_s + 8;
+    const uint32_t bar_e0 = bar_v0 + 8 * kPfStages;      // stage empty (all its products done)
+    const uint32_t bar_s0 = bar_e0 + 8 * kPfStages;      // S_X ready, X = 0 (A), 1 (B)
+    const uint32_t bar_p0 = bar_s0 + 16;                 // P_X written, O_X rescaled
+    const uint32_t bar_o0 = bar_p0 + 16;                 // P_X V done
     if (tid == 0) {
         tma_prefetch_desc(&p.qmap);
         tma_prefetch_desc(&p.kmap);
         tma_prefetch_desc(&p.vmap);
-        for (int i = 0; i < Gm::kBars; ++i) mbar_init(bar_q + 8 * i, 1);
+        mbar_init(bar_q, 1);
+        for (int i = 0; i < kPfStages; ++i) {
+            mbar_init(bar_k0 + 8 * i, 1);
+            mbar_init(bar_v0 + 8 * i, 1);
+            mbar_init(bar_e0 + 8 * i, 1);
+        }
+        for (int x = 0; x < 2; ++x) {
+            mbar_init(bar_s0 + 8 * x, 1);
+            mbar_init(bar_p0 + 8 * x, 4);  // one arrival per softmax warp
+            mbar_init(bar_o0 + 8 * x, 1);
+        }
         fence_barrier_init();
     }
-    if (warp == 0) {
+    if (warp == kPfMmaWarp) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                          smem_u32(&sh_tmem)),
                      "r"(kPfTmemCols)
@@ -287,250 +340,337 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = sh_tmem;
-    const uint32_t tmem_s = tmem, tmem_o = tmem + 128;
-    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
 
-    const int32_t *table = p.block_tables + (size_t)s * p.max_blocks_per_seq;
-    const int BR = p.box_rows;
-    // K/V tile jt -> stage: boxes of BR rows that overlap [kv_begin, L) are loaded
-    auto load_kv = [&](int jt) {  // thread 0 only
-        const int st = (jt - j0) % kPfStages;
-        const int kv0 = jt * kPfKeys;
-        int nload = 0;
-        bool ok = true;
-        for (int b = 0; b < kPfKeys / BR; ++b) {
-            const int r0 = kv0 + b * BR;
-            if (r0 < L && r0 + BR > kv_begin) {
-                ++nload;
-                const int blk = __ldg(table + (r0 >> p.bs_shift));
-                ok = ok && (unsigned)blk < (unsigned)p.num_blocks;
-            }
-        }
-        stage_ok[st] = ok ? 1 : 0;
-        const uint32_t bk = bar_k0 + 8 * st, bv = bar_v0 + 8 * st;
-        if (!ok) {
-            raise_error(PA_DEVERR_BLOCK_ID);
-            mbar_arrive(bk);
-            mbar_arrive(bv);
-            return;
-        }
-        const uint32_t bytes = (uint32_t)(nload * BR * 128 * Gm::kHalves);
-        mbar_arrive_expect_tx(bk, bytes);
-        mbar_arrive_expect_tx(bv, bytes);
-        const uint64_t pol = l2_policy_evict_first();
-        for (int b = 0; b < kPfKeys / BR; ++b) {
-            const int r0 = kv0 + b * BR;
-            if (r0 < L && r0 + BR > kv_begin) {
-                const int blk = __ldg(table + (r0 >> p.bs_shift));
-                const int y = (blk * p.num_kv_heads + g) * p.block_size + (r0 & (p.block_size - 1));
+    if (warp == kPfLoadWarp) {
+        // ============================ TMA producer (lane 0)
+        if (lane == 0) {
+            const int32_t *table = p.block_tables + (size_t)s * p.max_blocks_per_seq;
+            const int BR = p.box_rows;
+            const uint64_t pol = l2_policy_evict_first();
+            mbar_arrive_expect_tx(bar_q, (uint32_t)((tb.live ? 2 : 1) * Gm::kQ));
 #pragma unroll
-                for (int hf = 0; hf < Gm::kHalves; ++hf) {
-                    const uint32_t off = hf * Gm::kRegion + b * BR * 128;
-                    tma_load_2d(sk + st * Gm::kKV + off, &p.kmap, bk, 64 * hf, y, pol);
-                    tma_load_2d(sv + st * Gm::kKV + off, &p.vmap, bv, 64 * hf, y, pol);
+            for (int hf = 0; hf < Gm::kHalves; ++hf) {
+                tma_load_3d(sq + hf * Gm::kRegion, &p.qmap, bar_q, 64 * hf, g * G, q0 + ta.tok0);
+                if (tb.live)
+                    tma_load_3d(sq + Gm::kQ + hf * Gm::kRegion, &p.qmap, bar_q, 64 * hf, g * G,
+                                q0 + tb.tok0);
+            }
+            int issued = j0;
+            for (int jt = j0; jt < j1; ++jt) {
+                const int it = jt - j0, st = it % kPfStages;
+                if (it >= kPfStages &&
+                    !mbar_wait_bounded(bar_e0 + 8 * st, (uint32_t)(((it / kPfStages) - 1) & 1))) {
+                    raise_error(PA_DEVERR_TIMEOUT);
+                    sh_fail = 1;
+                    break;
                 }
-            }
-        }
-    };
-
-    int issued = j0;  // tiles whose K/V loads were issued: [j0, issued)
-    if (tid == 0) {
-        mbar_arrive_expect_tx(bar_q, (uint32_t)Gm::kQ);
-#pragma unroll
-        for (int hf = 0; hf < Gm::kHalves; ++hf)
-            tma_load_3d(sq + hf * Gm::kRegion, &p.qmap, bar_q, 64 * hf, g * G, q0 + tok0);
-        for (; issued < min(j1, j0 + kPfStages); ++issued) load_kv(issued);
-    }
-    __syncthreads();  // stage_ok of the first tiles
-
-    const uint32_t idesc_s = umma_idesc<T>(kPfRows, kPfKeys, false);
-    const uint32_t idesc_o = umma_idesc<T>(kPfRows, D, true);
-    float m_run = -INFINITY, l_run = 0.f;
-    bool failed = false;
-    // thread 0: parity of a commit not yet waited for, or -1 (for the cleanup)
-    int s_pending = -1, o_pending = -1;
-
-    for (int jt = j0; jt < j1; ++jt) {
-        const int it = jt - j0, st = it % kPfStages;
-        const uint32_t ph = (uint32_t)((it / kPfStages) & 1);
-        const int kv0 = jt * kPfKeys;
-        bool bad = false;
-        // (a) S = Q K^T
-        if (tid == 0) {
-            bool ok = (it > 0 || mbar_wait_bounded(bar_q, 0));
-            ok = ok && mbar_wait_bounded(bar_k0 + 8 * st, ph);
-            if (ok) {
-                tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t koff = (kk >> 2) * Gm::kRegion + (kk & 3) * 32;
-                    umma_f16(tmem_s, umma_desc_sw128(sq + koff, 16),
-                             umma_desc_sw128(sk + st * Gm::kKV + koff, 16), idesc_s, kk > 0);
+                if (sh_fail) break;
+                const int kv0 = jt * kPfKeys;
+                int nload = 0;
+                bool ok = true;
+                for (int b = 0; b < kPfKeys / BR; ++b) {
+                    const int r0 = kv0 + b * BR;
+                    if (r0 < L && r0 + BR > kv_begin) {
+                        ++nload;
+                        const int blk = __ldg(table + (r0 >> p.bs_shift));
+                        ok = ok && (unsigned)blk < (unsigned)p.num_blocks;
+                    }
                 }
-                umma_commit(bar_s);
-                s_pending = it & 1;
-            } else {
-                bad = true;
-            }
-        }
-        // (b) the previous tile's P V has finished (P and its stage are free again; the
-        // tensor core runs the S product above after it, so this rarely waits)
-        if (it > 0) {
-            const bool got = mbar_wait_bounded(bar_o, (uint32_t)((it - 1) & 1));
-            if (tid == 0 && got) o_pending = -1;
-            bad = bad || !got;
-            if (tid == 0 && got && issued < j1) load_kv(issued++);  // into the freed stage
-        }
-        // (c) softmax of row `tid` over the tile's keys
-        const bool got_s = mbar_wait_bounded(bar_s, (uint32_t)(it & 1));
-        if (tid == 0 && got_s) s_pending = -1;
-        bad = bad || !got_s;
-        tc_fence_after();
-        const bool tile_ok = stage_ok[st] != 0;
-        float mx = -INFINITY;
-#pragma unroll
-        for (int cc = 0; cc < kPfKeys / 32; ++cc) {
-            uint32_t v[32];
-            tmem_ld32(tmem_s + lane_off + cc * 32, v);
-            tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 32; ++e) {
-                const int key = kv0 + cc * 32 + e;
-                const bool ok = tile_ok && key <= rpos && key >= rlo;
-                mx = fmaxf(mx, ok ? __uint_as_float(v[e]) * p.scale_log2 : -INFINITY);
-            }
-        }
-        const float m_new = fmaxf(m_run, mx);
-        const float alpha = (m_new == -INFINITY) ? 1.f : fast_exp2(m_run - m_new);
-        float sum = 0.f;
-#pragma unroll
-        for (int cc = 0; cc < kPfKeys / 32; ++cc) {
-            uint32_t v[32];
-            tmem_ld32(tmem_s + lane_off + cc * 32, v);
-            tmem_wait_ld();
-            // P = hi + lo: hi = RN(p), lo = RN(p - hi) in the input type, so that the two
-            // P V products keep ~16 significant bits of every weight
-            uint32_t ph_[16], pl_[16];
-#pragma unroll
-            for (int e = 0; e < 32; e += 2) {
-                const int key = kv0 + cc * 32 + e;
-                const bool ok0 = tile_ok && key <= rpos && key >= rlo;
-                const bool ok1 = tile_ok && key + 1 <= rpos && key + 1 >= rlo;
-                const float p0 =
-                    ok0 ? fast_exp2(__uint_as_float(v[e]) * p.scale_log2 - m_new) : 0.f;
-                const float p1 =
-                    ok1 ? fast_exp2(__uint_as_float(v[e + 1]) * p.scale_log2 - m_new) : 0.f;
-                sum += p0 + p1;
-                ph_[e >> 1] = Fmt<T>::pack_rn(p0, p1);
-                const float2 h = Fmt<T>::unpack(ph_[e >> 1]);
-                pl_[e >> 1] = Fmt<T>::pack_rn(p0 - h.x, p1 - h.y);
-            }
-            // keys cc*32 .. +31 of row tid: column block cc/2, 16-byte chunks 4(cc%2) .. +3
-#pragma unroll
-            for (int c4 = 0; c4 < 4; ++c4) {
-                const int ch = (cc & 1) * 4 + c4;
-                const uint32_t off = (cc >> 1) * Gm::kRegion + tid * 128 + ((ch ^ (tid & 7)) << 4);
-                sts_v4(sp + off, ph_[4 * c4], ph_[4 * c4 + 1], ph_[4 * c4 + 2], ph_[4 * c4 + 3]);
-                sts_v4(splo + off, pl_[4 * c4], pl_[4 * c4 + 1], pl_[4 * c4 + 2], pl_[4 * c4 + 3]);
-            }
-        }
-        l_run = l_run * alpha + sum;
-        m_run = m_new;
-        // (d) rescale the running output in tensor memory by alpha (rows of this warp)
-        if (it > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
-#pragma unroll
-            for (int cc = 0; cc < D / 32; ++cc) {
-                uint32_t v[32];
-                tmem_ld32(tmem_o + lane_off + cc * 32, v);
-                tmem_wait_ld();
-#pragma unroll
-                for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * alpha);
-                tmem_st32(tmem_o + lane_off + cc * 32, v);
-            }
-            tmem_wait_st();
-        }
-        // V rows outside [kv_begin, L) (not loaded, or past the context) -> 0, so that
-        // their zero probabilities cannot meet a NaN
-        const bool edge = !tile_ok || kv0 < kv_begin || kv0 + kPfKeys > L;
-        if (edge) {
-            bad = bad || !mbar_wait_bounded(bar_v0 + 8 * st, ph);
-            const int key = kv0 + tid;
-            if (!tile_ok || key < kv_begin || key >= L) {
-#pragma unroll
-                for (int hf = 0; hf < Gm::kHalves; ++hf)
-#pragma unroll
-                    for (int c = 0; c < 8; ++c)
-                        sts_v4(sv + st * Gm::kKV + hf * Gm::kRegion + tid * 128 + c * 16, 0, 0,
-                               0, 0);
-            }
-        }
-        fence_proxy_async_smem();  // P (and zeroed V rows) -> the tensor-core reads
-        tc_fence_before();
-        if (__syncthreads_or(bad)) {
-            failed = true;
-            break;
-        }
-        // (e) O += P V
-        if (tid == 0) {
-            tc_fence_after();
-            if (mbar_wait_bounded(bar_v0 + 8 * st, ph)) {
-#pragma unroll
-                for (int kk = 0; kk < 2 * (kPfKeys / 16); ++kk) {  // P_hi V, then P_lo V
-                    const int k = kk % (kPfKeys / 16);
-                    const uint32_t aoff = (kk < kPfKeys / 16 ? sp : splo) + (k >> 2) * Gm::kRegion +
-                                          (k & 3) * 32;
-                    umma_f16(tmem_o, umma_desc_sw128(aoff, 16),
-                             umma_desc_sw128(sv + st * Gm::kKV + k * 16 * 128, Gm::kRegion),
-                             idesc_o, (it > 0 || kk > 0) ? 1u : 0u);
+                const uint32_t bk = bar_k0 + 8 * st, bv = bar_v0 + 8 * st;
+                if (!ok) {
+                    // nothing loaded: the consumers see the stage as all-masked
+                    raise_error(PA_DEVERR_BLOCK_ID);
+                    nload = 0;
                 }
-                umma_commit(bar_o);
-                o_pending = it & 1;
-            } else {
-                // nothing was issued: the next wait on bar_o times out and ends the tile
-                // loop through the barrier above
+                const uint32_t bytes = (uint32_t)(nload * BR * 128 * Gm::kHalves);
+                mbar_arrive_expect_tx(bk, bytes);
+                mbar_arrive_expect_tx(bv, bytes);
+                if (ok) {
+                    for (int b = 0; b < kPfKeys / BR; ++b) {
+                        const int r0 = kv0 + b * BR;
+                        if (r0 < L && r0 + BR > kv_begin) {
+                            const int blk = __ldg(table + (r0 >> p.bs_shift));
+                            const int y = (blk * p.num_kv_heads + g) * p.block_size +
+                                          (r0 & (p.block_size - 1));
+#pragma unroll
+                            for (int hf = 0; hf < Gm::kHalves; ++hf) {
+                                const uint32_t off = hf * Gm::kRegion + b * BR * 128;
+                                tma_load_2d(sk + st * Gm::kKV + off, &p.kmap, bk, 64 * hf, y, pol);
+                                tma_load_2d(sv + st * Gm::kKV + off, &p.vmap, bv, 64 * hf, y, pol);
+                            }
+                        }
+                    }
+                }
+                issued = jt + 1;
             }
-        }
-    }
-    // the last P V
-    if (!failed && j1 > j0) {
-        const bool got = mbar_wait_bounded(bar_o, (uint32_t)((j1 - j0 - 1) & 1));
-        if (tid == 0 && got) o_pending = -1;
-        failed = __syncthreads_or(!got);
-    }
-
-    if (failed) {
-        if (tid == 0) {
-            raise_error(PA_DEVERR_TIMEOUT);
-            // let the copies and matrix operations in flight finish (bounded)
+            // cleanup: the loads this CTA issued have landed (bounded)
             (void)mbar_wait_bounded(bar_q, 0);
-            for (int jt = j0; jt < issued; ++jt) {
+            for (int jt = max(j0, issued - kPfStages); jt < issued; ++jt) {
                 const int it = jt - j0, st = it % kPfStages;
                 const uint32_t ph = (uint32_t)((it / kPfStages) & 1);
                 (void)mbar_wait_bounded(bar_k0 + 8 * st, ph);
                 (void)mbar_wait_bounded(bar_v0 + 8 * st, ph);
             }
-            if (s_pending >= 0) (void)mbar_wait_bounded(bar_s, (uint32_t)s_pending);
-            if (o_pending >= 0) (void)mbar_wait_bounded(bar_o, (uint32_t)o_pending);
         }
+    } else if (warp == kPfMmaWarp) {
+        // ============================ matrix products (lane 0 issues; the warp waits)
+        const uint32_t idesc_s = umma_idesc<T>(kPfRows, kPfKeys, false);
+        const uint32_t idesc_o = umma_idesc<T>(kPfRows, D, true);
+        auto wait_all = [&](uint32_t bar, uint32_t par) {
+            return __all_sync(0xffffffffu, mbar_wait_bounded(bar, par));
+        };
+        bool ok = wait_all(bar_q, 0);
+        auto need = [&](const PfTile &t, int jt) { return t.live && jt >= t.j0 && jt < t.j1; };
+        auto issue_s = [&](int x, int jt) {  // S_X = Q_X K_jt
+            const int st = (jt - j0) % kPfStages;
+            if (lane == 0) {
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t koff = (kk >> 2) * Gm::kRegion + (kk & 3) * 32;
+                    umma_f16(tmem + 256 * x, umma_desc_sw128(sq + x * Gm::kQ + koff, 16),
+                             umma_desc_sw128(sk + st * Gm::kKV + koff, 16), idesc_s, kk > 0);
+                }
+                umma_commit(bar_s0 + 8 * x);
+            }
+            __syncwarp();
+        };
+        auto issue_pv = [&](int x, int jt, bool first) {  // O_X += P_X V_jt (high, low)
+            const int st = (jt - j0) % kPfStages;
+            if (lane == 0) {
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < 2 * (kPfKeys / 16); ++kk) {
+                    const int k = kk % (kPfKeys / 16);
+                    const uint32_t acol = 256 * x + (k >> 2) * 64 + (kk >= kPfKeys / 16 ? 32 : 0) +
+                                          (k & 3) * 8;
+                    umma_f16_ts(tmem + 256 * x + 128, tmem + acol,
+                                umma_desc_sw128(sv + st * Gm::kKV + k * 16 * 128, Gm::kRegion),
+                                idesc_o, (!first || kk > 0) ? 1u : 0u);
+                }
+                umma_commit(bar_o0 + 8 * x);
+            }
+            __syncwarp();
+        };
+        // per-tile counters of the products already issued (for the barrier parities)
+        int ns[2] = {0, 0}, npv[2] = {0, 0};
+        const PfTile *tl[2] = {&ta, &tb};
+        if (ok && !__any_sync(0xffffffffu, sh_fail != 0)) {
+            ok = wait_all(bar_k0, 0);
+            if (ok) {
+                for (int x = 0; x < 2; ++x)
+                    if (need(*tl[x], j0)) issue_s(x, j0), ++ns[x];
+            }
+        }
+        for (int jt = j0; ok && jt < j1; ++jt) {
+            if (__any_sync(0xffffffffu, sh_fail != 0)) {
+                ok = false;
+                break;
+            }
+            const int it = jt - j0, st = it % kPfStages;
+            const uint32_t ph = (uint32_t)((it / kPfStages) & 1);
+            const int kv0 = jt * kPfKeys;
+            // V of this tile; rows outside [kv_begin, L) (not loaded, or past the context)
+            // -> 0 so that zero weights cannot meet a NaN
+            ok = wait_all(bar_v0 + 8 * st, ph);
+            if (!ok) break;
+            if (kv0 < kv_begin || kv0 + kPfKeys > L) {
+                const int lo = max(0, kv_begin - kv0), hi = min(kPfKeys, L - kv0);
+                for (int idx = lane; idx < kPfKeys * Gm::kHalves * 8; idx += 32) {
+                    const int r = idx / (Gm::kHalves * 8), c = idx % (Gm::kHalves * 8);
+                    if (r < lo || r >= hi)
+                        asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(
+                                         sv + st * Gm::kKV + (c >> 3) * Gm::kRegion + r * 128 +
+                                         (c & 7) * 16),
+                                     "r"(0)
+                                     : "memory");
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+            }
+            const bool has_next = jt + 1 < j1;
+            if (has_next) {
+                const int st1 = (it + 1) % kPfStages;
+                ok = wait_all(bar_k0 + 8 * st1, (uint32_t)(((it + 1) / kPfStages) & 1));
+                if (!ok) break;
+            }
+            for (int x = 0; x < 2 && ok; ++x) {
+                const PfTile &t = *tl[x];
+                if (need(t, jt)) {
+                    ok = wait_all(bar_p0 + 8 * x, (uint32_t)(npv[x] & 1));
+                    if (!ok) break;
+                    issue_pv(x, jt, npv[x] == 0);
+                    ++npv[x];
+                }
+                if (has_next && need(t, jt + 1)) {
+                    if (need(t, jt)) {  // P_X (in S_X's columns) has been read: O_X done
+                        ok = wait_all(bar_o0 + 8 * x, (uint32_t)((npv[x] - 1) & 1));
+                        if (!ok) break;
+                    }
+                    issue_s(x, jt + 1);
+                    ++ns[x];
+                }
+            }
+            if (!ok) break;
+            if (lane == 0) umma_commit(bar_e0 + 8 * st);  // every product reading stage st
+            __syncwarp();
+        }
+        if (!ok) {
+            if (lane == 0) raise_error(PA_DEVERR_TIMEOUT);
+            sh_fail = 1;
+        }
+        // cleanup: the newest products have finished (bounded)
+        for (int x = 0; x < 2; ++x)
+            if (npv[x] > 0) (void)mbar_wait_bounded(bar_o0 + 8 * x, (uint32_t)((npv[x] - 1) & 1));
+        (void)ns;
     } else {
-        tc_fence_after();
-        const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-        T *dst = reinterpret_cast<T *>(p.out) +
-                 ((size_t)(q0 + tok0 + rtok) * p.num_q_heads + (size_t)g * G + rh) * D;
+        // ============================ softmax warpgroup X (rows = threads 128X .. 128X+127)
+        const int x = warp / 4;
+        const PfTile &t = x == 0 ? ta : tb;
+        const int row = tid & 127;
+        const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+        const uint32_t tS = tmem + 256 * x + lane_off, tO = tS + 128;
+        const int rtok = row / G, rh = row % G;
+        const bool rvalid = t.live && rtok < t.ntok;
+        const int rpos = rvalid ? t.pos0 + rtok : -1;
+        const int rlo = (W > 0 && rvalid) ? rpos - W + 1 : 0;
+        // every row of the tile attends keys [key_all_lo, key_all_hi] (valid tokens only)
+        const bool all_rows = t.live && t.ntok == kTpt;
+        const int key_all_hi = t.pos0;                          // min over rows of rpos
+        const int key_all_lo = W > 0 ? t.pos0 + t.ntok - W : 0;  // max over rows of rlo
+        float m_run = -INFINITY, l_run = 0.f;
+        bool ok = true;
+        int i = 0;
+        for (int jt = t.j0; t.live && jt < t.j1; ++jt, ++i) {
+            if (__any_sync(0xffffffffu, sh_fail != 0)) {
+                ok = false;
+                break;
+            }
+            const int kv0 = jt * kPfKeys;
+            ok = mbar_wait_bounded(bar_s0 + 8 * x, (uint32_t)(i & 1));
+            if (!__all_sync(0xffffffffu, ok)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            // keys inside every row's range, and nothing past the context or before the
+            // loaded keys: no per-element mask
+            const bool full = all_rows && kv0 + kPfKeys - 1 <= key_all_hi && kv0 >= key_all_lo &&
+                              kv0 >= kv_begin;
+            // scaled, masked scores of keys 64h .. 64h+63 of this row
+            auto load_half = [&](int h, uint32_t (&v)[64]) {
+                tmem_ld32(tS + 64 * h, *reinterpret_cast<uint32_t(*)[32]>(v));
+                tmem_ld32(tS + 64 * h + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
+                tmem_wait_ld();
+                if (full) {
 #pragma unroll
-        for (int cc = 0; cc < D / 32; ++cc) {
-            uint32_t v[32];
-            tmem_ld32(tmem_o + lane_off + cc * 32, v);
-            tmem_wait_ld();
-            if (rvalid) {
+                    for (int e = 0; e < 64; ++e)
+                        v[e] = __float_as_uint(__uint_as_float(v[e]) * p.scale_log2);
+                } else {
 #pragma unroll
-                for (int e = 0; e < 32; e += 8) {
-                    uint4 w;
-                    w.x = Fmt<T>::pack_rn(__uint_as_float(v[e]) * inv, __uint_as_float(v[e + 1]) * inv);
-                    w.y = Fmt<T>::pack_rn(__uint_as_float(v[e + 2]) * inv, __uint_as_float(v[e + 3]) * inv);
-                    w.z = Fmt<T>::pack_rn(__uint_as_float(v[e + 4]) * inv, __uint_as_float(v[e + 5]) * inv);
-                    w.w = Fmt<T>::pack_rn(__uint_as_float(v[e + 6]) * inv, __uint_as_float(v[e + 7]) * inv);
-                    *reinterpret_cast<uint4 *>(dst + cc * 32 + e) = w;
+                    for (int e = 0; e < 64; ++e) {
+                        const int key = kv0 + 64 * h + e;
+                        const bool in = key <= rpos && key >= rlo && key >= kv_begin;
+                        v[e] = __float_as_uint(in ? __uint_as_float(v[e]) * p.scale_log2
+                                                  : -INFINITY);
+                    }
+                }
+            };
+            float mx = -INFINITY;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                uint32_t v[64];
+                load_half(h, v);
+#pragma unroll
+                for (int e = 0; e < 64; ++e) mx = fmaxf(mx, __uint_as_float(v[e]));
+            }
+            const float m_new = fmaxf(m_run, mx);
+            const float alpha = (m_new == -INFINITY) ? 1.f : fast_exp2(m_run - m_new);
+            // the previous P_X V has finished: rescale O_X (and P_X's columns are free)
+            if (i > 0) {
+                ok = mbar_wait_bounded(bar_o0 + 8 * x, (uint32_t)((i - 1) & 1));
+                if (!__all_sync(0xffffffffu, ok)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                if (__any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll
+                    for (int cc = 0; cc < D / 32; ++cc) {
+                        uint32_t o[32];
+                        tmem_ld32(tO + cc * 32, o);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int e = 0; e < 32; ++e)
+                            o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+                        tmem_st32(tO + cc * 32, o);
+                    }
+                }
+            }
+            // P = hi + lo, written over S: keys 64h .. 64h+63 -> high part in columns
+            // 64h .. 64h+31, low part in 64h+32 .. 64h+63 (two keys per column).  A row
+            // with nothing attended yet (m = -inf) gets zeros.  Each half is read again
+            // before any of it is overwritten.
+            const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
+            float sum = 0.f;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                uint32_t v[64];
+                load_half(h, v);
+#pragma unroll
+                for (int c = 0; c < 2; ++c) {
+                    uint32_t ph_[16], pl_[16];
+#pragma unroll
+                    for (int e = 0; e < 32; e += 2) {
+                        const float p0 = fast_exp2(__uint_as_float(v[32 * c + e]) - m_use);
+                        const float p1 = fast_exp2(__uint_as_float(v[32 * c + e + 1]) - m_use);
+                        sum += p0 + p1;
+                        ph_[e >> 1] = Fmt<T>::pack_rn(p0, p1);
+                        const float2 hv = Fmt<T>::unpack(ph_[e >> 1]);
+                        pl_[e >> 1] = Fmt<T>::pack_rn(p0 - hv.x, p1 - hv.y);
+                    }
+                    tmem_st16(tS + 64 * h + 16 * c, ph_);
+                    tmem_st16(tS + 64 * h + 32 + 16 * c, pl_);
+                }
+            }
+            tmem_wait_st();
+            l_run = l_run * alpha + sum;
+            m_run = m_new;
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_p0 + 8 * x);
+        }
+        if (t.live && ok && i > 0) {
+            ok = mbar_wait_bounded(bar_o0 + 8 * x, (uint32_t)((i - 1) & 1));
+            ok = __all_sync(0xffffffffu, ok);
+        }
+        if (!ok) {
+            if (lane == 0) raise_error(PA_DEVERR_TIMEOUT);
+            sh_fail = 1;
+        } else if (t.live) {
+            tc_fence_after();
+            const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+            T *dst = reinterpret_cast<T *>(p.out) +
+                     ((size_t)(q0 + t.tok0 + rtok) * p.num_q_heads + (size_t)g * G + rh) * D;
+#pragma unroll
+            for (int cc = 0; cc < D / 32; ++cc) {
+                uint32_t v[32];
+                tmem_ld32(tO + cc * 32, v);
+                tmem_wait_ld();
+                if (rvalid) {
+#pragma unroll
+                    for (int e = 0; e < 32; e += 8) {
+                        uint4 w;
+                        w.x = Fmt<T>::pack_rn(__uint_as_float(v[e]) * inv,
+                                              __uint_as_float(v[e + 1]) * inv);
+                        w.y = Fmt<T>::pack_rn(__uint_as_float(v[e + 2]) * inv,
+                                              __uint_as_float(v[e + 3]) * inv);
+                        w.z = Fmt<T>::pack_rn(__uint_as_float(v[e + 4]) * inv,
+                                              __uint_as_float(v[e + 5]) * inv);
+                        w.w = Fmt<T>::pack_rn(__uint_as_float(v[e + 6]) * inv,
+                                              __uint_as_float(v[e + 7]) * inv);
+                        *reinterpret_cast<uint4 *>(dst + cc * 32 + e) = w;
+                    }
                 }
             }
         }
@@ -539,7 +679,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     // ---- teardown: free the tensor memory (the warp that allocated it)
     tc_fence_before();
     __syncthreads();
-    if (warp == 0) {
+    if (warp == kPfMmaWarp) {
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
                      "r"(kPfTmemCols)
