@@ -12,9 +12,11 @@
 // Work decomposition.  A query tile is 128 rows of one (sequence, kv head): 128/G
 // consecutive tokens times the G query heads that share the kv head (row r = token r / G,
 // head r % G), so one K/V tile read serves all G heads.  A CTA owns two consecutive
-// query tiles, A and B, and walks the keys they need in tiles of 128:
-//   S_X   = Q_X K^T     tcgen05.mma (M 128, N 128, K head_dim): Q_X and K K-major in
-//                       128-byte swizzled shared memory, fp32 S_X in tensor memory;
+// query tiles, A and B, and walks the keys they need in tiles of 64:
+//   S_X   = Q_X K^T     tcgen05.mma (M 128, N 64, K head_dim): Q_X and K K-major in
+//                       128-byte swizzled shared memory, fp32 S_X in tensor memory, two
+//                       buffers per query tile so that the product for key tile j+2 can
+//                       run while the softmax of tile j+1 and P V of tile j are pending;
 //   softmax             a warpgroup per query tile; row r is thread r is tensor-memory
 //                       lane r.  The row is read once into registers (tcgen05.ld),
 //                       masked (causal, window, context end; tiles wholly inside every
@@ -28,9 +30,10 @@
 //                       (skipped in a warp where no row raised its maximum).
 // Roles (warp specialisation): warps 0-3 softmax A, warps 4-7 softmax B, warp 8 issues the
 // matrix products (and zeroes V rows outside the attended keys), warp 9 issues the TMA
-// loads of Q and of a two-stage K/V ring.  The products of one tile overlap the softmax
-// of the other: the tensor core runs P_A V and S_A for the next key tile while the B
-// warpgroup works, and the other way round.  Scores are kept in the log2 domain (scale *
+// loads of Q and of a four-stage K/V ring.  The products of one query tile overlap the
+// softmax of the other, and a query tile's next scores are computed while its current
+// softmax runs.  The reference maximum of a row moves only when the row maximum exceeds
+// it by more than 2^8, so most key tiles need no rescale of O.  Scores are kept in the log2 domain (scale *
 // log2 e folded in), as in the decode kernels.
 //
 // Every wait is bounded: on a timeout a role records PA_DEVERR_TIMEOUT and stops, the
@@ -43,17 +46,20 @@
 namespace pa {
 
 constexpr int kPfRows = 128;        // query rows per tile = UMMA M = tensor-memory lanes
-constexpr int kPfKeys = 128;        // keys per tile = UMMA N of S and K of P.V
+constexpr int kPfKeys = 64;         // keys per tile = UMMA N of S and K of P.V
 constexpr int kPfSoftWarps = 8;     // two softmax warpgroups
 constexpr int kPfMmaWarp = 8;
 constexpr int kPfLoadWarp = 9;
 constexpr int kPfThreads = 320;
-constexpr int kPfStages = 2;        // K/V ring depth
-constexpr int kPfTmemCols = 512;    // tile X: S/P at [256X, 256X + 128), O at [256X + 128, ...)
+constexpr int kPfStages = 4;        // K/V ring depth
+// tensor memory of query tile X: two S/P buffers at [256X, 256X + 64) and [256X + 64,
+// 256X + 128) (key tile i of X uses buffer i % 2), O at [256X + 128, 256X + 128 + D)
+constexpr int kPfTmemCols = 512;
+constexpr float kPfRescaleLog2 = 8.f;  // move the softmax reference max only past 2^8
 
 struct PrefillParams {
     CUtensorMap qmap;  // 3-D [num_tokens][Hq][D] 16-bit, box {64, G, 128/G}, swizzle 128B
-    CUtensorMap kmap;  // 2-D [num_blocks * Hkv * bs][D], box {64, min(bs, 128)}, swizzle 128B
+    CUtensorMap kmap;  // 2-D [num_blocks * Hkv * bs][D], box {64, min(bs, 64)}, swizzle 128B
     CUtensorMap vmap;
     void *out;
     const int32_t *block_tables;
@@ -65,7 +71,7 @@ struct PrefillParams {
     int num_kv_heads;
     int block_size;
     int bs_shift;
-    int box_rows;  // min(block_size, 128)
+    int box_rows;  // min(block_size, 64)
     int num_blocks;
     int max_blocks_per_seq;
     int sliding_window;
@@ -75,14 +81,15 @@ struct PrefillParams {
 template <int D>
 struct PfGeom {
     static constexpr int kHalves = D / 64;                // 128-byte column blocks of a row
-    static constexpr int kRegion = 128 * 128;             // 128 rows of one column block
+    static constexpr int kRegion = kPfRows * 128;         // 128 query rows of one column block
+    static constexpr int kKVRegion = kPfKeys * 128;       // 64 key rows of one column block
     static constexpr int kQ = kHalves * kRegion;          // one Q tile
-    static constexpr int kKV = kHalves * kRegion;         // one K (or V) stage
+    static constexpr int kKV = kHalves * kKVRegion;       // one K (or V) stage
     static constexpr int kOffK = 2 * kQ;
     static constexpr int kOffV = kOffK + kPfStages * kKV;
     static constexpr int kOffBar = kOffV + kPfStages * kKV;
-    // q, k[2], v[2], empty[2], s[2], p[2], o[2]
-    static constexpr int kBars = 1 + 4 * kPfStages + 6;
+    // q, k[stages], v[stages], empty[stages], s[2][2], p[2][2], o[2], fin[2]
+    static constexpr int kBars = 1 + 3 * kPfStages + 12;
     static constexpr int kSmem = kOffBar + 8 * kBars + 1024;  // + alignment slack
 };
 
@@ -174,6 +181,21 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t *r) {
 
 __device__ __forceinline__ void tmem_wait_st() {
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// tcgen05.wait::ld that also names the 32 registers of the load it completes, so the
+// compiler cannot move their uses above it.
+__device__ __forceinline__ void tmem_wait_ld_regs(uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.wait::ld.sync.aligned;"
+        : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),
+          "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]),
+          "+r"(r[13]), "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]),
+          "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]), "+r"(r[24]),
+          "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]),
+          "+r"(r[31])
+        :
+        : "memory");
 }
 
 __device__ __forceinline__ void tmem_wait_ld() {
@@ -309,9 +331,12 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     const uint32_t bar_q = base + Gm::kOffBar;
     const uint32_t bar_k0 = bar_q + 8, bar_v0 = bar_k0 + 8 * kPfStages;
     const uint32_t bar_e0 = bar_v0 + 8 * kPfStages;      // stage empty (all its products done)
-    const uint32_t bar_s0 = bar_e0 + 8 * kPfStages;      // S_X ready, X = 0 (A), 1 (B)
-    const uint32_t bar_p0 = bar_s0 + 16;                 // P_X written, O_X rescaled
-    const uint32_t bar_o0 = bar_p0 + 16;                 // P_X V done
+    // per query tile X = 0 (A), 1 (B) and S/P buffer b: S ready, P written (one barrier
+    // per buffer, so that neither side can get two phases ahead of the other)
+    const uint32_t bar_s0 = bar_e0 + 8 * kPfStages;      // + 8 (2X + b)
+    const uint32_t bar_p0 = bar_s0 + 32;                 // + 8 (2X + b)
+    const uint32_t bar_o0 = bar_p0 + 32;                 // + 8X: P_X V done
+    const uint32_t bar_f0 = bar_o0 + 16;                 // + 8X: every product of X done
     if (tid == 0) {
         tma_prefetch_desc(&p.qmap);
         tma_prefetch_desc(&p.kmap);
@@ -322,10 +347,13 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             mbar_init(bar_v0 + 8 * i, 1);
             mbar_init(bar_e0 + 8 * i, 1);
         }
+        for (int i = 0; i < 4; ++i) {
+            mbar_init(bar_s0 + 8 * i, 1);
+            mbar_init(bar_p0 + 8 * i, 4);  // one arrival per softmax warp
+        }
         for (int x = 0; x < 2; ++x) {
-            mbar_init(bar_s0 + 8 * x, 1);
-            mbar_init(bar_p0 + 8 * x, 4);  // one arrival per softmax warp
             mbar_init(bar_o0 + 8 * x, 1);
+            mbar_init(bar_f0 + 8 * x, 1);
         }
         fence_barrier_init();
     }
@@ -394,7 +422,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                                           (r0 & (p.block_size - 1));
 #pragma unroll
                             for (int hf = 0; hf < Gm::kHalves; ++hf) {
-                                const uint32_t off = hf * Gm::kRegion + b * BR * 128;
+                                const uint32_t off = hf * Gm::kKVRegion + b * BR * 128;
                                 tma_load_2d(sk + st * Gm::kKV + off, &p.kmap, bk, 64 * hf, y, pol);
                                 tma_load_2d(sv + st * Gm::kKV + off, &p.vmap, bv, 64 * hf, y, pol);
                             }
@@ -421,58 +449,64 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         };
         bool ok = wait_all(bar_q, 0);
         auto need = [&](const PfTile &t, int jt) { return t.live && jt >= t.j0 && jt < t.j1; };
-        auto issue_s = [&](int x, int jt) {  // S_X = Q_X K_jt
-            const int st = (jt - j0) % kPfStages;
+        const PfTile *tl[2] = {&ta, &tb};
+        auto stage_of = [&](int jt) { return (jt - j0) % kPfStages; };
+        auto phase_of = [&](int jt) { return (uint32_t)(((jt - j0) / kPfStages) & 1); };
+        // S_X = Q_X K_jt into X's buffer (jt - j0_X) % 2
+        auto issue_s = [&](int x, int jt) {
+            const int st = stage_of(jt);
+            const int b = (jt - tl[x]->j0) & 1;
+            const uint32_t dcol = 256 * x + 64 * b;
             if (lane == 0) {
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t koff = (kk >> 2) * Gm::kRegion + (kk & 3) * 32;
-                    umma_f16(tmem + 256 * x, umma_desc_sw128(sq + x * Gm::kQ + koff, 16),
+                    const uint32_t qoff = (kk >> 2) * Gm::kRegion + (kk & 3) * 32;
+                    const uint32_t koff = (kk >> 2) * Gm::kKVRegion + (kk & 3) * 32;
+                    umma_f16(tmem + dcol, umma_desc_sw128(sq + x * Gm::kQ + qoff, 16),
                              umma_desc_sw128(sk + st * Gm::kKV + koff, 16), idesc_s, kk > 0);
                 }
-                umma_commit(bar_s0 + 8 * x);
+                umma_commit(bar_s0 + 8 * (2 * x + b));
             }
             __syncwarp();
         };
-        auto issue_pv = [&](int x, int jt, bool first) {  // O_X += P_X V_jt (high, low)
-            const int st = (jt - j0) % kPfStages;
+        // O_X += P_X V_jt (high, then low part of P from X's buffer)
+        auto issue_pv = [&](int x, int jt) {
+            const int st = stage_of(jt);
+            const uint32_t pcol = 256 * x + 64 * ((jt - tl[x]->j0) & 1);
+            const bool first = jt == tl[x]->j0;
             if (lane == 0) {
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < 2 * (kPfKeys / 16); ++kk) {
                     const int k = kk % (kPfKeys / 16);
-                    const uint32_t acol = 256 * x + (k >> 2) * 64 + (kk >= kPfKeys / 16 ? 32 : 0) +
-                                          (k & 3) * 8;
+                    const uint32_t acol = pcol + (kk >= kPfKeys / 16 ? 32 : 0) + k * 8;
                     umma_f16_ts(tmem + 256 * x + 128, tmem + acol,
-                                umma_desc_sw128(sv + st * Gm::kKV + k * 16 * 128, Gm::kRegion),
+                                umma_desc_sw128(sv + st * Gm::kKV + k * 16 * 128, Gm::kKVRegion),
                                 idesc_o, (!first || kk > 0) ? 1u : 0u);
                 }
                 umma_commit(bar_o0 + 8 * x);
             }
             __syncwarp();
         };
-        // per-tile counters of the products already issued (for the barrier parities)
-        int ns[2] = {0, 0}, npv[2] = {0, 0};
-        const PfTile *tl[2] = {&ta, &tb};
-        if (ok && !__any_sync(0xffffffffu, sh_fail != 0)) {
-            ok = wait_all(bar_k0, 0);
-            if (ok) {
-                for (int x = 0; x < 2; ++x)
-                    if (need(*tl[x], j0)) issue_s(x, j0), ++ns[x];
-            }
+        int npv[2] = {0, 0};
+        // prologue: S of the first two key tiles
+        for (int jn = j0; ok && jn < min(j1, j0 + 2); ++jn) {
+            ok = wait_all(bar_k0 + 8 * stage_of(jn), phase_of(jn));
+            if (!ok) break;
+            for (int x = 0; x < 2; ++x)
+                if (need(*tl[x], jn)) issue_s(x, jn);
         }
         for (int jt = j0; ok && jt < j1; ++jt) {
             if (__any_sync(0xffffffffu, sh_fail != 0)) {
                 ok = false;
                 break;
             }
-            const int it = jt - j0, st = it % kPfStages;
-            const uint32_t ph = (uint32_t)((it / kPfStages) & 1);
+            const int st = stage_of(jt);
             const int kv0 = jt * kPfKeys;
             // V of this tile; rows outside [kv_begin, L) (not loaded, or past the context)
             // -> 0 so that zero weights cannot meet a NaN
-            ok = wait_all(bar_v0 + 8 * st, ph);
+            ok = wait_all(bar_v0 + 8 * st, phase_of(jt));
             if (!ok) break;
             if (kv0 < kv_begin || kv0 + kPfKeys > L) {
                 const int lo = max(0, kv_begin - kv0), hi = min(kPfKeys, L - kv0);
@@ -480,7 +514,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                     const int r = idx / (Gm::kHalves * 8), c = idx % (Gm::kHalves * 8);
                     if (r < lo || r >= hi)
                         asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(
-                                         sv + st * Gm::kKV + (c >> 3) * Gm::kRegion + r * 128 +
+                                         sv + st * Gm::kKV + (c >> 3) * Gm::kKVRegion + r * 128 +
                                          (c & 7) * 16),
                                      "r"(0)
                                      : "memory");
@@ -488,48 +522,56 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                 fence_proxy_async_smem();
                 __syncwarp();
             }
-            const bool has_next = jt + 1 < j1;
-            if (has_next) {
-                const int st1 = (it + 1) % kPfStages;
-                ok = wait_all(bar_k0 + 8 * st1, (uint32_t)(((it + 1) / kPfStages) & 1));
-                if (!ok) break;
-            }
             for (int x = 0; x < 2 && ok; ++x) {
-                const PfTile &t = *tl[x];
-                if (need(t, jt)) {
-                    ok = wait_all(bar_p0 + 8 * x, (uint32_t)(npv[x] & 1));
-                    if (!ok) break;
-                    issue_pv(x, jt, npv[x] == 0);
-                    ++npv[x];
-                }
-                if (has_next && need(t, jt + 1)) {
-                    if (need(t, jt)) {  // P_X (in S_X's columns) has been read: O_X done
+                if (!need(*tl[x], jt)) continue;
+                const int i = jt - tl[x]->j0;
+                ok = wait_all(bar_p0 + 8 * (2 * x + (i & 1)), (uint32_t)((i >> 1) & 1));
+                if (!ok) break;
+                issue_pv(x, jt);
+                ++npv[x];
+            }
+            // S two key tiles ahead, into the buffer this tile's P V reads: after that
+            // P V has finished
+            const int jn = jt + 2;
+            if (ok && jn < j1) {
+                ok = wait_all(bar_k0 + 8 * stage_of(jn), phase_of(jn));
+                for (int x = 0; x < 2 && ok; ++x) {
+                    if (!need(*tl[x], jn)) continue;
+                    if (need(*tl[x], jt)) {
                         ok = wait_all(bar_o0 + 8 * x, (uint32_t)((npv[x] - 1) & 1));
                         if (!ok) break;
                     }
-                    issue_s(x, jt + 1);
-                    ++ns[x];
+                    issue_s(x, jn);
                 }
             }
             if (!ok) break;
             if (lane == 0) umma_commit(bar_e0 + 8 * st);  // every product reading stage st
             __syncwarp();
         }
-        if (!ok) {
+        if (ok) {
+            // one commit per live query tile: completes when every product issued so far
+            // (its last P V included) has finished
+            if (lane == 0)
+                for (int x = 0; x < 2; ++x)
+                    if (tl[x]->live) umma_commit(bar_f0 + 8 * x);
+            __syncwarp();
+        } else {
             if (lane == 0) raise_error(PA_DEVERR_TIMEOUT);
             sh_fail = 1;
+            // cleanup: the products issued so far have finished (bounded)
+            if (lane == 0) {
+                umma_commit(bar_f0);
+                (void)mbar_wait_bounded(bar_f0, 0);
+            }
+            __syncwarp();
         }
-        // cleanup: the newest products have finished (bounded)
-        for (int x = 0; x < 2; ++x)
-            if (npv[x] > 0) (void)mbar_wait_bounded(bar_o0 + 8 * x, (uint32_t)((npv[x] - 1) & 1));
-        (void)ns;
     } else {
         // ============================ softmax warpgroup X (rows = threads 128X .. 128X+127)
         const int x = warp / 4;
         const PfTile &t = x == 0 ? ta : tb;
         const int row = tid & 127;
         const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-        const uint32_t tS = tmem + 256 * x + lane_off, tO = tS + 128;
+        const uint32_t tO = tmem + 256 * x + 128 + lane_off;
         const int rtok = row / G, rh = row % G;
         const bool rvalid = t.live && rtok < t.ntok;
         const int rpos = rvalid ? t.pos0 + rtok : -1;
@@ -547,7 +589,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                 break;
             }
             const int kv0 = jt * kPfKeys;
-            ok = mbar_wait_bounded(bar_s0 + 8 * x, (uint32_t)(i & 1));
+            const uint32_t tS = tmem + 256 * x + 64 * (i & 1) + lane_off;  // S/P buffer
+            ok = mbar_wait_bounded(bar_s0 + 8 * (2 * x + (i & 1)), (uint32_t)((i >> 1) & 1));
             if (!__all_sync(0xffffffffu, ok)) {
                 ok = false;
                 break;
@@ -557,80 +600,95 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             // loaded keys: no per-element mask
             const bool full = all_rows && kv0 + kPfKeys - 1 <= key_all_hi && kv0 >= key_all_lo &&
                               kv0 >= kv_begin;
-            // scaled, masked scores of keys 64h .. 64h+63 of this row
-            auto load_half = [&](int h, uint32_t (&v)[64]) {
-                tmem_ld32(tS + 64 * h, *reinterpret_cast<uint32_t(*)[32]>(v));
-                tmem_ld32(tS + 64 * h + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
-                tmem_wait_ld();
+            // scaled, masked scores of keys 32c .. 32c+31 of this row, in place
+            auto scale_mask = [&](int c, uint32_t (&v)[32]) {
                 if (full) {
 #pragma unroll
-                    for (int e = 0; e < 64; ++e)
+                    for (int e = 0; e < 32; ++e)
                         v[e] = __float_as_uint(__uint_as_float(v[e]) * p.scale_log2);
                 } else {
 #pragma unroll
-                    for (int e = 0; e < 64; ++e) {
-                        const int key = kv0 + 64 * h + e;
+                    for (int e = 0; e < 32; ++e) {
+                        const int key = kv0 + 32 * c + e;
                         const bool in = key <= rpos && key >= rlo && key >= kv_begin;
                         v[e] = __float_as_uint(in ? __uint_as_float(v[e]) * p.scale_log2
                                                   : -INFINITY);
                     }
                 }
             };
+            // pass 1: the tile's row maximum; the load of chunk c+1 overlaps chunk c
             float mx = -INFINITY;
+            {
+                uint32_t va[32], vb[32];
+                tmem_ld32(tS, va);
+                tmem_wait_ld_regs(va);
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                uint32_t v[64];
-                load_half(h, v);
+                for (int c = 0; c < kPfKeys / 32; ++c) {
+                    uint32_t(&cur)[32] = (c & 1) ? vb : va;
+                    uint32_t(&nxt)[32] = (c & 1) ? va : vb;
+                    if (c + 1 < kPfKeys / 32) tmem_ld32(tS + 32 * (c + 1), nxt);
+                    scale_mask(c, cur);
 #pragma unroll
-                for (int e = 0; e < 64; ++e) mx = fmaxf(mx, __uint_as_float(v[e]));
+                    for (int e = 0; e < 32; ++e) mx = fmaxf(mx, __uint_as_float(cur[e]));
+                    if (c + 1 < kPfKeys / 32) tmem_wait_ld_regs(nxt);
+                }
             }
-            const float m_new = fmaxf(m_run, mx);
-            const float alpha = (m_new == -INFINITY) ? 1.f : fast_exp2(m_run - m_new);
-            // the previous P_X V has finished: rescale O_X (and P_X's columns are free)
-            if (i > 0) {
+            // The reference maximum moves only when the row maximum exceeds it by more
+            // than 2^8 (weights stay <= 256; O and l share the reference, so the result is
+            // exact either way) -- most tiles then need no rescale of O.
+            const bool upd = mx > m_run + kPfRescaleLog2 || (m_run == -INFINITY && mx > -INFINITY);
+            const float m_new = upd ? mx : m_run;
+            const float alpha = (upd && m_run != -INFINITY) ? fast_exp2(m_run - m_new) : 1.f;
+            // a row of this warp moved its reference: once the previous P_X V has
+            // finished, rescale the warp's rows of O_X (otherwise the next P V simply
+            // accumulates onto O_X after the previous one, same accumulator, in order)
+            if (i > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
                 ok = mbar_wait_bounded(bar_o0 + 8 * x, (uint32_t)((i - 1) & 1));
                 if (!__all_sync(0xffffffffu, ok)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                if (__any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll
-                    for (int cc = 0; cc < D / 32; ++cc) {
-                        uint32_t o[32];
-                        tmem_ld32(tO + cc * 32, o);
-                        tmem_wait_ld();
+                for (int cc = 0; cc < D / 32; ++cc) {
+                    uint32_t o[32];
+                    tmem_ld32(tO + cc * 32, o);
+                    tmem_wait_ld_regs(o);
 #pragma unroll
-                        for (int e = 0; e < 32; ++e)
-                            o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-                        tmem_st32(tO + cc * 32, o);
-                    }
+                    for (int e = 0; e < 32; ++e)
+                        o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+                    tmem_st32(tO + cc * 32, o);
                 }
             }
-            // P = hi + lo, written over S: keys 64h .. 64h+63 -> high part in columns
-            // 64h .. 64h+31, low part in 64h+32 .. 64h+63 (two keys per column).  A row
-            // with nothing attended yet (m = -inf) gets zeros.  Each half is read again
-            // before any of it is overwritten.
+            // pass 2: P = hi + lo, written over S in its buffer: the 64 keys' high part in
+            // columns 0 .. 31, the low part in 32 .. 63 (two keys per column).  A row with
+            // nothing attended yet (m = -inf) gets zeros.  Chunk 1 is loaded before chunk 0
+            // is stored (chunk 0's low part lands in chunk 1's columns).
             const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
             float sum = 0.f;
+            {
+                uint32_t va[32], vb[32];
+                tmem_ld32(tS, va);
+                tmem_wait_ld_regs(va);
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                uint32_t v[64];
-                load_half(h, v);
-#pragma unroll
-                for (int c = 0; c < 2; ++c) {
+                for (int c = 0; c < kPfKeys / 32; ++c) {
+                    uint32_t(&cur)[32] = (c & 1) ? vb : va;
+                    uint32_t(&nxt)[32] = (c & 1) ? va : vb;
+                    if (c + 1 < kPfKeys / 32) tmem_ld32(tS + 32 * (c + 1), nxt);
+                    scale_mask(c, cur);
                     uint32_t ph_[16], pl_[16];
 #pragma unroll
                     for (int e = 0; e < 32; e += 2) {
-                        const float p0 = fast_exp2(__uint_as_float(v[32 * c + e]) - m_use);
-                        const float p1 = fast_exp2(__uint_as_float(v[32 * c + e + 1]) - m_use);
+                        const float p0 = fast_exp2(__uint_as_float(cur[e]) - m_use);
+                        const float p1 = fast_exp2(__uint_as_float(cur[e + 1]) - m_use);
                         sum += p0 + p1;
                         ph_[e >> 1] = Fmt<T>::pack_rn(p0, p1);
                         const float2 hv = Fmt<T>::unpack(ph_[e >> 1]);
                         pl_[e >> 1] = Fmt<T>::pack_rn(p0 - hv.x, p1 - hv.y);
                     }
-                    tmem_st16(tS + 64 * h + 16 * c, ph_);
-                    tmem_st16(tS + 64 * h + 32 + 16 * c, pl_);
+                    if (c + 1 < kPfKeys / 32) tmem_wait_ld_regs(nxt);
+                    tmem_st16(tS + 16 * c, ph_);
+                    tmem_st16(tS + 32 + 16 * c, pl_);
                 }
             }
             tmem_wait_st();
@@ -638,10 +696,10 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             m_run = m_new;
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(bar_p0 + 8 * x);
+            if (lane == 0) mbar_arrive(bar_p0 + 8 * (2 * x + (i & 1)));
         }
         if (t.live && ok && i > 0) {
-            ok = mbar_wait_bounded(bar_o0 + 8 * x, (uint32_t)((i - 1) & 1));
+            ok = mbar_wait_bounded(bar_f0 + 8 * x, 0);
             ok = __all_sync(0xffffffffu, ok);
         }
         if (!ok) {
@@ -656,7 +714,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             for (int cc = 0; cc < D / 32; ++cc) {
                 uint32_t v[32];
                 tmem_ld32(tO + cc * 32, v);
-                tmem_wait_ld();
+                tmem_wait_ld_regs(v);
                 if (rvalid) {
 #pragma unroll
                     for (int e = 0; e < 32; e += 8) {
