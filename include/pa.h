@@ -261,6 +261,7 @@ pa_status pa_decode_static_scratch(void *out, const void *q, const void *k_cache
  *
  * q, out          : [num_tokens][num_q_heads][head_dim], contiguous, 16-byte aligned.
  * query_start_loc : int32 [num_seqs + 1], non-decreasing, [0] = 0, [num_seqs] = num_tokens.
+ * scale           : > 0 (1/sqrt(d_k)); other values are PA_ERR_INVALID_ARG.
  * Other arguments : as pa_decode (head_dim 64 or 128, G in {1, 2, 4, 8}, block_size a
  *                   power of two in [8, 512]).
  * Math: S = Q K^T and O = P V on the tcgen05 tensor cores (fp32 accumulation in tensor

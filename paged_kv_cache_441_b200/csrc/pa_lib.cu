@@ -807,7 +807,7 @@ extern "C" pa_status pa_prefill(void *out, const void *q, const void *k_cache,
     if (dtype != PA_FP16 && dtype != PA_BF16) return PA_ERR_INVALID_ARG;
     if (num_seqs < 0 || num_tokens < 0 || num_q_heads <= 0 || num_kv_heads <= 0 ||
         num_blocks <= 0 || max_blocks_per_seq <= 0 || sliding_window < 0 ||
-        !std::isfinite(scale))
+        !std::isfinite(scale) || !(scale > 0.f))
         return PA_ERR_INVALID_ARG;
     if (num_q_heads % num_kv_heads != 0) return PA_ERR_INVALID_ARG;
     const int G = num_q_heads / num_kv_heads;

@@ -56,6 +56,11 @@ constexpr int kPfStages = 4;        // K/V ring depth
 // 256X + 128) (key tile i of X uses buffer i % 2), O at [256X + 128, 256X + 128 + D)
 constexpr int kPfTmemCols = 512;
 constexpr float kPfRescaleLog2 = 8.f;  // move the softmax reference max only past 2^8
+#ifndef PA_PREFILL_SPLIT_P
+#define PA_PREFILL_SPLIT_P 1
+#endif
+// P as high + low 16-bit parts (two P V products): weights keep ~16 significant bits
+constexpr bool kPfSplitP = PA_PREFILL_SPLIT_P != 0;
 
 struct PrefillParams {
     CUtensorMap qmap;  // 3-D [num_tokens][Hq][D] 16-bit, box {64, G, 128/G}, swizzle 128B
@@ -478,7 +483,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             if (lane == 0) {
                 tc_fence_after();
 #pragma unroll
-                for (int kk = 0; kk < 2 * (kPfKeys / 16); ++kk) {
+                for (int kk = 0; kk < (kPfSplitP ? 2 : 1) * (kPfKeys / 16); ++kk) {
                     const int k = kk % (kPfKeys / 16);
                     const uint32_t acol = pcol + (kk >= kPfKeys / 16 ? 32 : 0) + k * 8;
                     umma_f16_ts(tmem + 256 * x + 128, tmem + acol,
@@ -600,24 +605,12 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             // loaded keys: no per-element mask
             const bool full = all_rows && kv0 + kPfKeys - 1 <= key_all_hi && kv0 >= key_all_lo &&
                               kv0 >= kv_begin;
-            // scaled, masked scores of keys 32c .. 32c+31 of this row, in place
-            auto scale_mask = [&](int c, uint32_t (&v)[32]) {
-                if (full) {
+            const float c2 = p.scale_log2;  // > 0 (checked on the host)
+            // pass 1: the tile's row maximum of the raw scores (8 independent partial
+            // maxima; scale > 0 keeps the order); the load of chunk c+1 overlaps chunk c
+            float mxp[8];
 #pragma unroll
-                    for (int e = 0; e < 32; ++e)
-                        v[e] = __float_as_uint(__uint_as_float(v[e]) * p.scale_log2);
-                } else {
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        const int key = kv0 + 32 * c + e;
-                        const bool in = key <= rpos && key >= rlo && key >= kv_begin;
-                        v[e] = __float_as_uint(in ? __uint_as_float(v[e]) * p.scale_log2
-                                                  : -INFINITY);
-                    }
-                }
-            };
-            // pass 1: the tile's row maximum; the load of chunk c+1 overlaps chunk c
-            float mx = -INFINITY;
+            for (int k = 0; k < 8; ++k) mxp[k] = -INFINITY;
             {
                 uint32_t va[32], vb[32];
                 tmem_ld32(tS, va);
@@ -627,12 +620,24 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                     uint32_t(&cur)[32] = (c & 1) ? vb : va;
                     uint32_t(&nxt)[32] = (c & 1) ? va : vb;
                     if (c + 1 < kPfKeys / 32) tmem_ld32(tS + 32 * (c + 1), nxt);
-                    scale_mask(c, cur);
+                    if (full) {
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) mx = fmaxf(mx, __uint_as_float(cur[e]));
+                        for (int e = 0; e < 32; ++e)
+                            mxp[e & 7] = fmaxf(mxp[e & 7], __uint_as_float(cur[e]));
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) {
+                            const int key = kv0 + 32 * c + e;
+                            const bool in = key <= rpos && key >= rlo && key >= kv_begin;
+                            mxp[e & 7] = fmaxf(mxp[e & 7], in ? __uint_as_float(cur[e]) : -INFINITY);
+                        }
+                    }
                     if (c + 1 < kPfKeys / 32) tmem_wait_ld_regs(nxt);
                 }
             }
+            const float mraw = fmaxf(fmaxf(fmaxf(mxp[0], mxp[1]), fmaxf(mxp[2], mxp[3])),
+                                     fmaxf(fmaxf(mxp[4], mxp[5]), fmaxf(mxp[6], mxp[7])));
+            const float mx = mraw * c2;  // -inf stays -inf
             // The reference maximum moves only when the row maximum exceeds it by more
             // than 2^8 (weights stay <= 256; O and l share the reference, so the result is
             // exact either way) -- most tiles then need no rescale of O.
@@ -665,7 +670,9 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             // nothing attended yet (m = -inf) gets zeros.  Chunk 1 is loaded before chunk 0
             // is stored (chunk 0's low part lands in chunk 1's columns).
             const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-            float sum = 0.f;
+            float sump[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) sump[k] = 0.f;
             {
                 uint32_t va[32], vb[32];
                 tmem_ld32(tS, va);
@@ -675,23 +682,39 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                     uint32_t(&cur)[32] = (c & 1) ? vb : va;
                     uint32_t(&nxt)[32] = (c & 1) ? va : vb;
                     if (c + 1 < kPfKeys / 32) tmem_ld32(tS + 32 * (c + 1), nxt);
-                    scale_mask(c, cur);
+                    // exponent = score * scale log2 e - reference, one FFMA; masked -> 0
+                    float xe[32];
+                    if (full) {
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) xe[e] = fmaf(__uint_as_float(cur[e]), c2, -m_use);
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) {
+                            const int key = kv0 + 32 * c + e;
+                            const bool in = key <= rpos && key >= rlo && key >= kv_begin;
+                            xe[e] = in ? fmaf(__uint_as_float(cur[e]), c2, -m_use) : -INFINITY;
+                        }
+                    }
                     uint32_t ph_[16], pl_[16];
 #pragma unroll
                     for (int e = 0; e < 32; e += 2) {
-                        const float p0 = fast_exp2(__uint_as_float(cur[e]) - m_use);
-                        const float p1 = fast_exp2(__uint_as_float(cur[e + 1]) - m_use);
-                        sum += p0 + p1;
+                        const float p0 = fast_exp2(xe[e]);
+                        const float p1 = fast_exp2(xe[e + 1]);
+                        sump[(e >> 1) & 7] += p0 + p1;
                         ph_[e >> 1] = Fmt<T>::pack_rn(p0, p1);
-                        const float2 hv = Fmt<T>::unpack(ph_[e >> 1]);
-                        pl_[e >> 1] = Fmt<T>::pack_rn(p0 - hv.x, p1 - hv.y);
+                        if (kPfSplitP) {
+                            const float2 hv = Fmt<T>::unpack(ph_[e >> 1]);
+                            pl_[e >> 1] = Fmt<T>::pack_rn(p0 - hv.x, p1 - hv.y);
+                        }
                     }
                     if (c + 1 < kPfKeys / 32) tmem_wait_ld_regs(nxt);
                     tmem_st16(tS + 16 * c, ph_);
-                    tmem_st16(tS + 32 + 16 * c, pl_);
+                    if (kPfSplitP) tmem_st16(tS + 32 + 16 * c, pl_);
                 }
             }
             tmem_wait_st();
+            const float sum = ((sump[0] + sump[1]) + (sump[2] + sump[3])) +
+                              ((sump[4] + sump[5]) + (sump[6] + sump[7]));
             l_run = l_run * alpha + sum;
             m_run = m_new;
             tc_fence_before();

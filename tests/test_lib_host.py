@@ -136,7 +136,8 @@ def _call_prefill(lib, **over):
 @pytest.mark.parametrize("over,code", [
     (dict(d=96), 2), (dict(hq=6), 2), (dict(hq=7), 1), (dict(hq=32), 2), (dict(bs=24), 2),
     (dict(bs=1024), 2), (dict(q=0), 1), (dict(q=24), 1), (dict(qsl=0), 1), (dict(qsl=2), 1),
-    (dict(win=-1), 1), (dict(scale=float("nan")), 1), (dict(dt=7), 1), (dict(T=-1), 1),
+    (dict(win=-1), 1), (dict(scale=float("nan")), 1), (dict(scale=0.0), 1),
+    (dict(scale=-0.1), 1), (dict(dt=7), 1), (dict(T=-1), 1),
     (dict(B=0), 0), (dict(T=0), 0),
 ])
 def test_prefill_rejects_before_launch(lib, over, code):
