@@ -28,9 +28,9 @@
 //                       products (high and low part) so the weights keep ~16 bits; before
 //                       it the warpgroup rescales its rows of O_X by 2^(m_old - m_new)
 //                       (skipped in a warp where no row raised its maximum).
-// Roles (warp specialisation): warps 0-3 softmax A, warps 4-7 softmax B, warp 8 issues the
-// matrix products (and zeroes V rows outside the attended keys), warp 9 issues the TMA
-// loads of Q and of a four-stage K/V ring.  The products of one query tile overlap the
+// Roles (warp specialisation): warps 0-3 softmax A, warps 4-7 softmax B, warps 8 and 9
+// issue the matrix products of A and of B, warp 10 issues the TMA loads of Q and of a
+// four-stage K/V ring (and zeroes the V rows of edge tiles outside the attended keys).  The products of one query tile overlap the
 // softmax of the other, and a query tile's next scores are computed while its current
 // softmax runs.  The reference maximum of a row moves only when the row maximum exceeds
 // it by more than 2^8, so most key tiles need no rescale of O.  Scores are kept in the log2 domain (scale *
@@ -48,9 +48,9 @@ namespace pa {
 constexpr int kPfRows = 128;        // query rows per tile = UMMA M = tensor-memory lanes
 constexpr int kPfKeys = 64;         // keys per tile = UMMA N of S and K of P.V
 constexpr int kPfSoftWarps = 8;     // two softmax warpgroups
-constexpr int kPfMmaWarp = 8;
-constexpr int kPfLoadWarp = 9;
-constexpr int kPfThreads = 320;
+constexpr int kPfMmaWarp = 8;       // warps 8 and 9: the products of query tiles A and B
+constexpr int kPfLoadWarp = 10;
+constexpr int kPfThreads = 352;
 constexpr int kPfStages = 4;        // K/V ring depth
 // tensor memory of query tile X: two S/P buffers at [256X, 256X + 64) and [256X + 64,
 // 256X + 128) (key tile i of X uses buffer i % 2), O at [256X + 128, 256X + 128 + D)
@@ -93,8 +93,8 @@ struct PfGeom {
     static constexpr int kOffK = 2 * kQ;
     static constexpr int kOffV = kOffK + kPfStages * kKV;
     static constexpr int kOffBar = kOffV + kPfStages * kKV;
-    // q, k[stages], v[stages], empty[stages], s[2][2], p[2][2], o[2], fin[2]
-    static constexpr int kBars = 1 + 3 * kPfStages + 12;
+    // q, k[stages], v[stages], v_edge[stages], empty[stages], s[2][2], p[2][2], o[2], fin[2]
+    static constexpr int kBars = 1 + 4 * kPfStages + 12;
     static constexpr int kSmem = kOffBar + 8 * kBars + 1024;  // + alignment slack
 };
 
@@ -335,7 +335,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     const uint32_t sq = base, sk = base + Gm::kOffK, sv = base + Gm::kOffV;
     const uint32_t bar_q = base + Gm::kOffBar;
     const uint32_t bar_k0 = bar_q + 8, bar_v0 = bar_k0 + 8 * kPfStages;
-    const uint32_t bar_e0 = bar_v0 + 8 * kPfStages;      // stage empty (all its products done)
+    const uint32_t bar_vt0 = bar_v0 + 8 * kPfStages;     // V of an edge tile landed (producer)
+    const uint32_t bar_e0 = bar_vt0 + 8 * kPfStages;     // stage empty (both MMA warps)
     // per query tile X = 0 (A), 1 (B) and S/P buffer b: S ready, P written (one barrier
     // per buffer, so that neither side can get two phases ahead of the other)
     const uint32_t bar_s0 = bar_e0 + 8 * kPfStages;      // + 8 (2X + b)
@@ -350,7 +351,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         for (int i = 0; i < kPfStages; ++i) {
             mbar_init(bar_k0 + 8 * i, 1);
             mbar_init(bar_v0 + 8 * i, 1);
-            mbar_init(bar_e0 + 8 * i, 1);
+            mbar_init(bar_vt0 + 8 * i, 1);
+            mbar_init(bar_e0 + 8 * i, 2);  // one commit per MMA warp
         }
         for (int i = 0; i < 4; ++i) {
             mbar_init(bar_s0 + 8 * i, 1);
@@ -362,7 +364,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         }
         fence_barrier_init();
     }
-    if (warp == kPfMmaWarp) {
+    if (warp == kPfLoadWarp) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                          smem_u32(&sh_tmem)),
                      "r"(kPfTmemCols)
@@ -375,11 +377,11 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     const uint32_t tmem = sh_tmem;
 
     if (warp == kPfLoadWarp) {
-        // ============================ TMA producer (lane 0)
+        // ============================ TMA producer (lane 0 issues; the warp zeroes edge V)
+        const int32_t *table = p.block_tables + (size_t)s * p.max_blocks_per_seq;
+        const int BR = p.box_rows;
+        const uint64_t pol = l2_policy_evict_first();
         if (lane == 0) {
-            const int32_t *table = p.block_tables + (size_t)s * p.max_blocks_per_seq;
-            const int BR = p.box_rows;
-            const uint64_t pol = l2_policy_evict_first();
             mbar_arrive_expect_tx(bar_q, (uint32_t)((tb.live ? 2 : 1) * Gm::kQ));
 #pragma unroll
             for (int hf = 0; hf < Gm::kHalves; ++hf) {
@@ -388,37 +390,47 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                     tma_load_3d(sq + Gm::kQ + hf * Gm::kRegion, &p.qmap, bar_q, 64 * hf, g * G,
                                 q0 + tb.tok0);
             }
-            int issued = j0;
-            for (int jt = j0; jt < j1; ++jt) {
-                const int it = jt - j0, st = it % kPfStages;
-                if (it >= kPfStages &&
-                    !mbar_wait_bounded(bar_e0 + 8 * st, (uint32_t)(((it / kPfStages) - 1) & 1))) {
-                    raise_error(PA_DEVERR_TIMEOUT);
-                    sh_fail = 1;
-                    break;
+        }
+        int issued = j0;
+        int vt_uses[kPfStages];
+#pragma unroll
+        for (int i = 0; i < kPfStages; ++i) vt_uses[i] = 0;
+        bool ok = true;
+        for (int jt = j0; jt < j1 && ok; ++jt) {
+            const int it = jt - j0, st = it % kPfStages;
+            if (it >= kPfStages) {
+                ok = __all_sync(0xffffffffu, mbar_wait_bounded(
+                                                 bar_e0 + 8 * st,
+                                                 (uint32_t)(((it / kPfStages) - 1) & 1)));
+                if (!ok) break;
+            }
+            if (__any_sync(0xffffffffu, sh_fail != 0)) {
+                ok = false;
+                break;
+            }
+            const int kv0 = jt * kPfKeys;
+            int nload = 0;
+            bool tab_ok = true;
+            for (int b = 0; b < kPfKeys / BR; ++b) {
+                const int r0 = kv0 + b * BR;
+                if (r0 < L && r0 + BR > kv_begin) {
+                    ++nload;
+                    const int blk = __ldg(table + (r0 >> p.bs_shift));
+                    tab_ok = tab_ok && (unsigned)blk < (unsigned)p.num_blocks;
                 }
-                if (sh_fail) break;
-                const int kv0 = jt * kPfKeys;
-                int nload = 0;
-                bool ok = true;
-                for (int b = 0; b < kPfKeys / BR; ++b) {
-                    const int r0 = kv0 + b * BR;
-                    if (r0 < L && r0 + BR > kv_begin) {
-                        ++nload;
-                        const int blk = __ldg(table + (r0 >> p.bs_shift));
-                        ok = ok && (unsigned)blk < (unsigned)p.num_blocks;
-                    }
-                }
-                const uint32_t bk = bar_k0 + 8 * st, bv = bar_v0 + 8 * st;
-                if (!ok) {
-                    // nothing loaded: the consumers see the stage as all-masked
-                    raise_error(PA_DEVERR_BLOCK_ID);
-                    nload = 0;
-                }
-                const uint32_t bytes = (uint32_t)(nload * BR * 128 * Gm::kHalves);
+            }
+            if (!tab_ok) nload = 0;  // nothing loaded: the tile reads as all-masked
+            // an edge tile (keys outside [kv_begin, L), or a bad table entry): its V lands
+            // on a private barrier, the rows outside the attended keys are zeroed, then V
+            // is released
+            const bool edge = !tab_ok || kv0 < kv_begin || kv0 + kPfKeys > L;
+            const uint32_t bk = bar_k0 + 8 * st, bv = bar_v0 + 8 * st, bvt = bar_vt0 + 8 * st;
+            const uint32_t bytes = (uint32_t)(nload * BR * 128 * Gm::kHalves);
+            if (lane == 0) {
+                if (!tab_ok) raise_error(PA_DEVERR_BLOCK_ID);
                 mbar_arrive_expect_tx(bk, bytes);
-                mbar_arrive_expect_tx(bv, bytes);
-                if (ok) {
+                mbar_arrive_expect_tx(edge ? bvt : bv, bytes);
+                if (tab_ok) {
                     for (int b = 0; b < kPfKeys / BR; ++b) {
                         const int r0 = kv0 + b * BR;
                         if (r0 < L && r0 + BR > kv_begin) {
@@ -429,92 +441,22 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                             for (int hf = 0; hf < Gm::kHalves; ++hf) {
                                 const uint32_t off = hf * Gm::kKVRegion + b * BR * 128;
                                 tma_load_2d(sk + st * Gm::kKV + off, &p.kmap, bk, 64 * hf, y, pol);
-                                tma_load_2d(sv + st * Gm::kKV + off, &p.vmap, bv, 64 * hf, y, pol);
+                                tma_load_2d(sv + st * Gm::kKV + off, &p.vmap, edge ? bvt : bv,
+                                            64 * hf, y, pol);
                             }
                         }
                     }
                 }
-                issued = jt + 1;
-            }
-            // cleanup: the loads this CTA issued have landed (bounded)
-            (void)mbar_wait_bounded(bar_q, 0);
-            for (int jt = max(j0, issued - kPfStages); jt < issued; ++jt) {
-                const int it = jt - j0, st = it % kPfStages;
-                const uint32_t ph = (uint32_t)((it / kPfStages) & 1);
-                (void)mbar_wait_bounded(bar_k0 + 8 * st, ph);
-                (void)mbar_wait_bounded(bar_v0 + 8 * st, ph);
-            }
-        }
-    } else if (warp == kPfMmaWarp) {
-        // ============================ matrix products (lane 0 issues; the warp waits)
-        const uint32_t idesc_s = umma_idesc<T>(kPfRows, kPfKeys, false);
-        const uint32_t idesc_o = umma_idesc<T>(kPfRows, D, true);
-        auto wait_all = [&](uint32_t bar, uint32_t par) {
-            return __all_sync(0xffffffffu, mbar_wait_bounded(bar, par));
-        };
-        bool ok = wait_all(bar_q, 0);
-        auto need = [&](const PfTile &t, int jt) { return t.live && jt >= t.j0 && jt < t.j1; };
-        const PfTile *tl[2] = {&ta, &tb};
-        auto stage_of = [&](int jt) { return (jt - j0) % kPfStages; };
-        auto phase_of = [&](int jt) { return (uint32_t)(((jt - j0) / kPfStages) & 1); };
-        // S_X = Q_X K_jt into X's buffer (jt - j0_X) % 2
-        auto issue_s = [&](int x, int jt) {
-            const int st = stage_of(jt);
-            const int b = (jt - tl[x]->j0) & 1;
-            const uint32_t dcol = 256 * x + 64 * b;
-            if (lane == 0) {
-                tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t qoff = (kk >> 2) * Gm::kRegion + (kk & 3) * 32;
-                    const uint32_t koff = (kk >> 2) * Gm::kKVRegion + (kk & 3) * 32;
-                    umma_f16(tmem + dcol, umma_desc_sw128(sq + x * Gm::kQ + qoff, 16),
-                             umma_desc_sw128(sk + st * Gm::kKV + koff, 16), idesc_s, kk > 0);
-                }
-                umma_commit(bar_s0 + 8 * (2 * x + b));
             }
             __syncwarp();
-        };
-        // O_X += P_X V_jt (high, then low part of P from X's buffer)
-        auto issue_pv = [&](int x, int jt) {
-            const int st = stage_of(jt);
-            const uint32_t pcol = 256 * x + 64 * ((jt - tl[x]->j0) & 1);
-            const bool first = jt == tl[x]->j0;
-            if (lane == 0) {
-                tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < (kPfSplitP ? 2 : 1) * (kPfKeys / 16); ++kk) {
-                    const int k = kk % (kPfKeys / 16);
-                    const uint32_t acol = pcol + (kk >= kPfKeys / 16 ? 32 : 0) + k * 8;
-                    umma_f16_ts(tmem + 256 * x + 128, tmem + acol,
-                                umma_desc_sw128(sv + st * Gm::kKV + k * 16 * 128, Gm::kKVRegion),
-                                idesc_o, (!first || kk > 0) ? 1u : 0u);
-                }
-                umma_commit(bar_o0 + 8 * x);
-            }
-            __syncwarp();
-        };
-        int npv[2] = {0, 0};
-        // prologue: S of the first two key tiles
-        for (int jn = j0; ok && jn < min(j1, j0 + 2); ++jn) {
-            ok = wait_all(bar_k0 + 8 * stage_of(jn), phase_of(jn));
-            if (!ok) break;
-            for (int x = 0; x < 2; ++x)
-                if (need(*tl[x], jn)) issue_s(x, jn);
-        }
-        for (int jt = j0; ok && jt < j1; ++jt) {
-            if (__any_sync(0xffffffffu, sh_fail != 0)) {
-                ok = false;
-                break;
-            }
-            const int st = stage_of(jt);
-            const int kv0 = jt * kPfKeys;
-            // V of this tile; rows outside [kv_begin, L) (not loaded, or past the context)
-            // -> 0 so that zero weights cannot meet a NaN
-            ok = wait_all(bar_v0 + 8 * st, phase_of(jt));
-            if (!ok) break;
-            if (kv0 < kv_begin || kv0 + kPfKeys > L) {
-                const int lo = max(0, kv_begin - kv0), hi = min(kPfKeys, L - kv0);
+            issued = jt + 1;
+            if (edge) {
+                ok = __all_sync(0xffffffffu,
+                                mbar_wait_bounded(bvt, (uint32_t)(vt_uses[st] & 1)));
+                ++vt_uses[st];
+                if (!ok) break;
+                const int lo = tab_ok ? max(0, kv_begin - kv0) : kPfKeys;
+                const int hi = tab_ok ? min(kPfKeys, L - kv0) : 0;
                 for (int idx = lane; idx < kPfKeys * Gm::kHalves * 8; idx += 32) {
                     const int r = idx / (Gm::kHalves * 8), c = idx % (Gm::kHalves * 8);
                     if (r < lo || r >= hi)
@@ -526,47 +468,127 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                 }
                 fence_proxy_async_smem();
                 __syncwarp();
+                if (lane == 0) mbar_arrive(bv);
             }
-            for (int x = 0; x < 2 && ok; ++x) {
-                if (!need(*tl[x], jt)) continue;
-                const int i = jt - tl[x]->j0;
+        }
+        if (!ok) {
+            if (lane == 0) raise_error(PA_DEVERR_TIMEOUT);
+            sh_fail = 1;
+        }
+        // cleanup: the loads this CTA issued have landed (bounded)
+        if (lane == 0) {
+            (void)mbar_wait_bounded(bar_q, 0);
+            for (int jt = max(j0, issued - kPfStages); jt < issued; ++jt) {
+                const int it = jt - j0, st = it % kPfStages;
+                const uint32_t ph = (uint32_t)((it / kPfStages) & 1);
+                (void)mbar_wait_bounded(bar_k0 + 8 * st, ph);
+                (void)mbar_wait_bounded(bar_v0 + 8 * st, ph);
+            }
+        }
+        __syncwarp();
+    } else if (warp >= kPfMmaWarp) {
+        // ============================ products of query tile X (lane 0 issues)
+        const int x = warp - kPfMmaWarp;
+        const PfTile &t = x == 0 ? ta : tb;
+        const uint32_t idesc_s = umma_idesc<T>(kPfRows, kPfKeys, false);
+        const uint32_t idesc_o = umma_idesc<T>(kPfRows, D, true);
+        auto wait_all = [&](uint32_t bar, uint32_t par) {
+            return __all_sync(0xffffffffu, mbar_wait_bounded(bar, par));
+        };
+        auto need = [&](int jt) { return t.live && jt >= t.j0 && jt < t.j1; };
+        auto stage_of = [&](int jt) { return (jt - j0) % kPfStages; };
+        auto phase_of = [&](int jt) { return (uint32_t)(((jt - j0) / kPfStages) & 1); };
+        // descriptors built once; each product adds a constant start-address offset
+        const uint64_t dq = umma_desc_sw128(sq + x * Gm::kQ, 16);
+        const uint64_t dk = umma_desc_sw128(sk, 16);
+        const uint64_t dv = umma_desc_sw128(sv, Gm::kKVRegion);
+        // S_X = Q_X K_jt into X's buffer (jt - j0_X) % 2
+        auto issue_s = [&](int jt) {
+            const int st = stage_of(jt);
+            const int b = (jt - t.j0) & 1;
+            if (lane == 0) {
+                tc_fence_after();
+                const uint64_t dks = dk + (uint64_t)((st * Gm::kKV) >> 4);
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t qoff = ((kk >> 2) * Gm::kRegion + (kk & 3) * 32) >> 4;
+                    const uint32_t koff = ((kk >> 2) * Gm::kKVRegion + (kk & 3) * 32) >> 4;
+                    umma_f16(tmem + 256 * x + 64 * b, dq + qoff, dks + koff, idesc_s, kk > 0);
+                }
+                umma_commit(bar_s0 + 8 * (2 * x + b));
+            }
+            __syncwarp();
+        };
+        // O_X += P_X V_jt (high, then low part of P from X's buffer)
+        auto issue_pv = [&](int jt) {
+            const int st = stage_of(jt);
+            const uint32_t pcol = 256 * x + 64 * ((jt - t.j0) & 1);
+            const bool first = jt == t.j0;
+            if (lane == 0) {
+                tc_fence_after();
+                const uint64_t dvs = dv + (uint64_t)((st * Gm::kKV) >> 4);
+#pragma unroll
+                for (int kk = 0; kk < (kPfSplitP ? 2 : 1) * (kPfKeys / 16); ++kk) {
+                    const int k = kk % (kPfKeys / 16);
+                    const uint32_t acol = pcol + (kk >= kPfKeys / 16 ? 32 : 0) + k * 8;
+                    umma_f16_ts(tmem + 256 * x + 128, tmem + acol, dvs + (uint64_t)((k * 16 * 128) >> 4),
+                                idesc_o, (!first || kk > 0) ? 1u : 0u);
+                }
+                umma_commit(bar_o0 + 8 * x);
+            }
+            __syncwarp();
+        };
+        bool ok = wait_all(bar_q, 0);
+        int npv = 0;
+        // S of the first two key tiles
+        for (int jn = j0; ok && jn < min(j1, j0 + 2); ++jn) {
+            if (!need(jn)) continue;
+            ok = wait_all(bar_k0 + 8 * stage_of(jn), phase_of(jn));
+            if (ok) issue_s(jn);
+        }
+        for (int jt = j0; ok && jt < j1; ++jt) {
+            if (__any_sync(0xffffffffu, sh_fail != 0)) {
+                ok = false;
+                break;
+            }
+            const int st = stage_of(jt);
+            // every warp waits each tile's V, so that neither commits a stage's release
+            // a ring's length ahead of the loads
+            ok = wait_all(bar_v0 + 8 * st, phase_of(jt));
+            if (!ok) break;
+            if (need(jt)) {
+                const int i = jt - t.j0;
                 ok = wait_all(bar_p0 + 8 * (2 * x + (i & 1)), (uint32_t)((i >> 1) & 1));
                 if (!ok) break;
-                issue_pv(x, jt);
-                ++npv[x];
+                issue_pv(jt);
+                ++npv;
             }
             // S two key tiles ahead, into the buffer this tile's P V reads: after that
             // P V has finished
             const int jn = jt + 2;
-            if (ok && jn < j1) {
-                ok = wait_all(bar_k0 + 8 * stage_of(jn), phase_of(jn));
-                for (int x = 0; x < 2 && ok; ++x) {
-                    if (!need(*tl[x], jn)) continue;
-                    if (need(*tl[x], jt)) {
-                        ok = wait_all(bar_o0 + 8 * x, (uint32_t)((npv[x] - 1) & 1));
-                        if (!ok) break;
-                    }
-                    issue_s(x, jn);
+            if (jn < j1 && need(jn)) {
+                if (need(jt)) {
+                    ok = wait_all(bar_o0 + 8 * x, (uint32_t)((npv - 1) & 1));
+                    if (!ok) break;
                 }
+                ok = wait_all(bar_k0 + 8 * stage_of(jn), phase_of(jn));
+                if (!ok) break;
+                issue_s(jn);
             }
-            if (!ok) break;
-            if (lane == 0) umma_commit(bar_e0 + 8 * st);  // every product reading stage st
+            if (lane == 0) umma_commit(bar_e0 + 8 * st);  // this warp's products on stage st
             __syncwarp();
         }
         if (ok) {
-            // one commit per live query tile: completes when every product issued so far
-            // (its last P V included) has finished
-            if (lane == 0)
-                for (int x = 0; x < 2; ++x)
-                    if (tl[x]->live) umma_commit(bar_f0 + 8 * x);
+            // completes when every product of this warp (its last P V included) is done
+            if (lane == 0 && t.live) umma_commit(bar_f0 + 8 * x);
             __syncwarp();
         } else {
             if (lane == 0) raise_error(PA_DEVERR_TIMEOUT);
             sh_fail = 1;
             // cleanup: the products issued so far have finished (bounded)
             if (lane == 0) {
-                umma_commit(bar_f0);
-                (void)mbar_wait_bounded(bar_f0, 0);
+                umma_commit(bar_f0 + 8 * x);
+                (void)mbar_wait_bounded(bar_f0 + 8 * x, 0);
             }
             __syncwarp();
         }
@@ -760,7 +782,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     // ---- teardown: free the tensor memory (the warp that allocated it)
     tc_fence_before();
     __syncthreads();
-    if (warp == kPfMmaWarp) {
+    if (warp == kPfLoadWarp) {
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
                      "r"(kPfTmemCols)
