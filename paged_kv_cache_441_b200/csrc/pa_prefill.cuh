@@ -18,23 +18,24 @@
 //                       buffers per query tile so that the product for key tile j+2 can
 //                       run while the softmax of tile j+1 and P V of tile j are pending;
 //   softmax             a warpgroup per query tile; row r is thread r is tensor-memory
-//                       lane r.  The row is read once into registers (tcgen05.ld),
-//                       masked (causal, window, context end; tiles wholly inside every
-//                       row's range skip the masks), and the online-softmax state
-//                       (m, l) updated in fp32; the probabilities go back over S_X in
-//                       tensor memory as a high and a low 16-bit part (tcgen05.st);
+//                       lane r.  The row is read from tensor memory in two 32-column
+//                       chunks (double-buffered), masked (causal, window, context end;
+//                       tiles wholly inside every row's range skip the masks), and the
+//                       online-softmax state (m, l) updated in fp32; the probabilities go
+//                       back over S_X in tensor memory as a high and a low 16-bit part
+//                       (tcgen05.st);
 //   O_X  += P_X V       tcgen05.mma with P_X read from tensor memory and V as an MN-major
 //                       shared-memory operand (the cache rows as TMA lays them down), two
-//                       products (high and low part) so the weights keep ~16 bits; before
-//                       it the warpgroup rescales its rows of O_X by 2^(m_old - m_new)
-//                       (skipped in a warp where no row raised its maximum).
+//                       products (high and low part) so the weights keep ~16 bits.  The
+//                       reference maximum of a row moves only when the row maximum
+//                       exceeds it by more than 2^8; only then does the warp rescale its
+//                       rows of O_X (in tensor memory) by 2^(m_old - m_new).
 // Roles (warp specialisation): warps 0-3 softmax A, warps 4-7 softmax B, warps 8 and 9
 // issue the matrix products of A and of B, warp 10 issues the TMA loads of Q and of a
-// four-stage K/V ring (and zeroes the V rows of edge tiles outside the attended keys).  The products of one query tile overlap the
-// softmax of the other, and a query tile's next scores are computed while its current
-// softmax runs.  The reference maximum of a row moves only when the row maximum exceeds
-// it by more than 2^8, so most key tiles need no rescale of O.  Scores are kept in the log2 domain (scale *
-// log2 e folded in), as in the decode kernels.
+// four-stage K/V ring (and zeroes the V rows of edge tiles outside the attended keys).
+// The products of one query tile overlap the softmax of the other, and a query tile's next
+// scores are computed while its current softmax runs.  Scores are kept in the log2 domain
+// (scale * log2 e folded into one FFMA), as in the decode kernels.
 //
 // Every wait is bounded: on a timeout a role records PA_DEVERR_TIMEOUT and stops, the
 // others see the shared failure flag (or time out themselves), the copies and products
