@@ -138,3 +138,86 @@ def test_block_manager_serving_loop(hq, hkv, bs, fused, preempt, window):
     torch.cuda.synchronize()
     assert pa.device_error(0) == 0
     assert np.array_equal(bits(kc), kc_h) and np.array_equal(bits(vc), vc_h)
+
+
+@pytest.mark.parametrize("window", [0, 50])
+def test_engine_loop_prefill_then_decode(window):
+    """The block manager drives a whole engine loop on the GPU: prompts arrive and are
+    prefilled (whole, or in two chunks), then every live sequence decodes step by step;
+    under a sliding window the manager gives back the blocks that fall out of it.  Every
+    attention output is checked against the oracle, and the device cache against a host
+    mirror."""
+    rng = np.random.default_rng(900 + window)
+    nb, bs, hq, hkv, d, width = 400, 16, 16, 4, 128, 64
+    scale = 1 / math.sqrt(d)
+    bm = pa.BlockManager(nb, bs)
+    bm.set_sliding_window(window)
+    kc_h = np.full((nb, hkv, bs, d), 0x7FC0, np.uint16)
+    vc_h = kc_h.copy()
+    kc, vc = dev16(kc_h, "bf16"), dev16(vc_h, "bf16")
+    live, next_id = [], 0
+
+    def write(key, val, slots):
+        oracle.kv_write(key, val, slots, kc_h, vc_h)
+        pa.kv_write(dev16(key, "bf16"), dev16(val, "bf16"), dev(slots), kc, vc)
+
+    def prefill_check(sids, chunk_lo, chunk_hi, ctx):
+        """Chunk [chunk_lo[i], chunk_hi[i]) of each listed sequence, contexts ctx[i]."""
+        n = [h - l for l, h in zip(chunk_lo, chunk_hi)]
+        qsl = np.concatenate([[0], np.cumsum(n)]).astype(np.int32)
+        q = _rand_bits(rng, (int(qsl[-1]), hq, d))
+        bt, _ = bm.block_tables(sids, width)
+        cl = np.array(ctx, np.int32)
+        out = torch.empty(int(qsl[-1]), hq, d, dtype=torch.bfloat16, device="cuda")
+        pa.prefill(out, dev16(q, "bf16"), kc, vc, dev(bt), dev(cl), dev(qsl), scale,
+                   sliding_window=window)
+        want, bad = oracle.prefill(q, kc_h, vc_h, bt, cl, qsl, scale, "bf16",
+                                   sliding_window=window, return_bad=True)
+        assert bad == 0
+        err = np.max(np.abs(to_f64(out) - want))
+        assert np.isfinite(err) and err <= TOL["bf16"], err
+
+    def arrive(chunked):
+        nonlocal next_id
+        n = int(rng.integers(40, 300))
+        sid = next_id
+        next_id += 1
+        bm.allocate(sid, n)
+        slots = np.array([bm.slot(sid, i) for i in range(n)], np.int64)
+        write(_rand_bits(rng, (n, hkv, d)), _rand_bits(rng, (n, hkv, d)), slots)
+        if chunked:  # the first part, then the rest on top of it
+            n1 = int(rng.integers(1, n))
+            prefill_check([sid], [0], [n1], [n1])
+            prefill_check([sid], [n1], [n], [n])
+        else:
+            prefill_check([sid], [0], [n], [n])
+        live.append(sid)
+
+    for k in range(4):
+        arrive(chunked=(k % 2 == 1))
+    for step in range(12):
+        if step % 5 == 4:
+            bm.free(live.pop(0))
+            arrive(chunked=True)
+        slots, pairs = bm.append_slots(live)
+        assert pairs.shape[0] == 0  # no sharing in this loop
+        key = _rand_bits(rng, (len(live), hkv, d))
+        val = _rand_bits(rng, (len(live), hkv, d))
+        write(key, val, slots)
+        bt, cl = bm.block_tables(live, width)
+        q = _rand_bits(rng, (len(live), hq, d))
+        out = torch.empty(len(live), hq, d, dtype=torch.bfloat16, device="cuda")
+        pa.decode(out, dev16(q, "bf16"), kc, vc, dev(bt), dev(cl), scale,
+                  max_context_len=int(cl.max()), sliding_window=window)
+        want, bad = oracle.decode(q, kc_h, vc_h, bt, cl, scale, "bf16", return_bad=True,
+                                  sliding_window=window)
+        assert bad == 0
+        err = np.max(np.abs(to_f64(out) - want))
+        assert np.isfinite(err) and err <= TOL["bf16"], (step, err)
+        if window:  # blocks wholly before every window have gone back to the pool
+            held = sum(int((bt[i] >= 0).sum()) for i in range(len(live)))
+            need = sum(-(-int(L) // bs) - max(int(L) - window, 0) // bs for L in cl)
+            assert held == need
+    torch.cuda.synchronize()
+    assert pa.device_error(0) == 0
+    assert np.array_equal(bits(kc), kc_h) and np.array_equal(bits(vc), vc_h)
