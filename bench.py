@@ -97,28 +97,29 @@ def peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def kernel_sources_sha() -> str:
-    """Identity of the decode partition kernel's sources (the kernel the ncu traffic
-    figure was taken from)."""
+def kernel_sources_sha(names=("pa_common.cuh", "pa_decode.cuh")) -> str:
+    """Identity of a kernel's sources (the kernel an ncu traffic figure was taken from);
+    the decode partition kernel by default."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "paged_kv_cache_441_b200", "csrc")
-    for name in ("pa_common.cuh", "pa_decode.cuh"):
+    for name in names:
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode())
             h.update(f.read())
     return h.hexdigest()[:16]
 
 
-def traffic_from_profile(workload: str):
-    """Per-launch DRAM bytes of pa_decode from the committed ncu summary, or None when
-    the kernels changed since it was captured."""
-    path = os.path.join(ROOT, "profiles", "decode_traffic.json")
+def traffic_from_profile(workload: str, file: str = "decode_traffic.json",
+                         names=("pa_common.cuh", "pa_decode.cuh")):
+    """Per-launch DRAM bytes of a kernel from its committed ncu summary, or None when
+    the kernel's sources changed since it was captured."""
+    path = os.path.join(ROOT, "profiles", file)
     try:
         with open(path) as f:
             j = json.load(f)
     except Exception:
         return None
-    if j.get("sources_sha") != kernel_sources_sha():
+    if j.get("sources_sha") != kernel_sources_sha(names):
         return None
     entry = j.get("workloads", {}).get(workload)
     return None if entry is None else entry.get("dram_bytes_per_call")
@@ -873,7 +874,8 @@ def run_prefill(args):
                                          "P's second product and masked tile work not "
                                          "counted) / mean CUDA-event time per call, events "
                                          "around groups of 10 calls",
-                         "traffic": None},
+                         "traffic": traffic_from_profile(args.workload, "prefill_traffic.json",
+                                                         ("pa_common.cuh", "pa_prefill.cuh"))},
             "clocks": clocks,
             "cpu_baseline": cpu,
         }
@@ -881,6 +883,117 @@ def run_prefill(args):
         dist.barrier()
         dist.destroy_process_group()
     return result
+
+
+def run_cache_op(args):
+    """pa_kv_write or pa_copy_blocks alone: algorithmic bytes (read + written) / the median
+    CUDA-event time of one call, with L2 flushed (256 MB written) before every call."""
+    import torch
+    import paged_kv_cache_441_b200 as pa
+    torch.cuda.set_device(0)
+    device = torch.device("cuda", 0)
+    from workloads import make_config, make_prefill_config
+    if args.workload in PREFILL_WORKLOADS:
+        case = make_prefill_config(args.workload, poison=False)
+        desc = PREFILL_WORKLOADS[args.workload] + " (the chunk's cache write)"
+    else:
+        name, kw, desc = WORKLOADS[args.workload]
+        case = make_config(name, poison=False, **kw)
+    tdt = torch.bfloat16 if case.dtype == "bf16" else torch.float16
+
+    def d16(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(device).view(tdt)
+
+    kc, vc = d16(case.k_cache), d16(case.v_cache)
+    key, val = d16(case.key), d16(case.value)
+    sm = torch.from_numpy(case.slot_mapping).to(device)
+    pairs = torch.from_numpy(np.ascontiguousarray(
+        getattr(case, "copy_pairs", np.zeros((0, 2), np.int64)).reshape(-1, 2).astype(np.int64))).to(device)
+    T = int(case.slot_mapping.shape[0])
+    hkv, bs, d = case.num_kv_heads, case.block_size, case.head_dim
+    if args.op == "kv_write":
+        nbytes = 2 * 2 * T * hkv * d * 2 + 8 * T
+        fn = lambda: pa.kv_write(key, val, sm, kc, vc)  # noqa: E731
+        what = f"{T} tokens x {hkv} kv heads x {d}"
+    else:
+        if pairs.shape[0] == 0:
+            raise SystemExit("--op copy_blocks needs a workload with copy-on-write pairs")
+        P = int(pairs.shape[0])
+        nbytes = 2 * 2 * P * hkv * bs * d * 2 + 16 * P
+        fn = lambda: pa.copy_blocks(kc, vc, pairs)  # noqa: E731
+        what = f"{P} block pairs x 2 caches x {hkv * bs * d * 2} B"
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    for _ in range(args.warmup):
+        fn()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(0)
+    sampler.start()
+    times = []
+    for _ in range(args.steps):
+        flush.zero_()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        fn()
+        b.record()
+        b.synchronize()
+        times.append(a.elapsed_time(b))
+    clocks = sampler.stop()
+    err = pa.device_error(0)
+    if err:
+        raise RuntimeError(f"device error word {err:#x}")
+    ms = statistics.median(times)
+    value = nbytes / (ms * 1e-3) / 1e9
+    # end to end: the op's inputs from pinned host memory, then the op (one stream)
+    hk = torch.from_numpy(case.key.view(np.int16)).view(tdt).pin_memory()
+    hv = torch.from_numpy(case.value.view(np.int16)).view(tdt).pin_memory()
+    hs = torch.from_numpy(case.slot_mapping).pin_memory()
+    hp = pairs.cpu().pin_memory()
+    e2e_n = max(1, min(args.steps, 50))
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(e2e_n):
+        if args.op == "kv_write":
+            key.copy_(hk, non_blocking=True)
+            val.copy_(hv, non_blocking=True)
+            sm.copy_(hs, non_blocking=True)
+        else:
+            pairs.copy_(hp, non_blocking=True)
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    h2d = (hk.numel() * 2 + hv.numel() * 2 + hs.numel() * 8) if args.op == "kv_write" else hp.numel() * 8
+    peak, peak_kind = peaks()
+    # CPU oracle of the same op on the host cores
+    import oracle
+    kh, vh = case.k_cache.copy(), case.v_cache.copy()
+    t0 = time.perf_counter()
+    reps = 0
+    while time.perf_counter() - t0 < min(args.cpu_budget, 5.0) or reps == 0:
+        if args.op == "kv_write":
+            oracle.kv_write(case.key, case.value, case.slot_mapping, kh, vh)
+        else:
+            oracle.copy_blocks(kh, vh, case.copy_pairs)
+        reps += 1
+    cpu_s = (time.perf_counter() - t0) / reps
+    return {
+        "metric": f"pa_{args.op} GB/s (algorithmic bytes read + written)",
+        "value": round(value, 2), "unit": "GB/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms, 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": case.dtype, "data": "synthetic",
+        "config": {"workload": desc, "op": what, "bytes_per_call": nbytes,
+                   "l2": "flushed (256 MB written) before every timed call; median of the calls"},
+        "e2e": {"value": round(nbytes * e2e_n / (e0.elapsed_time(e1) * 1e-3) / 1e9, 2),
+                "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": 0},
+        "gpu_launches": args.steps,
+        "roofline": {"bound": "hbm", "achieved": round(value, 2), "peak": peak,
+                     "peak_kind": f"{peak_kind} HBM copy GB/s", "unit": "GB/s",
+                     "frac": round(value / peak, 4), "kernel": f"pa_{args.op}", "traffic": None},
+        "clocks": clocks,
+        "cpu_baseline": {"value": round(nbytes / cpu_s / 1e9, 4), "unit": "GB/s", "cores": 1,
+                         "kind": "oracle", "sample": f"the whole op, {reps} repetitions"},
+    }
 
 
 def run_reference(args):
@@ -937,7 +1050,8 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=10.0)
     ap.add_argument("--reference-budget", type=float, default=60.0)
-    ap.add_argument("--op", choices=["step", "swap", "prefill"], default="step",
+    ap.add_argument("--op", choices=["step", "swap", "prefill", "kv_write", "copy_blocks"],
+                    default="step",
                     help="swap: time the preemption swap of the workload instead of the step; "
                          "prefill: the prefill / chunked-prefill step (--workload prefill_*)")
     ap.add_argument("--swap-seqs", type=int, default=8,
@@ -947,6 +1061,13 @@ def main(argv=None):
         ap.error("--warmup must be >= 3")
     if args.workload is None:
         args.workload = "prefill_2k_gqa" if args.op == "prefill" else "llama2_7b"
+    if args.op in ("kv_write", "copy_blocks"):
+        if args.workload is None or (args.op == "copy_blocks" and args.workload == "llama2_7b"):
+            args.workload = "prefix_cow" if args.op == "copy_blocks" else args.workload
+        res = run_cache_op(args) if args.impl == "ours" else None
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
     if (args.op == "prefill") != (args.workload in PREFILL_WORKLOADS):
         ap.error("prefill workloads go with --op prefill, the others with --op step/swap")
     if args.op == "prefill":
