@@ -71,6 +71,8 @@ typedef enum { PA_FP16 = 0, PA_BF16 = 1 } pa_dtype;
  * Alignment       : key, value, k_cache, v_cache 16-byte aligned.
  * Duplicate slots within one call give an unspecified winner.
  * Bit-exact copy of the 16-bit patterns.  head_dim multiple of 8, block_size >= 1.
+ * One call moves at most 2^31 - 1 16-byte chunks (num_tokens * num_kv_heads *
+ * head_dim / 8); larger calls return PA_ERR_UNSUPPORTED (split them).
  */
 pa_status pa_kv_write(const void *key, const void *value, const int64_t *slot_mapping,
                       int num_tokens, int num_kv_heads, int head_dim, int64_t key_token_stride,

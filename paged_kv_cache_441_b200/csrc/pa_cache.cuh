@@ -23,31 +23,45 @@ struct KvWriteParams {
     int block_size;
 };
 
-// One thread per 16-byte chunk of one (token, kv head) row, for K and V together.
+constexpr int kKvwThreads = 256;
+constexpr int kKvwUnroll = 4;
+
+// One CTA per kKvwThreads * kKvwUnroll consecutive 16-byte chunks of the (token, kv head,
+// chunk) rows, K and V together; each thread issues its kKvwUnroll K and V loads before any
+// store (32-bit index math: the host keeps the chunk count below 2^31).
 // "Every generated token's K and V are stored in the KV cache" (PagedAttention and
 // dynamic memory blog): the store goes to k_cache[slot / bs][h][slot % bs][:].
-__global__ void __launch_bounds__(256) pa_kv_write_kernel(const __grid_constant__ KvWriteParams p) {
+__global__ void __launch_bounds__(kKvwThreads) pa_kv_write_kernel(const __grid_constant__ KvWriteParams p) {
     pdl_wait_and_release();
-    const long long per_tok = (long long)p.num_kv_heads * p.row_chunks;
-    const long long total = per_tok * p.num_tokens;
-    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
-         i += (long long)gridDim.x * blockDim.x) {
-        const int t = (int)(i / per_tok);
-        const int rem = (int)(i % per_tok);
-        const int h = rem / p.row_chunks, c = rem % p.row_chunks;
+    const unsigned per_tok = (unsigned)(p.num_kv_heads * p.row_chunks);
+    const unsigned total = per_tok * (unsigned)p.num_tokens;
+    const unsigned i0 = blockIdx.x * (unsigned)(kKvwThreads * kKvwUnroll) + threadIdx.x;
+    uint4 kv[kKvwUnroll], vv[kKvwUnroll];
+    long long dst[kKvwUnroll];
+#pragma unroll
+    for (int u = 0; u < kKvwUnroll; ++u) {
+        const unsigned i = i0 + (unsigned)(u * kKvwThreads);
+        dst[u] = -1;
+        if (i >= total) continue;
+        const unsigned t = i / per_tok, rem = i - t * per_tok;
+        const unsigned h = rem / (unsigned)p.row_chunks, c = rem - h * (unsigned)p.row_chunks;
         const long long slot = p.slot_mapping[t];
         if (slot < 0) continue;
         if (slot >= p.num_slots) {
             if (rem == 0) raise_error(PA_DEVERR_SLOT);
             continue;
         }
-        const long long blk = slot / p.block_size, off = slot % p.block_size;
-        const long long row = ((blk * p.num_kv_heads + h) * p.block_size + off) * p.row_chunks + c;
-        const long long src_off = (long long)(h * p.row_chunks + c) * 16;
-        const uint4 kv = ld_global_nc_v4(p.key + t * p.key_stride_b + src_off);
-        const uint4 vv = ld_global_nc_v4(p.value + t * p.value_stride_b + src_off);
-        reinterpret_cast<uint4 *>(p.k_cache)[row] = kv;
-        reinterpret_cast<uint4 *>(p.v_cache)[row] = vv;
+        const long long blk = slot / p.block_size, off = slot - blk * p.block_size;
+        dst[u] = ((blk * p.num_kv_heads + h) * p.block_size + off) * p.row_chunks + c;
+        const long long src_off = (long long)rem * 16;
+        kv[u] = ld_global_nc_v4(p.key + (long long)t * p.key_stride_b + src_off);
+        vv[u] = ld_global_nc_v4(p.value + (long long)t * p.value_stride_b + src_off);
+    }
+#pragma unroll
+    for (int u = 0; u < kKvwUnroll; ++u) {
+        if (dst[u] < 0) continue;
+        reinterpret_cast<uint4 *>(p.k_cache)[dst[u]] = kv[u];
+        reinterpret_cast<uint4 *>(p.v_cache)[dst[u]] = vv[u];
     }
 }
 

@@ -435,9 +435,10 @@ pa_status pa_kv_write(const void *key, const void *value, const int64_t *slot_ma
     p.row_chunks = head_dim / 8;
     p.block_size = block_size;
     const long long total = (long long)num_tokens * num_kv_heads * p.row_chunks;
-    const long long blocks = (total + 255) / 256;
-    const int grid = (int)(blocks < 148 * 32 ? blocks : 148 * 32);
-    return launch_pdl(pa_kv_write_kernel, dim3(grid), dim3(256), 0,
+    if (total >= (1ll << 31)) return PA_ERR_UNSUPPORTED;  // split the call
+    const long long per_cta = (long long)kKvwThreads * kKvwUnroll;
+    const unsigned grid = (unsigned)((total + per_cta - 1) / per_cta);
+    return launch_pdl(pa_kv_write_kernel, dim3(grid), dim3(kKvwThreads), 0,
                       static_cast<cudaStream_t>(stream), p) == cudaSuccess
                ? PA_OK
                : PA_ERR_CUDA;
