@@ -143,3 +143,11 @@ def _call_prefill(lib, **over):
 def test_prefill_rejects_before_launch(lib, over, code):
     # every case is settled by host checks (or has nothing to do): no CUDA call is made
     assert _call_prefill(lib, **over) == code
+
+
+def test_kv_write_refuses_oversized_call(lib):
+    # 2^28 tokens x 8 heads x 16 chunks = 2^35 chunks: refused before any launch
+    P = ctypes.c_void_p
+    st = lib.pa_kv_write(P(16), P(16), P(16), 1 << 28, 8, 128, 1024, 1024, P(16), P(16), 1 << 20,
+                         16, 1, None)
+    assert st == 2  # PA_ERR_UNSUPPORTED
