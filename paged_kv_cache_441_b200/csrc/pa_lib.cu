@@ -232,7 +232,9 @@ cudaError_t launch_partition(const DecodeParams &p, dim3 grid, cudaStream_t st, 
 
 template <typename T, int D>
 cudaError_t launch_merge(const MergeParams &p, dim3 grid, cudaStream_t st) {
-    return launch_pdl(pa_merge_kernel<T, D>, grid, dim3(kMergeThreads), 0, st, p);
+    if (p.num_parts <= kMergeFew)
+        return launch_pdl(pa_merge_kernel<T, D, false>, grid, dim3(kMergeThreads), 0, st, p);
+    return launch_pdl(pa_merge_kernel<T, D, true>, grid, dim3(kMergeThreads), 0, st, p);
 }
 
 template <typename T, int D, int G>

@@ -25,6 +25,7 @@ namespace pa {
 constexpr int kMergeThreads = 256;
 constexpr int kMergeChunk = 512;
 constexpr int kMergeFew = 8;  // up to this many partials: one load round per thread
+constexpr int kMergeMid = 64; // up to this many: one load round, partials split over groups
 
 template <int D, typename RecFn>
 __device__ __forceinline__ float lse_merge_block(int n, RecFn rec, const float *rm,
@@ -132,8 +133,10 @@ struct MergeParams {
     int sliding_window;  // as in DecodeParams: partitions start at span_begin(L, W)
 };
 
-// One CTA per (q head, sequence) with more than one partition.
-template <typename T, int D>
+// One CTA per (q head, sequence) with more than one partition.  WIDE: compiled with the
+// medium and block paths (more than kMergeFew partitions possible); the instance for at
+// most kMergeFew keeps its register count, and so its occupancy, low.
+template <typename T, int D, bool WIDE>
 __global__ void __launch_bounds__(kMergeThreads) pa_merge_kernel(const __grid_constant__ MergeParams p) {
     pdl_wait_and_release();
     const int h = blockIdx.x, s = blockIdx.y;
@@ -143,7 +146,7 @@ __global__ void __launch_bounds__(kMergeThreads) pa_merge_kernel(const __grid_co
     if (n <= 1) return;
     n = min(n, p.num_parts);
     const long long base = ((long long)s * p.num_q_heads + h) * p.num_parts;
-    if (n <= kMergeFew) {
+    if (!WIDE || n <= kMergeFew) {
         // few partitions: every load of this thread's element is issued at once
         const int d = threadIdx.x;
         if (d >= D) return;
@@ -167,6 +170,55 @@ __global__ void __launch_bounds__(kMergeThreads) pa_merge_kernel(const __grid_co
         }
         T *out = reinterpret_cast<T *>(p.out) + ((size_t)s * p.num_q_heads + h) * D;
         out[d] = Fmt<T>::from_float(den > 0.f ? num / den : 0.f);
+        return;
+    }
+    if constexpr (!WIDE) return;
+    if (n <= kMergeMid) {
+        // medium: kMergeThreads / D groups of D threads; group g owns partials
+        // g*kPer .. g*kPer+kPer-1 and thread d of it element d: all its loads at once, then
+        // the groups' maxima and sums are combined in shared memory
+        constexpr int kGroups = kMergeThreads / D, kPer = kMergeMid / kGroups;
+        __shared__ float gmax[kGroups], gden[kGroups];
+        __shared__ float gnum[kGroups][D];
+        const int d = threadIdx.x % D, grp = threadIdx.x / D;
+        float m[kPer], l[kPer], o[kPer];
+#pragma unroll
+        for (int i = 0; i < kPer; ++i) {
+            const int idx = grp * kPer + i;
+            const bool in = idx < n;
+            m[i] = in ? p.ws_m[base + idx] : -INFINITY;
+            l[i] = in ? p.ws_l[base + idx] : 0.f;
+            o[i] = in ? p.ws_o[(base + idx) * D + d] : 0.f;
+        }
+        float Mg = -INFINITY;
+#pragma unroll
+        for (int i = 0; i < kPer; ++i) Mg = fmaxf(Mg, m[i]);
+        if (d == 0) gmax[grp] = Mg;
+        __syncthreads();
+        float M = -INFINITY;
+#pragma unroll
+        for (int g2 = 0; g2 < kGroups; ++g2) M = fmaxf(M, gmax[g2]);
+        float num = 0.f, den = 0.f;
+#pragma unroll
+        for (int i = 0; i < kPer; ++i) {
+            if (m[i] == -INFINITY) continue;  // no record: its slot is not used
+            const float w = l[i] * fast_exp2(m[i] - M);
+            num = fmaf(w, o[i], num);
+            den += w;
+        }
+        gnum[grp][d] = num;
+        if (d == 0) gden[grp] = den;
+        __syncthreads();
+        if (grp == 0) {
+            float nt = 0.f, dt = 0.f;
+#pragma unroll
+            for (int g2 = 0; g2 < kGroups; ++g2) {
+                nt += gnum[g2][d];
+                dt += gden[g2];
+            }
+            T *out = reinterpret_cast<T *>(p.out) + ((size_t)s * p.num_q_heads + h) * D;
+            out[d] = Fmt<T>::from_float(dt > 0.f ? nt / dt : 0.f);
+        }
         return;
     }
     const float v = lse_merge_block<D>(
