@@ -13,6 +13,14 @@ pinned host inputs copied in and the output copied out inside the timed region;
 `cpu_baseline` = the fp64 CPU oracle on the host cores.
 
 `--impl reference` times that oracle alone (rank 0) in the same JSON format.
+
+Other operations of the library, one JSON line each (`--op`):
+  swap         preemption swap of a group of the workload's sequences to a pinned host
+               pool and back (GB/s over the host link, against a pinned memcpy);
+  prefill      causal multi-query attention of a prefill workload (--workload prefill_*;
+               algorithmic TFLOP/s against the measured bf16 tensor rate);
+  kv_write     the cache write alone (GB/s, L2 flushed before every call);
+  copy_blocks  the copy-on-write block copy alone (the prefix workload).
 """
 from __future__ import annotations
 

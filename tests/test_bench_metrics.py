@@ -1,0 +1,46 @@
+"""The benchmark's algorithmic-work counts against brute-force enumerations on tiny cases:
+decode bytes (K/V of every attended token and kv head, q and out, the table entries of the
+attended pages, the lengths) and prefill FLOPs (4 d per attended (query, head, key)), with
+and without a sliding window."""
+import numpy as np
+
+import bench
+from workloads import make_case, make_prefill_case
+
+
+def _decode_bytes_brute(case):
+    eb, total = 2, 0
+    pages = set()
+    for s, L in enumerate(case.context_lens.tolist()):
+        lo = L - case.window if 0 < case.window < L else 0
+        for t in range(lo, L):
+            total += 2 * case.num_kv_heads * case.head_dim * eb  # K and V of every kv head
+            pages.add((s, t // case.block_size))
+    total += 2 * case.num_seqs * case.num_q_heads * case.head_dim * eb  # q and out
+    total += 4 * case.num_kv_heads * len(pages)  # one table entry per page and kv head
+    return total + 4 * case.num_seqs
+
+
+def test_decode_bytes_match_brute_force():
+    lens = [1, 15, 16, 17, 100, 333]
+    for window in (0, 1, 20, 64):
+        case = make_case("m", 3, len(lens), 8, 2, 64, 16, lambda r: np.array(lens, np.int32),
+                         window=window, poison=False)
+        assert bench.decode_bytes(case) == _decode_bytes_brute(case), window
+
+
+def test_prefill_flops_match_brute_force():
+    specs = [(5, 5), (3, 40), (1, 7), (17, 17)]
+    for window in (0, 1, 4, 10):
+        case = make_prefill_case("m", 4, specs, 8, 2, 64, 16, window=window, poison=False)
+        qsl = case.query_start_loc
+        want = 0
+        for s, (n, L) in enumerate(specs):
+            for i in range(n):
+                p = L - n + i
+                keys = [u for u in range(p + 1) if window <= 0 or u > p - window]
+                want += 4 * case.head_dim * case.num_q_heads * len(keys)
+        assert bench.prefill_flops(case) == want, window
+        # the per-sample count used by the CPU baseline agrees on the whole set
+        sel = np.array([(t, h) for t in range(int(qsl[-1])) for h in range(case.num_q_heads)])
+        assert bench.prefill_sample_flops(case, sel) == want
