@@ -2,7 +2,12 @@
  * libpa -- paged KV-cache decode attention for NVIDIA B200 (sm_100a).
  *
  * C ABI.  Every pointer argument is DEVICE memory owned by the caller unless the
- * comment says otherwise; the library allocates nothing on these paths.  Every
+ * comment says otherwise; the library allocates nothing on these paths.  Device
+ * pointers are not queried on the launch paths (only pa_swap_blocks, which accepts
+ * host pools, asks the runtime what each pool is): a host pointer, or memory of
+ * another device than the current one, where device memory is required is
+ * undefined behaviour.  The Python binding checks device, dtype, contiguity and
+ * shapes of its tensors before it calls in.  Every
  * call is asynchronous on `stream` (a cudaStream_t passed as void*, NULL = the
  * legacy default stream) and never synchronises the device, except
  * pa_get_device_error, which says so.

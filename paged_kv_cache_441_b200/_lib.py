@@ -1,8 +1,11 @@
 """ctypes binding of libpa (include/pa.h).  Argument marshalling only.
 
-Every function takes torch CUDA tensors, reads their pointers, shapes and the
-current CUDA stream, and calls the C entry point of the same name.  There is no
-fallback: if ``libpa.so`` is missing or a call fails, an exception is raised.
+Every function takes torch CUDA tensors, checks that they are what the C entry
+point reads (device, dtype, contiguity, shapes that agree), then passes their
+pointers, shapes and the tensors' device's current CUDA stream to the C entry
+point of the same name.  A failed check raises PAError before anything reaches
+the library.  There is no fallback: if ``libpa.so`` is missing or a call fails,
+an exception is raised.
 """
 from __future__ import annotations
 
@@ -91,11 +94,87 @@ def _dtype(t) -> int:
     raise PAError(f"unsupported dtype {t.dtype}")
 
 
-def _stream(stream):
+# Device type every tensor of a launch must live on.  The marshalling tests run the
+# same checks on CPU tensors against a stand-in library by switching this to "cpu".
+_DEVICE_TYPE = "cuda"
+
+
+def _fail(what: str, msg: str):
+    raise PAError(f"{what}: {msg}")
+
+
+def _args(what: str, half: dict, ints: dict = None, rows: dict = None, device=None):
+    """Check the tensors of one call before their pointers reach the library.
+
+    half: 16-bit float tensors (q, out, caches), one dtype, contiguous.
+    ints: name -> (tensor, torch dtype); contiguous (block tables, lengths, slots).
+    rows: 16-bit tensors [T, H, d] whose heads are contiguous but whose token stride
+          is free (a key or value slice of a wider projection).
+    All of them on one device of type _DEVICE_TYPE (``device`` if given).
+    Returns that device."""
+    ints, rows = ints or {}, rows or {}
+    first = next(iter(half.values()))
+    dev = first.device if device is None else device
+    if dev.type != _DEVICE_TYPE:
+        _fail(what, f"tensors must be on a {_DEVICE_TYPE} device, got {dev}")
+    for name, t in {**half, **rows}.items():
+        if t.dtype != first.dtype:
+            _fail(what, f"{name} is {t.dtype}, expected {first.dtype}")
+        if t.device != dev:
+            _fail(what, f"{name} is on device {t.device}, expected {dev}")
+    _dtype(first)
+    for name, t in half.items():
+        if not t.is_contiguous():
+            _fail(what, f"{name} must be contiguous")
+    for name, t in rows.items():
+        if not (t.dim() == 3 and t.stride(2) == 1 and t.stride(1) == t.shape[2]):
+            _fail(what, f"{name} must be [tokens, heads, head_dim] with contiguous heads")
+    for name, (t, dt) in ints.items():
+        if t.dtype != dt:
+            _fail(what, f"{name} is {t.dtype}, expected {dt}")
+        if t.device != dev:
+            _fail(what, f"{name} is on device {t.device}, expected {dev}")
+        if not t.is_contiguous():
+            _fail(what, f"{name} must be contiguous")
+    return dev
+
+
+def _cache_shape(what: str, k_cache, v_cache, num_kv_heads=None, head_dim=None):
+    if not (k_cache.dim() == 4 and tuple(v_cache.shape) == tuple(k_cache.shape)):
+        _fail(what, f"k_cache {tuple(k_cache.shape)} and v_cache {tuple(v_cache.shape)} must "
+              "both be [num_blocks, num_kv_heads, block_size, head_dim]")
+    nb, hkv, bs, d = k_cache.shape
+    if num_kv_heads is not None and hkv != num_kv_heads:
+        _fail(what, f"cache has {hkv} kv heads, the tokens {num_kv_heads}")
+    if head_dim is not None and d != head_dim:
+        _fail(what, f"cache head_dim {d} != {head_dim}")
+    return nb, hkv, bs, d
+
+
+def _tables(what: str, block_tables, context_lens, num_seqs):
+    if not (block_tables.dim() == 2 and block_tables.shape[0] == num_seqs):
+        _fail(what, f"block_tables {tuple(block_tables.shape)} must be "
+              f"[{num_seqs}, max_blocks]")
+    if tuple(context_lens.shape) != (num_seqs,):
+        _fail(what, f"context_lens {tuple(context_lens.shape)} must be [{num_seqs}]")
+
+
+def _stream(stream, device=None):
     import torch
     if stream is None:
-        stream = torch.cuda.current_stream()
+        stream = torch.cuda.current_stream(device)
     return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _on(device):
+    """Make ``device`` current for the launch (the library launches on the current
+    device; a tensor on another GPU would be read through the wrong context)."""
+    import contextlib
+    import torch
+    if device is None or device.type != "cuda" or device.index is None or \
+            device.index == torch.cuda.current_device():
+        return contextlib.nullcontext()
+    return torch.cuda.device(device)
 
 
 def _ptr(t):
@@ -104,29 +183,66 @@ def _ptr(t):
 
 def kv_write(key, value, slot_mapping, k_cache, v_cache, stream=None) -> None:
     """key/value [T, Hkv, d] (token stride may exceed Hkv*d), slot_mapping int64 [T]."""
+    import torch
+    what = "pa_kv_write"
+    if not (key.dim() == 3 and tuple(value.shape) == tuple(key.shape)):
+        _fail(what, f"key {tuple(key.shape)} and value {tuple(value.shape)} must both be "
+              "[T, Hkv, d]")
     T, hkv, d = key.shape
-    assert key.stride(2) == 1 and key.stride(1) == d and value.stride(1) == d
-    nb, _, bs, _ = k_cache.shape
-    _check(load().pa_kv_write(_ptr(key), _ptr(value), _ptr(slot_mapping), T, hkv, d,
-                              key.stride(0), value.stride(0), _ptr(k_cache), _ptr(v_cache), nb, bs,
-                              _dtype(k_cache), _stream(stream)), "pa_kv_write")
+    nb, _, bs, _ = _cache_shape(what, k_cache, v_cache, hkv, d)
+    if tuple(slot_mapping.shape) != (T,):
+        _fail(what, f"slot_mapping must be [{T}]")
+    dev = _args(what, {"k_cache": k_cache, "v_cache": v_cache}, rows={"key": key, "value": value},
+                ints={"slot_mapping": (slot_mapping, torch.int64)})
+    with _on(dev):
+        _check(load().pa_kv_write(_ptr(key), _ptr(value), _ptr(slot_mapping), T, hkv, d,
+                                  key.stride(0), value.stride(0), _ptr(k_cache), _ptr(v_cache),
+                                  nb, bs, _dtype(k_cache), _stream(stream, dev)), what)
 
 
 def copy_blocks(k_cache, v_cache, pairs, stream=None) -> None:
     """pairs int64 [P, 2] (src, dst) on the device."""
-    nb, hkv, bs, d = k_cache.shape
-    _check(load().pa_copy_blocks(_ptr(k_cache), _ptr(v_cache), _ptr(pairs), pairs.shape[0], hkv,
-                                 bs, d, nb, _dtype(k_cache), _stream(stream)), "pa_copy_blocks")
+    import torch
+    what = "pa_copy_blocks"
+    nb, hkv, bs, d = _cache_shape(what, k_cache, v_cache)
+    if not (pairs.dim() == 2 and pairs.shape[1] == 2):
+        _fail(what, "pairs must be [P, 2]")
+    dev = _args(what, {"k_cache": k_cache, "v_cache": v_cache},
+                ints={"pairs": (pairs, torch.int64)})
+    with _on(dev):
+        _check(load().pa_copy_blocks(_ptr(k_cache), _ptr(v_cache), _ptr(pairs), pairs.shape[0],
+                                     hkv, bs, d, nb, _dtype(k_cache), _stream(stream, dev)), what)
 
 
 def swap_blocks(dst_k_cache, dst_v_cache, src_k_cache, src_v_cache, pairs, stream=None) -> None:
     """Copy blocks pairs[:, 0] of the source pool to blocks pairs[:, 1] of the destination
-    pool; either pool may be a pinned host tensor.  pairs: int64 [P, 2] (device or pinned)."""
-    snb, hkv, bs, d = src_k_cache.shape
-    dnb = dst_k_cache.shape[0]
-    _check(load().pa_swap_blocks(_ptr(dst_k_cache), _ptr(dst_v_cache), _ptr(src_k_cache),
-                                 _ptr(src_v_cache), _ptr(pairs), pairs.shape[0], hkv, bs, d, snb,
-                                 dnb, _dtype(src_k_cache), _stream(stream)), "pa_swap_blocks")
+    pool; either pool may be a pinned host tensor.  pairs: int64 [P, 2] (device or pinned).
+    Whether a host pool is pinned is checked by the library."""
+    import torch
+    what = "pa_swap_blocks"
+    snb, hkv, bs, d = _cache_shape(what, src_k_cache, src_v_cache)
+    dnb, dh, dbs, dd = _cache_shape(what, dst_k_cache, dst_v_cache)
+    if (dh, dbs, dd) != (hkv, bs, d):
+        _fail(what, "source and destination blocks differ in shape")
+    if not (pairs.dim() == 2 and pairs.shape[1] == 2):
+        _fail(what, "pairs must be [P, 2]")
+    pools = {"dst_k_cache": dst_k_cache, "dst_v_cache": dst_v_cache,
+             "src_k_cache": src_k_cache, "src_v_cache": src_v_cache}
+    for name, t in pools.items():
+        if t.dtype != src_k_cache.dtype:
+            _fail(what, f"{name} is {t.dtype}, expected {src_k_cache.dtype}")
+        if not t.is_contiguous():
+            _fail(what, f"{name} must be contiguous")
+    if not (pairs.dtype == torch.int64 and pairs.is_contiguous()):
+        _fail(what, "pairs must be contiguous int64")
+    gpus = {t.device for t in (*pools.values(), pairs) if t.device.type == _DEVICE_TYPE}
+    if len(gpus) > 1:
+        _fail(what, f"tensors on more than one device: {sorted(map(str, gpus))}")
+    dev = next(iter(gpus)) if gpus else None
+    with _on(dev):
+        _check(load().pa_swap_blocks(_ptr(dst_k_cache), _ptr(dst_v_cache), _ptr(src_k_cache),
+                                     _ptr(src_v_cache), _ptr(pairs), pairs.shape[0], hkv, bs, d,
+                                     snb, dnb, _dtype(src_k_cache), _stream(stream, dev)), what)
 
 
 def decode_workspace_bytes(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
@@ -145,29 +261,54 @@ def decode_partition_tokens(num_seqs, num_q_heads, num_kv_heads, head_dim, block
                                                  sliding_window, partition_size))
 
 
+def _decode_shapes(what, out, q, k_cache, v_cache, block_tables, context_lens, block_size):
+    """Shapes shared by the decode entry points: (B, Hq, d, NB, Hkv, bs, W)."""
+    if not (q.dim() == 3 and tuple(out.shape) == tuple(q.shape)):
+        _fail(what, f"q {tuple(q.shape)} and out {tuple(out.shape)} must both be [B, Hq, d]")
+    B, hq, d = q.shape
+    nb, hkv, bs, _ = _cache_shape(what, k_cache, v_cache, head_dim=d)
+    if block_size is not None and block_size != bs:
+        _fail(what, f"block_size {block_size} != cache block size {bs}")
+    _tables(what, block_tables, context_lens, B)
+    return B, hq, d, nb, hkv, bs, block_tables.shape[1]
+
+
+def _workspace(what, workspace, need, dev):
+    """(pointer, bytes) of the split-K workspace; allocated with torch when the plan needs
+    one and the caller gave none."""
+    import torch
+    if workspace is None:
+        if not need:
+            return None, 0
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    if not (workspace.device == dev and workspace.is_contiguous()):
+        _fail(what, f"workspace must be a contiguous tensor on {dev}")
+    return _ptr(workspace), workspace.numel() * workspace.element_size()
+
+
 def decode(out, q, k_cache, v_cache, block_tables, context_lens, scale, block_size=None,
            max_context_len=0, partition_size=0, workspace=None, stream=None,
            sliding_window=0) -> None:
     """out, q [B, Hq, d]; caches [NB, Hkv, bs, d]; block_tables int32 [B, W];
-    context_lens int32 [B].  ``workspace`` (a uint8 CUDA tensor) is allocated here
+    context_lens int32 [B].  ``workspace`` (a contiguous CUDA tensor) is allocated here
     with torch when the plan needs one and none is given.  ``sliding_window`` > 0:
     each query attends to the last that many tokens of its context."""
     import torch
-    B, hq, d = q.shape
-    nb, hkv, bs, _ = k_cache.shape
-    if block_size is not None and block_size != bs:
-        raise PAError(f"block_size {block_size} != cache block size {bs}")
-    W = block_tables.shape[1]
-    need = decode_workspace_bytes(B, hq, hkv, d, bs, W, max_context_len, partition_size,
-                                  sliding_window)
-    if need and workspace is None:
-        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
-    wptr = _ptr(workspace) if workspace is not None else None
-    wbytes = workspace.numel() if workspace is not None else 0
-    _check(load().pa_decode(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
-                            _ptr(context_lens), B, hq, hkv, d, bs, nb, W, float(scale),
-                            int(max_context_len), int(sliding_window), int(partition_size), wptr,
-                            wbytes, _dtype(q), _stream(stream)), "pa_decode")
+    what = "pa_decode"
+    B, hq, d, nb, hkv, bs, W = _decode_shapes(what, out, q, k_cache, v_cache, block_tables,
+                                              context_lens, block_size)
+    dev = _args(what, {"q": q, "out": out, "k_cache": k_cache, "v_cache": v_cache},
+                ints={"block_tables": (block_tables, torch.int32),
+                      "context_lens": (context_lens, torch.int32)})
+    with _on(dev):
+        need = decode_workspace_bytes(B, hq, hkv, d, bs, W, max_context_len, partition_size,
+                                      sliding_window)
+        wptr, wbytes = _workspace(what, workspace, need, dev)
+        _check(load().pa_decode(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                                _ptr(block_tables), _ptr(context_lens), B, hq, hkv, d, bs, nb, W,
+                                float(scale), int(max_context_len), int(sliding_window),
+                                int(partition_size), wptr, wbytes, _dtype(q),
+                                _stream(stream, dev)), what)
 
 
 def decode_append(out, q, key, value, k_cache, v_cache, block_tables, context_lens, scale,
@@ -176,23 +317,26 @@ def decode_append(out, q, key, value, k_cache, v_cache, block_tables, context_le
     """Cache write of each sequence's new token (key/value [B, Hkv, d], stored at
     position context_lens[s]-1) fused with decode; same result as kv_write + decode."""
     import torch
-    B, hq, d = q.shape
-    nb, hkv, bs, _ = k_cache.shape
-    assert key.shape[0] == B and key.stride(2) == 1 and key.stride(1) == d
-    assert value.stride(2) == 1 and value.stride(1) == d
-    W = block_tables.shape[1]
-    need = decode_workspace_bytes(B, hq, hkv, d, bs, W, max_context_len, partition_size,
-                                  sliding_window)
-    if need and workspace is None:
-        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
-    wptr = _ptr(workspace) if workspace is not None else None
-    wbytes = workspace.numel() if workspace is not None else 0
-    _check(load().pa_decode_append(_ptr(out), _ptr(q), _ptr(key), _ptr(value), key.stride(0),
-                                   value.stride(0), _ptr(k_cache), _ptr(v_cache),
-                                   _ptr(block_tables), _ptr(context_lens), B, hq, hkv, d, bs, nb,
-                                   W, float(scale), int(max_context_len), int(sliding_window),
-                                   int(partition_size), wptr, wbytes, _dtype(q), _stream(stream)),
-           "pa_decode_append")
+    what = "pa_decode_append"
+    B, hq, d, nb, hkv, bs, W = _decode_shapes(what, out, q, k_cache, v_cache, block_tables,
+                                              context_lens, None)
+    if not (tuple(key.shape) == (B, hkv, d) and tuple(value.shape) == (B, hkv, d)):
+        _fail(what, f"key {tuple(key.shape)} and value {tuple(value.shape)} must both be "
+              f"[{B}, {hkv}, {d}]")
+    dev = _args(what, {"q": q, "out": out, "k_cache": k_cache, "v_cache": v_cache},
+                rows={"key": key, "value": value},
+                ints={"block_tables": (block_tables, torch.int32),
+                      "context_lens": (context_lens, torch.int32)})
+    with _on(dev):
+        need = decode_workspace_bytes(B, hq, hkv, d, bs, W, max_context_len, partition_size,
+                                      sliding_window)
+        wptr, wbytes = _workspace(what, workspace, need, dev)
+        _check(load().pa_decode_append(_ptr(out), _ptr(q), _ptr(key), _ptr(value),
+                                       key.stride(0), value.stride(0), _ptr(k_cache),
+                                       _ptr(v_cache), _ptr(block_tables), _ptr(context_lens), B,
+                                       hq, hkv, d, bs, nb, W, float(scale), int(max_context_len),
+                                       int(sliding_window), int(partition_size), wptr, wbytes,
+                                       _dtype(q), _stream(stream, dev)), what)
 
 
 def decode_static_scratch(out, q, k_cache, v_cache, block_tables, context_lens, scale,
@@ -201,22 +345,23 @@ def decode_static_scratch(out, q, k_cache, v_cache, block_tables, context_lens, 
     """``decode`` for callers that cannot allocate device memory: the split-K partial
     results go to the library's own fixed scratch array (STATIC_SCRATCH_BYTES per
     GPU) instead of a workspace.  Calls that overlap on the GPU race on that array."""
-    B, hq, d = q.shape
-    nb, hkv, bs, _ = k_cache.shape
-    if block_size is not None and block_size != bs:
-        raise PAError(f"block_size {block_size} != cache block size {bs}")
-    W = block_tables.shape[1]
+    import torch
+    what = "pa_decode_static_scratch"
+    B, hq, d, nb, hkv, bs, W = _decode_shapes(what, out, q, k_cache, v_cache, block_tables,
+                                              context_lens, block_size)
+    dev = _args(what, {"q": q, "out": out, "k_cache": k_cache, "v_cache": v_cache},
+                ints={"block_tables": (block_tables, torch.int32),
+                      "context_lens": (context_lens, torch.int32)})
     need = decode_workspace_bytes(B, hq, hkv, d, bs, W, max_context_len, partition_size,
                                   sliding_window)
     if need > STATIC_SCRATCH_BYTES:
-        raise PAError(f"pa_decode_static_scratch: these sizes need {need} bytes of scratch, "
-                      f"more than the library's fixed {STATIC_SCRATCH_BYTES}; use decode() "
-                      "with a workspace")
-    _check(load().pa_decode_static_scratch(
-        _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
-        _ptr(context_lens), B, hq, hkv, d, bs, nb, W, float(scale), int(max_context_len),
-        int(sliding_window), int(partition_size), _dtype(q), _stream(stream)),
-        "pa_decode_static_scratch")
+        _fail(what, f"these sizes need {need} bytes of scratch, more "
+              f"than the library's fixed {STATIC_SCRATCH_BYTES}; use decode() with a workspace")
+    with _on(dev):
+        _check(load().pa_decode_static_scratch(
+            _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
+            _ptr(context_lens), B, hq, hkv, d, bs, nb, W, float(scale), int(max_context_len),
+            int(sliding_window), int(partition_size), _dtype(q), _stream(stream, dev)), what)
 
 
 def prefill(out, q, k_cache, v_cache, block_tables, context_lens, query_start_loc, scale,
@@ -225,14 +370,27 @@ def prefill(out, q, k_cache, v_cache, block_tables, context_lens, query_start_lo
     sequence s in rows query_start_loc[s] .. [s+1]); caches [NB, Hkv, bs, d];
     block_tables int32 [B, W]; context_lens int32 [B] (tokens in the cache, the chunk
     included); query_start_loc int32 [B + 1]."""
+    import torch
+    what = "pa_prefill"
+    if not (q.dim() == 3 and tuple(out.shape) == tuple(q.shape)):
+        _fail(what, f"q {tuple(q.shape)} and out {tuple(out.shape)} must both be [T, Hq, d]")
     T, hq, d = q.shape
-    nb, hkv, bs, _ = k_cache.shape
+    nb, hkv, bs, _ = _cache_shape(what, k_cache, v_cache, head_dim=d)
+    if context_lens.dim() != 1:
+        _fail(what, "context_lens must be [B]")
     B = context_lens.shape[0]
-    assert query_start_loc.shape[0] == B + 1
-    _check(load().pa_prefill(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache),
-                             _ptr(block_tables), _ptr(context_lens), _ptr(query_start_loc), B, T,
-                             hq, hkv, d, bs, nb, block_tables.shape[1], float(scale),
-                             int(sliding_window), _dtype(q), _stream(stream)), "pa_prefill")
+    _tables(what, block_tables, context_lens, B)
+    if tuple(query_start_loc.shape) != (B + 1,):
+        _fail(what, f"query_start_loc must be [{B + 1}]")
+    dev = _args(what, {"q": q, "out": out, "k_cache": k_cache, "v_cache": v_cache},
+                ints={"block_tables": (block_tables, torch.int32),
+                      "context_lens": (context_lens, torch.int32),
+                      "query_start_loc": (query_start_loc, torch.int32)})
+    with _on(dev):
+        _check(load().pa_prefill(_ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                                 _ptr(block_tables), _ptr(context_lens), _ptr(query_start_loc),
+                                 B, T, hq, hkv, d, bs, nb, block_tables.shape[1], float(scale),
+                                 int(sliding_window), _dtype(q), _stream(stream, dev)), what)
 
 
 def device_error(device: int = 0, clear: bool = True) -> int:

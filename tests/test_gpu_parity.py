@@ -301,9 +301,19 @@ def test_device_errors_are_flagged_not_fatal():
 def test_host_rejects_bad_arguments():
     case = _rand_case(15, "bf16", 2, 8, 2, 128, 16, [10, 200])
     dc = DeviceCase(case)
-    with pytest.raises(pa.PAError):
-        pa.decode(dc.out, dc.q[:, :6], dc.k_cache, dc.v_cache, dc.block_tables, dc.context_lens,
-                  0.1)  # 6 q heads over 2 kv heads: group 3 not supported
+    q6 = dc.q[:, :6].contiguous()
+    with pytest.raises(pa.PAError, match="unsupported"):  # refused by the library itself
+        pa.decode(torch.empty_like(q6), q6, dc.k_cache, dc.v_cache, dc.block_tables,
+                  dc.context_lens, 0.1)  # 6 q heads over 2 kv heads: group 3 not supported
+    with pytest.raises(pa.PAError, match="contiguous"):  # refused by the binding
+        pa.decode(dc.out[:, :6], dc.q[:, :6], dc.k_cache, dc.v_cache, dc.block_tables,
+                  dc.context_lens, 0.1)
+    with pytest.raises(pa.PAError, match="expected torch.int32"):
+        pa.decode(dc.out, dc.q, dc.k_cache, dc.v_cache, dc.block_tables.long(),
+                  dc.context_lens, 0.1)
+    with pytest.raises(pa.PAError, match="device"):  # a host tensor never reaches a kernel
+        pa.decode(dc.out, dc.q, dc.k_cache, dc.v_cache, dc.block_tables.cpu(),
+                  dc.context_lens, 0.1)
     with pytest.raises(pa.PAError):  # workspace too small for the split it needs
         pa.decode(dc.out, dc.q, dc.k_cache, dc.v_cache, dc.block_tables, dc.context_lens, 0.1,
                   partition_size=64, max_context_len=0,
