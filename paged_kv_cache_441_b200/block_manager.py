@@ -70,9 +70,11 @@ def _p(a):
 
 
 class BlockManager:
-    """Reference-counted block pool with per-sequence page tables."""
+    """Reference-counted block pool with per-sequence page tables.  Not thread-safe: one
+    manager per engine thread."""
 
     def __init__(self, num_blocks: int, block_size: int):
+        self._h = None  # so that __del__ is safe if the library cannot be loaded
         self._lib = _lib()
         self._h = self._lib.pa_bm_create(num_blocks, block_size)
         if not self._h:
@@ -88,25 +90,30 @@ class BlockManager:
     def __del__(self):
         self.close()
 
+    def _live(self):
+        if not self._h:
+            raise PAError("the block manager has been closed")
+        return self._h
+
     @property
     def num_free_blocks(self) -> int:
-        return int(self._lib.pa_bm_num_free_blocks(self._h))
+        return int(self._lib.pa_bm_num_free_blocks(self._live()))
 
     @property
     def usage_ratio(self) -> float:
-        return float(self._lib.pa_bm_usage_ratio(self._h))
+        return float(self._lib.pa_bm_usage_ratio(self._live()))
 
     def can_allocate(self, num_tokens: int) -> bool:
-        return bool(self._lib.pa_bm_can_allocate(self._h, num_tokens))
+        return bool(self._lib.pa_bm_can_allocate(self._live(), num_tokens))
 
     def allocate(self, seq_id: int, num_tokens: int) -> None:
-        _check(self._lib.pa_bm_allocate(self._h, seq_id, num_tokens), "pa_bm_allocate")
+        _check(self._lib.pa_bm_allocate(self._live(), seq_id, num_tokens), "pa_bm_allocate")
 
     def fork(self, parent_id: int, child_id: int) -> None:
-        _check(self._lib.pa_bm_fork(self._h, parent_id, child_id), "pa_bm_fork")
+        _check(self._lib.pa_bm_fork(self._live(), parent_id, child_id), "pa_bm_fork")
 
     def free(self, seq_id: int) -> None:
-        _check(self._lib.pa_bm_free(self._h, seq_id), "pa_bm_free")
+        _check(self._lib.pa_bm_free(self._live(), seq_id), "pa_bm_free")
 
     def append_slots(self, seq_ids):
         """One new token per sequence -> (slot_mapping int64 [n], copy pairs int64 [p, 2])."""
@@ -115,40 +122,44 @@ class BlockManager:
         slots = np.empty(n, np.int64)
         pairs = np.empty((max(n, 1), 2), np.int64)
         npairs = ctypes.c_int(0)
-        _check(self._lib.pa_bm_append_slots(self._h, _p(ids), n, _p(slots), _p(pairs), n,
+        _check(self._lib.pa_bm_append_slots(self._live(), _p(ids), n, _p(slots), _p(pairs), n,
                                             ctypes.byref(npairs)), "pa_bm_append_slots")
         return slots, pairs[:npairs.value].copy()
 
     def slot(self, seq_id: int, pos: int) -> int:
-        return int(self._lib.pa_bm_slot(self._h, seq_id, pos))
+        """Slot of token position ``pos``; -1 where the position has no block (past the
+        sequence's end, or released by the sliding window), which a cache write skips."""
+        return int(self._lib.pa_bm_slot(self._live(), seq_id, pos))
 
     def seq_len(self, seq_id: int) -> int:
-        return int(self._lib.pa_bm_seq_len(self._h, seq_id))
+        """Context length of a sequence; -1 for an unknown sequence."""
+        return int(self._lib.pa_bm_seq_len(self._live(), seq_id))
 
     def refcount(self, block: int) -> int:
-        return int(self._lib.pa_bm_block_refcount(self._h, block))
+        """Reference count of a physical block (0 = free); -1 for an id outside the pool."""
+        return int(self._lib.pa_bm_block_refcount(self._live(), block))
 
     def set_sliding_window(self, window: int) -> None:
         """Keep only each sequence's last ``window`` positions: blocks wholly before them
         go back to the pool (table entry -1).  Only while no sequence exists."""
-        _check(self._lib.pa_bm_set_sliding_window(self._h, window), "pa_bm_set_sliding_window")
+        _check(self._lib.pa_bm_set_sliding_window(self._live(), window), "pa_bm_set_sliding_window")
 
     def set_cpu_pool(self, num_cpu_blocks: int) -> None:
-        _check(self._lib.pa_bm_set_cpu_pool(self._h, num_cpu_blocks), "pa_bm_set_cpu_pool")
+        _check(self._lib.pa_bm_set_cpu_pool(self._live(), num_cpu_blocks), "pa_bm_set_cpu_pool")
 
     @property
     def num_free_cpu_blocks(self) -> int:
-        return int(self._lib.pa_bm_num_free_cpu_blocks(self._h))
+        return int(self._lib.pa_bm_num_free_cpu_blocks(self._live()))
 
     def is_swapped(self, seq_id: int) -> bool:
-        return self._lib.pa_bm_is_swapped(self._h, seq_id) == 1
+        return self._lib.pa_bm_is_swapped(self._live(), seq_id) == 1
 
     def _move(self, fn, seq_ids, what):
         ids = np.ascontiguousarray(seq_ids, np.int64)
         cap = max(1, int(self.num_blocks))
         pairs = np.empty((cap, 2), np.int64)
         npairs = ctypes.c_int(0)
-        _check(fn(self._h, _p(ids), ids.shape[0], _p(pairs), cap, ctypes.byref(npairs)), what)
+        _check(fn(self._live(), _p(ids), ids.shape[0], _p(pairs), cap, ctypes.byref(npairs)), what)
         return pairs[:npairs.value].copy()
 
     def swap_out(self, seq_ids):
@@ -165,6 +176,6 @@ class BlockManager:
         n = ids.shape[0]
         bt = np.empty((n, width), np.int32)
         cl = np.empty(n, np.int32)
-        _check(self._lib.pa_bm_block_tables(self._h, _p(ids), n, _p(bt), width, _p(cl)),
+        _check(self._lib.pa_bm_block_tables(self._live(), _p(ids), n, _p(bt), width, _p(cl)),
                "pa_bm_block_tables")
         return bt, cl

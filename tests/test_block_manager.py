@@ -279,3 +279,14 @@ def test_logical_token_streams_through_tables(window):
                 got = oracle_np.gather_positions(kc, bt[0], lo, L, g)
                 want = np.concatenate([t[:, g] for t in toks[lo:]])
                 assert np.array_equal(got, want), (step, s)
+
+
+def test_closed_manager_refuses_calls():
+    bm = pa.BlockManager(8, 16)
+    bm.allocate(1, 20)
+    bm.close()
+    bm.close()  # idempotent
+    with pytest.raises(pa.PAError, match="closed"):
+        bm.allocate(2, 5)
+    with pytest.raises(pa.PAError, match="closed"):
+        _ = bm.num_free_blocks
