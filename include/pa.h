@@ -7,10 +7,9 @@
  * host pools, asks the runtime what each pool is): a host pointer, or memory of
  * another device than the current one, where device memory is required is
  * undefined behaviour.  The Python binding checks device, dtype, contiguity and
- * shapes of its tensors before it calls in.  Every
- * call is asynchronous on `stream` (a cudaStream_t passed as void*, NULL = the
- * legacy default stream) and never synchronises the device, except
- * pa_get_device_error, which says so.
+ * shapes of its tensors before it calls in.  Every call is asynchronous on
+ * `stream` (a cudaStream_t passed as void*, NULL = the legacy default stream) and
+ * never synchronises the device, except pa_get_device_error, which says so.
  *
  * Data layout (both caches, the same for every call):
  *   k_cache, v_cache : [num_blocks][num_kv_heads][block_size][head_dim], 16-bit
@@ -46,7 +45,8 @@ extern "C" {
 typedef enum {
     PA_OK = 0,
     PA_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad size, workspace too small */
-    PA_ERR_UNSUPPORTED = 2, /* head_dim, block size or group size not built */
+    PA_ERR_UNSUPPORTED = 2, /* head_dim, block size or group size not built, or a size
+                               past a launch limit the entry point states (split the call) */
     PA_ERR_CUDA = 3,        /* a CUDA runtime call failed (launch, attribute, ...) */
     PA_ERR_OUT_OF_RANGE = 4,
     PA_ERR_TIMEOUT = 5,
@@ -93,6 +93,9 @@ pa_status pa_kv_write(const void *key, const void *value, const int64_t *slot_ma
  * (all kv heads, all block_size slots).  src_dst_pairs: int64 [num_pairs][2], device.
  * Destinations must be distinct and no destination may be a source of the same call.
  * Bit-exact.  Caches 16-byte aligned; num_kv_heads*block_size*head_dim multiple of 8.
+ * A pair id outside [0, num_blocks) sets PA_DEVERR_PAIR and that pair is skipped.
+ * At most 65535 pairs per call, and a block of at most 65535 x 2048 16-byte chunks;
+ * larger calls return PA_ERR_UNSUPPORTED (split them).
  */
 pa_status pa_copy_blocks(void *k_cache, void *v_cache, const int64_t *src_dst_pairs,
                          int num_pairs, int num_kv_heads, int block_size, int head_dim,
@@ -112,7 +115,10 @@ pa_status pa_copy_blocks(void *k_cache, void *v_cache, const int64_t *src_dst_pa
  * unified addressing).  src_dst_pairs: int64 [num_pairs][2] in device memory (or
  * mapped pinned memory).  Destination blocks must be distinct and the two pools must
  * not overlap.  One launch; bit-exact.  A pair id outside its pool sets
- * PA_DEVERR_PAIR and that pair is skipped.  Pointers 16-byte aligned.
+ * PA_DEVERR_PAIR and that pair is skipped.  Pointers 16-byte aligned.  Every pointer
+ * is checked with the runtime before the launch: pageable host memory returns
+ * PA_ERR_INVALID_ARG.  A block of at most 65535 x 2048 16-byte chunks (else
+ * PA_ERR_UNSUPPORTED).
  */
 pa_status pa_swap_blocks(void *dst_k_cache, void *dst_v_cache, const void *src_k_cache,
                          const void *src_v_cache, const int64_t *src_dst_pairs, int num_pairs,
