@@ -39,6 +39,13 @@ MUTANTS = [
      "int pos = L - n + (tok - query_start_loc[s]) + (n < L);"),
     ("prefill_wrong_seq", "query_start_loc[s] <= tok && tok < query_start_loc[s + 1]",
      "query_start_loc[s] <= tok && tok <= query_start_loc[s + 1]"),
+    ("prefill_not_causal", "pos + 1, h,", "L, h,"),
+    ("prefill_q_head", "q + ((size_t)tok * num_q_heads + h) * head_dim",
+     "q + ((size_t)tok * num_q_heads + 0) * head_dim"),
+    ("prefill_window_ignored", "dtype,\n                    window) != 0)",
+     "dtype,\n                    0) != 0)"),
+    ("softmax_skips_first", "for (int t = t_lo; t < L; ++t) {\n            z[t] = exp",
+     "for (int t = t_lo + 1; t < L; ++t) {\n            z[t] = exp"),
 ]
 
 
