@@ -5,6 +5,8 @@ import os
 import re
 
 import pytest
+from hypothesis import given, settings
+from hypothesis import strategies as st
 
 import paged_kv_cache_441_b200 as pa
 from paged_kv_cache_441_b200 import build as pa_build
@@ -151,3 +153,41 @@ def test_kv_write_refuses_oversized_call(lib):
     st = lib.pa_kv_write(P(16), P(16), P(16), 1 << 28, 8, 128, 1024, 1024, P(16), P(16), 1 << 20,
                          16, 1, None)
     assert st == 2  # PA_ERR_UNSUPPORTED
+
+
+def _attend_bound(W, bs, mcl, win):
+    """Most tokens one context's partitions must cover: the table's capacity, cut by the
+    max_context_len hint and, under a window, by the window plus the tile it starts in."""
+    bound = W * bs
+    if 0 < mcl < bound:
+        bound = mcl
+    if win > 0:
+        bound = min(bound, win + 15)
+    return max(bound, 1)
+
+
+@settings(max_examples=400, derandomize=True, deadline=None)
+@given(B=st.integers(1, 600), G=st.sampled_from([1, 2, 4, 8]), hkv=st.integers(1, 16),
+       d=st.sampled_from([64, 128]), bs=st.sampled_from([8, 16, 32, 64, 128, 256, 512]),
+       W=st.integers(1, 4096), mcl=st.integers(0, 300000), win=st.integers(0, 70000),
+       ps=st.sampled_from([0, 0, 64, 128, 512, 1024, 4096]))
+def test_workspace_plan_invariants(lib, B, G, hkv, d, bs, W, mcl, win, ps):
+    """The fixed split covers every token a context may attend, a single pass needs no
+    workspace, and a split's workspace holds one (d + 2)-float record per (sequence, q
+    head, partition), 256-byte aligned; a longer hint or window never shrinks it."""
+    hq = G * hkv
+    P = pa.decode_partition_tokens(B, hq, hkv, d, bs, W, mcl, ps, win)
+    ws = pa.decode_workspace_bytes(B, hq, hkv, d, bs, W, mcl, ps, win)
+    bound = _attend_bound(W, bs, mcl, win)
+    assert P > 0 and P % 64 == 0
+    if ps > 0:
+        assert P == ps
+    parts = -(-bound // P)
+    if parts == 1:
+        assert ws == 0
+    else:
+        assert ws % 256 == 0 and ws >= B * hq * parts * (d + 2) * 4
+    if ps > 0:  # monotone in the hint and the window (the automatic size may switch)
+        assert ws <= pa.decode_workspace_bytes(B, hq, hkv, d, bs, W, mcl + 4096, ps, win)
+        if win > 0:
+            assert ws <= pa.decode_workspace_bytes(B, hq, hkv, d, bs, W, mcl, ps, win + 4096)
