@@ -188,6 +188,15 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+def workload_config(case, desc, ws):
+    """The keys that identify a decode workload, the same in both arms' JSON lines."""
+    return {"workload": desc, "num_seqs": case.num_seqs, "num_q_heads": case.num_q_heads,
+            "num_kv_heads": case.num_kv_heads, "head_dim": case.head_dim,
+            "block_size": case.block_size, "num_blocks": case.num_blocks,
+            "kv_tokens": int(case.context_lens.sum()), "max_context_len": case.max_context_len,
+            "sliding_window": case.window, "parallelism": f"dp{ws} (independent replicas)"}
+
+
 def dist_env():
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -514,14 +523,9 @@ def run_ours(args):
             "vs_baseline": None,
             "dtype": dt,
             "data": "synthetic (seeded N(0,1) q/K/V rounded to bf16, shuffled block pool)",
-            "config": {"workload": desc, "num_seqs": case.num_seqs,
-                       "num_q_heads": case.num_q_heads, "num_kv_heads": case.num_kv_heads,
-                       "head_dim": case.head_dim, "block_size": case.block_size,
-                       "num_blocks": case.num_blocks, "kv_tokens": int(case.context_lens.sum()),
-                       "max_context_len": mcl, "sliding_window": win,
+            "config": {**workload_config(case, desc, ws),
                        "split": ("balanced over persistent warps (stream-K) + LSE merge"
                                  if ptoks == 0 else f"fixed {ptoks}-token partitions, {nparts} max"),
-                       "parallelism": f"dp{ws} (independent replicas)",
                        "step": ("pa_decode_append (cache write fused into decode)" if fused
                                 else "pa_copy_blocks + pa_kv_write + pa_decode"),
                        "l2": f"inputs larger than L2: {decode_bytes(case) / 1e9:.2f} GB of K/V "
@@ -1038,7 +1042,8 @@ def run_reference(args):
             "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(tot_t / args.steps * 1e3, 4), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": desc},
+            "config": {**workload_config(case, desc, ws),
+                       "step": "fp64 CPU oracle of the step's attention outputs"},
             "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": nthreads,
                              "kind": "oracle", "sample": sample},
             "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
