@@ -272,10 +272,22 @@ def cpu_baseline(case, budget_s=10.0):
         if reps >= 50:
             break
     gbs = decode_bytes(case) * reps / t_all / 1e9
+    # the same oracle on one thread, over a seeded sample of (seq, q head) pairs sized to
+    # about a third of the budget
+    rng = np.random.default_rng(0)
+    probe = all_sel[rng.permutation(len(all_sel))[:8]]
+    per_pair = oracle_step_time(case, sel=probe, nthreads=1) / len(probe)
+    n1 = int(max(1, min(len(all_sel), budget_s / 3 / max(per_pair, 1e-9))))
+    sel1 = all_sel[rng.permutation(len(all_sel))[:n1]]
+    t1 = oracle_step_time(case, sel=sel1, nthreads=1)
     return {"value": round(gbs, 4), "unit": "GB/s", "cores": nthreads, "kind": "oracle",
             "sample": f"full workload decode (all {case.num_seqs} seqs x {case.num_q_heads} "
                       f"q heads), fp64 C oracle with OpenMP, repeated {reps}x in {t_all:.1f} s",
-            "seq_steps_per_s": round(case.num_seqs * reps / t_all, 3)}
+            "seq_steps_per_s": round(case.num_seqs * reps / t_all, 3),
+            "single_thread": {"value": round(sel_bytes(case, sel1) / t1 / 1e9, 4),
+                              "unit": "GB/s", "cores": 1,
+                              "sample": f"{n1} of {len(all_sel)} (seq, q head) pairs, seeded, "
+                                        f"{t1:.1f} s"}}
 
 
 # ----------------------------------------------------------------------------- GPU arm
