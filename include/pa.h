@@ -50,7 +50,8 @@ typedef enum {
     PA_ERR_CUDA = 3,        /* a CUDA runtime call failed (launch, attribute, ...) */
     PA_ERR_OUT_OF_RANGE = 4,
     PA_ERR_TIMEOUT = 5,
-    PA_ERR_NO_FREE_BLOCK = 6 /* host block manager: the pool cannot satisfy the request */
+    PA_ERR_NO_FREE_BLOCK = 6, /* host block manager: the pool cannot satisfy the request */
+    PA_ERR_HOST_ALLOC = 7     /* host block manager: a host allocation failed; nothing changed */
 } pa_status;
 
 typedef enum { PA_FP16 = 0, PA_BF16 = 1 } pa_dtype;
@@ -299,7 +300,7 @@ pa_status pa_get_device_error(int device, uint32_t *bits_out, int clear);
 /* Static description of a status code.  Never NULL. */
 const char *pa_status_str(pa_status status);
 
-/* Library ABI version (major * 100 + minor). */
+/* Library ABI version (major * 100 + minor): 201. */
 int pa_version(void);
 
 #ifdef __cplusplus

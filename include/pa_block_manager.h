@@ -22,8 +22,9 @@
  * Not thread-safe: one manager per engine thread.  Operations other than swap-in and
  * free on a swapped-out sequence return PA_ERR_INVALID_ARG.  Sequence ids are caller-chosen
  * int64 values.  Errors: PA_ERR_INVALID_ARG (null pointer, unknown or duplicate
- * sequence id, bad size), PA_ERR_NO_FREE_BLOCK (the pool cannot satisfy the request;
- * nothing is changed).
+ * sequence id, bad size), PA_ERR_NO_FREE_BLOCK (the pool cannot satisfy the request),
+ * PA_ERR_HOST_ALLOC (a host allocation for the manager's bookkeeping failed).  A call
+ * that returns an error has changed nothing; no exception crosses this interface.
  */
 #ifndef PA_BLOCK_MANAGER_H
 #define PA_BLOCK_MANAGER_H
@@ -38,7 +39,8 @@ extern "C" {
 
 typedef struct pa_block_manager pa_block_manager;
 
-/* Pool of num_blocks blocks of block_size tokens; NULL on bad arguments. */
+/* Pool of num_blocks blocks of block_size tokens; NULL on bad arguments or when the
+ * host memory for the pool's bookkeeping cannot be allocated. */
 pa_block_manager *pa_bm_create(int num_blocks, int block_size);
 void pa_bm_destroy(pa_block_manager *bm);
 

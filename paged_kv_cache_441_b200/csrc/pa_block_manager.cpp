@@ -6,7 +6,15 @@
 // copy first (copy-on-write), reported as a (src, dst) pair for pa_copy_blocks.
 // Under a sliding window of W tokens, a block that lies wholly before the last W
 // positions of its sequence is given back and its table entry becomes -1.
+//
+// Failure atomicity: every entry point either does all of its work or changes nothing.
+// Those that allocate host memory do every allocation (or reserve the capacity they
+// will fill) before the first change, and a failed allocation becomes
+// PA_ERR_HOST_ALLOC at the C boundary instead of an exception.  The free lists never
+// grow past the capacity reserved when their pool was made, so giving blocks back
+// cannot fail.
 #include <cstdint>
+#include <memory>
 #include <new>
 #include <unordered_map>
 #include <vector>
@@ -64,6 +72,17 @@ struct pa_block_manager {
 
 namespace {
 
+// Runs an entry point's body; an exception (a failed host allocation) becomes
+// PA_ERR_HOST_ALLOC.  The bodies allocate before they change anything.
+template <typename Body>
+pa_status no_throw(Body &&body) {
+    try {
+        return body();
+    } catch (...) {
+        return PA_ERR_HOST_ALLOC;
+    }
+}
+
 // Moves the listed sequences between the pools: `from` (refcounts, free list) -> `to`.
 pa_status move_group(pa_block_manager *bm, const int64_t *seq_ids, int n, int64_t *pairs,
                      int max_pairs, int *num_pairs, bool out) {
@@ -91,21 +110,24 @@ pa_status move_group(pa_block_manager *bm, const int64_t *seq_ids, int n, int64_
         if (uses[b] != from_ref[b]) return PA_ERR_INVALID_ARG;  // shared outside the group
     if ((int)order.size() > (int)to_free.size()) return PA_ERR_NO_FREE_BLOCK;
     if ((int)order.size() > max_pairs) return PA_ERR_INVALID_ARG;
+    // the destination of every block, decided (and allocated) before anything moves
     std::unordered_map<int, int> moved;
+    moved.reserve(order.size());
+    for (size_t i = 0; i < order.size(); ++i)
+        moved.emplace(order[i], to_free[to_free.size() - 1 - i]);
     for (size_t i = 0; i < order.size(); ++i) {
         const int b = order[i];
         const int nb = to_free.back();
         to_free.pop_back();
         to_ref[nb] = from_ref[b];
         from_ref[b] = 0;
-        from_free.push_back(b);
-        moved[b] = nb;
+        from_free.push_back(b);  // within the capacity reserved for that pool
         pairs[2 * i] = b;
         pairs[2 * i + 1] = nb;
     }
     for (pa_block_manager::Seq *g : group) {
         for (int &b : g->blocks)
-            if (b >= 0) b = moved[b];
+            if (b >= 0) b = moved.find(b)->second;
         g->on_cpu = out;
     }
     *num_pairs = (int)order.size();
@@ -118,10 +140,15 @@ extern "C" {
 
 pa_status pa_bm_set_cpu_pool(pa_block_manager *bm, int num_cpu_blocks) {
     if (!bm || num_cpu_blocks <= 0 || bm->num_cpu_blocks != 0) return PA_ERR_INVALID_ARG;
-    bm->num_cpu_blocks = num_cpu_blocks;
-    bm->cpu_refcount.assign(num_cpu_blocks, 0);
-    for (int b = num_cpu_blocks - 1; b >= 0; --b) bm->cpu_free_list.push_back(b);
-    return PA_OK;
+    return no_throw([&] {
+        std::vector<int> ref(num_cpu_blocks, 0), free_list;
+        free_list.reserve(num_cpu_blocks);
+        for (int b = num_cpu_blocks - 1; b >= 0; --b) free_list.push_back(b);
+        bm->cpu_refcount.swap(ref);
+        bm->cpu_free_list.swap(free_list);
+        bm->num_cpu_blocks = num_cpu_blocks;
+        return PA_OK;
+    });
 }
 
 int pa_bm_num_free_cpu_blocks(const pa_block_manager *bm) {
@@ -136,12 +163,13 @@ int pa_bm_is_swapped(const pa_block_manager *bm, int64_t seq_id) {
 
 pa_status pa_bm_swap_out(pa_block_manager *bm, const int64_t *seq_ids, int n, int64_t *pairs,
                          int max_pairs, int *num_pairs) {
-    return move_group(bm, seq_ids, n, pairs, max_pairs, num_pairs, true);
+    return no_throw([&] { return move_group(bm, seq_ids, n, pairs, max_pairs, num_pairs, true); });
 }
 
 pa_status pa_bm_swap_in(pa_block_manager *bm, const int64_t *seq_ids, int n, int64_t *pairs,
                         int max_pairs, int *num_pairs) {
-    return move_group(bm, seq_ids, n, pairs, max_pairs, num_pairs, false);
+    return no_throw(
+        [&] { return move_group(bm, seq_ids, n, pairs, max_pairs, num_pairs, false); });
 }
 
 pa_status pa_bm_set_sliding_window(pa_block_manager *bm, int window) {
@@ -152,16 +180,19 @@ pa_status pa_bm_set_sliding_window(pa_block_manager *bm, int window) {
 
 pa_block_manager *pa_bm_create(int num_blocks, int block_size) {
     if (num_blocks <= 0 || block_size <= 0) return nullptr;
-    pa_block_manager *bm = new (std::nothrow) pa_block_manager();
-    if (!bm) return nullptr;
-    bm->num_blocks = num_blocks;
-    bm->block_size = block_size;
-    bm->refcount.assign(num_blocks, 0);
-    bm->released.assign(num_blocks, 0);
-    bm->released_stamp.assign(num_blocks, 0);
-    bm->free_list.reserve(num_blocks);
-    for (int b = num_blocks - 1; b >= 0; --b) bm->free_list.push_back(b);  // hands out 0, 1, ...
-    return bm;
+    try {
+        std::unique_ptr<pa_block_manager> bm(new pa_block_manager());
+        bm->num_blocks = num_blocks;
+        bm->block_size = block_size;
+        bm->refcount.assign(num_blocks, 0);
+        bm->released.assign(num_blocks, 0);
+        bm->released_stamp.assign(num_blocks, 0);
+        bm->free_list.reserve(num_blocks);
+        for (int b = num_blocks - 1; b >= 0; --b) bm->free_list.push_back(b);  // hands out 0, 1, ...
+        return bm.release();
+    } catch (...) {
+        return nullptr;  // out of host memory
+    }
 }
 
 void pa_bm_destroy(pa_block_manager *bm) { delete bm; }
@@ -192,12 +223,14 @@ pa_status pa_bm_allocate(pa_block_manager *bm, int64_t seq_id, int num_tokens) {
     // takes all its blocks; those before the window go back at its next append
     const int need = pa_bm_blocks_needed(num_tokens, bm->block_size);
     if (need > (int)bm->free_list.size()) return PA_ERR_NO_FREE_BLOCK;
-    pa_block_manager::Seq s;
-    s.blocks.reserve(need);
-    for (int i = 0; i < need; ++i) s.blocks.push_back(bm->take());
-    s.len = num_tokens;
-    bm->seqs.emplace(seq_id, std::move(s));
-    return PA_OK;
+    return no_throw([&] {
+        pa_block_manager::Seq s;
+        s.blocks.reserve(need);
+        pa_block_manager::Seq &t = bm->seqs.emplace(seq_id, std::move(s)).first->second;
+        for (int i = 0; i < need; ++i) t.blocks.push_back(bm->take());  // within capacity
+        t.len = num_tokens;
+        return PA_OK;
+    });
 }
 
 pa_status pa_bm_fork(pa_block_manager *bm, int64_t parent_id, int64_t child_id) {
@@ -205,12 +238,14 @@ pa_status pa_bm_fork(pa_block_manager *bm, int64_t parent_id, int64_t child_id) 
     auto it = bm->seqs.find(parent_id);
     if (it == bm->seqs.end() || it->second.on_cpu || bm->seqs.count(child_id))
         return PA_ERR_INVALID_ARG;
-    pa_block_manager::Seq child = it->second;
-    child.stamp = 0;
-    for (int b : child.blocks)
-        if (b >= 0) ++bm->refcount[b];
-    bm->seqs.emplace(child_id, std::move(child));
-    return PA_OK;
+    return no_throw([&] {
+        // the copy and the insertion allocate; the reference counts change after them
+        pa_block_manager::Seq &child = bm->seqs.emplace(child_id, it->second).first->second;
+        child.stamp = 0;
+        for (int b : child.blocks)
+            if (b >= 0) ++bm->refcount[b];
+        return PA_OK;
+    });
 }
 
 pa_status pa_bm_free(pa_block_manager *bm, int64_t seq_id) {
@@ -241,7 +276,11 @@ pa_status pa_bm_append_slots(pa_block_manager *bm, const int64_t *seq_ids, int n
     // anything), following the reference counts as earlier entries of the batch
     // would change them
     const unsigned stamp = ++bm->batch;
-    bm->batch_seqs.resize(n);
+    if (no_throw([&] {
+            bm->batch_seqs.resize(n);
+            return PA_OK;
+        }) != PA_OK)
+        return PA_ERR_HOST_ALLOC;
     int fresh = 0, pairs = 0;
     for (int i = 0; i < n; ++i) {
         auto it = bm->seqs.find(seq_ids[i]);
@@ -254,6 +293,16 @@ pa_status pa_bm_append_slots(pa_block_manager *bm, const int64_t *seq_ids, int n
         bm->batch_seqs[i] = &s;
         if (s.len % bs == 0) {
             ++fresh;
+            // room for the block pass 2 appends, so that pass 2 cannot fail half-way
+            std::vector<int> &b = s.blocks;
+            if (b.size() == b.capacity() &&
+                no_throw([&] {
+                    b.reserve(b.empty() ? 4 : 2 * b.size());
+                    return PA_OK;
+                }) != PA_OK) {
+                for (int j = 0; j <= i; ++j) bm->batch_seqs[j]->stamp = 0;
+                return PA_ERR_HOST_ALLOC;
+            }
         } else {
             const int last = s.blocks.back();
             int &rel = bm->released[last];
@@ -280,7 +329,7 @@ pa_status pa_bm_append_slots(pa_block_manager *bm, const int64_t *seq_ids, int n
         int blk;
         if (off == 0) {
             blk = bm->take();
-            s.blocks.push_back(blk);
+            s.blocks.push_back(blk);  // within the capacity reserved in pass 1
         } else {
             blk = s.blocks.back();
             if (bm->refcount[blk] > 1) {

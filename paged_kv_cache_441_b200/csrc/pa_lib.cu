@@ -372,7 +372,7 @@ pa_status check_decode_shape(int num_seqs, int num_q_heads, int num_kv_heads, in
 
 extern "C" {
 
-int pa_version(void) { return 200; }
+int pa_version(void) { return 201; }
 
 const char *pa_status_str(pa_status s) {
     switch (s) {
@@ -383,6 +383,7 @@ const char *pa_status_str(pa_status s) {
         case PA_ERR_OUT_OF_RANGE: return "index out of range (device error word)";
         case PA_ERR_TIMEOUT: return "bounded wait expired (device error word)";
         case PA_ERR_NO_FREE_BLOCK: return "no free block in the pool";
+        case PA_ERR_HOST_ALLOC: return "host memory allocation failed";
     }
     return "unknown status";
 }

@@ -44,7 +44,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_status_strings_and_version(lib):
-    assert pa.version() == 200
+    assert pa.version() == 201
     for code in range(7):
         assert lib.pa_status_str(code) != b"unknown status"
     assert lib.pa_status_str(77) == b"unknown status"
