@@ -64,3 +64,61 @@ def test_prefix_cow_structure():
     dst = c.copy_pairs[:, 1]
     assert len(set(dst.tolist())) == len(dst) and not set(dst) & set(c.copy_pairs[:, 0])
     assert len(set(c.slot_mapping.tolist())) == len(c.slot_mapping)
+
+
+def test_prefill_case_structure():
+    """Chunks sit at the end of their contexts, each new token's slot is its position's
+    page and offset, pages are distinct across sequences, and poison covers exactly the
+    slots that are neither earlier context nor written by the step."""
+    from workloads import make_prefill_case
+    specs = [(9, 9), (5, 30), (1, 12), (0, 7), (17, 17)]
+    c = make_prefill_case("pfs", 3, specs, 8, 2, 32, 8, dtype="fp16")
+    bs, qsl = c.block_size, c.query_start_loc
+    assert qsl.tolist() == [0, 9, 14, 15, 15, 32] and c.num_tokens == 32
+    assert c.context_lens.tolist() == [L for _, L in specs]
+    used, need = _check_tables(c)
+    assert len(set(used)) == len(used) <= c.num_blocks
+    for s, (n, L) in enumerate(specs):
+        for i in range(n):
+            p = L - n + i
+            blk, off = divmod(int(c.slot_mapping[qsl[s] + i]), bs)
+            assert blk == c.block_tables[s, p // bs] and off == p % bs
+    assert len(set(c.slot_mapping.tolist())) == c.num_tokens
+    nan = NAN_BITS["fp16"]
+    earlier = {(int(c.block_tables[s, p // bs]), p % bs)
+               for s, (n, L) in enumerate(specs) for p in range(L - n)}
+    for b in range(c.num_blocks):
+        for o in range(bs):
+            poisoned = bool(np.all(c.k_cache[b, :, o] == nan))
+            assert poisoned == ((b, o) not in earlier), (b, o)
+
+
+def test_prefill_workloads_shapes():
+    from workloads import make_prefill_config
+    a = make_prefill_config("prefill_2k_gqa", poison=False)
+    assert (a.num_seqs, a.num_tokens, a.num_q_heads, a.num_kv_heads, a.head_dim) == \
+        (8, 8 * 2048, 32, 8, 128)
+    b = make_prefill_config("prefill_chunk512_gqa", poison=False)
+    n = np.diff(b.query_start_loc)
+    assert b.num_seqs == 16 and np.all(n == 512)
+    assert sorted(set(b.context_lens.tolist())) == sorted({2048 + 128 * (i % 13) for i in range(16)})
+
+
+def test_window_case_holds_only_the_windows_pages():
+    """Under a sliding window the pages wholly before each sequence's window are -1 and
+    the pool holds the window pages plus spare; the new token's slot is still L - 1."""
+    from workloads import make_case
+    W, bs = 20, 8
+    c = make_case("win", 5, 6, 4, 2, 32, bs, lambda r: np.array([1, 19, 20, 21, 60, 100],
+                                                              np.int32), window=W)
+    held = []
+    for s, L in enumerate(c.context_lens.tolist()):
+        need = -(-L // bs)
+        dead = max(L - W, 0) // bs
+        row = c.block_tables[s]
+        assert np.all(row[:dead] == -1) and np.all(row[dead:need] >= 0)
+        assert np.all(row[need:] == -1)
+        held.extend(row[dead:need].tolist())
+        blk, off = divmod(int(c.slot_mapping[s]), bs)
+        assert blk == row[(L - 1) // bs] and off == (L - 1) % bs
+    assert len(set(held)) == len(held) <= c.num_blocks
