@@ -46,6 +46,10 @@ MUTANTS = [
      "dtype,\n                    0) != 0)"),
     ("softmax_skips_first", "for (int t = t_lo; t < L; ++t) {\n            z[t] = exp",
      "for (int t = t_lo + 1; t < L; ++t) {\n            z[t] = exp"),
+    ("fp16_subnormal", "ldexp((double)f, -24)", "ldexp((double)f, -23)"),
+    ("copy_v_from_k", "v_cache[(size_t)dst * blk + i] = v_cache[(size_t)src * blk + i];",
+     "v_cache[(size_t)dst * blk + i] = k_cache[(size_t)src * blk + i];"),
+    ("write_v_from_key", "v_cache[dst + i] = vs[i];", "v_cache[dst + i] = ks[i];"),
 ]
 
 
