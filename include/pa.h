@@ -9,7 +9,11 @@
  * undefined behaviour.  The Python binding checks device, dtype, contiguity and
  * shapes of its tensors before it calls in.  Every call is asynchronous on
  * `stream` (a cudaStream_t passed as void*, NULL = the legacy default stream) and
- * never synchronises the device, except pa_get_device_error, which says so.
+ * never synchronises the device, except pa_get_device_error, which says so.  The
+ * launch entry points may be called from several host threads at once: they keep no
+ * host state besides a once-initialised driver entry point and per-device caches, and
+ * on the device they share only the sticky error word (and the scratch array of
+ * pa_decode_static_scratch, which says so).
  *
  * Data layout (both caches, the same for every call):
  *   k_cache, v_cache : [num_blocks][num_kv_heads][block_size][head_dim], 16-bit
