@@ -283,7 +283,9 @@ pa_status pa_decode_static_scratch(void *out, const void *q, const void *k_cache
  * Other arguments : as pa_decode (head_dim 64 or 128, G in {1, 2, 4, 8}, block_size a
  *                   power of two in [8, 512]).
  * Math: S = Q K^T and O = P V on the tcgen05 tensor cores (fp32 accumulation in tensor
- * memory), softmax in fp32 with P rounded to the input type for the P V product.
+ * memory), softmax in fp32; P enters the P V product as two values of the input type, a
+ * high part and the rounded remainder, so it keeps about twice the input type's
+ * precision (the accuracy bar of the output, not the tensor rate, sets this).
  * One launch, no workspace.  Errors: host-checkable problems as pa_decode; n_s > L_s
  * or L_s beyond the table sets PA_DEVERR_CONTEXT (that sequence's rows are not
  * written); an out-of-range table entry sets PA_DEVERR_BLOCK_ID.
