@@ -103,18 +103,18 @@ def _fail(what: str, msg: str):
     raise PAError(f"{what}: {msg}")
 
 
-def _args(what: str, half: dict, ints: dict = None, rows: dict = None, device=None):
+def _args(what: str, half: dict, ints: dict = None, rows: dict = None):
     """Check the tensors of one call before their pointers reach the library.
 
     half: 16-bit float tensors (q, out, caches), one dtype, contiguous.
     ints: name -> (tensor, torch dtype); contiguous (block tables, lengths, slots).
     rows: 16-bit tensors [T, H, d] whose heads are contiguous but whose token stride
           is free (a key or value slice of a wider projection).
-    All of them on one device of type _DEVICE_TYPE (``device`` if given).
+    All of them on the first half tensor's device, which must be of type _DEVICE_TYPE.
     Returns that device."""
     ints, rows = ints or {}, rows or {}
     first = next(iter(half.values()))
-    dev = first.device if device is None else device
+    dev = first.device
     if dev.type != _DEVICE_TYPE:
         _fail(what, f"tensors must be on a {_DEVICE_TYPE} device, got {dev}")
     for name, t in {**half, **rows}.items():
