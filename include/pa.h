@@ -20,8 +20,12 @@
  *                      elements (pa_dtype); one (block, kv head) is one contiguous run.
  *   block_tables     : int32 [num_seqs][max_blocks_per_seq]; entry j of row s is the
  *                      physical block that holds logical tokens [j*bs, (j+1)*bs) of
- *                      sequence s.  Entries at or past ceil(context_lens[s] / bs) are
- *                      never read.
+ *                      sequence s.  Entries at or past ceil(context_lens[s] / bs) never
+ *                      select a page: the decode kernels may load them (a
+ *                      partition's whole table range is fetched before its length
+ *                      is known) but never use their values, so they may hold any
+ *                      value, -1 and out-of-range ids included.  Every load stays
+ *                      inside row s (max_blocks_per_seq entries).
  *   slot             : block * block_size + offset inside the block.
  *
  * Errors.  A problem the host can see (null or misaligned pointer, unsupported
@@ -247,7 +251,11 @@ int pa_decode_partition_tokens(int num_seqs, int num_q_heads, int num_kv_heads, 
  *    launch; use pa_decode with a caller workspace for those.
  *  - The first call on a device looks up the array's device address on that device
  *    (cudaGetSymbolAddress, with the device current); make that first call before
- *    any stream capture.  Later calls reuse the address.
+ *    any stream capture.  Later calls reuse the address, which the library keeps
+ *    for the life of the process: after cudaDeviceReset on a device the module
+ *    may be loaded at another address, so this entry point must not be called on
+ *    that device again in the same process (pa_decode with a workspace is not
+ *    affected).
  *  - Every call on a device shares the one array, and it keeps the last call's
  *    contents.  No part of it needs clearing (each call writes every partial result
  *    it reads), but calls that overlap on the GPU race on it: serialise them (one

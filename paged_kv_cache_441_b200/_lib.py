@@ -352,12 +352,13 @@ def decode_static_scratch(out, q, k_cache, v_cache, block_tables, context_lens, 
     dev = _args(what, {"q": q, "out": out, "k_cache": k_cache, "v_cache": v_cache},
                 ints={"block_tables": (block_tables, torch.int32),
                       "context_lens": (context_lens, torch.int32)})
-    need = decode_workspace_bytes(B, hq, hkv, d, bs, W, max_context_len, partition_size,
-                                  sliding_window)
-    if need > STATIC_SCRATCH_BYTES:
-        _fail(what, f"these sizes need {need} bytes of scratch, more "
-              f"than the library's fixed {STATIC_SCRATCH_BYTES}; use decode() with a workspace")
     with _on(dev):
+        # sized on the tensors' device: the balanced split's need grows with its SM count
+        need = decode_workspace_bytes(B, hq, hkv, d, bs, W, max_context_len, partition_size,
+                                      sliding_window)
+        if need > STATIC_SCRATCH_BYTES:
+            _fail(what, f"these sizes need {need} bytes of scratch, more than the library's "
+                  f"fixed {STATIC_SCRATCH_BYTES}; use decode() with a workspace")
         _check(load().pa_decode_static_scratch(
             _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
             _ptr(context_lens), B, hq, hkv, d, bs, nb, W, float(scale), int(max_context_len),

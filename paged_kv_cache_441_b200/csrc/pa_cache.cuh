@@ -29,8 +29,9 @@ constexpr int kKvwUnroll = 4;
 // One CTA per kKvwThreads * kKvwUnroll consecutive 16-byte chunks of the (token, kv head,
 // chunk) rows, K and V together; each thread issues its kKvwUnroll K and V loads before any
 // store (32-bit index math: the host keeps the chunk count below 2^31).
-// "Every generated token's K and V are stored in the KV cache" (PagedAttention and
-// dynamic memory blog): the store goes to k_cache[slot / bs][h][slot % bs][:].
+// PagedAttention and dynamic memory management blog, first section: the cache keeps the
+// K and V of each token the model produces; here that store goes to
+// k_cache[slot / bs][h][slot % bs][:] (and the same for V).
 __global__ void __launch_bounds__(kKvwThreads) pa_kv_write_kernel(const __grid_constant__ KvWriteParams p) {
     pdl_wait_and_release();
     const unsigned per_tok = (unsigned)(p.num_kv_heads * p.row_chunks);

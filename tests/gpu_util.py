@@ -75,16 +75,3 @@ class DeviceCase:
                   partition_size=partition_size, workspace=workspace,
                   sliding_window=sliding_window)
         return self.out
-
-
-def sample_pairs(case, n=48, seed=0):
-    """(seq, q head) pairs: the shortest and longest sequences plus a seeded sample."""
-    rng = np.random.default_rng(seed)
-    lens = case.context_lens
-    seqs = {int(np.argmin(lens)), int(np.argmax(lens))}
-    seqs |= set(int(x) for x in rng.integers(0, case.num_seqs, size=n))
-    pairs = []
-    for s in sorted(seqs):
-        for h in {0, case.num_q_heads - 1, int(rng.integers(0, case.num_q_heads))}:
-            pairs.append((s, h))
-    return np.array(pairs, np.int32)

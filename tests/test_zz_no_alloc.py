@@ -3,11 +3,13 @@
 Such callers (an engine that handed all free HBM to its KV-cache pool and offers no
 allocator, or code that must not run cudaMalloc inside its decode loop) cannot pass
 pa_decode a workspace.  This entry point keeps the split-K partials in the library's
-own fixed scratch array instead.  The test calls it through the C ABI twice in a
-row, on different inputs that both need several partitions, and checks each output
-against pa_decode with a caller workspace; the second call must not be disturbed by
-what the first left in the shared array.  It also checks that sizes over the fixed
-limit are refused before any launch.  This file sorts last so that a stop-at-first-
+own fixed scratch array instead.  The test calls it through the C ABI several times
+in a row, on different inputs that all need several partitions, and checks each
+output bit for bit against pa_decode with a caller workspace (the same kernels on
+the same plan) and against the fp64 oracle within the bf16 bar; a later call must
+not be disturbed by what an earlier one left in the shared array.  It also checks
+that sizes over the fixed limit are refused before any launch, for the fixed and
+the balanced split.  This file sorts last so that a stop-at-first-
 failure run has run every other test before it.
 """
 import ctypes
@@ -16,8 +18,9 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 import paged_kv_cache_441_b200 as pa
-from tests.gpu_util import TOL, dev, dev16, to_f64
+from tests.gpu_util import TOL, bits, dev, dev16, to_f64
 from workloads import make_case
 
 pytestmark = [pytest.mark.gpu,
@@ -62,7 +65,9 @@ def test_static_scratch_matches_workspace_path_twice():
         pa.decode(want, t["q"], t["kc"], t["vc"], t["bt"], t["cl"], case.scale,
                   max_context_len=case.max_context_len, partition_size=ps)
         torch.cuda.synchronize()
-        err = np.max(np.abs(to_f64(got) - to_f64(want)))
+        assert np.array_equal(bits(got), bits(want)), seed
+        ref, _, _ = oracle.step(case)
+        err = np.max(np.abs(to_f64(got) - ref))
         assert err <= TOL["bf16"], (seed, err)
     assert pa.device_error(0) == 0
 
@@ -75,5 +80,19 @@ def test_static_scratch_refuses_sizes_over_the_limit():
     assert need > pa.STATIC_SCRATCH_BYTES
     out = torch.zeros_like(t["q"])
     assert _c_static(case, t, out, 64) == 1  # PA_ERR_INVALID_ARG, nothing launched
+    torch.cuda.synchronize()
+    assert torch.count_nonzero(out.float()) == 0
+
+
+def test_static_scratch_refuses_balanced_split_over_the_limit():
+    """The balanced split sizes its partial results by the GPU's SM count and the
+    group size: a group of 8 at head_dim 128 needs more than the fixed array."""
+    case, t = _inputs(25, [5000, 7000, 300, 9000], hq=16, hkv=2)
+    need = pa.decode_workspace_bytes(case.num_seqs, case.num_q_heads, case.num_kv_heads,
+                                     case.head_dim, case.block_size, case.max_blocks_per_seq,
+                                     case.max_context_len, -1)
+    assert need > pa.STATIC_SCRATCH_BYTES
+    out = torch.zeros_like(t["q"])
+    assert _c_static(case, t, out, -1) == 1  # PA_ERR_INVALID_ARG, nothing launched
     torch.cuda.synchronize()
     assert torch.count_nonzero(out.float()) == 0

@@ -14,7 +14,9 @@ Layout produced (the library's layout):
 * ``copy_pairs``: ``int64 [P, 2]`` (src, dst) copy-on-write block pairs.
 
 Draw order for a seed: context lengths, the pool permutation, q, K pool, V pool, the
-new tokens' key, value.  Values are N(0, 1) in fp32 rounded to nearest-even.
+new tokens' key, value.  Values are N(0, 1) in fp32 rounded to nearest-even; an array
+of more than 2^24 values takes one key from the seed's stream and draws its chunks of
+2^24 values from generators seeded with (key, chunk index), on host threads.
 
 Poisoning (``poison=True``): every cache slot that the decode step must not read
 (spare blocks, slots at or past ``L-1`` of each sequence's last block, and slot
@@ -24,6 +26,8 @@ a missing write shows up as NaN in the result.
 from __future__ import annotations
 
 import math
+import os
+from concurrent.futures import ThreadPoolExecutor
 from dataclasses import dataclass, field
 
 import numpy as np
@@ -55,11 +59,25 @@ def bits_to_f32(b: np.ndarray, dtype: str) -> np.ndarray:
 
 
 def _draw(rng: np.random.Generator, shape, dtype: str) -> np.ndarray:
+    """N(0, 1) values rounded to `dtype`.  Up to _CHUNK values come from `rng` itself;
+    a larger array takes one 63-bit key from `rng` and fills chunk i from a generator
+    seeded with (key, i), on host threads, so the values do not depend on the thread
+    count."""
     n = int(np.prod(shape))
     out = np.empty(n, dtype=np.uint16)
-    for i in range(0, n, _CHUNK):
+    if n <= _CHUNK:
+        out[:] = round_to_bits(rng.standard_normal(n, dtype=np.float32), dtype)
+        return out.reshape(shape)
+    key = int(rng.integers(0, 2**63 - 1))
+
+    def fill(i: int) -> None:
         m = min(_CHUNK, n - i)
-        out[i:i + m] = round_to_bits(rng.standard_normal(m, dtype=np.float32), dtype)
+        sub = np.random.default_rng([key, i // _CHUNK])
+        out[i:i + m] = round_to_bits(sub.standard_normal(m, dtype=np.float32), dtype)
+
+    workers = max(1, min(16, os.cpu_count() or 1))
+    with ThreadPoolExecutor(max_workers=workers) as ex:
+        list(ex.map(fill, range(0, n, _CHUNK)))
     return out.reshape(shape)
 
 
