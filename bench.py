@@ -292,6 +292,176 @@ def cpu_baseline(case, budget_s=10.0):
 
 # ----------------------------------------------------------------------------- GPU arm
 
+# The Llama-shaped decode workloads on which pa_decode is held to >= 70% of 8 TB/s; the
+# default run times each of them beside the headline workload (one GPU).
+PER_CONFIG = ["llama2_7b", "gqa_llama3_8b", "gqa_llama3_8b_bs32", "long_8_1", "long_8_1_bs512",
+              "long_32_8", "long_32_8_bs512"]
+ROOF_GROUP = 10        # consecutive calls between two events
+ROOF_MIN_GROUPS = 20   # at least 200 calls ...
+ROOF_MIN_S = 0.5       # ... and at least half a second of device time
+FLUSH_CALLS = 50       # L2-flushed pass: median of this many single calls
+FLUSH_BYTES = 256 << 20
+
+
+class DecodeStep:
+    """A decode workload resident on the device and its step: copy-on-write pairs (when
+    the workload has them), the cache write and paged decode -- fused into one call
+    (pa_decode_append) when every sequence appends exactly one token and nothing is
+    copied."""
+
+    def __init__(self, torch, pa, case, device, partition_size):
+        self.case, self.pa = case, pa
+        dt = case.dtype
+
+        def d16(a):
+            return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(device).view(
+                torch.bfloat16 if dt == "bf16" else torch.float16)
+
+        def di(a):
+            return torch.from_numpy(np.ascontiguousarray(a)).to(device)
+
+        self.q, self.kc, self.vc = d16(case.q), d16(case.k_cache), d16(case.v_cache)
+        self.key, self.val = d16(case.key), d16(case.value)
+        self.sm, self.bt, self.cl = di(case.slot_mapping), di(case.block_tables), di(case.context_lens)
+        self.pairs = di(case.copy_pairs.reshape(-1, 2).astype(np.int64))
+        self.out = torch.empty_like(self.q)
+        self.ps = partition_size
+        W, mcl, win = case.max_blocks_per_seq, case.max_context_len, case.window
+        need = pa.decode_workspace_bytes(case.num_seqs, case.num_q_heads, case.num_kv_heads,
+                                         case.head_dim, case.block_size, W, mcl, partition_size,
+                                         win)
+        self.workspace = torch.zeros(max(need, 256), dtype=torch.uint8, device=device)
+        ptoks = pa.decode_partition_tokens(case.num_seqs, case.num_q_heads, case.num_kv_heads,
+                                           case.head_dim, case.block_size, W, mcl,
+                                           partition_size, win)
+        span = min(mcl, W * case.block_size, win + 15 if win > 0 else mcl)
+        nparts = 0 if ptoks == 0 else -(-span // ptoks)
+        self.has_pairs = case.copy_pairs.shape[0] > 0
+        self.fused = ((not self.has_pairs) and case.key.shape[0] == case.num_seqs
+                      and partition_size >= 0)
+        decode_launches = 1 if nparts == 1 else 2
+        self.launches_per_step = decode_launches + (0 if self.fused else
+                                                    1 + (1 if self.has_pairs else 0))
+        self.split = ("balanced over persistent warps (stream-K) + LSE merge" if ptoks == 0
+                      else f"fixed {ptoks}-token partitions, {nparts} max")
+        self.kind = ("pa_decode_append (cache write fused into decode)" if self.fused
+                     else "pa_copy_blocks + pa_kv_write + pa_decode" if self.has_pairs
+                     else "pa_kv_write + pa_decode")
+        self.step_bytes = (decode_bytes(case) + write_bytes(case)
+                           + (copy_bytes(case) if self.has_pairs else 0))
+
+    def decode(self, b=None):
+        """The attention call of the step (with the fused write when the step has it)."""
+        c, pa = self.case, self.pa
+        b = b or {}
+        out, q = b.get("out", self.out), b.get("q", self.q)
+        bt, cl = b.get("bt", self.bt), b.get("cl", self.cl)
+        if self.fused:
+            pa.decode_append(out, q, b.get("key", self.key), b.get("val", self.val), self.kc,
+                             self.vc, bt, cl, c.scale, max_context_len=c.max_context_len,
+                             partition_size=self.ps, workspace=self.workspace,
+                             sliding_window=c.window)
+        else:
+            pa.decode(out, q, self.kc, self.vc, bt, cl, c.scale, max_context_len=c.max_context_len,
+                      partition_size=self.ps, workspace=self.workspace, sliding_window=c.window)
+
+    def step(self, b=None):
+        b = b or {}
+        if not self.fused:
+            if self.has_pairs:
+                self.pa.copy_blocks(self.kc, self.vc, b.get("pairs", self.pairs))
+            self.pa.kv_write(b.get("key", self.key), b.get("val", self.val),
+                             b.get("sm", self.sm), self.kc, self.vc)
+        self.decode(b)
+
+
+def time_groups(torch, fn, stream, est_ms):
+    """Per-call device time of `fn`: CUDA events on the launching stream around groups of
+    ROOF_GROUP consecutive calls (an event between every two launches would stop each
+    kernel from being scheduled while the previous one drains), for at least
+    ROOF_MIN_GROUPS groups and ROOF_MIN_S seconds.  Returns (median ms per call over the
+    groups, number of calls)."""
+    n = max(ROOF_MIN_GROUPS, int(math.ceil(ROOF_MIN_S * 1e3 / (ROOF_GROUP * max(est_ms, 1e-3)))))
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(n)]
+    for i in range(n):
+        ev[i][0].record(stream)
+        for _ in range(ROOF_GROUP):
+            fn()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    return statistics.median(a.elapsed_time(b) / ROOF_GROUP for a, b in ev), n * ROOF_GROUP
+
+
+class L2Flush:
+    """Leaves L2 cold and clean: writes a FLUSH_BYTES buffer (twice the 126 MB L2), then
+    reads another, so the written lines are evicted -- and written back -- before the
+    timed call instead of during it."""
+
+    def __init__(self, torch, device):
+        self.w = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=device)
+        self.r = torch.ones(FLUSH_BYTES // 4, dtype=torch.float32, device=device)
+        self.k = 0
+
+    def __call__(self):
+        self.k += 1
+        self.w.fill_(float(self.k))
+        self.r.sum()
+
+
+def time_flushed(torch, fn, stream, flush):
+    """Median device time of FLUSH_CALLS single calls of `fn`, L2 flushed before each."""
+    times = []
+    for _ in range(FLUSH_CALLS):
+        flush()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        fn()
+        b.record(stream)
+        b.synchronize()
+        times.append(a.elapsed_time(b))
+    return statistics.median(times)
+
+
+def measure_config(torch, pa, name, device, stream, args, peak, flush):
+    """One per-config entry: the workload's step on its own, timed like the headline's
+    roofline pass (median over groups of consecutive calls) and L2-flushed."""
+    wname, kw, desc = WORKLOADS[name]
+    from workloads import make_config
+    case = make_config(wname, poison=False, **kw)
+    ds = DecodeStep(torch, pa, case, device, args.partition_size)
+    for _ in range(args.warmup):
+        ds.step()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(device.index)
+    sampler.start()
+    time.sleep(0.2)
+    t = time.perf_counter()
+    ds.decode()
+    torch.cuda.synchronize()
+    est = (time.perf_counter() - t) * 1e3
+    ms, ncalls = time_groups(torch, ds.decode, stream, est)
+    clocks = sampler.stop()
+    ms_flushed = time_flushed(torch, ds.decode, stream, flush)
+    err = pa.device_error(device.index)
+    if err:
+        raise RuntimeError(f"device error word {err:#x} in the {name} pass")
+    db = decode_bytes(case)
+    ach, ach_f = db / (ms * 1e-3) / 1e9, db / (ms_flushed * 1e-3) / 1e9
+    entry = {"workload": desc, "block_size": case.block_size, "split": ds.split, "call": ds.kind,
+             "value": round(ach, 1), "unit": "GB/s", "ms_per_call": round(ms, 6),
+             "pct_of_8tbs": round(100 * ach / 8000.0, 2), "meets_70pct_of_8tbs": ach >= 5600.0,
+             "roofline": {"achieved": round(ach, 1), "frac": round(ach / peak, 4),
+                          "frac_l2_flushed": round(ach_f / peak, 4),
+                          "ms_per_call_l2_flushed": round(ms_flushed, 6),
+                          "algorithmic_bytes_per_call": db, "calls": ncalls,
+                          "traffic": traffic_from_profile(name)},
+             "clocks": clocks}
+    del ds
+    torch.cuda.empty_cache()
+    return entry
+
+
 def run_ours(args):
     import torch
     ws, rank, local = dist_env()
@@ -314,56 +484,12 @@ def run_ours(args):
         desc = f"{desc} [profiling subset: first {args.seqs} seqs' distribution]"
     case = make_config(name, poison=False, **kw)
     dt = case.dtype
-
-    def d16(a):
-        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(device).view(
-            torch.bfloat16 if dt == "bf16" else torch.float16)
-
-    def di(a):
-        return torch.from_numpy(np.ascontiguousarray(a)).to(device)
-
-    q, kc, vc = d16(case.q), d16(case.k_cache), d16(case.v_cache)
-    key, val = d16(case.key), d16(case.value)
-    sm, bt, cl = di(case.slot_mapping), di(case.block_tables), di(case.context_lens)
-    pairs = di(case.copy_pairs.reshape(-1, 2).astype(np.int64))
-    out = torch.empty_like(q)
-    W = case.max_blocks_per_seq
-    mcl = case.max_context_len
-    win = case.window
-    need = pa.decode_workspace_bytes(case.num_seqs, case.num_q_heads, case.num_kv_heads,
-                                     case.head_dim, case.block_size, W, mcl, args.partition_size,
-                                     win)
-    workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=device)
-    ptoks = pa.decode_partition_tokens(case.num_seqs, case.num_q_heads, case.num_kv_heads,
-                                       case.head_dim, case.block_size, W, mcl,
-                                       args.partition_size, win)
-    # partition_tokens 0: balanced split over persistent warps (decode + merge kernels)
-    span = min(mcl, W * case.block_size, win + 15 if win > 0 else mcl)
-    nparts = 0 if ptoks == 0 else -(-span // ptoks)
-    has_pairs = case.copy_pairs.shape[0] > 0
-    launches_per_step = 1 + (1 if nparts == 1 else 2) + (1 if has_pairs else 0)
+    ds = DecodeStep(torch, pa, case, device, args.partition_size)
+    q, out = ds.q, ds.out
     stream = torch.cuda.current_stream()
 
-    # One new token per sequence (no copy-on-write): the cache write is fused into the
-    # decode (pa_decode_append).  Otherwise: copy pairs, cache write, decode.
-    fused = (not has_pairs) and case.key.shape[0] == case.num_seqs and args.partition_size >= 0
-    launches_per_step = ((1 if nparts == 1 else 2) if fused else launches_per_step)
-
-    def step():
-        if fused:
-            pa.decode_append(out, q, key, val, kc, vc, bt, cl, case.scale, max_context_len=mcl,
-                             partition_size=args.partition_size, workspace=workspace,
-                             sliding_window=win)
-            return
-        if has_pairs:
-            pa.copy_blocks(kc, vc, pairs)
-        pa.kv_write(key, val, sm, kc, vc)
-        pa.decode(out, q, kc, vc, bt, cl, case.scale, max_context_len=mcl,
-                  partition_size=args.partition_size, workspace=workspace,
-                  sliding_window=win)
-
     for _ in range(args.warmup):
-        step()
+        ds.step()
     torch.cuda.synchronize()
     pa.device_error(torch.cuda.current_device())  # clears; warm-up must be clean
 
@@ -378,40 +504,24 @@ def run_ours(args):
     t1 = torch.cuda.Event(enable_timing=True)
     t0.record(stream)
     for i in range(args.steps):
-        step()
+        ds.step()
     t1.record(stream)
     torch.cuda.synchronize()
     if ws > 1:
         dist.barrier()
     elapsed_ms = t0.elapsed_time(t1)
-    # Roofline pass: the same K steps again, timed with CUDA events on the launching
-    # stream around groups of 10 consecutive decode calls (an event between every two
-    # launches would stop each kernel from being scheduled while the previous one
-    # drains).  With the fused step the group holds only decode calls; otherwise events
-    # bracket each pa_decode call.
-    group = 10 if fused else 1
-    ngroups = max(1, args.steps // group)
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(ngroups)]
-    for i in range(ngroups):
-        if fused:
-            ev[i][0].record(stream)
-            for _ in range(group):
-                pa.decode_append(out, q, key, val, kc, vc, bt, cl, case.scale,
-                                 max_context_len=mcl, partition_size=args.partition_size,
-                                 workspace=workspace, sliding_window=win)
-            ev[i][1].record(stream)
-        else:
-            if has_pairs:
-                pa.copy_blocks(kc, vc, pairs)
-            pa.kv_write(key, val, sm, kc, vc)
-            ev[i][0].record(stream)
-            pa.decode(out, q, kc, vc, bt, cl, case.scale, max_context_len=mcl,
-                      partition_size=args.partition_size, workspace=workspace,
-                             sliding_window=win)
-            ev[i][1].record(stream)
-    torch.cuda.synchronize()
     clocks = sampler.stop()
-    dec_ms = [a.elapsed_time(b) / group for a, b in ev]
+
+    # Roofline pass: the attention call alone (the fused call when the step has it), a
+    # fixed length independent of --steps, with its own clock record; then single calls
+    # after an L2 flush.
+    roof_sampler = ClockSampler(torch.cuda.current_device())
+    roof_sampler.start()
+    time.sleep(0.2)
+    dec_ms, roof_calls = time_groups(torch, ds.decode, stream, elapsed_ms / max(args.steps, 1))
+    roof_clocks = roof_sampler.stop()
+    flush = L2Flush(torch, device)
+    dec_ms_flushed = time_flushed(torch, ds.decode, stream, flush)
     errbits = pa.device_error(torch.cuda.current_device())
     if errbits:
         raise RuntimeError(f"device error word {errbits:#x} during the timed loop")
@@ -426,7 +536,7 @@ def run_ours(args):
     h_pairs = torch.from_numpy(case.copy_pairs.reshape(-1, 2).astype(np.int64)).pin_memory()
     h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
     h2d_bytes = sum(t.numel() * t.element_size() for t in (h_q, h_key, h_val, h_sm, h_bt, h_cl))
-    h2d_bytes += h_pairs.numel() * 8 if has_pairs else 0
+    h2d_bytes += h_pairs.numel() * 8 if ds.has_pairs else 0
     d2h_bytes = h_out.numel() * h_out.element_size()
     e2e_steps = max(1, min(args.steps, args.e2e_steps))
 
@@ -435,9 +545,9 @@ def run_ours(args):
     # stream, and step i's output is read back on that stream as soon as it is ready.
     # Every step still copies all of its own inputs in and its output out.
     copy_stream = torch.cuda.Stream(device=device)
-    bufs = [dict(q=torch.empty_like(q), key=torch.empty_like(key), val=torch.empty_like(val),
-                 sm=torch.empty_like(sm), bt=torch.empty_like(bt), cl=torch.empty_like(cl),
-                 pairs=torch.empty_like(pairs), out=torch.empty_like(out)) for _ in range(2)]
+    bufs = [dict(q=torch.empty_like(q), key=torch.empty_like(ds.key), val=torch.empty_like(ds.val),
+                 sm=torch.empty_like(ds.sm), bt=torch.empty_like(ds.bt), cl=torch.empty_like(ds.cl),
+                 pairs=torch.empty_like(ds.pairs), out=torch.empty_like(out)) for _ in range(2)]
     h_outs = [h_out, torch.empty(out.shape, dtype=out.dtype).pin_memory()]
     ev_in = [torch.cuda.Event() for _ in range(2)]
     ev_done = [torch.cuda.Event() for _ in range(2)]
@@ -454,7 +564,7 @@ def run_ours(args):
             b["sm"].copy_(h_sm, non_blocking=True)
             b["bt"].copy_(h_bt, non_blocking=True)
             b["cl"].copy_(h_cl, non_blocking=True)
-            if has_pairs:
+            if ds.has_pairs:
                 b["pairs"].copy_(h_pairs, non_blocking=True)
             ev_in[i % 2].record(copy_stream)
 
@@ -463,18 +573,7 @@ def run_ours(args):
         stream.wait_event(ev_in[i % 2])
         if i >= 2:
             stream.wait_event(ev_read[i % 2])  # step i-2's output has been read back
-        if fused:
-            pa.decode_append(b["out"], b["q"], b["key"], b["val"], kc, vc, b["bt"], b["cl"],
-                             case.scale, max_context_len=mcl,
-                             partition_size=args.partition_size, workspace=workspace,
-                             sliding_window=win)
-        else:
-            if has_pairs:
-                pa.copy_blocks(kc, vc, b["pairs"])
-            pa.kv_write(b["key"], b["val"], b["sm"], kc, vc)
-            pa.decode(b["out"], b["q"], kc, vc, b["bt"], b["cl"], case.scale,
-                      max_context_len=mcl, partition_size=args.partition_size,
-                      workspace=workspace, sliding_window=win)
+        ds.step(b)
         ev_done[i % 2].record(stream)
 
     def d2h(i):
@@ -509,18 +608,38 @@ def run_ours(args):
     torch.testing.assert_close(h_outs[(e2e_steps - 1) % 2], out.cpu(), rtol=0, atol=0)
 
     # ---- aggregate over ranks
-    step_bytes = decode_bytes(case) + write_bytes(case) + (copy_bytes(case) if has_pairs else 0)
     max_ms = max_over_ranks(elapsed_ms, ws, device)
     max_e2e_ms = max_over_ranks(e2e_ms, ws, device)
-    tot_bytes = sum_over_ranks(float(step_bytes), ws, device)
+    tot_bytes = sum_over_ranks(float(ds.step_bytes), ws, device)
     ms_per_step = max_ms / args.steps
     value = tot_bytes / (ms_per_step * 1e-3) / 1e9
     e2e_value = tot_bytes / (max_e2e_ms / e2e_steps * 1e-3) / 1e9
-    dec_avg_ms = sum(dec_ms) / len(dec_ms)
-    achieved = decode_bytes(case) / (dec_avg_ms * 1e-3) / 1e9
+    achieved = decode_bytes(case) / (dec_ms * 1e-3) / 1e9
+    achieved_flushed = decode_bytes(case) / (dec_ms_flushed * 1e-3) / 1e9
     peak, peak_kind = peaks()
     result = None
     if rank == 0:
+        # The other Llama-shaped configs, each timed on its own (one GPU only: the
+        # per-rank replicas of a multi-GPU run are the headline workload).
+        per_config = None
+        if ws == 1 and not args.no_per_config and args.workload in PER_CONFIG:
+            head = {"workload": desc, "block_size": case.block_size, "split": ds.split,
+                    "call": ds.kind, "value": round(achieved, 1), "unit": "GB/s",
+                    "ms_per_call": round(dec_ms, 6),
+                    "pct_of_8tbs": round(100 * achieved / 8000.0, 2),
+                    "meets_70pct_of_8tbs": achieved >= 5600.0,
+                    "roofline": {"achieved": round(achieved, 1), "frac": round(achieved / peak, 4),
+                                 "frac_l2_flushed": round(achieved_flushed / peak, 4),
+                                 "ms_per_call_l2_flushed": round(dec_ms_flushed, 6),
+                                 "algorithmic_bytes_per_call": decode_bytes(case),
+                                 "calls": roof_calls,
+                                 "traffic": traffic_from_profile(args.workload)},
+                    "clocks": roof_clocks}
+            per_config = {}
+            for cname in PER_CONFIG:
+                per_config[cname] = (head if cname == args.workload else
+                                     measure_config(torch, pa, cname, device, stream, args, peak,
+                                                    flush))
         cpu = None if args.no_cpu_baseline or ws > 1 else cpu_baseline(case, args.cpu_budget)
         result = {
             "metric": METRIC,
@@ -535,13 +654,12 @@ def run_ours(args):
             "vs_baseline": None,
             "dtype": dt,
             "data": "synthetic (seeded N(0,1) q/K/V rounded to bf16, shuffled block pool)",
-            "config": {**workload_config(case, desc, ws),
-                       "split": ("balanced over persistent warps (stream-K) + LSE merge"
-                                 if ptoks == 0 else f"fixed {ptoks}-token partitions, {nparts} max"),
-                       "step": ("pa_decode_append (cache write fused into decode)" if fused
-                                else "pa_copy_blocks + pa_kv_write + pa_decode"),
-                       "l2": f"inputs larger than L2: {decode_bytes(case) / 1e9:.2f} GB of K/V "
-                             f"read per step vs 126 MB L2; no flush"},
+            "config": workload_config(case, desc, ws),
+            "plan": {"split": ds.split, "step": ds.kind,
+                     "l2": f"inputs larger than L2 ({decode_bytes(case) / 1e9:.2f} GB of K/V "
+                           f"read per step vs 126 MB); the timed steps run back to back "
+                           f"without a flush; roofline.frac_l2_flushed times single calls "
+                           f"after a {FLUSH_BYTES >> 20} MB write + read"},
             "seq_steps_per_s": round(case.num_seqs * ws / (ms_per_step * 1e-3), 1),
             "pct_of_8tbs": round(100 * value / 8000.0, 2),
             "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d_bytes,
@@ -549,22 +667,27 @@ def run_ours(args):
                     "how": "pa_* calls on double-buffered device inputs; each step's inputs "
                            "copied from pinned host memory and its output read back on a copy "
                            "stream that overlaps the previous step's compute"},
-            "gpu_launches": launches_per_step * args.steps,
+            "gpu_launches": ds.launches_per_step * args.steps,
             "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
-                         "peak_kind": f"{peak_kind} HBM copy GB/s",
+                         "peak_kind": f"{peak_kind} HBM copy GB/s (burst)",
                          "unit": "GB/s", "frac": round(achieved / peak, 4),
+                         "frac_l2_flushed": round(achieved_flushed / peak, 4),
                          "kernel": ("pa_decode_append (cache write fused into the partition "
-                                    "pass) + LSE merge" if fused else
+                                    "pass) + LSE merge" if ds.fused else
                                     "pa_decode (partition pass + LSE merge when split)"),
-                         "achieved_how": ("algorithmic bytes / mean CUDA-event time per call over "
-                                          "a second pass of the K timed steps, events around "
-                                          "groups of 10 consecutive calls" if fused else
-                                          "algorithmic bytes / mean CUDA-event time of each "
-                                          "pa_decode call over a second pass of the K steps"),
+                         "achieved_how": (f"algorithmic bytes / median per-call CUDA-event time "
+                                          f"over groups of {ROOF_GROUP} consecutive calls "
+                                          f"({roof_calls} calls, >= {ROOF_MIN_S} s, a pass of "
+                                          f"its own after the timed steps); frac_l2_flushed: "
+                                          f"median of {FLUSH_CALLS} single calls, each after an "
+                                          f"L2 flush"),
                          "algorithmic_bytes_per_call": decode_bytes(case),
-                         "avg_call_us": round(dec_avg_ms * 1e3, 2),
-                         "traffic": traffic_from_profile(args.workload)},
+                         "avg_call_us": round(dec_ms * 1e3, 2),
+                         "call_us_l2_flushed": round(dec_ms_flushed * 1e3, 2),
+                         "traffic": traffic_from_profile(args.workload),
+                         "clocks": roof_clocks},
             "clocks": clocks,
+            "per_config": per_config,
             "cpu_baseline": cpu,
         }
     if ws > 1:
@@ -1054,8 +1177,8 @@ def run_reference(args):
             "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(tot_t / args.steps * 1e3, 4), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {**workload_config(case, desc, ws),
-                       "step": "fp64 CPU oracle of the step's attention outputs"},
+            "config": workload_config(case, desc, ws),
+            "plan": {"step": "fp64 CPU oracle of the step's attention outputs"},
             "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": nthreads,
                              "kind": "oracle", "sample": sample},
             "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
@@ -1075,6 +1198,8 @@ def main(argv=None):
                     help="profiling only: build the workload with this many sequences")
     ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="skip timing the other Llama-shaped workloads after the headline one")
     ap.add_argument("--cpu-budget", type=float, default=10.0)
     ap.add_argument("--reference-budget", type=float, default=60.0)
     ap.add_argument("--op", choices=["step", "swap", "prefill", "kv_write", "copy_blocks"],

@@ -70,6 +70,7 @@ typedef enum { PA_FP16 = 0, PA_BF16 = 1 } pa_dtype;
 #define PA_DEVERR_PAIR 0x4u     /* a copy pair id outside [0, num_blocks) */
 #define PA_DEVERR_CONTEXT 0x8u  /* context longer than its table or the partition grid */
 #define PA_DEVERR_TIMEOUT 0x10u /* a bounded wait on a copy expired */
+#define PA_DEVERR_WORKSPACE 0x20u /* dynamic split: the workspace's counters were not zero */
 
 /*
  * Cache write ("PagedAttention and dynamic memory management" blog, first section:
@@ -169,12 +170,27 @@ pa_status pa_swap_blocks(void *dst_k_cache, void *dst_v_cache, const void *src_k
  *                         work, cutting contexts wherever the shares end (needs
  *                         num_seqs <= 16383 for head_dim 128, 8191 for 64; otherwise
  *                         fixed partitions are used);
- *                     0: the library chooses.
+ *                     PA_PARTITION_DYNAMIC (-2): dynamic split for a few long contexts
+ *                         -- persistent CTAs (3 per SM), each (sequence, kv head) unit
+ *                         served by CTAs in proportion to its length, whose warps claim
+ *                         32-token chunks of it from a counter while they run, so warps
+ *                         on faster SMs take more.  Needs num_seqs * num_kv_heads <=
+ *                         min(3 * SMs, 1024) (otherwise the library's fixed split is
+ *                         used) and the workspace rule below.  The split of each sum
+ *                         varies between calls, so results may differ in the last bits
+ *                         from call to call;
+ *                     0: the library chooses (a fixed split: the same inputs always
+ *                         give the same bits).
  * workspace       : fp32 scratch for those partial results, at least
  *                   pa_decode_workspace_bytes(...) bytes, 256-byte aligned; may be
  *                   NULL when no context needs more than one partition.  Its contents
- *                   need no initialisation and are overwritten.  Calls that share a
- *                   workspace must not overlap on the GPU.
+ *                   are overwritten, except that with PA_PARTITION_DYNAMIC its first
+ *                   PA_WORKSPACE_ZERO_BYTES bytes hold counters: they must be
+ *                   zero before the workspace's first such call (one cudaMemset after
+ *                   allocating it), and every call leaves them zero (a call that finds
+ *                   them otherwise sets PA_DEVERR_WORKSPACE).  No other split needs any
+ *                   initialisation.  Calls that share a workspace must not overlap on
+ *                   the GPU.
  * Launches 1 kernel (one partition per sequence) or 2 (partition pass + merge).
  */
 pa_status pa_decode(void *out, const void *q, const void *k_cache, const void *v_cache,
@@ -185,6 +201,8 @@ pa_status pa_decode(void *out, const void *q, const void *k_cache, const void *v
                     size_t workspace_bytes, pa_dtype dtype, void *stream);
 
 #define PA_PARTITION_BALANCED (-1)
+#define PA_PARTITION_DYNAMIC (-2)
+#define PA_WORKSPACE_ZERO_BYTES 8192
 
 /*
  * One decode step with its cache write fused in: the cache write of each sequence's
@@ -194,9 +212,10 @@ pa_status pa_decode(void *out, const void *q, const void *k_cache, const void *v
  *   v_cache[...] likewise from value,
  * then the attention of pa_decode over [0, L) (or the last sliding_window tokens of
  * it) -- which therefore includes the new token.
- * The write is done by the CTA that owns the last partition of (s, h) before it reads
- * that position, so the result equals pa_kv_write (with slot = the slot of position L-1)
- * followed by pa_decode, bit for bit.
+ * The write is done by the CTA (the warp, under PA_PARTITION_DYNAMIC) that reads the
+ * last tile of (s, h), before it reads that position, so the result equals pa_kv_write
+ * (with slot = the slot of position L-1) followed by pa_decode -- bit for bit under a
+ * fixed split.
  * key, value : [num_seqs][...] rows, heads contiguous, token strides in elements
  *              (multiples of 8), 16-byte aligned.
  * Sequences must not share the block that holds their position L-1 (copy a shared
@@ -216,8 +235,9 @@ pa_status pa_decode_append(void *out, const void *q, const void *key, const void
 /*
  * Bytes of workspace pa_decode needs for these sizes and this partition_size.
  * Host-side; it reads the current device's SM count (cudaDeviceGetAttribute, no
- * synchronisation; 148 when no device is visible), because the balanced split keeps
- * two partial records per resident warp.  Returns 0 when no merge is needed.
+ * synchronisation; 148 when no device is visible), because the balanced and dynamic
+ * splits keep partial records per resident warp or CTA.  Returns 0 when no merge is
+ * needed.
  */
 size_t pa_decode_workspace_bytes(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
                                  int block_size, int max_blocks_per_seq, int max_context_len,
@@ -225,7 +245,8 @@ size_t pa_decode_workspace_bytes(int num_seqs, int num_q_heads, int num_kv_heads
 
 /*
  * The partition size (tokens) pa_decode uses for these arguments when its
- * partition_size argument is `partition_size`: 0 means the balanced split is used;
+ * partition_size argument is `partition_size`: 0 means the balanced or the dynamic
+ * split is used;
  * a value >= the longest context means one pass per sequence.  Host-side, as
  * pa_decode_workspace_bytes.
  */

@@ -22,8 +22,11 @@ from ._lib import (  # noqa: F401
     DEVERR,
     EXPORTS,
     LIB_PATH,
+    PARTITION_BALANCED,
+    PARTITION_DYNAMIC,
     PAError,
     STATIC_SCRATCH_BYTES,
+    WORKSPACE_ZERO_BYTES,
     copy_blocks,
     decode,
     decode_append,

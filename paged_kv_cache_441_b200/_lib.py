@@ -16,7 +16,8 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libpa.so")
 
 PA_FP16, PA_BF16 = 0, 1
-DEVERR = {"block_id": 0x1, "slot": 0x2, "pair": 0x4, "context": 0x8, "timeout": 0x10}
+DEVERR = {"block_id": 0x1, "slot": 0x2, "pair": 0x4, "context": 0x8, "timeout": 0x10,
+          "workspace": 0x20}
 EXPORTS = ("pa_kv_write", "pa_copy_blocks", "pa_decode", "pa_decode_workspace_bytes",
            "pa_decode_partition_tokens", "pa_get_device_error", "pa_status_str", "pa_version",
            "pa_decode_static_scratch", "pa_decode_append", "pa_swap_blocks", "pa_prefill",
@@ -28,6 +29,9 @@ EXPORTS = ("pa_kv_write", "pa_copy_blocks", "pa_decode", "pa_decode_workspace_by
            "pa_bm_num_free_cpu_blocks", "pa_bm_is_swapped", "pa_bm_swap_out", "pa_bm_swap_in",
            "pa_bm_set_sliding_window")
 STATIC_SCRATCH_BYTES = 16 << 20  # PA_STATIC_SCRATCH_BYTES in include/pa.h
+PARTITION_BALANCED = -1  # PA_PARTITION_BALANCED
+PARTITION_DYNAMIC = -2  # PA_PARTITION_DYNAMIC
+WORKSPACE_ZERO_BYTES = 8192  # PA_WORKSPACE_ZERO_BYTES
 
 _lib = None
 
@@ -275,12 +279,13 @@ def _decode_shapes(what, out, q, k_cache, v_cache, block_tables, context_lens, b
 
 def _workspace(what, workspace, need, dev):
     """(pointer, bytes) of the split-K workspace; allocated with torch when the plan needs
-    one and the caller gave none."""
+    one and the caller gave none (zero-filled: the dynamic split keeps its claim counters
+    in the first WORKSPACE_ZERO_BYTES, which must start at zero)."""
     import torch
     if workspace is None:
         if not need:
             return None, 0
-        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+        workspace = torch.zeros(need, dtype=torch.uint8, device=dev)
     if not (workspace.device == dev and workspace.is_contiguous()):
         _fail(what, f"workspace must be a contiguous tensor on {dev}")
     return _ptr(workspace), workspace.numel() * workspace.element_size()

@@ -13,6 +13,7 @@
 #include "pa_decode.cuh"
 #include "pa_merge.cuh"
 #include "pa_decode_streamk.cuh"
+#include "pa_decode_dynamic.cuh"
 #include "pa_prefill.cuh"
 
 using namespace pa;
@@ -88,13 +89,16 @@ bool make_q_map(CUtensorMap *m, const void *base, int num_tokens, int Hq, int D,
 
 struct Plan {
     bool streamk = false;   // balanced split over persistent warps
-    int grid = 0;           // stream-K CTAs
+    bool dynamic = false;   // dynamic split over persistent CTAs
+    int grid = 0;           // stream-K / dynamic CTAs
     int partition_tokens = 0;
     int num_parts = 1;
     size_t ws_bytes = 0;
     size_t off_m = 0, off_l = 0, off_pre = 0;
     size_t off_co = 0, off_cm = 0, off_cl = 0;  // balanced split: CTA-level records
+    size_t off_us = 0, off_ro = 0, off_rm = 0, off_rl = 0;  // dynamic split
 };
+
 
 constexpr int kSmPerSmBytes = 233472;  // shared memory per SM usable by CTAs (228 KiB)
 
@@ -145,6 +149,22 @@ Plan make_plan(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, in
     const bool fits32 = (long long)num_seqs * ((cap + kTile - 1) / kTile) < (1LL << 31);
     const bool balanced_ok = num_seqs <= max_seqs && fits32;
     const bool want_balanced = partition_size == PA_PARTITION_BALANCED;
+    const long long units = (long long)num_seqs * num_kv_heads;
+    const int dyn_grid = sms * kDynCtasPerSm;
+    if (partition_size == PA_PARTITION_DYNAMIC && units >= 1 && units <= dyn_grid &&
+        units <= kDynMaxUnits && fits32) {
+        pl.dynamic = true;
+        pl.grid = dyn_grid;
+        const size_t recs = (size_t)dyn_grid * G;
+        pl.off_us = kDynCounterBytes;
+        pl.off_ro = pl.off_us + round_up(((size_t)units + 1) * sizeof(int32_t), 256);
+        pl.off_rm = pl.off_ro + round_up(recs * head_dim * sizeof(float), 256);
+        pl.off_rl = pl.off_rm + round_up(recs * sizeof(float), 256);
+        pl.ws_bytes = pl.off_rl + round_up(recs * sizeof(float), 256);
+        pl.partition_tokens = 0;
+        pl.num_parts = 0;
+        return pl;
+    }
     if (want_balanced && balanced_ok) {
         pl.streamk = true;
         const int per_sm = head_dim == 64 ? streamk_ctas_per_sm<64>() : streamk_ctas_per_sm<128>();
@@ -320,6 +340,57 @@ cudaError_t sk_merge(const SkMergeParams &p, dim3 grid, int D, cudaStream_t st) 
                                 p);
 }
 
+template <typename T, int D, int G, int BOXR>
+cudaError_t launch_dynamic(const DynParams &p, int grid, cudaStream_t st, int dev) {
+    static std::atomic<bool> flags[kMaxDevices];
+    static std::atomic<int> occ[kMaxDevices];
+    auto kernel = pa_decode_dynamic_kernel<T, D, G, BOXR>;
+    cudaError_t e = ensure_smem(kernel, Geom<D>::kSmem, flags, dev);
+    if (e != cudaSuccess) return e;
+    int n = occ[dev].load(std::memory_order_relaxed);
+    if (n == 0) {
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, kWarps * 32,
+                                                          Geom<D>::kSmem);
+        if (e != cudaSuccess) return e;
+        occ[dev].store(n, std::memory_order_relaxed);
+    }
+    // the plan gives every warp two chunks of its own: all CTAs must be resident at once
+    if (n < kDynCtasPerSm) return cudaErrorInvalidConfiguration;
+    return launch_pdl(kernel, dim3(grid), dim3(kWarps * 32), Geom<D>::kSmem, st, p);
+}
+
+template <typename T, int D, int G>
+cudaError_t dyn_dispatch_boxr(const DynParams &p, int grid, cudaStream_t st, int dev, int boxr) {
+    return boxr == 8 ? launch_dynamic<T, D, G, 8>(p, grid, st, dev)
+                     : launch_dynamic<T, D, G, 16>(p, grid, st, dev);
+}
+
+template <typename T, int D>
+cudaError_t dyn_dispatch_group(const DynParams &p, int grid, cudaStream_t st, int dev, int G,
+                               int boxr) {
+    switch (G) {
+        case 1: return dyn_dispatch_boxr<T, D, 1>(p, grid, st, dev, boxr);
+        case 2: return dyn_dispatch_boxr<T, D, 2>(p, grid, st, dev, boxr);
+        case 4: return dyn_dispatch_boxr<T, D, 4>(p, grid, st, dev, boxr);
+        case 8: return dyn_dispatch_boxr<T, D, 8>(p, grid, st, dev, boxr);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+template <typename T>
+cudaError_t dyn_dispatch(const DynParams &p, int grid, cudaStream_t st, int dev, int D, int G,
+                         int boxr) {
+    return D == 64 ? dyn_dispatch_group<T, 64>(p, grid, st, dev, G, boxr)
+                   : dyn_dispatch_group<T, 128>(p, grid, st, dev, G, boxr);
+}
+
+template <typename T>
+cudaError_t dyn_merge(const DynMergeParams &p, dim3 grid, int D, cudaStream_t st) {
+    return D == 64 ? launch_pdl(pa_merge_dynamic_kernel<T, 64>, grid, dim3(kMergeThreads), 0, st, p)
+                   : launch_pdl(pa_merge_dynamic_kernel<T, 128>, grid, dim3(kMergeThreads), 0, st,
+                                p);
+}
+
 template <typename T, int D, int G>
 cudaError_t launch_prefill(const PrefillParams &p, dim3 grid, cudaStream_t st, int dev) {
     static std::atomic<bool> flags[kMaxDevices];
@@ -353,7 +424,7 @@ pa_status check_decode_shape(int num_seqs, int num_q_heads, int num_kv_heads, in
                              int max_context_len, int sliding_window, int partition_size) {
     if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || num_blocks <= 0 ||
         max_blocks_per_seq <= 0 || max_context_len < 0 || sliding_window < 0 ||
-        partition_size < PA_PARTITION_BALANCED)
+        partition_size < PA_PARTITION_DYNAMIC)
         return PA_ERR_INVALID_ARG;
     if (num_q_heads % num_kv_heads != 0) return PA_ERR_INVALID_ARG;
     const int G = num_q_heads / num_kv_heads;
@@ -530,7 +601,7 @@ size_t pa_decode_workspace_bytes(int num_seqs, int num_q_heads, int num_kv_heads
                                  int block_size, int max_blocks_per_seq, int max_context_len,
                                  int sliding_window, int partition_size) {
     if (num_seqs <= 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 ||
-        block_size <= 0 || max_blocks_per_seq <= 0 || partition_size < PA_PARTITION_BALANCED ||
+        block_size <= 0 || max_blocks_per_seq <= 0 || partition_size < PA_PARTITION_DYNAMIC ||
         max_context_len < 0 || sliding_window < 0)
         return 0;
     return make_plan(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
@@ -543,7 +614,7 @@ int pa_decode_partition_tokens(int num_seqs, int num_q_heads, int num_kv_heads, 
                                int block_size, int max_blocks_per_seq, int max_context_len,
                                int sliding_window, int partition_size) {
     if (num_kv_heads <= 0 || block_size <= 0 || max_blocks_per_seq <= 0 ||
-        partition_size < PA_PARTITION_BALANCED || max_context_len < 0 || sliding_window < 0)
+        partition_size < PA_PARTITION_DYNAMIC || max_context_len < 0 || sliding_window < 0)
         return 0;
     return make_plan(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
                      max_blocks_per_seq, max_context_len, sliding_window, partition_size,
@@ -635,6 +706,61 @@ pa_status decode_impl(void *out, const void *q, const void *k_cache, const void 
         dim3 mgrid((unsigned)num_q_heads, (unsigned)num_seqs);
         e = dtype == PA_BF16 ? sk_merge<__nv_bfloat16>(mp, mgrid, head_dim, st_)
                              : sk_merge<__half>(mp, mgrid, head_dim, st_);
+        return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+    }
+
+    if (pl.dynamic) {
+        DynParams dp;
+        std::memset(&dp, 0, sizeof dp);
+        if (!make_cache_map(&dp.kmap, k_cache, rows, head_dim, dtype, boxr) ||
+            !make_cache_map(&dp.vmap, v_cache, rows, head_dim, dtype, boxr))
+            return PA_ERR_CUDA;
+        uint8_t *ws = static_cast<uint8_t *>(workspace);
+        dp.out = out;
+        dp.q = q;
+        dp.block_tables = block_tables;
+        dp.context_lens = context_lens;
+        dp.claim = reinterpret_cast<int32_t *>(ws);
+        dp.done = dp.claim + kDynMaxUnits;
+        dp.ustart = reinterpret_cast<int32_t *>(ws + pl.off_us);
+        dp.rec_o = reinterpret_cast<float *>(ws + pl.off_ro);
+        dp.rec_m = reinterpret_cast<float *>(ws + pl.off_rm);
+        dp.rec_l = reinterpret_cast<float *>(ws + pl.off_rl);
+        dp.num_seqs = num_seqs;
+        dp.num_q_heads = num_q_heads;
+        dp.num_kv_heads = num_kv_heads;
+        dp.block_size = block_size;
+        dp.bs_shift = ilog2_host(block_size);
+        dp.num_blocks = num_blocks;
+        dp.max_blocks_per_seq = max_blocks_per_seq;
+        dp.sliding_window = sliding_window;
+        dp.scale_log2 = scale * 1.4426950408889634f;
+        dp.new_k = new_k;
+        dp.new_v = new_v;
+        dp.new_k_stride = new_k_stride;
+        dp.new_v_stride = new_v_stride;
+        dp.k_cache = const_cast<void *>(k_cache);
+        dp.v_cache = const_cast<void *>(v_cache);
+        cudaError_t e = dtype == PA_BF16
+                            ? dyn_dispatch<__nv_bfloat16>(dp, pl.grid, st_, dev, head_dim, G, boxr)
+                            : dyn_dispatch<__half>(dp, pl.grid, st_, dev, head_dim, G, boxr);
+        if (e != cudaSuccess) return PA_ERR_CUDA;
+        DynMergeParams mp;
+        mp.out = out;
+        mp.context_lens = context_lens;
+        mp.claim = dp.claim;
+        mp.done = dp.done;
+        mp.ustart = dp.ustart;
+        mp.rec_o = dp.rec_o;
+        mp.rec_m = dp.rec_m;
+        mp.rec_l = dp.rec_l;
+        mp.num_q_heads = num_q_heads;
+        mp.num_kv_heads = num_kv_heads;
+        mp.cap = max_blocks_per_seq * block_size;
+        mp.sliding_window = sliding_window;
+        dim3 mgrid((unsigned)num_q_heads, (unsigned)num_seqs);
+        e = dtype == PA_BF16 ? dyn_merge<__nv_bfloat16>(mp, mgrid, head_dim, st_)
+                             : dyn_merge<__half>(mp, mgrid, head_dim, st_);
         return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
     }
 

@@ -66,10 +66,13 @@ class DeviceCase:
         mcl = c.max_context_len if max_context_len is None else max_context_len
         if workspace is None:
             # all-ones bytes = NaN floats: nothing may be read that this call did not write
+            # (except the dynamic split's counters, which must start at zero)
             need = pa.decode_workspace_bytes(c.num_seqs, c.num_q_heads, c.num_kv_heads,
                                              c.head_dim, c.block_size, c.max_blocks_per_seq,
                                              mcl, partition_size, sliding_window)
             workspace = torch.full((max(need, 256),), 255, dtype=torch.uint8, device=self.q.device)
+            if partition_size == pa.PARTITION_DYNAMIC:
+                workspace[:pa.WORKSPACE_ZERO_BYTES] = 0
         pa.decode(self.out, self.q, self.k_cache, self.v_cache, self.block_tables,
                   self.context_lens, c.scale, max_context_len=mcl,
                   partition_size=partition_size, workspace=workspace,

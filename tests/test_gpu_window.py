@@ -77,7 +77,7 @@ def test_window_every_kernel_variant(dtype, G, d, bs):
     lens = [1, 15, 16, 17, 40, 63, 64, 65, 130, 333, 700]
     for window in (1, 9, 16, 17, 100, 333):
         case = _case(11 + window, dtype, hkv * G, hkv, d, bs, lens, window)
-        for ps in (-1, 0, 64, 192):
+        for ps in (-2, -1, 0, 64, 192):
             _check(case, window, ps)
 
 
@@ -130,7 +130,7 @@ def test_window_long_contexts(window):
     few thousand tokens: only the window's pages are read, in every split; every
     output compared."""
     case = _recycle(make_config("long_32_8", block_size=16, num_seqs=4), window)
-    for ps in (-1, 0, 512):
+    for ps in (-2, -1, 0, 512):
         _check(case, window, ps)
 
 

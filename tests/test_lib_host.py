@@ -72,6 +72,17 @@ def test_workspace_plan(lib):
     assert pa.decode_workspace_bytes(B, hq, hkv, d, bs, W, 2011, -1) >= 2 * warps * (d + 2) * 4
     assert pa.decode_partition_tokens(8, 8, 1, d, bs, 8192, 131072, 512) == 512
     assert pa.decode_workspace_bytes(B, hq, hkv, d, bs, W, 0, 128) >= B * hq * 16 * (d + 2) * 4
+    # dynamic split: the counters (zeroed by the caller once), the units' first CTAs and
+    # one record per resident CTA (148 SMs x 3), independent of the lengths
+    ctas = 148 * 3
+    assert pa.decode_partition_tokens(8, 8, 1, d, bs, 8192, 131072, -2) == 0
+    need = pa.decode_workspace_bytes(8, 8, 1, d, bs, 8192, 131072, -2)
+    assert need % 256 == 0 and need >= pa.WORKSPACE_ZERO_BYTES + ctas * 8 * (d + 2) * 4
+    assert need == pa.decode_workspace_bytes(8, 8, 1, d, bs, 8192, 0, -2)
+    # ... and more units than resident CTAs fall back to the fixed split
+    assert pa.decode_partition_tokens(B, hq, hkv, d, bs, W, 2011, -2) == 1024
+    assert pa.decode_workspace_bytes(B, hq, hkv, d, bs, W, 2011, -2) == pa.decode_workspace_bytes(
+        B, hq, hkv, d, bs, W, 2011)
     # sliding window: the tiles of a context span at most W + 15 tokens, whatever L is
     assert pa.decode_partition_tokens(8, 8, 1, d, bs, 8192, 131072, 0, 1000) == 1024
     assert pa.decode_workspace_bytes(8, 8, 1, d, bs, 8192, 131072, 0, 1000) == 0
@@ -99,7 +110,8 @@ def _call_decode(lib, a):
     (dict(d=96), 2), (dict(hq=6), 2), (dict(hq=7), 1), (dict(bs=24), 2), (dict(bs=4), 2),
     (dict(bs=1024), 2), (dict(q=0), 1), (dict(q=24), 1), (dict(out=8), 1), (dict(ps=100), 1),
     (dict(scale=float("inf")), 1), (dict(dt=5), 1), (dict(nb=0), 1), (dict(W=0), 1),
-    (dict(ps=-2), 1), (dict(ps=-1), 1),  # balanced split needs a workspace
+    (dict(ps=-2), 1), (dict(ps=-1), 1),  # balanced and dynamic splits need a workspace
+    (dict(ps=-3), 1),
     (dict(mcl=-1), 1), (dict(B=-1), 1), (dict(hkv=0), 1), (dict(win=-1), 1),
     (dict(ps=64, W=100), 1),  # needs a workspace, none given
 ])
