@@ -375,13 +375,13 @@ class DecodeStep:
         self.decode(b)
 
 
-def time_groups(torch, fn, stream, est_ms):
+def time_groups(torch, fn, stream, est_ms, min_s=ROOF_MIN_S):
     """Per-call device time of `fn`: CUDA events on the launching stream around groups of
     ROOF_GROUP consecutive calls (an event between every two launches would stop each
     kernel from being scheduled while the previous one drains), for at least
-    ROOF_MIN_GROUPS groups and ROOF_MIN_S seconds.  Returns (median ms per call over the
+    ROOF_MIN_GROUPS groups and `min_s` seconds.  Returns (median ms per call over the
     groups, number of calls)."""
-    n = max(ROOF_MIN_GROUPS, int(math.ceil(ROOF_MIN_S * 1e3 / (ROOF_GROUP * max(est_ms, 1e-3)))))
+    n = max(ROOF_MIN_GROUPS, int(math.ceil(min_s * 1e3 / (ROOF_GROUP * max(est_ms, 1e-3)))))
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(n)]
     for i in range(n):
         ev[i][0].record(stream)
@@ -440,7 +440,7 @@ def measure_config(torch, pa, name, device, stream, args, peak, flush):
     ds.decode()
     torch.cuda.synchronize()
     est = (time.perf_counter() - t) * 1e3
-    ms, ncalls = time_groups(torch, ds.decode, stream, est)
+    ms, ncalls = time_groups(torch, ds.decode, stream, est, args.roofline_s)
     clocks = sampler.stop()
     ms_flushed = time_flushed(torch, ds.decode, stream, flush)
     err = pa.device_error(device.index)
@@ -518,7 +518,8 @@ def run_ours(args):
     roof_sampler = ClockSampler(torch.cuda.current_device())
     roof_sampler.start()
     time.sleep(0.2)
-    dec_ms, roof_calls = time_groups(torch, ds.decode, stream, elapsed_ms / max(args.steps, 1))
+    dec_ms, roof_calls = time_groups(torch, ds.decode, stream, elapsed_ms / max(args.steps, 1),
+                                     args.roofline_s)
     roof_clocks = roof_sampler.stop()
     flush = L2Flush(torch, device)
     dec_ms_flushed = time_flushed(torch, ds.decode, stream, flush)
@@ -605,7 +606,10 @@ def run_ours(args):
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1)
-    torch.testing.assert_close(h_outs[(e2e_steps - 1) % 2], out.cpu(), rtol=0, atol=0)
+    # the end-to-end loop computes the same step: bit for bit under a fixed split; the
+    # dynamic split's sums vary in the last bits from call to call
+    torch.testing.assert_close(h_outs[(e2e_steps - 1) % 2].float(), out.cpu().float(), rtol=0,
+                               atol=0 if args.partition_size != -2 else 1e-3)
 
     # ---- aggregate over ranks
     max_ms = max_over_ranks(elapsed_ms, ws, device)
@@ -677,7 +681,7 @@ def run_ours(args):
                                     "pa_decode (partition pass + LSE merge when split)"),
                          "achieved_how": (f"algorithmic bytes / median per-call CUDA-event time "
                                           f"over groups of {ROOF_GROUP} consecutive calls "
-                                          f"({roof_calls} calls, >= {ROOF_MIN_S} s, a pass of "
+                                          f"({roof_calls} calls, >= {args.roofline_s} s, a pass of "
                                           f"its own after the timed steps); frac_l2_flushed: "
                                           f"median of {FLUSH_CALLS} single calls, each after an "
                                           f"L2 flush"),
@@ -1198,6 +1202,9 @@ def main(argv=None):
                     help="profiling only: build the workload with this many sequences")
     ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--roofline-s", type=float, default=ROOF_MIN_S,
+                    help="minimum device seconds of each roofline pass (at least "
+                         f"{ROOF_MIN_GROUPS * ROOF_GROUP} calls either way)")
     ap.add_argument("--no-per-config", action="store_true",
                     help="skip timing the other Llama-shaped workloads after the headline one")
     ap.add_argument("--cpu-budget", type=float, default=10.0)
