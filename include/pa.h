@@ -188,9 +188,10 @@ pa_status pa_swap_blocks(void *dst_k_cache, void *dst_v_cache, const void *src_k
  *                   PA_WORKSPACE_ZERO_BYTES bytes hold counters: they must be
  *                   zero before the workspace's first such call (one cudaMemset after
  *                   allocating it), and every call leaves them zero (a call that finds
- *                   them otherwise sets PA_DEVERR_WORKSPACE).  No other split needs any
- *                   initialisation.  Calls that share a workspace must not overlap on
- *                   the GPU.
+ *                   them otherwise sets PA_DEVERR_WORKSPACE).  No split writes those
+ *                   bytes otherwise, so one workspace can serve calls with different
+ *                   splits, and no other split needs any initialisation.  Calls that
+ *                   share a workspace must not overlap on the GPU.
  * Launches 1 kernel (one partition per sequence) or 2 (partition pass + merge).
  */
 pa_status pa_decode(void *out, const void *q, const void *k_cache, const void *v_cache,
@@ -278,9 +279,11 @@ int pa_decode_partition_tokens(int num_seqs, int num_q_heads, int num_kv_heads, 
  *    that device again in the same process (pa_decode with a workspace is not
  *    affected).
  *  - Every call on a device shares the one array, and it keeps the last call's
- *    contents.  No part of it needs clearing (each call writes every partial result
- *    it reads), but calls that overlap on the GPU race on it: serialise them (one
- *    stream, or events between streams).
+ *    contents.  Its partial results need no clearing (each call writes every one it
+ *    reads); its first PA_WORKSPACE_ZERO_BYTES, the counters of PA_PARTITION_DYNAMIC,
+ *    are zero when the library loads and every call leaves them zero.  Calls that
+ *    overlap on the GPU race on the array: serialise them (one stream, or events
+ *    between streams).
  */
 #define PA_STATIC_SCRATCH_BYTES ((size_t)16 << 20) /* 16 MiB per GPU */
 

@@ -71,6 +71,7 @@ struct DecodeParams {
     int partition_tokens;
     int num_parts;
     int sliding_window;  // > 0: attend to the last sliding_window tokens only; 0: all
+    int rotate;          // != 0: each warp starts its tiles at a pseudo-random offset
     float scale_log2;
     // Cache write fused into the decode (pa_decode_append): the new token of sequence s
     // (key/value rows new_k + s * new_k_stride, heads contiguous) is stored at position
@@ -616,6 +617,20 @@ __global__ void __launch_bounds__(kWarps * 32)
     const int nt = qd + (warp < rm ? 1 : 0);
     const int tok_begin = t0 + wt0 * kTile;
     const int tok_end = min(tok_begin + nt * kTile, t1);
+    // With large pages every warp's range starts at the same offset of a page, and all
+    // warps would walk their pages in step; `rotate` starts each warp at its own offset
+    // and wraps around (the softmax is order-independent; the order is fixed per call
+    // shape, so results stay the same from call to call).
+    int rot = 0;
+    if (p.rotate && nt > 1) {
+        const unsigned hsh = ((unsigned)s * 2654435761u) ^ ((unsigned)g * 2246822519u) ^
+                             ((unsigned)part * 3266489917u) ^ ((unsigned)warp * 668265263u);
+        rot = (int)((hsh >> 8) % (unsigned)nt);
+    }
+    auto tile_tok = [&](int jt) {
+        const int j = jt + rot < nt ? jt + rot : jt + rot - nt;
+        return tok_begin + j * kTile;
+    };
 
     const uint32_t bars_all = base + Gm::kRing;
     const uint32_t ring = base + warp * kStages * Gm::kStage;
@@ -646,7 +661,7 @@ __global__ void __launch_bounds__(kWarps * 32)
 
     auto produce = [&](int jt) {
         const int stage = jt % kStages;
-        const int tok = tok_begin + jt * kTile;
+        const int tok = tile_tok(jt);
         const int nrows = min(kTile, tok_end - tok);
         const int row_lo = WIN ? max(0, wlo - tok) : 0;
         constexpr int kBoxes = kTile / BOXR;
@@ -707,7 +722,7 @@ __global__ void __launch_bounds__(kWarps * 32)
             failed = true;
             break;
         }
-        const int tok = tok_begin + jt * kTile;
+        const int tok = tile_tok(jt);
         const int nrows = ((okmask >> stage) & 1u) ? min(kTile, tok_end - tok) : 0;
         const uint32_t kd = ring + stage * Gm::kStage, vd = kd + Gm::kMat;
         wc.tile(kd, vd, WIN ? max(0, wlo - tok) : 0, nrows, p.scale_log2, lane);

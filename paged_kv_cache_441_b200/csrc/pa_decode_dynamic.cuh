@@ -69,6 +69,7 @@ struct DynParams {
     int num_blocks;
     int max_blocks_per_seq;
     int sliding_window;
+    int cta_stride;    // coprime with the grid: CTA b takes plan slot (b * cta_stride) % grid
     float scale_log2;
     // fused cache write (pa_decode_append): the warp that produces the tile holding
     // position L-1 stores the new token's K and V row there before that tile's copy
@@ -111,20 +112,26 @@ __global__ void __launch_bounds__(kWarps * 32, kDynCtasPerSm)
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int B = p.num_seqs, Hkv = p.num_kv_heads, Hq = p.num_q_heads;
-    const int U = B * Hkv, C = gridDim.x, c = blockIdx.x;
+    // plan slot of this CTA: consecutive slots (the CTAs of one unit) are spread over
+    // the grid, so no unit sits on one corner of the GPU's SMs
+    const int U = B * Hkv, C = gridDim.x;
+    const int c = (int)(((long long)blockIdx.x * p.cta_stride) % C);
     const int W = p.sliding_window;
     const int cap = p.max_blocks_per_seq << p.bs_shift;
 
-    // ---- 1. plan: tiles per sequence, exclusive prefix (block scan, aliasing the ring)
+    // ---- 1. plan: tiles per sequence, exclusive prefix (block scan, aliasing the ring);
+    // the lengths are kept beside it
     int *pre = reinterpret_cast<int *>(base_ptr);
+    int *lens_sm = pre + (B + 1);
     {
         constexpr int nthr = kWarps * 32;
         const int per = (B + nthr - 1) / nthr;
         const int s_lo = min(B, tid * per), s_hi = min(B, s_lo + per);
         int local = 0;
         for (int s = s_lo; s < s_hi; ++s) {
-            int L = __ldg(p.context_lens + s);
-            L = L < 0 ? 0 : (L > cap ? cap : L);
+            const int L0 = __ldg(p.context_lens + s);
+            lens_sm[s] = L0;
+            const int L = L0 < 0 ? 0 : (L0 > cap ? cap : L0);
             local += (L - span_begin(L, W) + kTile - 1) / kTile;
         }
         int incl = local;
@@ -140,7 +147,7 @@ __global__ void __launch_bounds__(kWarps * 32, kDynCtasPerSm)
         for (int w = 0; w < warp; ++w) off += wsum[w];
         int run = off + incl - local;
         for (int s = s_lo; s < s_hi; ++s) {
-            int L = __ldg(p.context_lens + s);
+            int L = lens_sm[s];
             L = L < 0 ? 0 : (L > cap ? cap : L);
             pre[s] = run;
             run += (L - span_begin(L, W) + kTile - 1) / kTile;
@@ -171,18 +178,13 @@ __global__ void __launch_bounds__(kWarps * 32, kDynCtasPerSm)
     const int u = unit_s;
     const int s = u / Hkv, g = u - s * Hkv;
     const int c0 = ustart(u), nctas = ustart(u + 1) - c0;
-    __syncthreads();  // pre[] (in the ring) is no longer read
+    int L = lens_sm[s];
+    __syncthreads();  // pre[] and the lengths (in the ring) are no longer read
 
-    int L = __ldg(p.context_lens + s);
     if (L < 0 || L > cap) {
         if (tid == 0 && c == c0) raise_error(PA_DEVERR_CONTEXT);
         L = L < 0 ? 0 : cap;
     }
-    const T *q_item = reinterpret_cast<const T *>(p.q) + ((size_t)s * Hq + (size_t)g * G) * D;
-    T *out = reinterpret_cast<T *>(p.out) + ((size_t)s * Hq + (size_t)g * G) * D;
-    WarpCompute<T, D, G> wc;
-    wc.init(q_item, lane);
-
     const int wlo = window_lo(L, W), span0 = span_begin(L, W);
     const int ntile = (L - span0 + kTile - 1) / kTile;
     const int nch = (ntile + kDynChunk - 1) / kDynChunk;
@@ -191,18 +193,9 @@ __global__ void __launch_bounds__(kWarps * 32, kDynCtasPerSm)
     const int32_t *table = p.block_tables + (size_t)s * p.max_blocks_per_seq;
     int *claim = p.claim + u;
 
-    const uint32_t bars_all = base + Gm::kRing;
-    const uint32_t ring = base + warp * kStages * Gm::kStage;
-    const uint32_t bars = bars_all + warp * kStages * 8;
-    if (tid == 0) {
-        tma_prefetch_desc(&p.kmap);
-        tma_prefetch_desc(&p.vmap);
-        for (int i = 0; i < kWarps * kStages; ++i) mbar_init(bars_all + 8 * i, 1);
-        fence_barrier_init();
-    }
-
     // ---- 2. chunk pipeline of this warp (all values warp-uniform except the per-lane
-    // table entries and lane 0's claim result)
+    // table entries and lane 0's claim result).  The table entries of the first two
+    // chunks and the first claim are in flight while q is read.
     auto chunk_pages = [&](int ch, int &pg_lo) -> int {
         const int t_lo = span0 + ch * (kDynChunk * kTile);
         const int t_hi = min(t_lo + kDynChunk * kTile, L);
@@ -225,6 +218,22 @@ __global__ void __launch_bounds__(kWarps * 32, kDynCtasPerSm)
         pending = true;
     }
     int nchunks = q0 < nch ? 1 : 0;  // chunks this warp has started
+
+    const T *q_item = reinterpret_cast<const T *>(p.q) + ((size_t)s * Hq + (size_t)g * G) * D;
+    T *out = reinterpret_cast<T *>(p.out) + ((size_t)s * Hq + (size_t)g * G) * D;
+    WarpCompute<T, D, G> wc;
+    wc.init(q_item, lane);
+
+    const uint32_t bars_all = base + Gm::kRing;
+    const uint32_t ring = base + warp * kStages * Gm::kStage;
+    const uint32_t bars = bars_all + warp * kStages * 8;
+    if (tid == 0) {
+        tma_prefetch_desc(&p.kmap);
+        tma_prefetch_desc(&p.vmap);
+        for (int i = 0; i < kWarps * kStages; ++i) mbar_init(bars_all + 8 * i, 1);
+        fence_barrier_init();
+    }
+
     auto advance = [&]() {         // q0 exhausted: move to q1, resolve the claim
         q0 = q1;
         if (q0 < nch) ++nchunks;
@@ -412,19 +421,14 @@ struct DynMergeParams {
     int sliding_window;
 };
 
-constexpr int kDynMergeFast = 16;  // records per warp in the one-round path
-
-// One CTA of kMergeThreads per (q head, sequence).  Up to kMergeThreads / 32 *
-// kDynMergeFast records: warp w loads records w, w + 8, ... (o as one float4 per lane,
-// m and l broadcast) all at once, the maximum is combined in shared memory, and the
-// weighted sums are added across warps.  More records: lse_merge_block.
+// One CTA of kMergeThreads per (q head, sequence): the unit's CTA records merged in one
+// round of loads (lse_merge_warps), or by lse_merge_block when there are more of them.
 template <typename T, int D>
 __global__ void __launch_bounds__(kMergeThreads)
     pa_merge_dynamic_kernel(const __grid_constant__ DynMergeParams p) {
     pdl_wait_and_release();
-    constexpr int kW = kMergeThreads / 32, kV = D / 32;
+    constexpr int kW = kMergeThreads / 32;
     const int h = blockIdx.x, s = blockIdx.y, tid = threadIdx.x;
-    const int lane = tid & 31, wid = tid >> 5;
     const int Hkv = p.num_kv_heads, G = p.num_q_heads / Hkv;
     const int g = h / G, hh = h - g * G, u = s * Hkv + g;
     const int c0 = p.ustart[u], n = p.ustart[u + 1] - c0;
@@ -441,75 +445,11 @@ __global__ void __launch_bounds__(kMergeThreads)
     }
     if (n <= 1) return;  // the unit's only CTA wrote the output
     T *out = reinterpret_cast<T *>(p.out) + ((size_t)s * p.num_q_heads + h) * D;
-    if (n > kW * kDynMergeFast) {
-        const float v = lse_merge_block<D>(
-            n, [&](int i) -> long long { return (long long)(c0 + i) * G + hh; }, p.rec_m,
-            p.rec_l, p.rec_o);
-        if (tid < D) out[tid] = Fmt<T>::from_float(v);
-        return;
-    }
-    __shared__ float red[kW];
-    __shared__ float den_s[kW];
-    __shared__ float part[kW][D];
-    float m[kDynMergeFast], l[kDynMergeFast];
-    float o[kDynMergeFast][kV];
-#pragma unroll
-    for (int i = 0; i < kDynMergeFast; ++i) {
-        const int j = wid + i * kW;
-        m[i] = -INFINITY;
-        l[i] = 0.f;
-#pragma unroll
-        for (int e = 0; e < kV; ++e) o[i][e] = 0.f;
-        if (j < n) {
-            const long long rec = (long long)(c0 + j) * G + hh;
-            m[i] = p.rec_m[rec];
-            l[i] = p.rec_l[rec];
-            const float *src = p.rec_o + rec * D + lane * kV;
-            if constexpr (kV == 4) {
-                const float4 v = *reinterpret_cast<const float4 *>(src);
-                o[i][0] = v.x;
-                o[i][1] = v.y;
-                o[i][2] = v.z;
-                o[i][3] = v.w;
-            } else {
-                const float2 v = *reinterpret_cast<const float2 *>(src);
-                o[i][0] = v.x;
-                o[i][1] = v.y;
-            }
-        }
-    }
-    float Mw = -INFINITY;
-#pragma unroll
-    for (int i = 0; i < kDynMergeFast; ++i) Mw = fmaxf(Mw, m[i]);
-    if (lane == 0) red[wid] = Mw;
-    __syncthreads();
-    float M = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < kW; ++w) M = fmaxf(M, red[w]);
-    float acc[kV], den = 0.f;
-#pragma unroll
-    for (int e = 0; e < kV; ++e) acc[e] = 0.f;
-#pragma unroll
-    for (int i = 0; i < kDynMergeFast; ++i) {
-        if (m[i] == -INFINITY) continue;  // a CTA that got no tile, or no record
-        const float w = l[i] * fast_exp2(m[i] - M);
-        den += w;
-#pragma unroll
-        for (int e = 0; e < kV; ++e) acc[e] = fmaf(w, o[i][e], acc[e]);
-    }
-#pragma unroll
-    for (int e = 0; e < kV; ++e) part[wid][lane * kV + e] = acc[e];
-    if (lane == 0) den_s[wid] = den;
-    __syncthreads();
-    if (tid < D) {
-        float num = 0.f, dsum = 0.f;
-#pragma unroll
-        for (int w = 0; w < kW; ++w) {
-            num += part[w][tid];
-            dsum += den_s[w];
-        }
-        out[tid] = Fmt<T>::from_float(dsum > 0.f ? num / dsum : 0.f);
-    }
+    const auto rec = [&](int i) -> long long { return (long long)(c0 + i) * G + hh; };
+    const float v = n <= kW * kMergeWarpRecs
+                        ? lse_merge_warps<D>(n, rec, p.rec_m, p.rec_l, p.rec_o)
+                        : lse_merge_block<D>(n, rec, p.rec_m, p.rec_l, p.rec_o);
+    if (tid < D) out[tid] = Fmt<T>::from_float(v);
 }
 
 }  // namespace pa

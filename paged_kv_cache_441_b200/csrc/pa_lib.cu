@@ -27,6 +27,9 @@ constexpr int kMaxDevices = 64;
 constexpr int kAutoSplitTokens = 1024;
 constexpr int kAutoSplitTokensFew = 2048;
 constexpr int kAutoSingleMax = 1280;
+// Pages of at least this many tokens: warps start their tiles at rotated offsets (measured
+// on the long-context workload at 512-token pages: 59.8 -> 58.5 us per step; no gain at 16).
+constexpr int kRotateMinBlock = 64;
 
 bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 bool pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
@@ -94,7 +97,9 @@ struct Plan {
     int partition_tokens = 0;
     int num_parts = 1;
     size_t ws_bytes = 0;
-    size_t off_m = 0, off_l = 0, off_pre = 0;
+    // every split leaves the first kDynCounterBytes (the dynamic split's counters) alone,
+    // so that one workspace can serve calls with different splits
+    size_t off_o = kDynCounterBytes, off_m = 0, off_l = 0, off_pre = 0;
     size_t off_co = 0, off_cm = 0, off_cl = 0;  // balanced split: CTA-level records
     size_t off_us = 0, off_ro = 0, off_rm = 0, off_rl = 0;  // dynamic split
 };
@@ -175,9 +180,9 @@ Plan make_plan(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, in
         const size_t v_bytes = round_up(recs * sizeof(float), 256);
         const size_t co_bytes = round_up(crecs * head_dim * sizeof(float), 256);
         const size_t cv_bytes = round_up(crecs * sizeof(float), 256);
-        pl.off_m = o_bytes;
-        pl.off_l = o_bytes + v_bytes;
-        pl.off_co = o_bytes + 2 * v_bytes;
+        pl.off_m = pl.off_o + o_bytes;
+        pl.off_l = pl.off_m + v_bytes;
+        pl.off_co = pl.off_l + v_bytes;
         pl.off_cm = pl.off_co + co_bytes;
         pl.off_cl = pl.off_cm + cv_bytes;
         pl.off_pre = pl.off_cl + cv_bytes;
@@ -200,11 +205,19 @@ Plan make_plan(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, in
         const size_t n = (size_t)num_seqs * num_q_heads * pl.num_parts;
         const size_t o_bytes = round_up(n * head_dim * sizeof(float), 256);
         const size_t v_bytes = round_up(n * sizeof(float), 256);
-        pl.off_m = o_bytes;
-        pl.off_l = o_bytes + v_bytes;
-        pl.ws_bytes = o_bytes + 2 * v_bytes;
+        pl.off_m = pl.off_o + o_bytes;
+        pl.off_l = pl.off_m + v_bytes;
+        pl.ws_bytes = pl.off_l + v_bytes;
     }
     return pl;
+}
+
+// A stride coprime with n (a prime that does not divide it), so that b -> b * stride % n
+// permutes [0, n) and scatters consecutive values.
+int coprime_stride(int n) {
+    for (int pr : {97, 101, 103, 107, 109, 113, 127, 131, 137, 139})
+        if (n % pr != 0 && pr < n) return pr;
+    return 1;
 }
 
 // Launch with programmatic stream serialisation (see pdl_wait_and_release).
@@ -670,7 +683,7 @@ pa_status decode_impl(void *out, const void *q, const void *k_cache, const void 
         sp.q = q;
         sp.block_tables = block_tables;
         sp.context_lens = context_lens;
-        sp.rec_o = reinterpret_cast<float *>(ws);
+        sp.rec_o = reinterpret_cast<float *>(ws + pl.off_o);
         sp.rec_m = reinterpret_cast<float *>(ws + pl.off_m);
         sp.rec_l = reinterpret_cast<float *>(ws + pl.off_l);
         sp.crec_o = reinterpret_cast<float *>(ws + pl.off_co);
@@ -734,6 +747,7 @@ pa_status decode_impl(void *out, const void *q, const void *k_cache, const void 
         dp.num_blocks = num_blocks;
         dp.max_blocks_per_seq = max_blocks_per_seq;
         dp.sliding_window = sliding_window;
+        dp.cta_stride = coprime_stride(pl.grid);
         dp.scale_log2 = scale * 1.4426950408889634f;
         dp.new_k = new_k;
         dp.new_v = new_v;
@@ -775,7 +789,7 @@ pa_status decode_impl(void *out, const void *q, const void *k_cache, const void 
     p.context_lens = context_lens;
     if (pl.ws_bytes > 0) {
         uint8_t *ws = static_cast<uint8_t *>(workspace);
-        p.ws_o = reinterpret_cast<float *>(ws);
+        p.ws_o = reinterpret_cast<float *>(ws + pl.off_o);
         p.ws_m = reinterpret_cast<float *>(ws + pl.off_m);
         p.ws_l = reinterpret_cast<float *>(ws + pl.off_l);
     }
@@ -788,6 +802,7 @@ pa_status decode_impl(void *out, const void *q, const void *k_cache, const void 
     p.partition_tokens = pl.partition_tokens;
     p.num_parts = pl.num_parts;
     p.sliding_window = sliding_window;
+    p.rotate = block_size >= kRotateMinBlock ? 1 : 0;
     p.scale_log2 = scale * 1.4426950408889634f;
     p.new_k = new_k;
     p.new_v = new_v;

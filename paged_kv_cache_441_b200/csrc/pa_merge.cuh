@@ -25,7 +25,6 @@ namespace pa {
 constexpr int kMergeThreads = 256;
 constexpr int kMergeChunk = 512;
 constexpr int kMergeFew = 8;  // up to this many partials: one load round per thread
-constexpr int kMergeMid = 64; // up to this many: one load round, partials split over groups
 
 template <int D, typename RecFn>
 __device__ __forceinline__ float lse_merge_block(int n, RecFn rec, const float *rm,
@@ -120,6 +119,82 @@ __device__ __forceinline__ float lse_merge_block(int n, RecFn rec, const float *
     return dsum > 0.f ? num / dsum : 0.f;
 }
 
+// Log-sum-exp merge of n <= (kMergeThreads / 32) * kMergeWarpRecs partials in one round of
+// loads: warp w takes partials w, w + 8, w + 16, ... -- o as D/32 floats per lane in one
+// vector load, m and l as broadcast loads -- all issued before any is used; the maximum is
+// combined through shared memory, then each warp's weighted sum, and the warps' sums.
+// rec(i) as in lse_merge_block; a partial whose m is -inf (nothing attended) gets no
+// weight, and whatever its o slot holds is not used.  Thread e (e < D) returns element e.
+constexpr int kMergeWarpRecs = 16;
+
+template <int D, typename RecFn>
+__device__ __forceinline__ float lse_merge_warps(int n, RecFn rec, const float *rm,
+                                                 const float *rl, const float *ro) {
+    constexpr int kW = kMergeThreads / 32, kV = D / 32;
+    __shared__ float red[kW];
+    __shared__ float den_s[kW];
+    __shared__ float part[kW][D];
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    float m[kMergeWarpRecs], l[kMergeWarpRecs];
+    float o[kMergeWarpRecs][kV];
+#pragma unroll
+    for (int i = 0; i < kMergeWarpRecs; ++i) {
+        const int j = wid + i * kW;
+        m[i] = -INFINITY;
+        l[i] = 0.f;
+#pragma unroll
+        for (int e = 0; e < kV; ++e) o[i][e] = 0.f;
+        if (j < n) {
+            const long long r = rec(j);
+            m[i] = rm[r];
+            l[i] = rl[r];
+            const float *src = ro + r * D + lane * kV;
+            if constexpr (kV == 4) {
+                const float4 v = *reinterpret_cast<const float4 *>(src);
+                o[i][0] = v.x;
+                o[i][1] = v.y;
+                o[i][2] = v.z;
+                o[i][3] = v.w;
+            } else {
+                const float2 v = *reinterpret_cast<const float2 *>(src);
+                o[i][0] = v.x;
+                o[i][1] = v.y;
+            }
+        }
+    }
+    float Mw = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < kMergeWarpRecs; ++i) Mw = fmaxf(Mw, m[i]);
+    if (lane == 0) red[wid] = Mw;
+    __syncthreads();
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kW; ++w) M = fmaxf(M, red[w]);
+    float acc[kV], den = 0.f;
+#pragma unroll
+    for (int e = 0; e < kV; ++e) acc[e] = 0.f;
+#pragma unroll
+    for (int i = 0; i < kMergeWarpRecs; ++i) {
+        if (m[i] == -INFINITY) continue;
+        const float w = l[i] * fast_exp2(m[i] - M);
+        den += w;
+#pragma unroll
+        for (int e = 0; e < kV; ++e) acc[e] = fmaf(w, o[i][e], acc[e]);
+    }
+#pragma unroll
+    for (int e = 0; e < kV; ++e) part[wid][lane * kV + e] = acc[e];
+    if (lane == 0) den_s[wid] = den;
+    __syncthreads();
+    if (tid >= D) return 0.f;
+    float num = 0.f, dsum = 0.f;
+#pragma unroll
+    for (int w = 0; w < kW; ++w) {
+        num += part[w][tid];
+        dsum += den_s[w];
+    }
+    return dsum > 0.f ? num / dsum : 0.f;
+}
+
 struct MergeParams {
     void *out;
     const int32_t *context_lens;
@@ -134,7 +209,7 @@ struct MergeParams {
 };
 
 // One CTA per (q head, sequence) with more than one partition.  WIDE: compiled with the
-// medium and block paths (more than kMergeFew partitions possible); the instance for at
+// warp and block paths (more than kMergeFew partitions possible); the instance for at
 // most kMergeFew keeps its register count, and so its occupancy, low.
 template <typename T, int D, bool WIDE>
 __global__ void __launch_bounds__(kMergeThreads) pa_merge_kernel(const __grid_constant__ MergeParams p) {
@@ -173,57 +248,15 @@ __global__ void __launch_bounds__(kMergeThreads) pa_merge_kernel(const __grid_co
         return;
     }
     if constexpr (!WIDE) return;
-    if (n <= kMergeMid) {
-        // medium: kMergeThreads / D groups of D threads; group g owns partials
-        // g*kPer .. g*kPer+kPer-1 and thread d of it element d: all its loads at once, then
-        // the groups' maxima and sums are combined in shared memory
-        constexpr int kGroups = kMergeThreads / D, kPer = kMergeMid / kGroups;
-        __shared__ float gmax[kGroups], gden[kGroups];
-        __shared__ float gnum[kGroups][D];
-        const int d = threadIdx.x % D, grp = threadIdx.x / D;
-        float m[kPer], l[kPer], o[kPer];
-#pragma unroll
-        for (int i = 0; i < kPer; ++i) {
-            const int idx = grp * kPer + i;
-            const bool in = idx < n;
-            m[i] = in ? p.ws_m[base + idx] : -INFINITY;
-            l[i] = in ? p.ws_l[base + idx] : 0.f;
-            o[i] = in ? p.ws_o[(base + idx) * D + d] : 0.f;
-        }
-        float Mg = -INFINITY;
-#pragma unroll
-        for (int i = 0; i < kPer; ++i) Mg = fmaxf(Mg, m[i]);
-        if (d == 0) gmax[grp] = Mg;
-        __syncthreads();
-        float M = -INFINITY;
-#pragma unroll
-        for (int g2 = 0; g2 < kGroups; ++g2) M = fmaxf(M, gmax[g2]);
-        float num = 0.f, den = 0.f;
-#pragma unroll
-        for (int i = 0; i < kPer; ++i) {
-            if (m[i] == -INFINITY) continue;  // no record: its slot is not used
-            const float w = l[i] * fast_exp2(m[i] - M);
-            num = fmaf(w, o[i], num);
-            den += w;
-        }
-        gnum[grp][d] = num;
-        if (d == 0) gden[grp] = den;
-        __syncthreads();
-        if (grp == 0) {
-            float nt = 0.f, dt = 0.f;
-#pragma unroll
-            for (int g2 = 0; g2 < kGroups; ++g2) {
-                nt += gnum[g2][d];
-                dt += gden[g2];
-            }
-            T *out = reinterpret_cast<T *>(p.out) + ((size_t)s * p.num_q_heads + h) * D;
-            out[d] = Fmt<T>::from_float(dt > 0.f ? nt / dt : 0.f);
-        }
+    T *out = reinterpret_cast<T *>(p.out) + ((size_t)s * p.num_q_heads + h) * D;
+    if (n <= (kMergeThreads / 32) * kMergeWarpRecs) {
+        const float v = lse_merge_warps<D>(
+            n, [&](int i) -> long long { return base + i; }, p.ws_m, p.ws_l, p.ws_o);
+        if (threadIdx.x < D) out[threadIdx.x] = Fmt<T>::from_float(v);
         return;
     }
     const float v = lse_merge_block<D>(
         n, [&](int i) -> long long { return base + i; }, p.ws_m, p.ws_l, p.ws_o);
-    T *out = reinterpret_cast<T *>(p.out) + ((size_t)s * p.num_q_heads + h) * D;
     if (threadIdx.x < D) out[threadIdx.x] = Fmt<T>::from_float(v);
 }
 

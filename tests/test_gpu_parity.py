@@ -275,25 +275,28 @@ def test_decode_append_equals_write_then_decode(dtype, G, d, bs):
 # ------------------------------------------------------------------------ dynamic split
 
 def test_dynamic_split_reuses_its_workspace():
-    """Consecutive dynamic-split calls on one workspace: each leaves the counters at
-    zero for the next (no error bit) and each result is within the bar; a unit with
-    an empty context, units with one CTA and units with many in the same call."""
+    """Consecutive dynamic-split calls on one workspace, with fixed- and balanced-split
+    calls in between: each leaves the counters at zero for the next (no error bit) and
+    each result is within the bar; a unit with an empty context, units with one CTA and
+    units with many in the same call."""
     lens = [0, 1, 17, 5000, 40000, 300, 12000, 2]
     case = _rand_case(31, "bf16", len(lens), 16, 2, 128, 16, lens)
     dc = DeviceCase(case)
     dc.step(partition_size=-2)
     want, _, _ = oracle.step(case)
-    need = pa.decode_workspace_bytes(case.num_seqs, case.num_q_heads, case.num_kv_heads,
-                                     case.head_dim, case.block_size, case.max_blocks_per_seq,
-                                     case.max_context_len, -2)
+    need = max(pa.decode_workspace_bytes(case.num_seqs, case.num_q_heads, case.num_kv_heads,
+                                         case.head_dim, case.block_size,
+                                         case.max_blocks_per_seq, case.max_context_len, ps)
+               for ps in (-2, -1, 256))
     ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
-    for _ in range(3):
+    # the other splits share the workspace between dynamic calls and leave its counters be
+    for ps in (-2, 256, -2, -1, -2):
         dc.out.fill_(float("nan"))
-        dc.decode(partition_size=-2, workspace=ws)
+        dc.decode(partition_size=ps, workspace=ws)
         torch.cuda.synchronize()
-        assert np.max(np.abs(to_f64(dc.out) - want)) <= TOL["bf16"]
-        assert pa.device_error(0) == 0
-        assert torch.count_nonzero(ws[:pa.WORKSPACE_ZERO_BYTES]) == 0
+        assert np.max(np.abs(to_f64(dc.out) - want)) <= TOL["bf16"], ps
+        assert pa.device_error(0) == 0, ps
+        assert torch.count_nonzero(ws[:pa.WORKSPACE_ZERO_BYTES]) == 0, ps
 
 
 @pytest.mark.parametrize("fill", [0xFF, 0x01])

@@ -6,8 +6,10 @@ pa_decode a workspace.  This entry point keeps the split-K partials in the libra
 own fixed scratch array instead.  The test calls it through the C ABI several times
 in a row, on different inputs that all need several partitions, and checks each
 output bit for bit against pa_decode with a caller workspace (the same kernels on
-the same plan) and against the fp64 oracle within the bf16 bar; a later call must
-not be disturbed by what an earlier one left in the shared array.  It also checks
+the same plan; within the bf16 bar for the dynamic split, whose sums vary in the
+last bits) and against the fp64 oracle within the bf16 bar; a later call must not
+be disturbed by what an earlier one left in the shared array, and the dynamic
+split's counters, kept at its start, must read zero at each call.  It also checks
 that sizes over the fixed limit are refused before any launch, for the fixed and
 the balanced split.  This file sorts last so that a stop-at-first-
 failure run has run every other test before it.
@@ -52,7 +54,8 @@ def _c_static(case, t, out, partition_size):
 
 def test_static_scratch_matches_workspace_path_twice():
     runs = [(21, [3000, 17, 1290, 640, 2048], 128), (22, [700, 2500, 64, 1999], 256),
-            (24, [900, 0, 4100, 33], -1)]
+            (24, [900, 0, 4100, 33], -1), (26, [5000, 1, 2600, 700], -2),
+            (27, [3100, 64, 9000, 20], -2)]
     for seed, lens, ps in runs:
         case, t = _inputs(seed, lens)
         need = pa.decode_workspace_bytes(case.num_seqs, case.num_q_heads, case.num_kv_heads,
@@ -65,7 +68,12 @@ def test_static_scratch_matches_workspace_path_twice():
         pa.decode(want, t["q"], t["kc"], t["vc"], t["bt"], t["cl"], case.scale,
                   max_context_len=case.max_context_len, partition_size=ps)
         torch.cuda.synchronize()
-        assert np.array_equal(bits(got), bits(want)), seed
+        if ps == pa.PARTITION_DYNAMIC:
+            # the dynamic split's sums vary in the last bits from call to call; its
+            # counters live at the start of the scratch and each call leaves them zero
+            assert np.max(np.abs(to_f64(got) - to_f64(want))) <= TOL["bf16"], seed
+        else:
+            assert np.array_equal(bits(got), bits(want)), seed
         ref, _, _ = oracle.step(case)
         err = np.max(np.abs(to_f64(got) - ref))
         assert err <= TOL["bf16"], (seed, err)
