@@ -342,8 +342,10 @@ class DecodeStep:
         decode_launches = 1 if nparts == 1 else 2
         self.launches_per_step = decode_launches + (0 if self.fused else
                                                     1 + (1 if self.has_pairs else 0))
-        self.split = ("balanced over persistent warps (stream-K) + LSE merge" if ptoks == 0
-                      else f"fixed {ptoks}-token partitions, {nparts} max")
+        self.split = (f"fixed {ptoks}-token partitions, {nparts} max" if ptoks > 0 else
+                      "dynamic: persistent CTAs claim 32-token chunks + LSE merge"
+                      if partition_size == -2 else
+                      "balanced over persistent warps (stream-K) + LSE merge")
         self.kind = ("pa_decode_append (cache write fused into decode)" if self.fused
                      else "pa_copy_blocks + pa_kv_write + pa_decode" if self.has_pairs
                      else "pa_kv_write + pa_decode")
