@@ -50,8 +50,9 @@ constexpr int kPfRows = 128;        // query rows per tile = UMMA M = tensor-mem
 constexpr int kPfKeys = 64;         // keys per tile = UMMA N of S and K of P.V
 constexpr int kPfSoftWarps = 8;     // two softmax warpgroups
 constexpr int kPfMmaWarp = 8;       // warps 8 and 9: the products of query tiles A and B
-constexpr int kPfLoadWarp = 10;
-constexpr int kPfThreads = 352;
+constexpr int kPfLoadWarp = 10;     // TMA loads of Q and K (and the tensor-memory allocation)
+constexpr int kPfLoadWarpV = 11;    // TMA loads of V (and the zeroing of edge-tile V rows)
+constexpr int kPfThreads = 384;
 constexpr int kPfStages = 4;        // K/V ring depth
 // tensor memory of query tile X: two S/P buffers at [256X, 256X + 64) and [256X + 64,
 // 256X + 128) (key tile i of X uses buffer i % 2), O at [256X + 128, 256X + 128 + D)
@@ -94,8 +95,9 @@ struct PfGeom {
     static constexpr int kOffK = 2 * kQ;
     static constexpr int kOffV = kOffK + kPfStages * kKV;
     static constexpr int kOffBar = kOffV + kPfStages * kKV;
-    // q, k[stages], v[stages], v_edge[stages], empty[stages], s[2][2], p[2][2], o[2], fin[2]
-    static constexpr int kBars = 1 + 4 * kPfStages + 12;
+    // q, k[stages], v[stages], v_edge[stages], k_empty[stages], v_empty[stages], s[2][2],
+    // p[2][2], o[2], fin[2]
+    static constexpr int kBars = 1 + 5 * kPfStages + 12;
     static constexpr int kSmem = kOffBar + 8 * kBars + 1024;  // + alignment slack
 };
 
@@ -337,10 +339,13 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     const uint32_t bar_q = base + Gm::kOffBar;
     const uint32_t bar_k0 = bar_q + 8, bar_v0 = bar_k0 + 8 * kPfStages;
     const uint32_t bar_vt0 = bar_v0 + 8 * kPfStages;     // V of an edge tile landed (producer)
-    const uint32_t bar_e0 = bar_vt0 + 8 * kPfStages;     // stage empty (both MMA warps)
+    // a stage's K and its V are released separately (both MMA warps commit each): K once
+    // the S product that reads it has finished, V once the P V product has
+    const uint32_t bar_ek0 = bar_vt0 + 8 * kPfStages;
+    const uint32_t bar_ev0 = bar_ek0 + 8 * kPfStages;
     // per query tile X = 0 (A), 1 (B) and S/P buffer b: S ready, P written (one barrier
     // per buffer, so that neither side can get two phases ahead of the other)
-    const uint32_t bar_s0 = bar_e0 + 8 * kPfStages;      // + 8 (2X + b)
+    const uint32_t bar_s0 = bar_ev0 + 8 * kPfStages;     // + 8 (2X + b)
     const uint32_t bar_p0 = bar_s0 + 32;                 // + 8 (2X + b)
     const uint32_t bar_o0 = bar_p0 + 32;                 // + 8X: P_X V done
     const uint32_t bar_f0 = bar_o0 + 16;                 // + 8X: every product of X done
@@ -353,7 +358,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             mbar_init(bar_k0 + 8 * i, 1);
             mbar_init(bar_v0 + 8 * i, 1);
             mbar_init(bar_vt0 + 8 * i, 1);
-            mbar_init(bar_e0 + 8 * i, 2);  // one commit per MMA warp
+            mbar_init(bar_ek0 + 8 * i, 2);  // one commit per MMA warp
+            mbar_init(bar_ev0 + 8 * i, 2);
         }
         for (int i = 0; i < 4; ++i) {
             mbar_init(bar_s0 + 8 * i, 1);
@@ -377,12 +383,16 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     tc_fence_after();
     const uint32_t tmem = sh_tmem;
 
-    if (warp == kPfLoadWarp) {
-        // ============================ TMA producer (lane 0 issues; the warp zeroes edge V)
+    if (warp == kPfLoadWarp || warp == kPfLoadWarpV) {
+        // ============================ TMA producers (lane 0 issues): warp 10 loads Q and
+        // the K ring, warp 11 the V ring and zeroes edge V rows.  Each ring stage is reused
+        // once both MMA warps have released it: K after its S product, V after its P V, so
+        // the K loads run ahead of the V loads by the two key tiles S is computed ahead.
+        const bool is_k = warp == kPfLoadWarp;
         const int32_t *table = p.block_tables + (size_t)s * p.max_blocks_per_seq;
         const int BR = p.box_rows;
         const uint64_t pol = l2_policy_evict_first();
-        if (lane == 0) {
+        if (is_k && lane == 0) {
             mbar_arrive_expect_tx(bar_q, (uint32_t)((tb.live ? 2 : 1) * Gm::kQ));
 #pragma unroll
             for (int hf = 0; hf < Gm::kHalves; ++hf) {
@@ -392,6 +402,9 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                                 q0 + tb.tok0);
             }
         }
+        const uint32_t bar_empty0 = is_k ? bar_ek0 : bar_ev0;
+        const uint32_t sbase = is_k ? sk : sv;
+        const CUtensorMap *map = is_k ? &p.kmap : &p.vmap;
         int issued = j0;
         int vt_uses[kPfStages];
 #pragma unroll
@@ -401,7 +414,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             const int it = jt - j0, st = it % kPfStages;
             if (it >= kPfStages) {
                 ok = __all_sync(0xffffffffu, mbar_wait_bounded(
-                                                 bar_e0 + 8 * st,
+                                                 bar_empty0 + 8 * st,
                                                  (uint32_t)(((it / kPfStages) - 1) & 1)));
                 if (!ok) break;
             }
@@ -424,13 +437,13 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             // an edge tile (keys outside [kv_begin, L), or a bad table entry): its V lands
             // on a private barrier, the rows outside the attended keys are zeroed, then V
             // is released
-            const bool edge = !tab_ok || kv0 < kv_begin || kv0 + kPfKeys > L;
+            const bool edge = !is_k && (!tab_ok || kv0 < kv_begin || kv0 + kPfKeys > L);
             const uint32_t bk = bar_k0 + 8 * st, bv = bar_v0 + 8 * st, bvt = bar_vt0 + 8 * st;
+            const uint32_t bar = is_k ? bk : (edge ? bvt : bv);
             const uint32_t bytes = (uint32_t)(nload * BR * 128 * Gm::kHalves);
             if (lane == 0) {
-                if (!tab_ok) raise_error(PA_DEVERR_BLOCK_ID);
-                mbar_arrive_expect_tx(bk, bytes);
-                mbar_arrive_expect_tx(edge ? bvt : bv, bytes);
+                if (!tab_ok && is_k) raise_error(PA_DEVERR_BLOCK_ID);
+                mbar_arrive_expect_tx(bar, bytes);
                 if (tab_ok) {
                     for (int b = 0; b < kPfKeys / BR; ++b) {
                         const int r0 = kv0 + b * BR;
@@ -441,9 +454,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
 #pragma unroll
                             for (int hf = 0; hf < Gm::kHalves; ++hf) {
                                 const uint32_t off = hf * Gm::kKVRegion + b * BR * 128;
-                                tma_load_2d(sk + st * Gm::kKV + off, &p.kmap, bk, 64 * hf, y, pol);
-                                tma_load_2d(sv + st * Gm::kKV + off, &p.vmap, edge ? bvt : bv,
-                                            64 * hf, y, pol);
+                                tma_load_2d(sbase + st * Gm::kKV + off, map, bar, 64 * hf, y, pol);
                             }
                         }
                     }
@@ -476,14 +487,13 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             if (lane == 0) raise_error(PA_DEVERR_TIMEOUT);
             sh_fail = 1;
         }
-        // cleanup: the loads this CTA issued have landed (bounded)
+        // cleanup: the loads this warp issued have landed (bounded)
         if (lane == 0) {
-            (void)mbar_wait_bounded(bar_q, 0);
+            if (is_k) (void)mbar_wait_bounded(bar_q, 0);
             for (int jt = max(j0, issued - kPfStages); jt < issued; ++jt) {
                 const int it = jt - j0, st = it % kPfStages;
                 const uint32_t ph = (uint32_t)((it / kPfStages) & 1);
-                (void)mbar_wait_bounded(bar_k0 + 8 * st, ph);
-                (void)mbar_wait_bounded(bar_v0 + 8 * st, ph);
+                (void)mbar_wait_bounded((is_k ? bar_k0 : bar_v0) + 8 * st, ph);
             }
         }
         __syncwarp();
@@ -540,12 +550,16 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             __syncwarp();
         };
         bool ok = wait_all(bar_q, 0);
-        int npv = 0;
-        // S of the first two key tiles
+        // S of the first two key tiles; each tile's K is released (by both MMA warps,
+        // whether or not this one needs it) once the products issued so far are done.
+        // Every warp waits each K before releasing it, so that neither releases a stage a
+        // ring's length ahead of the loads.
         for (int jn = j0; ok && jn < min(j1, j0 + 2); ++jn) {
-            if (!need(jn)) continue;
             ok = wait_all(bar_k0 + 8 * stage_of(jn), phase_of(jn));
-            if (ok) issue_s(jn);
+            if (!ok) break;
+            if (need(jn)) issue_s(jn);
+            if (lane == 0) umma_commit(bar_ek0 + 8 * stage_of(jn));
+            __syncwarp();
         }
         for (int jt = j0; ok && jt < j1; ++jt) {
             if (__any_sync(0xffffffffu, sh_fail != 0)) {
@@ -562,22 +576,20 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                 ok = wait_all(bar_p0 + 8 * (2 * x + (i & 1)), (uint32_t)((i >> 1) & 1));
                 if (!ok) break;
                 issue_pv(jt);
-                ++npv;
             }
-            // S two key tiles ahead, into the buffer this tile's P V reads: after that
-            // P V has finished
+            if (lane == 0) umma_commit(bar_ev0 + 8 * st);  // V of stage st, after this P V
+            __syncwarp();
+            // S two key tiles ahead, into the buffer this tile's P V reads.  No wait for
+            // that P V: the products one thread issues run in issue order, so the P V has
+            // read P before the S product that follows it writes the buffer.
             const int jn = jt + 2;
-            if (jn < j1 && need(jn)) {
-                if (need(jt)) {
-                    ok = wait_all(bar_o0 + 8 * x, (uint32_t)((npv - 1) & 1));
-                    if (!ok) break;
-                }
+            if (jn < j1) {
                 ok = wait_all(bar_k0 + 8 * stage_of(jn), phase_of(jn));
                 if (!ok) break;
-                issue_s(jn);
+                if (need(jn)) issue_s(jn);
+                if (lane == 0) umma_commit(bar_ek0 + 8 * stage_of(jn));  // K of that stage
+                __syncwarp();
             }
-            if (lane == 0) umma_commit(bar_e0 + 8 * st);  // this warp's products on stage st
-            __syncwarp();
         }
         if (ok) {
             // completes when every product of this warp (its last P V included) is done
