@@ -409,6 +409,15 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         int vt_uses[kPfStages];
 #pragma unroll
         for (int i = 0; i < kPfStages; ++i) vt_uses[i] = 0;
+        // the table entries of a tile's boxes, one per lane (lane b: box b; the boxes of
+        // keys outside [kv_begin, L) read nothing), loaded one tile ahead of their use
+        const int nbox = kPfKeys / BR;
+        auto tab_load = [&](int jt) -> int {
+            const int r0 = jt * kPfKeys + lane * BR;
+            if (jt >= j1 || lane >= nbox || r0 >= L || r0 + BR <= kv_begin) return -1;
+            return __ldg(table + (r0 >> p.bs_shift));
+        };
+        int tab_next = tab_load(j0);
         bool ok = true;
         for (int jt = j0; jt < j1 && ok; ++jt) {
             const int it = jt - j0, st = it % kPfStages;
@@ -423,17 +432,21 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                 break;
             }
             const int kv0 = jt * kPfKeys;
-            int nload = 0;
-            bool tab_ok = true;
-            for (int b = 0; b < kPfKeys / BR; ++b) {
-                const int r0 = kv0 + b * BR;
-                if (r0 < L && r0 + BR > kv_begin) {
-                    ++nload;
-                    const int blk = __ldg(table + (r0 >> p.bs_shift));
-                    tab_ok = tab_ok && (unsigned)blk < (unsigned)p.num_blocks;
-                }
-            }
-            if (!tab_ok) nload = 0;  // nothing loaded: the tile reads as all-masked
+            const int tab_cur = tab_next;
+            tab_next = tab_load(jt + 1);
+            const int r0l = kv0 + lane * BR;
+            const bool live = lane < nbox && r0l < L && r0l + BR > kv_begin;
+            const unsigned live_mask = __ballot_sync(0xffffffffu, live);
+            const bool tab_ok =
+                !__any_sync(0xffffffffu, live && (unsigned)tab_cur >= (unsigned)p.num_blocks);
+            // nothing loaded after a bad entry: the tile reads as all-masked
+            const int nload = tab_ok ? __popc(live_mask) : 0;
+            const int y_l = live && tab_ok ? (tab_cur * p.num_kv_heads + g) * p.block_size +
+                                                 (r0l & (p.block_size - 1))
+                                           : 0;
+            int ys[kPfKeys / 8];  // box rows are at least 8
+#pragma unroll
+            for (int b = 0; b < kPfKeys / 8; ++b) ys[b] = __shfl_sync(0xffffffffu, y_l, b);
             // an edge tile (keys outside [kv_begin, L), or a bad table entry): its V lands
             // on a private barrier, the rows outside the attended keys are zeroed, then V
             // is released
@@ -445,16 +458,14 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                 if (!tab_ok && is_k) raise_error(PA_DEVERR_BLOCK_ID);
                 mbar_arrive_expect_tx(bar, bytes);
                 if (tab_ok) {
-                    for (int b = 0; b < kPfKeys / BR; ++b) {
-                        const int r0 = kv0 + b * BR;
-                        if (r0 < L && r0 + BR > kv_begin) {
-                            const int blk = __ldg(table + (r0 >> p.bs_shift));
-                            const int y = (blk * p.num_kv_heads + g) * p.block_size +
-                                          (r0 & (p.block_size - 1));
+#pragma unroll
+                    for (int b = 0; b < kPfKeys / 8; ++b) {
+                        if ((live_mask >> b) & 1u) {
 #pragma unroll
                             for (int hf = 0; hf < Gm::kHalves; ++hf) {
                                 const uint32_t off = hf * Gm::kKVRegion + b * BR * 128;
-                                tma_load_2d(sbase + st * Gm::kKV + off, map, bar, 64 * hf, y, pol);
+                                tma_load_2d(sbase + st * Gm::kKV + off, map, bar, 64 * hf, ys[b],
+                                            pol);
                             }
                         }
                     }
