@@ -49,10 +49,11 @@ namespace pa {
 constexpr int kPfRows = 128;        // query rows per tile = UMMA M = tensor-memory lanes
 constexpr int kPfKeys = 64;         // keys per tile = UMMA N of S and K of P.V
 constexpr int kPfSoftWarps = 8;     // two softmax warpgroups
-constexpr int kPfMmaWarp = 8;       // warps 8 and 9: the products of query tiles A and B
+constexpr int kPfMmaWarp = 8;       // warps 8 and 9: the P V products of query tiles A and B
 constexpr int kPfLoadWarp = 10;     // TMA loads of Q and K (and the tensor-memory allocation)
 constexpr int kPfLoadWarpV = 11;    // TMA loads of V (and the zeroing of edge-tile V rows)
-constexpr int kPfThreads = 384;
+constexpr int kPfSWarp = 12;        // warps 12 and 13: the S products of query tiles A and B
+constexpr int kPfThreads = 448;
 constexpr int kPfStages = 4;        // K/V ring depth
 // tensor memory of query tile X: two S/P buffers at [256X, 256X + 64) and [256X + 64,
 // 256X + 128) (key tile i of X uses buffer i % 2), O at [256X + 128, 256X + 128 + D)
@@ -96,8 +97,8 @@ struct PfGeom {
     static constexpr int kOffV = kOffK + kPfStages * kKV;
     static constexpr int kOffBar = kOffV + kPfStages * kKV;
     // q, k[stages], v[stages], v_edge[stages], k_empty[stages], v_empty[stages], s[2][2],
-    // p[2][2], o[2], fin[2]
-    static constexpr int kBars = 1 + 5 * kPfStages + 12;
+    // p[2][2], o[2], fin[2], pv_done[2][2], s_fin[2]
+    static constexpr int kBars = 1 + 5 * kPfStages + 18;
     static constexpr int kSmem = kOffBar + 8 * kBars + 1024;  // + alignment slack
 };
 
@@ -348,7 +349,11 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     const uint32_t bar_s0 = bar_ev0 + 8 * kPfStages;     // + 8 (2X + b)
     const uint32_t bar_p0 = bar_s0 + 32;                 // + 8 (2X + b)
     const uint32_t bar_o0 = bar_p0 + 32;                 // + 8X: P_X V done
-    const uint32_t bar_f0 = bar_o0 + 16;                 // + 8X: every product of X done
+    const uint32_t bar_f0 = bar_o0 + 16;                 // + 8X: every P V of X done
+    // per query tile X and buffer b: the P V that read the buffer's P has finished (the S
+    // warp may then overwrite it); one barrier per buffer, as for S and P
+    const uint32_t bar_pv0 = bar_f0 + 16;                // + 8 (2X + b)
+    const uint32_t bar_sf0 = bar_pv0 + 32;               // + 8X: every S product of X done
     if (tid == 0) {
         tma_prefetch_desc(&p.qmap);
         tma_prefetch_desc(&p.kmap);
@@ -368,7 +373,9 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         for (int x = 0; x < 2; ++x) {
             mbar_init(bar_o0 + 8 * x, 1);
             mbar_init(bar_f0 + 8 * x, 1);
+            mbar_init(bar_sf0 + 8 * x, 1);
         }
+        for (int i = 0; i < 4; ++i) mbar_init(bar_pv0 + 8 * i, 1);
         fence_barrier_init();
     }
     if (warp == kPfLoadWarp) {
@@ -509,8 +516,11 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         }
         __syncwarp();
     } else if (warp >= kPfMmaWarp) {
-        // ============================ products of query tile X (lane 0 issues)
-        const int x = warp - kPfMmaWarp;
+        // ============================ products of query tile X (lane 0 issues): warps 8
+        // and 9 the P V products, warps 12 and 13 the S products, so that the P V of a tile
+        // is issued as soon as its P is written, even while the S products queue
+        const bool s_role = warp >= kPfSWarp;
+        const int x = warp - (s_role ? kPfSWarp : kPfMmaWarp);
         const PfTile &t = x == 0 ? ta : tb;
         const uint32_t idesc_s = umma_idesc<T>(kPfRows, kPfKeys, false);
         const uint32_t idesc_o = umma_idesc<T>(kPfRows, D, true);
@@ -557,64 +567,83 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                                 idesc_o, (!first || kk > 0) ? 1u : 0u);
                 }
                 umma_commit(bar_o0 + 8 * x);
+                umma_commit(bar_pv0 + 8 * (2 * x + ((jt - t.j0) & 1)));
             }
             __syncwarp();
         };
-        bool ok = wait_all(bar_q, 0);
-        // S of the first two key tiles; each tile's K is released (by both MMA warps,
-        // whether or not this one needs it) once the products issued so far are done.
-        // Every warp waits each K before releasing it, so that neither releases a stage a
-        // ring's length ahead of the loads.
-        for (int jn = j0; ok && jn < min(j1, j0 + 2); ++jn) {
-            ok = wait_all(bar_k0 + 8 * stage_of(jn), phase_of(jn));
-            if (!ok) break;
-            if (need(jn)) issue_s(jn);
-            if (lane == 0) umma_commit(bar_ek0 + 8 * stage_of(jn));
-            __syncwarp();
-        }
-        for (int jt = j0; ok && jt < j1; ++jt) {
-            if (__any_sync(0xffffffffu, sh_fail != 0)) {
-                ok = false;
-                break;
-            }
-            const int st = stage_of(jt);
-            // every warp waits each tile's V, so that neither commits a stage's release
-            // a ring's length ahead of the loads
-            ok = wait_all(bar_v0 + 8 * st, phase_of(jt));
-            if (!ok) break;
-            if (need(jt)) {
-                const int i = jt - t.j0;
-                ok = wait_all(bar_p0 + 8 * (2 * x + (i & 1)), (uint32_t)((i >> 1) & 1));
-                if (!ok) break;
-                issue_pv(jt);
-            }
-            if (lane == 0) umma_commit(bar_ev0 + 8 * st);  // V of stage st, after this P V
-            __syncwarp();
-            // S two key tiles ahead, into the buffer this tile's P V reads.  No wait for
-            // that P V: the products one thread issues run in issue order, so the P V has
-            // read P before the S product that follows it writes the buffer.
-            const int jn = jt + 2;
-            if (jn < j1) {
+        if (s_role) {
+            // S of every key tile this query tile needs, two tiles ahead of its softmax:
+            // into buffer i % 2 once the P V that read that buffer (tile i - 2) is done.
+            // Each tile's K is released by both S warps (whether or not this one needs
+            // it) once the products issued so far are done; every S warp waits each K
+            // before releasing it, so that neither releases a stage a ring's length ahead
+            // of the loads.
+            bool ok = wait_all(bar_q, 0);
+            for (int jn = j0; ok && jn < j1; ++jn) {
+                if (__any_sync(0xffffffffu, sh_fail != 0)) {
+                    ok = false;
+                    break;
+                }
                 ok = wait_all(bar_k0 + 8 * stage_of(jn), phase_of(jn));
                 if (!ok) break;
-                if (need(jn)) issue_s(jn);
-                if (lane == 0) umma_commit(bar_ek0 + 8 * stage_of(jn));  // K of that stage
+                if (need(jn)) {
+                    const int i = jn - t.j0;
+                    if (i >= 2) {
+                        ok = wait_all(bar_pv0 + 8 * (2 * x + (i & 1)),
+                                      (uint32_t)(((i - 2) >> 1) & 1));
+                        if (!ok) break;
+                    }
+                    issue_s(jn);
+                }
+                if (lane == 0) umma_commit(bar_ek0 + 8 * stage_of(jn));
                 __syncwarp();
             }
-        }
-        if (ok) {
-            // completes when every product of this warp (its last P V included) is done
-            if (lane == 0 && t.live) umma_commit(bar_f0 + 8 * x);
-            __syncwarp();
-        } else {
-            if (lane == 0) raise_error(PA_DEVERR_TIMEOUT);
-            sh_fail = 1;
-            // cleanup: the products issued so far have finished (bounded)
+            if (!ok) {
+                if (lane == 0) raise_error(PA_DEVERR_TIMEOUT);
+                sh_fail = 1;
+            }
+            // the S products this warp issued have finished (bounded) before the tensor
+            // memory is freed
             if (lane == 0) {
-                umma_commit(bar_f0 + 8 * x);
-                (void)mbar_wait_bounded(bar_f0 + 8 * x, 0);
+                umma_commit(bar_sf0 + 8 * x);
+                (void)mbar_wait_bounded(bar_sf0 + 8 * x, 0);
             }
             __syncwarp();
+        } else {
+            bool ok = true;
+            for (int jt = j0; ok && jt < j1; ++jt) {
+                if (__any_sync(0xffffffffu, sh_fail != 0)) {
+                    ok = false;
+                    break;
+                }
+                const int st = stage_of(jt);
+                // every P V warp waits each tile's V, so that neither commits a stage's
+                // release a ring's length ahead of the loads
+                ok = wait_all(bar_v0 + 8 * st, phase_of(jt));
+                if (!ok) break;
+                if (need(jt)) {
+                    const int i = jt - t.j0;
+                    ok = wait_all(bar_p0 + 8 * (2 * x + (i & 1)), (uint32_t)((i >> 1) & 1));
+                    if (!ok) break;
+                    issue_pv(jt);
+                }
+                if (lane == 0) umma_commit(bar_ev0 + 8 * st);  // V of stage st, after this P V
+                __syncwarp();
+            }
+            if (ok) {
+                // completes when every P V of this query tile (its last included) is done
+                if (lane == 0 && t.live) umma_commit(bar_f0 + 8 * x);
+                __syncwarp();
+            } else {
+                if (lane == 0) raise_error(PA_DEVERR_TIMEOUT);
+                sh_fail = 1;
+                // cleanup: the products issued so far have finished (bounded)
+                if (lane == 0) {
+                    umma_commit(bar_f0 + 8 * x);
+                    (void)mbar_wait_bounded(bar_f0 + 8 * x, 0);
+                }
+                __syncwarp();
+            }
         }
     } else {
         // ============================ softmax warpgroup X (rows = threads 128X .. 128X+127)
