@@ -95,6 +95,22 @@ def copy_bytes(case) -> int:
 
 # ----------------------------------------------------------------------------- helpers
 
+def bf16_peaks():
+    """((burst TFLOP/s, kind), (sustained TFLOP/s, kind)): the measured cuBLAS bf16
+    rates, else the profiling recipe's figures for this pool (1.59 PFLOP/s burst, about
+    1.4 sustained under the 1 kW cap)."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            j = json.load(f)
+        burst = (float(j["bf16_tflops"]), "measured")
+    except Exception:
+        return (1590.0, "fallback"), (1400.0, "fallback")
+    try:
+        return burst, (float(j["bf16_tflops_sustained"]), "measured")
+    except Exception:
+        return burst, (1400.0, "fallback")
+
+
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -301,6 +317,8 @@ ROOF_MIN_GROUPS = 20   # at least 200 calls ...
 ROOF_MIN_S = 0.5       # ... and at least half a second of device time
 FLUSH_CALLS = 50       # L2-flushed pass: median of this many single calls
 FLUSH_BYTES = 256 << 20
+PF_BURSTS = 10         # prefill burst pass: bursts of 10 calls ...
+PF_BURST_IDLE_S = 0.05  # ... each after this idle pause (the clock recovers from the cap)
 
 
 class DecodeStep:
@@ -950,6 +968,20 @@ def run_prefill(args):
     torch.cuda.synchronize()
     clocks = sampler.stop()
     call_ms = sum(a.elapsed_time(b) for a, b in ev) / (ngroups * group)
+    # burst pass: the kernel timed alone at full clock -- bursts of 10 calls, each after
+    # an idle pause; under a long back-to-back loop the 1 kW power cap lowers the clock
+    burst_ms = []
+    for _ in range(PF_BURSTS):
+        time.sleep(PF_BURST_IDLE_S)
+        torch.cuda.synchronize()
+        a_, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a_.record(stream)
+        for _ in range(group):
+            pa.prefill(out, q, kc, vc, bt, cl, qsl, case.scale, sliding_window=win)
+        b_.record(stream)
+        torch.cuda.synchronize()
+        burst_ms.append(a_.elapsed_time(b_) / group)
+    burst_call_ms = statistics.median(burst_ms)
     err = pa.device_error(device.index)
     if err:
         raise RuntimeError(f"device error word {err:#x} during the timed loop")
@@ -988,11 +1020,8 @@ def run_prefill(args):
     value = flops * ws / (ms_step * 1e-3) / 1e12
     e2e_val = flops * ws / (max_over_ranks(e2e_ms, ws, device) / e2e_steps * 1e-3) / 1e12
     achieved = flops / (call_ms * 1e-3) / 1e12
-    try:
-        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
-            peak, peak_kind = float(json.load(f)["bf16_tflops"]), "measured"
-    except Exception:
-        peak, peak_kind = 1590.0, "fallback"
+    achieved_burst = flops / (burst_call_ms * 1e-3) / 1e12
+    (peak, peak_kind), (peak_s, peak_s_kind) = bf16_peaks()
     result = None
     if rank == 0:
         cpu = None
@@ -1019,14 +1048,23 @@ def run_prefill(args):
             "e2e": {"value": round(e2e_val, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "steps": e2e_steps},
             "gpu_launches": 2 * args.steps,
-            "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak,
-                         "peak_kind": f"{peak_kind} cuBLAS bf16 TFLOP/s (burst)", "unit": "TFLOP/s",
-                         "frac": round(achieved / peak, 4), "kernel": "pa_prefill",
+            "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak_s,
+                         "peak_kind": f"{peak_s_kind} cuBLAS bf16 TFLOP/s (sustained: this pass "
+                                      "is a long back-to-back loop under the power cap)",
+                         "unit": "TFLOP/s",
+                         "frac": round(achieved / peak_s, 4), "kernel": "pa_prefill",
                          "avg_call_us": round(call_ms * 1e3, 2),
                          "achieved_how": "algorithmic FLOPs (both products once; the split "
                                          "P's second product and masked tile work not "
                                          "counted) / mean CUDA-event time per call, events "
-                                         "around groups of 10 calls",
+                                         "around groups of 10 back-to-back calls after the "
+                                         "timed steps",
+                         "burst": {"achieved": round(achieved_burst, 2), "peak": peak,
+                                   "peak_kind": f"{peak_kind} cuBLAS bf16 TFLOP/s (burst)",
+                                   "frac": round(achieved_burst / peak, 4),
+                                   "avg_call_us": round(burst_call_ms * 1e3, 2),
+                                   "how": f"median over {PF_BURSTS} bursts of 10 calls, each "
+                                          f"after {PF_BURST_IDLE_S * 1e3:.0f} ms idle"},
                          "traffic": traffic_from_profile(args.workload, "prefill_traffic.json",
                                                          ("pa_common.cuh", "pa_prefill.cuh"))},
             "clocks": clocks,
