@@ -72,6 +72,7 @@ struct DecodeParams {
     int num_parts;
     int sliding_window;  // > 0: attend to the last sliding_window tokens only; 0: all
     int rotate;          // != 0: each warp starts its tiles at a pseudo-random offset
+    int sort_second;     // != 0 (two partitions, few sequences): second partitions longest first
     float scale_log2;
     // Cache write fused into the decode (pa_decode_append): the new token of sequence s
     // (key/value rows new_k + s * new_k_stride, heads contiguous) is stored at position
@@ -533,6 +534,45 @@ using WarpCompute = typename std::conditional<(G >= 4), MmaWarp<T, D, G>, SimtWa
 
 // ------------------------------------------------------------------ partition kernel
 
+constexpr int kSortMaxSeqs = kWarps * 32;  // one sequence per thread
+
+// Launches of at most two partitions per context: the second partitions -- the grid's
+// last CTAs, and so the tail -- are taken longest first.  Returns the sequence whose second
+// partition has rank k in that order (by decreasing length, ties by sequence), or -1
+// past the last one.  Every thread of the CTA calls it; at most kSortMaxSeqs sequences.
+template <bool WIN>
+__device__ __forceinline__ int second_partition_seq(const DecodeParams &p, int k, int S) {
+    __shared__ __align__(16) int sh_len2[kSortMaxSeqs];  // second partition's length, or -1
+    __shared__ int sh_sel;
+    const int tid = threadIdx.x;
+    const int P = p.partition_tokens;
+    const int cap = p.max_blocks_per_seq << p.bs_shift;
+    int r = -1;
+    if (tid < S) {
+        int L = __ldg(p.context_lens + tid);
+        L = L < 0 ? 0 : (L > cap ? cap : L);
+        const int len = WIN ? L - span_begin(L, p.sliding_window) : L;
+        r = len > P ? len - P : -1;
+    }
+    sh_len2[tid] = r;
+    if (tid == 0) sh_sel = -1;
+    __syncthreads();
+    if (r >= 0) {
+        int rank = 0;
+#pragma unroll 4
+        for (int t = 0; t < kSortMaxSeqs; t += 4) {
+            const int4 v = *reinterpret_cast<const int4 *>(sh_len2 + t);
+            rank += (v.x > r || (v.x == r && t < tid)) ? 1 : 0;
+            rank += (v.y > r || (v.y == r && t + 1 < tid)) ? 1 : 0;
+            rank += (v.z > r || (v.z == r && t + 2 < tid)) ? 1 : 0;
+            rank += (v.w > r || (v.w == r && t + 3 < tid)) ? 1 : 0;
+        }
+        if (rank == k) sh_sel = tid;
+    }
+    __syncthreads();
+    return sh_sel;
+}
+
 // WIN: compiled with sliding-window support (p.sliding_window > 0); the instances
 // without it keep the whole-context path free of the window's bookkeeping.
 template <typename T, int D, int G, int BOXR, bool WIN>
@@ -549,8 +589,15 @@ __global__ void __launch_bounds__(kWarps * 32)
     const int warp = tid >> 5, lane = tid & 31;
     // grid (kv head, sequence, partition): every first partition is scheduled before any
     // second one, so the smaller remainder partitions run last and shorten the tail, and
-    // CTAs scheduled together read neighbouring heads of the same physical blocks.
-    const int g = blockIdx.x, s = blockIdx.y, part = blockIdx.z;
+    // CTAs scheduled together read neighbouring heads of the same physical blocks.  With
+    // p.sort_second the second partitions are moreover taken longest first.
+    const int g = blockIdx.x;
+    int s = blockIdx.y;
+    const int part = blockIdx.z;
+    if (p.sort_second && part == 1) {
+        s = second_partition_seq<WIN>(p, (int)blockIdx.y, (int)gridDim.y);
+        if (s < 0) return;
+    }
     const int Hq = p.num_q_heads;
 
     // Start the three independent loads of this item at once: its context length, the

@@ -803,6 +803,7 @@ pa_status decode_impl(void *out, const void *q, const void *k_cache, const void 
     p.num_parts = pl.num_parts;
     p.sliding_window = sliding_window;
     p.rotate = block_size >= kRotateMinBlock ? 1 : 0;
+    p.sort_second = (pl.num_parts == 2 && num_seqs <= kSortMaxSeqs) ? 1 : 0;
     p.scale_log2 = scale * 1.4426950408889634f;
     p.new_k = new_k;
     p.new_v = new_v;

@@ -208,6 +208,21 @@ def test_balanced_split_ragged_and_empty(seed):
     _check_step(one, partition_size=-1, full=True)
 
 
+@pytest.mark.parametrize("B", [100, 128, 129])
+def test_second_partitions_longest_first(B):
+    """Two partitions per context (partitions of 64, contexts up to 128) and at most 128
+    contexts: the second partitions are taken longest first.  Ties in their length,
+    contexts without one, empty contexts and one-token second partitions must all land on
+    the right outputs (129 contexts keep the plain order)."""
+    rng = np.random.default_rng(B)
+    lens = rng.integers(0, 129, size=B)
+    lens[:10] = [0, 1, 64, 65, 65, 65, 128, 128, 100, 100]
+    for G in (1, 4):
+        case = _rand_case(B, "bf16", B, 2 * G, 2, 128, 16, lens)
+        case.slot_mapping[case.context_lens == 0] = -1
+        _check_step(case, partition_size=64, full=True)
+
+
 def test_table_width_bound():
     """Contexts exactly filling the table width (the largest the table allows)."""
     case = _rand_case(11, "bf16", 3, 8, 8, 128, 32, [32 * 20, 32 * 20, 1])

@@ -156,3 +156,15 @@ def test_window_workload_full_size(ps):
                          max_context_len=case.max_context_len, sliding_window=case.window)
         torch.cuda.synchronize()
         assert np.array_equal(bits(fused.out), bits(dc.out))
+
+
+@pytest.mark.parametrize("B", [60, 129])
+def test_window_second_partitions_longest_first(B):
+    """Two partitions per window (W = 100, partitions of 64): with at most 128 contexts the
+    second partitions are taken longest first.  Ties, contexts shorter than one partition
+    and long contexts whose window starts inside a page."""
+    rng = np.random.default_rng(B + 7)
+    lens = rng.integers(1, 400, size=B)
+    lens[:6] = [1, 64, 65, 100, 101, 399]
+    case = _case(B, "bf16", 8, 2, 128, 16, lens, 100)
+    _check(case, 100, 64)
