@@ -999,7 +999,9 @@ extern "C" pa_status pa_prefill(void *out, const void *q, const void *k_cache,
     const long long tpt = kPfRows / G;
     const long long pairs = (long long)num_tokens / (2 * tpt) + num_seqs;
     if (pairs >= (1ll << 31)) return PA_ERR_UNSUPPORTED;
-    const dim3 grid((unsigned)pairs, (unsigned)num_kv_heads);
+    p.heads_inner = pairs <= 65535 ? 1 : 0;
+    const dim3 grid = p.heads_inner ? dim3((unsigned)num_kv_heads, (unsigned)pairs)
+                                    : dim3((unsigned)pairs, (unsigned)num_kv_heads);
     cudaStream_t st_ = static_cast<cudaStream_t>(stream);
     const cudaError_t e = dtype == PA_BF16
                               ? prefill_dispatch<__nv_bfloat16>(p, grid, st_, dev, head_dim, G)

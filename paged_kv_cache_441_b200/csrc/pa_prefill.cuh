@@ -84,6 +84,7 @@ struct PrefillParams {
     int max_blocks_per_seq;
     int sliding_window;
     float scale_log2;
+    int heads_inner;  // 1: blockIdx.x is the kv head and blockIdx.y the tile pair; 0: swapped
 };
 
 template <int D>
@@ -261,8 +262,8 @@ __device__ __forceinline__ PfTile pf_tile(int qt, int tpt, int n, int L, int W) 
     return t;
 }
 
-// grid = (an upper bound of the number of tile pairs, kv heads); CTAs past the last pair
-// return at once.
+// grid = (kv heads, an upper bound of the number of tile pairs), or the two swapped when
+// the bound exceeds the grid's y limit; CTAs past the last pair return at once.
 template <typename T, int D, int G>
 __global__ void __launch_bounds__(kPfThreads, 1)
     pa_prefill_kernel(const __grid_constant__ PrefillParams p) {
@@ -278,8 +279,11 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     const uint32_t base = (raw + 1023u) & ~1023u;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int g = blockIdx.y;
-    const int cta = blockIdx.x;
+    // kv head and tile-pair slot.  With the kv head as blockIdx.x, the hardware hands out
+    // every head of one pair before the next pair, so the last CTAs are the shortest pairs
+    // of the last sequence instead of all pairs of the last kv head.
+    const int g = p.heads_inner ? blockIdx.x : blockIdx.y;
+    const int cta = p.heads_inner ? blockIdx.y : blockIdx.x;
 
     // ---- 1. this CTA's (sequence, tile pair): block-wide prefix sum of pairs per
     // sequence; within a sequence the last (longest-context) pair comes first.
