@@ -660,6 +660,13 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         const bool rvalid = t.live && rtok < t.ntok;
         const int rpos = rvalid ? t.pos0 + rtok : -1;
         const int rlo = (W > 0 && rvalid) ? rpos - W + 1 : 0;
+        // this row attends keys [key_base, key_base + key_span]: a key is in iff
+        // key - key_base <= key_span as unsigned (one compare per element); a row that
+        // attends nothing gets a base every key is below, modulo 2^32
+        const int key_lo = max(rlo, kv_begin);
+        const bool row_any = rpos >= key_lo;
+        const unsigned key_base = row_any ? (unsigned)key_lo : 0x80000000u;
+        const unsigned key_span = row_any ? (unsigned)(rpos - key_lo) : 0u;
         // every row of the tile attends keys [key_all_lo, key_all_hi] (valid tokens only)
         const bool all_rows = t.live && t.ntok == kTpt;
         const int key_all_hi = t.pos0;                          // min over rows of rpos
@@ -704,10 +711,10 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                         for (int e = 0; e < 32; ++e)
                             mxp[e & 7] = fmaxf(mxp[e & 7], __uint_as_float(cur[e]));
                     } else {
+                        const unsigned dlo = (unsigned)(kv0 + 32 * c) - key_base;
 #pragma unroll
                         for (int e = 0; e < 32; ++e) {
-                            const int key = kv0 + 32 * c + e;
-                            const bool in = key <= rpos && key >= rlo && key >= kv_begin;
+                            const bool in = dlo + (unsigned)e <= key_span;
                             mxp[e & 7] = fmaxf(mxp[e & 7], in ? __uint_as_float(cur[e]) : -INFINITY);
                         }
                     }
@@ -767,10 +774,10 @@ __global__ void __launch_bounds__(kPfThreads, 1)
 #pragma unroll
                         for (int e = 0; e < 32; ++e) xe[e] = fmaf(__uint_as_float(cur[e]), c2, -m_use);
                     } else {
+                        const unsigned dlo = (unsigned)(kv0 + 32 * c) - key_base;
 #pragma unroll
                         for (int e = 0; e < 32; ++e) {
-                            const int key = kv0 + 32 * c + e;
-                            const bool in = key <= rpos && key >= rlo && key >= kv_begin;
+                            const bool in = dlo + (unsigned)e <= key_span;
                             xe[e] = in ? fmaf(__uint_as_float(cur[e]), c2, -m_use) : -INFINITY;
                         }
                     }
