@@ -44,3 +44,15 @@ def test_prefill_flops_match_brute_force():
         # the per-sample count used by the CPU baseline agrees on the whole set
         sel = np.array([(t, h) for t in range(int(qsl[-1])) for h in range(case.num_q_heads)])
         assert bench.prefill_sample_flops(case, sel) == want
+
+
+def test_bf16_peaks_measured_and_fallback(tmp_path, monkeypatch):
+    """The prefill roofline's denominators: the measured burst and sustained cuBLAS
+    rates when the file has them, the recipe's 1,590 / 1,400 TFLOP/s otherwise."""
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.bf16_peaks() == ((1590.0, "fallback"), (1400.0, "fallback"))
+    (tmp_path / "MEASURED_PEAKS.json").write_text('{"bf16_tflops": 1665.0}')
+    assert bench.bf16_peaks() == ((1665.0, "measured"), (1400.0, "fallback"))
+    (tmp_path / "MEASURED_PEAKS.json").write_text(
+        '{"bf16_tflops": 1665.0, "bf16_tflops_sustained": 1339.0}')
+    assert bench.bf16_peaks() == ((1665.0, "measured"), (1339.0, "measured"))
