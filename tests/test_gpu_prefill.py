@@ -106,6 +106,26 @@ def test_prefill_one_token_chunks_match_decode():
         assert np.max(np.abs(to_f64(dec) - to_f64(out))) <= 2 * TOL["bf16"]
 
 
+def test_prefill_many_short_prompts():
+    """66,000 one- to three-token prompts (8 query heads on 1 kv head): the launch's bound
+    on tile pairs exceeds the grid's y limit, so the kernel takes the layout with the pair
+    in blockIdx.x and the kv head in blockIdx.y; every output against the oracle.  Among
+    34M outputs some reach magnitudes of 4 and more, where half a bf16 step (2^-6) is
+    itself above the 1e-2 bar, so each output may differ from the exact value by the larger
+    of the bar and half a bf16 step of that value (rounding the exact result gives the same
+    worst case)."""
+    specs = [(1, 1 + (i % 3)) for i in range(66000)]
+    case = make_prefill_case("many", 5, specs, 8, 1, 64, 16)
+    out, kc, vc = _run(case)
+    ref, _, _ = _oracle(case)
+    got = to_f64(out)
+    mag = np.maximum(np.abs(ref), 2.0 ** -126)
+    half_step = np.exp2(np.floor(np.log2(mag)) - 8)  # half the bf16 spacing at |ref|
+    bound = np.maximum(TOL[case.dtype], half_step)
+    err = np.abs(got - ref)
+    assert np.all(np.isfinite(got)) and np.all(err <= bound), float(np.max(err - bound))
+
+
 @pytest.mark.parametrize("name", ["prefill_2k_gqa", "prefill_chunk512_gqa"])
 def test_prefill_workloads_full_size(name):
     """The benchmark's prefill workloads at full size, every (token, head) output."""
