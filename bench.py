@@ -93,6 +93,13 @@ def copy_bytes(case) -> int:
     return 2 * 2 * P * case.num_kv_heads * case.block_size * case.head_dim * 2 + 16 * P
 
 
+def cow_bytes(case) -> int:
+    """The copies pa_decode_cow makes: the named rows of every kv head, read and written
+    in both caches, plus the per-sequence triples."""
+    rows = int(case.cow[case.cow[:, 0] >= 0, 2].sum()) if case.cow.shape[0] else 0
+    return 2 * 2 * rows * case.num_kv_heads * case.head_dim * 2 + 12 * case.cow.shape[0]
+
+
 # ----------------------------------------------------------------------------- helpers
 
 def bf16_peaks():
@@ -322,12 +329,13 @@ PF_BURST_IDLE_S = 0.05  # ... each after this idle pause (the clock recovers fro
 
 
 class DecodeStep:
-    """A decode workload resident on the device and its step: copy-on-write pairs (when
-    the workload has them), the cache write and paged decode -- fused into one call
-    (pa_decode_append) when every sequence appends exactly one token and nothing is
-    copied."""
+    """A decode workload resident on the device and its step: copy-on-write copies (when
+    the workload has them), the cache write and paged decode.  The write is fused into the
+    decode (pa_decode_append) when every sequence appends exactly one token and nothing is
+    copied; copies are done by the decode's own CTAs (pa_decode_cow, cow="folded") or by
+    a pa_copy_blocks launch before the write (cow="separate")."""
 
-    def __init__(self, torch, pa, case, device, partition_size):
+    def __init__(self, torch, pa, case, device, partition_size, cow="folded"):
         self.case, self.pa = case, pa
         dt = case.dtype
 
@@ -355,20 +363,26 @@ class DecodeStep:
         span = min(mcl, W * case.block_size, win + 15 if win > 0 else mcl)
         nparts = 0 if ptoks == 0 else -(-span // ptoks)
         self.has_pairs = case.copy_pairs.shape[0] > 0
+        self.cow_folded = (self.has_pairs and cow == "folded" and partition_size >= 0
+                           and case.cow.shape[0] == case.num_seqs)
+        self.cow = di(case.cow) if self.cow_folded else None
         self.fused = ((not self.has_pairs) and case.key.shape[0] == case.num_seqs
                       and partition_size >= 0)
         decode_launches = 1 if nparts == 1 else 2
-        self.launches_per_step = decode_launches + (0 if self.fused else
-                                                    1 + (1 if self.has_pairs else 0))
+        self.launches_per_step = decode_launches + (
+            0 if self.fused else 1 + (1 if self.has_pairs and not self.cow_folded else 0))
         self.split = (f"fixed {ptoks}-token partitions, {nparts} max" if ptoks > 0 else
                       "dynamic: persistent CTAs claim 32-token chunks + LSE merge"
                       if partition_size == -2 else
                       "balanced over persistent warps (stream-K) + LSE merge")
         self.kind = ("pa_decode_append (cache write fused into decode)" if self.fused
+                     else "pa_kv_write + pa_decode_cow (copy-on-write rows copied by the "
+                          "partition pass)" if self.cow_folded
                      else "pa_copy_blocks + pa_kv_write + pa_decode" if self.has_pairs
                      else "pa_kv_write + pa_decode")
         self.step_bytes = (decode_bytes(case) + write_bytes(case)
-                           + (copy_bytes(case) if self.has_pairs else 0))
+                           + (cow_bytes(case) if self.cow_folded else
+                              copy_bytes(case) if self.has_pairs else 0))
 
     def decode(self, b=None):
         """The attention call of the step (with the fused write when the step has it)."""
@@ -381,6 +395,10 @@ class DecodeStep:
                              self.vc, bt, cl, c.scale, max_context_len=c.max_context_len,
                              partition_size=self.ps, workspace=self.workspace,
                              sliding_window=c.window)
+        elif self.cow_folded:
+            pa.decode_cow(out, q, self.kc, self.vc, bt, cl, b.get("cow", self.cow), c.scale,
+                          max_context_len=c.max_context_len, partition_size=self.ps,
+                          workspace=self.workspace, sliding_window=c.window)
         else:
             pa.decode(out, q, self.kc, self.vc, bt, cl, c.scale, max_context_len=c.max_context_len,
                       partition_size=self.ps, workspace=self.workspace, sliding_window=c.window)
@@ -388,7 +406,7 @@ class DecodeStep:
     def step(self, b=None):
         b = b or {}
         if not self.fused:
-            if self.has_pairs:
+            if self.has_pairs and not self.cow_folded:
                 self.pa.copy_blocks(self.kc, self.vc, b.get("pairs", self.pairs))
             self.pa.kv_write(b.get("key", self.key), b.get("val", self.val),
                              b.get("sm", self.sm), self.kc, self.vc)
@@ -504,7 +522,7 @@ def run_ours(args):
         desc = f"{desc} [profiling subset: first {args.seqs} seqs' distribution]"
     case = make_config(name, poison=False, **kw)
     dt = case.dtype
-    ds = DecodeStep(torch, pa, case, device, args.partition_size)
+    ds = DecodeStep(torch, pa, case, device, args.partition_size, cow=args.cow)
     q, out = ds.q, ds.out
     stream = torch.cuda.current_stream()
 
@@ -555,9 +573,11 @@ def run_ours(args):
     h_bt = torch.from_numpy(case.block_tables).pin_memory()
     h_cl = torch.from_numpy(case.context_lens).pin_memory()
     h_pairs = torch.from_numpy(case.copy_pairs.reshape(-1, 2).astype(np.int64)).pin_memory()
+    h_cow = torch.from_numpy(case.cow).pin_memory()
     h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
     h2d_bytes = sum(t.numel() * t.element_size() for t in (h_q, h_key, h_val, h_sm, h_bt, h_cl))
-    h2d_bytes += h_pairs.numel() * 8 if ds.has_pairs else 0
+    h2d_bytes += (h_cow.numel() * 4 if ds.cow_folded else
+                  h_pairs.numel() * 8 if ds.has_pairs else 0)
     d2h_bytes = h_out.numel() * h_out.element_size()
     e2e_steps = max(1, min(args.steps, args.e2e_steps))
 
@@ -568,7 +588,8 @@ def run_ours(args):
     copy_stream = torch.cuda.Stream(device=device)
     bufs = [dict(q=torch.empty_like(q), key=torch.empty_like(ds.key), val=torch.empty_like(ds.val),
                  sm=torch.empty_like(ds.sm), bt=torch.empty_like(ds.bt), cl=torch.empty_like(ds.cl),
-                 pairs=torch.empty_like(ds.pairs), out=torch.empty_like(out)) for _ in range(2)]
+                 pairs=torch.empty_like(ds.pairs), out=torch.empty_like(out),
+                 cow=torch.empty_like(ds.cow) if ds.cow_folded else None) for _ in range(2)]
     h_outs = [h_out, torch.empty(out.shape, dtype=out.dtype).pin_memory()]
     ev_in = [torch.cuda.Event() for _ in range(2)]
     ev_done = [torch.cuda.Event() for _ in range(2)]
@@ -585,7 +606,9 @@ def run_ours(args):
             b["sm"].copy_(h_sm, non_blocking=True)
             b["bt"].copy_(h_bt, non_blocking=True)
             b["cl"].copy_(h_cl, non_blocking=True)
-            if ds.has_pairs:
+            if ds.cow_folded:
+                b["cow"].copy_(h_cow, non_blocking=True)
+            elif ds.has_pairs:
                 b["pairs"].copy_(h_pairs, non_blocking=True)
             ev_in[i % 2].record(copy_stream)
 
@@ -630,6 +653,31 @@ def run_ours(args):
     # dynamic split's sums vary in the last bits from call to call
     torch.testing.assert_close(h_outs[(e2e_steps - 1) % 2].float(), out.cpu().float(), rtol=0,
                                atol=0 if args.partition_size != -2 else 1e-3)
+
+    # ---- the same step with the copies in their own launch (or folded in), timed in
+    # alternation with this one: what folding the copy-on-write into the decode gives
+    cow_compare = None
+    if ds.has_pairs and ws == 1 and args.partition_size >= 0:
+        other = DecodeStep(torch, pa, case, device, args.partition_size,
+                           cow="separate" if ds.cow_folded else "folded")
+        for _ in range(args.warmup):
+            other.step()
+        torch.cuda.synchronize()
+        est = elapsed_ms / max(args.steps, 1)
+        t_this, t_other = [], []
+        for _ in range(2):
+            t_this.append(time_groups(torch, ds.step, stream, est, args.roofline_s / 2)[0])
+            t_other.append(time_groups(torch, other.step, stream, est, args.roofline_s / 2)[0])
+        if pa.device_error(device.index):
+            raise RuntimeError("device error word set in the copy-on-write comparison")
+        folded, separate = ((t_this, t_other) if ds.cow_folded else (t_other, t_this))
+        cow_compare = {
+            "folded_us_per_step": round(1e3 * statistics.mean(folded), 2),
+            "separate_us_per_step": round(1e3 * statistics.mean(separate), 2),
+            "folded": "pa_kv_write + pa_decode_cow (rows copied by the CTAs that read them)",
+            "separate": "pa_copy_blocks + pa_kv_write + pa_decode",
+            "how": "median over groups of consecutive steps, two alternating passes each"}
+        del other
 
     # ---- aggregate over ranks
     max_ms = max_over_ranks(elapsed_ms, ws, device)
@@ -684,6 +732,7 @@ def run_ours(args):
                            f"read per step vs 126 MB); the timed steps run back to back "
                            f"without a flush; roofline.frac_l2_flushed times single calls "
                            f"after a {FLUSH_BYTES >> 20} MB write + read"},
+            **({"cow_compare": cow_compare} if cow_compare else {}),
             "seq_steps_per_s": round(case.num_seqs * ws / (ms_per_step * 1e-3), 1),
             "pct_of_8tbs": round(100 * value / 8000.0, 2),
             "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d_bytes,
@@ -1275,6 +1324,9 @@ def main(argv=None):
                     default="step",
                     help="swap: time the preemption swap of the workload instead of the step; "
                          "prefill: the prefill / chunked-prefill step (--workload prefill_*)")
+    ap.add_argument("--cow", choices=["folded", "separate"], default="folded",
+                    help="workloads with copy-on-write: copies done by the decode's own CTAs "
+                         "(pa_decode_cow) or by a pa_copy_blocks launch before the step")
     ap.add_argument("--swap-seqs", type=int, default=8,
                     help="swap: number of sequences preempted and restored per step")
     args = ap.parse_args(argv)

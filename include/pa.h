@@ -234,6 +234,48 @@ pa_status pa_decode_append(void *out, const void *q, const void *key, const void
                            size_t workspace_bytes, pa_dtype dtype, void *stream);
 
 /*
+ * One decode step with the copy-on-write of a shared block folded into the attention
+ * pass (the pages let several requests share KV blocks -- "PagedAttention" summary,
+ * features 2 -- so a sequence that appends into a shared, partially filled block
+ * first needs a private copy of it).  Instead of a pa_copy_blocks launch before the
+ * step, each sequence names the block it copies, and the rows are copied by the CTAs
+ * that read them, just before they read them.
+ *
+ * cow : int32 [num_seqs][3] in device memory, 4-byte aligned.  For sequence s the
+ *       triple (src, lb, rows): src < 0 means no copy; otherwise, for every kv head
+ *       h and every r < rows,
+ *         k_cache[block_tables[s][lb]][h][r][:] = k_cache[src][h][r][:]
+ *       and likewise in v_cache, done before any of those rows is read.  Rows >= rows
+ *       of the destination are left as they are: they hold this sequence's own tokens
+ *       (written before the call, e.g. by pa_kv_write) or are unused.  With rows =
+ *       block_size this is pa_copy_blocks of the pair (src, block_tables[s][lb]).
+ *       Every row is copied whether or not the attention reads it (rows outside the
+ *       context or before the sliding window too).  src outside [0, num_blocks), lb
+ *       outside [0, max_blocks_per_seq) or rows outside [0, block_size] sets
+ *       PA_DEVERR_PAIR, and an entry block_tables[s][lb] outside [0, num_blocks) sets
+ *       PA_DEVERR_BLOCK_ID; that sequence's copy is skipped.  A destination must be
+ *       private to its sequence, must not be the source of any copy of the call, and
+ *       no other sequence of the call may read it; no row a copy reads may be one that
+ *       the call's fused cache write stores.
+ * key, value : both NULL (no cache write), or both given: the fused write of
+ *       pa_decode_append, done after the copy (so a written row wins over a copied
+ *       one).  Strides and alignment as pa_decode_append.
+ * The result equals pa_copy_blocks of the rows, then (with key) pa_kv_write of the
+ * new tokens, then pa_decode -- bit for bit.  partition_size as pa_decode, except
+ * that a call that would take the balanced or the dynamic split returns
+ * PA_ERR_UNSUPPORTED (the fixed split only).  Other arguments, errors and the
+ * workspace as pa_decode.  Launches as pa_decode.
+ */
+pa_status pa_decode_cow(void *out, const void *q, const void *key, const void *value,
+                        int64_t key_token_stride, int64_t value_token_stride, void *k_cache,
+                        void *v_cache, const int32_t *block_tables, const int32_t *context_lens,
+                        const int32_t *cow, int num_seqs, int num_q_heads, int num_kv_heads,
+                        int head_dim, int block_size, int num_blocks, int max_blocks_per_seq,
+                        float scale, int max_context_len, int sliding_window,
+                        int partition_size, void *workspace, size_t workspace_bytes,
+                        pa_dtype dtype, void *stream);
+
+/*
  * Bytes of workspace pa_decode needs for these sizes and this partition_size.
  * Host-side; it reads the current device's SM count (cudaDeviceGetAttribute, no
  * synchronisation; 148 when no device is visible), because the balanced and dynamic

@@ -11,6 +11,8 @@ The compute lives in ``libpa.so`` (CUDA kernels behind the C ABI in
   log-sum-exp merge; GQA served from one page read per kv head);
 * ``decode_append(out, q, key, value, k_cache, v_cache, ...)`` -- the step's cache
   write fused into the decode;
+* ``decode_cow(out, q, k_cache, v_cache, block_tables, context_lens, cow, scale, ...)``
+  -- each sequence's copy-on-write of a shared block folded into the decode;
 * ``prefill(out, q, k_cache, v_cache, block_tables, context_lens, query_start_loc,
   scale)`` -- causal multi-query attention for prompts and prompt chunks (tcgen05);
 * ``swap_blocks(...)`` -- block copies between the GPU cache and a pinned host pool;
@@ -30,6 +32,7 @@ from ._lib import (  # noqa: F401
     copy_blocks,
     decode,
     decode_append,
+    decode_cow,
     decode_static_scratch,
     decode_partition_tokens,
     decode_workspace_bytes,

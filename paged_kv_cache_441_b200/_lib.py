@@ -20,7 +20,8 @@ DEVERR = {"block_id": 0x1, "slot": 0x2, "pair": 0x4, "context": 0x8, "timeout": 
           "workspace": 0x20}
 EXPORTS = ("pa_kv_write", "pa_copy_blocks", "pa_decode", "pa_decode_workspace_bytes",
            "pa_decode_partition_tokens", "pa_get_device_error", "pa_status_str", "pa_version",
-           "pa_decode_static_scratch", "pa_decode_append", "pa_swap_blocks", "pa_prefill",
+           "pa_decode_static_scratch", "pa_decode_append", "pa_decode_cow", "pa_swap_blocks",
+           "pa_prefill",
            # host block manager (include/pa_block_manager.h)
            "pa_bm_create", "pa_bm_destroy", "pa_bm_blocks_needed", "pa_bm_num_free_blocks",
            "pa_bm_usage_ratio", "pa_bm_can_allocate", "pa_bm_allocate", "pa_bm_fork",
@@ -70,6 +71,9 @@ def load(path: str = LIB_PATH):
     lib.pa_decode_append.argtypes = [P, P, P, P, i64, i64, P, P, P, P, i32, i32, i32, i32, i32,
                                      i32, i32, f32, i32, i32, i32, P, sz, i32, P]
     lib.pa_decode_append.restype = i32
+    lib.pa_decode_cow.argtypes = [P, P, P, P, i64, i64, P, P, P, P, P, i32, i32, i32, i32, i32,
+                                  i32, i32, f32, i32, i32, i32, P, sz, i32, P]
+    lib.pa_decode_cow.restype = i32
     lib.pa_prefill.argtypes = [P, P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, i32, i32, f32,
                                i32, i32, P]
     lib.pa_prefill.restype = i32
@@ -342,6 +346,41 @@ def decode_append(out, q, key, value, k_cache, v_cache, block_tables, context_le
                                        hq, hkv, d, bs, nb, W, float(scale), int(max_context_len),
                                        int(sliding_window), int(partition_size), wptr, wbytes,
                                        _dtype(q), _stream(stream, dev)), what)
+
+
+def decode_cow(out, q, k_cache, v_cache, block_tables, context_lens, cow, scale, key=None,
+               value=None, max_context_len=0, partition_size=0, workspace=None, stream=None,
+               sliding_window=0) -> None:
+    """``decode`` with each sequence's copy-on-write done by the CTAs that read the rows:
+    cow int32 [B, 3] = (source block, logical block index, rows), source < 0 for none.
+    With key/value ([B, Hkv, d]) the new token's cache write of ``decode_append`` too."""
+    import torch
+    what = "pa_decode_cow"
+    B, hq, d, nb, hkv, bs, W = _decode_shapes(what, out, q, k_cache, v_cache, block_tables,
+                                              context_lens, None)
+    if (key is None) != (value is None):
+        _fail(what, "key and value must be given together")
+    if tuple(cow.shape) != (B, 3):
+        _fail(what, f"cow {tuple(cow.shape)} must be [{B}, 3]")
+    rows = {}
+    if key is not None:
+        if not (tuple(key.shape) == (B, hkv, d) and tuple(value.shape) == (B, hkv, d)):
+            _fail(what, f"key {tuple(key.shape)} and value {tuple(value.shape)} must both be "
+                  f"[{B}, {hkv}, {d}]")
+        rows = {"key": key, "value": value}
+    dev = _args(what, {"q": q, "out": out, "k_cache": k_cache, "v_cache": v_cache}, rows=rows,
+                ints={"block_tables": (block_tables, torch.int32),
+                      "context_lens": (context_lens, torch.int32),
+                      "cow": (cow, torch.int32)})
+    with _on(dev):
+        need = decode_workspace_bytes(B, hq, hkv, d, bs, W, max_context_len, partition_size,
+                                      sliding_window)
+        wptr, wbytes = _workspace(what, workspace, need, dev)
+        _check(load().pa_decode_cow(
+            _ptr(out), _ptr(q), _ptr(key), _ptr(value), key.stride(0) if key is not None else 0, value.stride(0) if value is not None else 0,
+            _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), _ptr(context_lens), _ptr(cow), B,
+            hq, hkv, d, bs, nb, W, float(scale), int(max_context_len), int(sliding_window),
+            int(partition_size), wptr, wbytes, _dtype(q), _stream(stream, dev)), what)
 
 
 def decode_static_scratch(out, q, k_cache, v_cache, block_tables, context_lens, scale,

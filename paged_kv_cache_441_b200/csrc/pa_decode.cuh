@@ -83,6 +83,11 @@ struct DecodeParams {
     long long new_v_stride;
     void *k_cache;
     void *v_cache;
+    // Copy-on-write folded into the decode (pa_decode_cow): int32 [B][3] = (source block,
+    // logical block index, rows); rows [0, rows) of every kv head of the source block are
+    // copied into the sequence's own block at that index before any of them is read.
+    // Source < 0: no copy for that sequence.  nullptr = no copies at all.
+    const int32_t *cow;
 };
 
 template <int D>
@@ -573,9 +578,29 @@ __device__ __forceinline__ int second_partition_seq(const DecodeParams &p, int k
     return sh_sel;
 }
 
+// Copy-on-write (p.cow): rows [a, b) of kv head g of block src into block dst, in both
+// caches, by `n` threads numbered `t` (a warp's lanes or the whole CTA).
+template <int D>
+__device__ __forceinline__ void cow_rows(const DecodeParams &p, int src, int dst, int g, int a,
+                                         int b, int t, int n) {
+    constexpr int kChunks = D / 8;  // 16-byte chunks of a head row
+    if (a >= b) return;
+    const size_t head_rows = (size_t)p.num_kv_heads * p.block_size;
+    const size_t from = ((size_t)src * head_rows + (size_t)g * p.block_size + a) * kChunks;
+    const size_t to = ((size_t)dst * head_rows + (size_t)g * p.block_size + a) * kChunks;
+    uint4 *kc = reinterpret_cast<uint4 *>(p.k_cache);
+    uint4 *vc = reinterpret_cast<uint4 *>(p.v_cache);
+    for (int c = t; c < (b - a) * kChunks; c += n) {
+        const uint4 k = ld_global_nc_v4(kc + from + c), v = ld_global_nc_v4(vc + from + c);
+        kc[to + c] = k;
+        vc[to + c] = v;
+    }
+}
+
 // WIN: compiled with sliding-window support (p.sliding_window > 0); the instances
-// without it keep the whole-context path free of the window's bookkeeping.
-template <typename T, int D, int G, int BOXR, bool WIN>
+// without it keep the whole-context path free of the window's bookkeeping.  COW: compiled
+// with the copy-on-write of p.cow, so that calls without copies run code without it.
+template <typename T, int D, int G, int BOXR, bool WIN, bool COW = false>
 __global__ void __launch_bounds__(kWarps * 32)
     pa_decode_partition_kernel(const __grid_constant__ DecodeParams p) {
     pdl_wait_and_release();
@@ -607,6 +632,12 @@ __global__ void __launch_bounds__(kWarps * 32)
     const int P = p.partition_tokens;
     const int W = WIN ? p.sliding_window : 0;
     const int32_t *table = p.block_tables + (size_t)s * p.max_blocks_per_seq;
+    int cw_src = -1, cw_lb = 0, cw_rows = 0;  // this sequence's copy-on-write, loaded early
+    if constexpr (COW) {
+        cw_src = __ldg(p.cow + 3 * (size_t)s);
+        cw_lb = __ldg(p.cow + 3 * (size_t)s + 1);
+        cw_rows = __ldg(p.cow + 3 * (size_t)s + 2);
+    }
     const int pg_first = (int)(((long long)part * P) >> p.bs_shift);
     const int pg_count = min((int)((((long long)part * P + P - 1) >> p.bs_shift) - pg_first + 1),
                              p.max_blocks_per_seq - pg_first);
@@ -626,8 +657,39 @@ __global__ void __launch_bounds__(kWarps * 32)
     const int wlo = WIN ? window_lo(L, W) : 0, span0 = WIN ? span_begin(L, W) : 0;
     const int nparts = (L - span0 + P - 1) / P;
     if (nparts > p.num_parts && tid == 0 && part == 0) raise_error(PA_DEVERR_CONTEXT);
+    // Copy-on-write: every row of the copied block goes to the CTA whose partition holds
+    // its position (rows before the first partition to the first, rows past the last to
+    // the last), so the CTA that reads a row copies it.  This CTA's share: rows [cr0, cr1).
+    int cr0 = 0, cr1 = 0;
+    long long cw_pos0 = 0;  // position of the block's first row
+    if constexpr (COW) {
+        const int owners = max(min(nparts, p.num_parts), 1);
+        if (cw_src >= 0 && part < owners) {
+            if (cw_src >= p.num_blocks || (unsigned)cw_lb >= (unsigned)p.max_blocks_per_seq ||
+                (unsigned)cw_rows > (unsigned)p.block_size) {
+                if (tid == 0 && part == 0 && g == 0) raise_error(PA_DEVERR_PAIR);
+            } else {
+                cw_pos0 = (long long)cw_lb << p.bs_shift;
+                const long long Pl = P;
+                const long long lo = part == 0 ? cw_pos0 : span0 + part * Pl;
+                const long long hi = part == owners - 1 ? cw_pos0 + cw_rows
+                                                        : span0 + (part + 1) * Pl;
+                cr0 = (int)max(0LL, min((long long)cw_rows, lo - cw_pos0));
+                cr1 = (int)max(0LL, min((long long)cw_rows, hi - cw_pos0));
+            }
+        }
+    }
     T *out = reinterpret_cast<T *>(p.out) + ((size_t)s * Hq + (size_t)g * G) * D;
     if (L == 0) {
+        if constexpr (COW) {
+            if (cr0 < cr1) {  // no tiles: the whole CTA copies the rows
+                const int dst = __ldg(table + cw_lb);
+                if ((unsigned)dst < (unsigned)p.num_blocks)
+                    cow_rows<D>(p, cw_src, dst, g, cr0, cr1, tid, kWarps * 32);
+                else if (tid == 0)
+                    raise_error(PA_DEVERR_BLOCK_ID);
+            }
+        }
         if (part == 0)
             for (int e = tid; e < G * D; e += kWarps * 32) out[e] = Fmt<T>::from_float(0.f);
         return;
@@ -753,6 +815,39 @@ __global__ void __launch_bounds__(kWarps * 32)
         okmask = ok ? (okmask | (1u << stage)) : (okmask & ~(1u << stage));
     };
 
+    // Copy-on-write rows of this CTA's share, after the barrier and before the first TMA:
+    // the warp whose tiles hold rows copies those (only that warp waits for the copy; the
+    // others start streaming), and the rows no tile of the call reads -- before the first
+    // tile or past the context -- are copied by the whole CTA.  The row the fused cache
+    // write stored is left out (the write wins either way).  Deferring the warp's copy
+    // until after its first TMA issues measured slower.
+    if constexpr (COW) {
+        if (cr0 < cr1) {  // CTA-uniform
+            const int o1 = (int)max((long long)cr0, min((long long)cr1, (long long)t0 - cw_pos0));
+            const int o2 = (int)min((long long)cr1, max((long long)cr0, (long long)t1 - cw_pos0));
+            long long wb = min((long long)cr1, (long long)tok_end - cw_pos0);
+            if (p.new_k != nullptr) wb = min(wb, (long long)(L - 1) - cw_pos0);
+            const int wa = (int)max((long long)cr0, (long long)tok_begin - cw_pos0);
+            const bool outside = cr0 < o1 || o2 < cr1;
+            const bool reads_rows = nt > 0 && wa < wb;  // warp-uniform
+            if (outside || reads_rows) {
+                const int dst = __ldg(table + cw_lb);
+                if ((unsigned)dst < (unsigned)p.num_blocks) {
+                    if (reads_rows) {
+                        cow_rows<D>(p, cw_src, dst, g, wa, (int)wb, lane, 32);
+                        fence_proxy_async_global();  // this warp's TMA reads the rows
+                    }
+                    if (outside) {
+                        cow_rows<D>(p, cw_src, dst, g, cr0, o1, tid, kWarps * 32);
+                        cow_rows<D>(p, cw_src, dst, g, o2, cr1, tid, kWarps * 32);
+                    }
+                } else if (lane == 0) {
+                    raise_error(PA_DEVERR_BLOCK_ID);
+                }
+                __syncwarp();
+            }
+        }
+    }
     const int npre = min(kStages, nt);
     for (int jt = 0; jt < npre; ++jt) produce(jt);
 
@@ -777,7 +872,6 @@ __global__ void __launch_bounds__(kWarps * 32)
         if (jt + kStages < nt) produce(jt + kStages);
     }
     if (failed) wc.init(q_item, lane);  // contributes nothing (m = -inf, l = 0)
-
     // ---- merge the warps' partial softmax states (each warp uses its own ring)
     float *mine = reinterpret_cast<float *>(base_ptr + warp * kStages * Gm::kStage);
     wc.finish(mine, lane);

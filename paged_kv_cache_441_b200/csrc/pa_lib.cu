@@ -254,10 +254,10 @@ cudaError_t ensure_smem(K kernel, int bytes, std::atomic<bool> *flags, int dev) 
     return e;
 }
 
-template <typename T, int D, int G, int BOXR, bool WIN>
+template <typename T, int D, int G, int BOXR, bool WIN, bool COW = false>
 cudaError_t launch_partition(const DecodeParams &p, dim3 grid, cudaStream_t st, int dev) {
     static std::atomic<bool> flags[kMaxDevices];
-    auto kernel = pa_decode_partition_kernel<T, D, G, BOXR, WIN>;
+    auto kernel = pa_decode_partition_kernel<T, D, G, BOXR, WIN, COW>;
     cudaError_t e = ensure_smem(kernel, Geom<D>::kSmem, flags, dev);
     if (e != cudaSuccess) return e;
     return launch_pdl(kernel, grid, dim3(kWarps * 32), Geom<D>::kSmem, st, p);
@@ -272,6 +272,12 @@ cudaError_t launch_merge(const MergeParams &p, dim3 grid, cudaStream_t st) {
 
 template <typename T, int D, int G>
 cudaError_t dispatch_boxr(const DecodeParams &p, dim3 grid, cudaStream_t st, int dev, int boxr) {
+    if (p.cow != nullptr && p.sliding_window > 0)  // the instances with copy-on-write
+        return boxr == 8 ? launch_partition<T, D, G, 8, true, true>(p, grid, st, dev)
+                         : launch_partition<T, D, G, 16, true, true>(p, grid, st, dev);
+    if (p.cow != nullptr)
+        return boxr == 8 ? launch_partition<T, D, G, 8, false, true>(p, grid, st, dev)
+                         : launch_partition<T, D, G, 16, false, true>(p, grid, st, dev);
     if (p.sliding_window > 0)
         return boxr == 8 ? launch_partition<T, D, G, 8, true>(p, grid, st, dev)
                          : launch_partition<T, D, G, 16, true>(p, grid, st, dev);
@@ -646,7 +652,8 @@ pa_status decode_impl(void *out, const void *q, const void *k_cache, const void 
                       int num_blocks, int max_blocks_per_seq, float scale, int max_context_len,
                       int sliding_window, int partition_size, void *workspace,
                       size_t workspace_bytes, pa_dtype dtype, void *stream, const void *new_k,
-                      const void *new_v, long long new_k_stride, long long new_v_stride) {
+                      const void *new_v, long long new_k_stride, long long new_v_stride,
+                      const int32_t *cow = nullptr) {
     if (dtype != PA_FP16 && dtype != PA_BF16) return PA_ERR_INVALID_ARG;
     pa_status st = check_decode_shape(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
                                       num_blocks, max_blocks_per_seq, max_context_len,
@@ -672,6 +679,7 @@ pa_status decode_impl(void *out, const void *q, const void *k_cache, const void 
     cudaStream_t st_ = static_cast<cudaStream_t>(stream);
     const unsigned long long rows = (unsigned long long)num_blocks * num_kv_heads * block_size;
     if (pl.streamk && new_k != nullptr) return PA_ERR_UNSUPPORTED;  // fixed split only
+    if ((pl.streamk || pl.dynamic) && cow != nullptr) return PA_ERR_UNSUPPORTED;
     if (pl.streamk) {
         StreamKParams sp;
         std::memset(&sp, 0, sizeof sp);
@@ -811,6 +819,7 @@ pa_status decode_impl(void *out, const void *q, const void *k_cache, const void 
     p.new_v_stride = new_v_stride;
     p.k_cache = const_cast<void *>(k_cache);
     p.v_cache = const_cast<void *>(v_cache);
+    p.cow = cow;
 
     if (pl.num_parts > 65535) return PA_ERR_UNSUPPORTED;  // use a larger partition_size
     dim3 grid((unsigned)num_kv_heads, (unsigned)num_seqs, (unsigned)pl.num_parts);
@@ -879,6 +888,33 @@ pa_status pa_decode_append(void *out, const void *q, const void *key, const void
                        max_blocks_per_seq, scale, max_context_len, sliding_window,
                        partition_size, workspace, workspace_bytes, dtype, stream, key, value,
                        key_token_stride, value_token_stride);
+}
+
+pa_status pa_decode_cow(void *out, const void *q, const void *key, const void *value,
+                        int64_t key_token_stride, int64_t value_token_stride, void *k_cache,
+                        void *v_cache, const int32_t *block_tables, const int32_t *context_lens,
+                        const int32_t *cow, int num_seqs, int num_q_heads, int num_kv_heads,
+                        int head_dim, int block_size, int num_blocks, int max_blocks_per_seq,
+                        float scale, int max_context_len, int sliding_window,
+                        int partition_size, void *workspace, size_t workspace_bytes,
+                        pa_dtype dtype, void *stream) {
+    if (num_seqs > 0) {
+        if (!cow || !aligned(cow, 4)) return PA_ERR_INVALID_ARG;
+        if ((key == nullptr) != (value == nullptr)) return PA_ERR_INVALID_ARG;
+        if (key != nullptr) {
+            if (!aligned(key, 16) || !aligned(value, 16)) return PA_ERR_INVALID_ARG;
+            if (key_token_stride % 8 != 0 || value_token_stride % 8 != 0 ||
+                key_token_stride < (int64_t)num_kv_heads * head_dim ||
+                value_token_stride < (int64_t)num_kv_heads * head_dim)
+                return PA_ERR_INVALID_ARG;
+        }
+    }
+    return decode_impl(out, q, k_cache, v_cache, block_tables, context_lens, num_seqs,
+                       num_q_heads, num_kv_heads, head_dim, block_size, num_blocks,
+                       max_blocks_per_seq, scale, max_context_len, sliding_window,
+                       partition_size, workspace, workspace_bytes, dtype, stream, key, value,
+                       key != nullptr ? key_token_stride : 0,
+                       value != nullptr ? value_token_stride : 0, cow);
 }
 
 }  // extern "C"

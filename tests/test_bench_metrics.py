@@ -56,3 +56,13 @@ def test_bf16_peaks_measured_and_fallback(tmp_path, monkeypatch):
     (tmp_path / "MEASURED_PEAKS.json").write_text(
         '{"bf16_tflops": 1665.0, "bf16_tflops_sustained": 1339.0}')
     assert bench.bf16_peaks() == ((1665.0, "measured"), (1339.0, "measured"))
+
+
+def test_cow_bytes_count_the_named_rows():
+    """The folded copies move the named rows of every kv head (read and written, K and
+    V) plus one triple per sequence; the separate block copy moves whole blocks."""
+    from workloads.gen import make_prefix_cow
+    c = make_prefix_cow(groups=2, samples=8, max_suffix=20, num_kv_heads=4, head_dim=64)
+    rows = 2 * 7 * 8  # 7 copies per group, 8 prompt rows each
+    assert bench.cow_bytes(c) == 2 * 2 * rows * 4 * 64 * 2 + 12 * 16
+    assert bench.copy_bytes(c) == 2 * 2 * 14 * 4 * 16 * 64 * 2 + 16 * 14

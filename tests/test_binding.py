@@ -126,6 +126,31 @@ def test_decode_append_and_prefill_marshalling(fake):
     assert args[16] == 9
 
 
+def test_decode_cow_marshalling(fake):
+    a = _decode_args()
+    cow = torch.tensor([[4, 1, 8], [-1, 0, 0], [7, 0, 16]], dtype=torch.int32)
+    _lib.decode_cow(a["out"], a["q"], a["k_cache"], a["v_cache"], a["block_tables"],
+                    a["context_lens"], cow, 0.2, stream=STREAM)
+    args = [_v(x) for x in fake.last("pa_decode_cow")]
+    assert args[2] is None and args[3] is None and args[4:6] == [0, 0]  # no cache write
+    assert args[10] == cow.data_ptr() and args[11:18] == [3, 8, 2, 64, 16, 10, 5]
+    key = torch.zeros(3, 2, 64, dtype=torch.bfloat16)
+    _lib.decode_cow(a["out"], a["q"], a["k_cache"], a["v_cache"], a["block_tables"],
+                    a["context_lens"], cow, 0.2, key=key, value=torch.zeros_like(key),
+                    stream=STREAM)
+    args = [_v(x) for x in fake.last("pa_decode_cow")]
+    assert args[2] == key.data_ptr() and args[4:6] == [2 * 64, 2 * 64]
+    with pytest.raises(_lib.PAError, match="together"):
+        _lib.decode_cow(a["out"], a["q"], a["k_cache"], a["v_cache"], a["block_tables"],
+                        a["context_lens"], cow, 0.2, key=key, stream=STREAM)
+    with pytest.raises(_lib.PAError, match=r"must be \[3, 3\]"):
+        _lib.decode_cow(a["out"], a["q"], a["k_cache"], a["v_cache"], a["block_tables"],
+                        a["context_lens"], cow[:2], 0.2, stream=STREAM)
+    with pytest.raises(_lib.PAError, match="int32"):
+        _lib.decode_cow(a["out"], a["q"], a["k_cache"], a["v_cache"], a["block_tables"],
+                        a["context_lens"], cow.long(), 0.2, stream=STREAM)
+
+
 def test_swap_blocks_host_and_device_pools(fake):
     dev_k = torch.zeros(8, 2, 16, 64, dtype=torch.bfloat16)
     host_k = torch.zeros(5, 2, 16, 64, dtype=torch.bfloat16)

@@ -120,6 +120,31 @@ def test_decode_rejects_before_launch(lib, over, code):
     assert _call_decode(lib, _decode_args(**over)) == code
 
 
+def _call_decode_cow(lib, a, key=None, value=None, cow=16, ks=256, vs=256):
+    P = ctypes.c_void_p
+    return lib.pa_decode_cow(P(a["out"]), P(a["q"]), P(key) if key else None,
+                             P(value) if value else None, ks, vs, P(a["kc"]), P(a["vc"]),
+                             P(a["bt"]), P(a["cl"]), P(cow) if cow else None, a["B"], a["hq"],
+                             a["hkv"], a["d"], a["bs"], a["nb"], a["W"], a["scale"], a["mcl"],
+                             a["win"], a["ps"], a["ws"], a["wsb"], a["dt"], a["stream"])
+
+
+@pytest.mark.parametrize("over,extra,code", [
+    ({}, dict(cow=None), 1),                      # no copy list
+    ({}, dict(cow=2), 1),                         # misaligned copy list
+    ({}, dict(key=16), 1),                        # key without value
+    ({}, dict(key=8, value=16), 1),               # misaligned key
+    ({}, dict(key=16, value=16, ks=100), 1),      # token stride not a multiple of 8
+    ({}, dict(key=16, value=16, vs=128), 1),      # token stride below Hkv * d
+    # the balanced and dynamic splits do not take copies (a workspace is given)
+    (dict(ps=-1, ws=256, wsb=1 << 40), {}, 2),
+    (dict(ps=-2, ws=256, wsb=1 << 40), {}, 2),
+    (dict(d=96), {}, 2),                          # the checks of pa_decode apply too
+])
+def test_decode_cow_rejects_before_launch(lib, over, extra, code):
+    assert _call_decode_cow(lib, _decode_args(**over), **extra) == code
+
+
 def test_zero_sized_calls_are_noops(lib):
     P = ctypes.c_void_p
     assert _call_decode(lib, _decode_args(B=0, out=0, q=0)) == 0

@@ -64,6 +64,18 @@ def test_prefix_cow_structure():
     dst = c.copy_pairs[:, 1]
     assert len(set(dst.tolist())) == len(dst) and not set(dst) & set(c.copy_pairs[:, 0])
     assert len(set(c.slot_mapping.tolist())) == len(c.slot_mapping)
+    # the per-sample copy list names the same copies, restricted to the prompt's 8 rows
+    # of block 62 (the slots past them are the ones the step writes)
+    assert c.cow.shape == (24, 3) and c.cow.dtype == np.int32
+    named = {(int(s), int(c.block_tables[i, lb])) for i, (s, lb, r) in enumerate(c.cow)
+             if s >= 0}
+    assert named == {(int(a), int(b)) for a, b in c.copy_pairs}
+    assert np.all(c.cow[c.cow[:, 0] >= 0, 1:] == [62, 1000 - 62 * 16])
+    assert np.all(c.cow[7::8, 0] == -1)  # the sample that keeps the shared block
+    written = {(int(x) // 16, int(x) % 16) for x in c.slot_mapping}
+    for i, (s, lb, r) in enumerate(c.cow):
+        if s >= 0:
+            assert not any((int(c.block_tables[i, lb]), k) in written for k in range(r))
 
 
 def test_prefill_case_structure():

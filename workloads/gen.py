@@ -11,7 +11,9 @@ Layout produced (the library's layout):
 * ``context_lens``: ``int32 [num_seqs]``, counting the token appended in this step.
 * ``key``/``value``: ``uint16 [T, num_kv_heads, head_dim]`` new tokens, ``slot_mapping``:
   ``int64 [T]`` with ``slot = block * block_size + offset``.
-* ``copy_pairs``: ``int64 [P, 2]`` (src, dst) copy-on-write block pairs.
+* ``copy_pairs``: ``int64 [P, 2]`` (src, dst) copy-on-write block pairs; ``cow``:
+  ``int32 [num_seqs, 3]`` the same copies per sequence (source block, logical block
+  index, rows), source ``-1`` for none.
 
 Draw order for a seed: context lengths, the pool permutation, q, K pool, V pool, the
 new tokens' key, value.  Values are N(0, 1) in fp32 rounded to nearest-even; an array
@@ -101,6 +103,10 @@ class DecodeCase:
     value: np.ndarray
     slot_mapping: np.ndarray
     copy_pairs: np.ndarray = field(default_factory=lambda: np.zeros((0, 2), np.int64))
+    # the same copies per sequence, for a decode that does them itself: int32 [B, 3] =
+    # (source block, logical block index, rows to copy), source -1 for none; empty when
+    # the case has no copies
+    cow: np.ndarray = field(default_factory=lambda: np.zeros((0, 3), np.int32))
     seed: int = 0
     window: int = 0  # sliding window the decode uses (0 = whole contexts)
 
@@ -198,7 +204,9 @@ def make_prefix_cow(seed: int = 5, groups: int = 64, samples: int = 8, prefix: i
 
     Each group's prompt of ``prefix`` tokens sits in shared blocks (reference count
     ``samples``); its last block is partially filled.  Samples ``0..samples-2`` get a
-    private copy of that block (``copy_pairs``), the last sample keeps the original.
+    private copy of that block (``copy_pairs``), the last sample keeps the original;
+    ``cow`` names the same copies per sample, restricted to the prompt's rows of the
+    block (the rows past them receive the sample's own tokens in this step).
     Each sample then has ``u ~ U{0..max_suffix}`` suffix tokens plus the new token,
     ``L = prefix + u + 1``.  The step is: copy the pairs, write the tokens that land in
     the (copied) partial block plus the new token, decode.  Suffix tokens that land in
@@ -221,6 +229,8 @@ def make_prefix_cow(seed: int = 5, groups: int = 64, samples: int = 8, prefix: i
     width = int(max(n_shared + f for f in fresh))
     tables = np.full((nseq, width), -1, dtype=np.int32)
     pairs = []
+    cow = np.full((nseq, 3), -1, dtype=np.int32)
+    cow[:, 1:] = 0
     pos = 0
     for g in range(groups):
         shared = perm[pos:pos + n_shared]
@@ -233,6 +243,7 @@ def make_prefix_cow(seed: int = 5, groups: int = 64, samples: int = 8, prefix: i
                 pos += 1
                 tables[s, n_full] = cp
                 pairs.append((int(shared[-1]), int(cp)))
+                cow[s] = (int(shared[-1]), n_full, part_fill)  # the prompt's rows of it
             f = fresh[s]
             tables[s, n_shared:n_shared + f] = perm[pos:pos + f]
             pos += f
@@ -272,7 +283,7 @@ def make_prefix_cow(seed: int = 5, groups: int = 64, samples: int = 8, prefix: i
     return DecodeCase("prefix_cow", dtype, nseq, num_q_heads, num_kv_heads, head_dim, bs, nb,
                       1.0 / math.sqrt(head_dim), lens, tables, q, k_cache, v_cache, key, value,
                       slots, copy_pairs=np.asarray(pairs, dtype=np.int64).reshape(-1, 2),
-                      seed=seed)
+                      cow=cow, seed=seed)
 
 
 @dataclass
