@@ -225,6 +225,7 @@ def test_workspace_plan_invariants(lib, B, G, hkv, d, bs, W, mcl, win, ps):
     else:
         assert ws % 256 == 0 and ws >= B * hq * parts * (d + 2) * 4
     if ps > 0:  # monotone in the hint and the window (the automatic size may switch)
-        assert ws <= pa.decode_workspace_bytes(B, hq, hkv, d, bs, W, mcl + 4096, ps, win)
+        if mcl > 0:  # a hint of 0 means the table's capacity, which may exceed mcl + 4096
+            assert ws <= pa.decode_workspace_bytes(B, hq, hkv, d, bs, W, mcl + 4096, ps, win)
         if win > 0:
             assert ws <= pa.decode_workspace_bytes(B, hq, hkv, d, bs, W, mcl, ps, win + 4096)
