@@ -17,7 +17,9 @@
  *
  * The decode step that uses it:  pa_bm_append_slots (one new token per sequence)
  * -> pa_copy_blocks(pairs) -> pa_kv_write(slot_mapping) -> pa_decode(tables, lens);
- * pa_bm_block_tables fills the table and length arrays for the listed sequences.
+ * or, with the copies done by the decode itself, pa_bm_append_slots_cow ->
+ * pa_decode_cow(tables, lens, copy list, new tokens).  pa_bm_block_tables fills the
+ * table and length arrays for the listed sequences.
  *
  * Not thread-safe: one manager per engine thread.  Operations other than swap-in and
  * free on a swapped-out sequence return PA_ERR_INVALID_ARG.  Sequence ids are caller-chosen
@@ -95,6 +97,19 @@ pa_status pa_bm_free(pa_block_manager *bm, int64_t seq_id);
 pa_status pa_bm_append_slots(pa_block_manager *bm, const int64_t *seq_ids, int n,
                              int64_t *slot_mapping, int64_t *copy_pairs, int max_pairs,
                              int *num_pairs);
+
+/*
+ * pa_bm_append_slots for a decode step that makes its copies itself (pa_decode_cow):
+ * the same reservations, with each private copy reported per sequence instead of as a
+ * pair.  cow, int32 [n][3], receives for sequence i (source block, logical index of
+ * its last block, rows of that block filled before the new token) when its last block
+ * was copied, else (-1, 0, 0) -- pa_decode_cow's copy list, in the order of seq_ids;
+ * *num_copies the number of copies.  The new token goes to the row past the copied
+ * ones, so the copy and the token's cache write touch different rows.  Errors and
+ * all-or-nothing as pa_bm_append_slots.
+ */
+pa_status pa_bm_append_slots_cow(pa_block_manager *bm, const int64_t *seq_ids, int n,
+                                 int64_t *slot_mapping, int32_t *cow, int *num_copies);
 
 /* Slot of token position pos of a sequence (block * bs + offset), -1 if out of range. */
 int64_t pa_bm_slot(const pa_block_manager *bm, int64_t seq_id, int pos);

@@ -25,7 +25,8 @@ EXPORTS = ("pa_kv_write", "pa_copy_blocks", "pa_decode", "pa_decode_workspace_by
            # host block manager (include/pa_block_manager.h)
            "pa_bm_create", "pa_bm_destroy", "pa_bm_blocks_needed", "pa_bm_num_free_blocks",
            "pa_bm_usage_ratio", "pa_bm_can_allocate", "pa_bm_allocate", "pa_bm_fork",
-           "pa_bm_free", "pa_bm_append_slots", "pa_bm_slot", "pa_bm_seq_len",
+           "pa_bm_free", "pa_bm_append_slots", "pa_bm_append_slots_cow", "pa_bm_slot",
+           "pa_bm_seq_len",
            "pa_bm_block_refcount", "pa_bm_block_tables", "pa_bm_set_cpu_pool",
            "pa_bm_num_free_cpu_blocks", "pa_bm_is_swapped", "pa_bm_swap_out", "pa_bm_swap_in",
            "pa_bm_set_sliding_window")

@@ -38,6 +38,8 @@ def _lib():
         lib.pa_bm_free.restype = i32
         lib.pa_bm_append_slots.argtypes = [P, P, i32, P, P, i32, ctypes.POINTER(i32)]
         lib.pa_bm_append_slots.restype = i32
+        lib.pa_bm_append_slots_cow.argtypes = [P, P, i32, P, P, ctypes.POINTER(i32)]
+        lib.pa_bm_append_slots_cow.restype = i32
         lib.pa_bm_slot.argtypes = [P, i64, i32]
         lib.pa_bm_slot.restype = i64
         lib.pa_bm_seq_len.argtypes = [P, i64]
@@ -125,6 +127,20 @@ class BlockManager:
         _check(self._lib.pa_bm_append_slots(self._live(), _p(ids), n, _p(slots), _p(pairs), n,
                                             ctypes.byref(npairs)), "pa_bm_append_slots")
         return slots, pairs[:npairs.value].copy()
+
+    def append_slots_cow(self, seq_ids):
+        """One new token per sequence -> (slot_mapping int64 [n], copy list int32 [n, 3]):
+        the same reservations as append_slots, each private copy given per sequence as
+        (source block, logical block index, rows filled before the token), (-1, 0, 0)
+        where nothing is copied -- the copy list of decode_cow."""
+        ids = np.ascontiguousarray(seq_ids, np.int64)
+        n = ids.shape[0]
+        slots = np.empty(n, np.int64)
+        cow = np.empty((max(n, 1), 3), np.int32)
+        ncopies = ctypes.c_int(0)
+        _check(self._lib.pa_bm_append_slots_cow(self._live(), _p(ids), n, _p(slots), _p(cow),
+                                                ctypes.byref(ncopies)), "pa_bm_append_slots_cow")
+        return slots, cow[:n].copy()
 
     def slot(self, seq_id: int, pos: int) -> int:
         """Slot of token position ``pos``; -1 where the position has no block (past the

@@ -265,12 +265,13 @@ pa_status pa_bm_free(pa_block_manager *bm, int64_t seq_id) {
     return PA_OK;
 }
 
-pa_status pa_bm_append_slots(pa_block_manager *bm, const int64_t *seq_ids, int n,
-                             int64_t *slot_mapping, int64_t *copy_pairs, int max_pairs,
-                             int *num_pairs) {
-    if (!bm || n < 0 || (n > 0 && (!seq_ids || !slot_mapping)) || !num_pairs || max_pairs < 0 ||
-        (max_pairs > 0 && !copy_pairs))
-        return PA_ERR_INVALID_ARG;
+namespace {
+
+// pa_bm_append_slots, reporting each private copy as a pair (copy_pairs) or per sequence
+// (cow: source block, logical index of the copied block, rows filled before the token).
+pa_status append_slots(pa_block_manager *bm, const int64_t *seq_ids, int n,
+                       int64_t *slot_mapping, int64_t *copy_pairs, int max_pairs,
+                       int *num_pairs, int32_t *cow) {
     const int bs = bm->block_size;
     // pass 1: validate and count the fresh blocks the batch needs (without changing
     // anything), following the reference counts as earlier entries of the batch
@@ -334,8 +335,15 @@ pa_status pa_bm_append_slots(pa_block_manager *bm, const int64_t *seq_ids, int n
             blk = s.blocks.back();
             if (bm->refcount[blk] > 1) {
                 const int copy = bm->take();
-                copy_pairs[2 * np] = blk;
-                copy_pairs[2 * np + 1] = copy;
+                if (copy_pairs) {
+                    copy_pairs[2 * np] = blk;
+                    copy_pairs[2 * np + 1] = copy;
+                }
+                if (cow) {
+                    cow[3 * i] = blk;
+                    cow[3 * i + 1] = (int32_t)s.blocks.size() - 1;
+                    cow[3 * i + 2] = off;
+                }
                 ++np;
                 bm->drop(blk);
                 s.blocks.back() = copy;
@@ -350,6 +358,31 @@ pa_status pa_bm_append_slots(pa_block_manager *bm, const int64_t *seq_ids, int n
         for (int i = 0; i < n; ++i) bm->release_before_window(*bm->batch_seqs[i]);
     *num_pairs = np;
     return PA_OK;
+}
+
+}  // namespace
+
+pa_status pa_bm_append_slots(pa_block_manager *bm, const int64_t *seq_ids, int n,
+                             int64_t *slot_mapping, int64_t *copy_pairs, int max_pairs,
+                             int *num_pairs) {
+    if (!bm || n < 0 || (n > 0 && (!seq_ids || !slot_mapping)) || !num_pairs || max_pairs < 0 ||
+        (max_pairs > 0 && !copy_pairs))
+        return PA_ERR_INVALID_ARG;
+    return append_slots(bm, seq_ids, n, slot_mapping, copy_pairs, max_pairs, num_pairs,
+                        nullptr);
+}
+
+pa_status pa_bm_append_slots_cow(pa_block_manager *bm, const int64_t *seq_ids, int n,
+                                 int64_t *slot_mapping, int32_t *cow, int *num_copies) {
+    if (!bm || n < 0 || (n > 0 && (!seq_ids || !slot_mapping || !cow)) || !num_copies)
+        return PA_ERR_INVALID_ARG;
+    for (int i = 0; i < n; ++i) {  // no copy unless pass 2 records one
+        cow[3 * i] = -1;
+        cow[3 * i + 1] = 0;
+        cow[3 * i + 2] = 0;
+    }
+    // at most one copy per listed sequence, so the pair bound never binds
+    return append_slots(bm, seq_ids, n, slot_mapping, nullptr, n, num_copies, cow);
 }
 
 int64_t pa_bm_slot(const pa_block_manager *bm, int64_t seq_id, int pos) {

@@ -34,7 +34,7 @@ int main(void) {
         (any_fn)pa_bm_set_sliding_window, (any_fn)pa_bm_blocks_needed,
         (any_fn)pa_bm_num_free_blocks, (any_fn)pa_bm_usage_ratio, (any_fn)pa_bm_can_allocate,
         (any_fn)pa_bm_allocate, (any_fn)pa_bm_fork, (any_fn)pa_bm_free,
-        (any_fn)pa_bm_append_slots, (any_fn)pa_bm_slot, (any_fn)pa_bm_seq_len,
+        (any_fn)pa_bm_append_slots, (any_fn)pa_bm_append_slots_cow, (any_fn)pa_bm_slot, (any_fn)pa_bm_seq_len,
         (any_fn)pa_bm_block_refcount, (any_fn)pa_bm_set_cpu_pool,
         (any_fn)pa_bm_num_free_cpu_blocks, (any_fn)pa_bm_is_swapped, (any_fn)pa_bm_swap_out,
         (any_fn)pa_bm_swap_in, (any_fn)pa_bm_block_tables};
@@ -66,6 +66,16 @@ int main(void) {
     CHECK(slots[0] == (int64_t)tables[2] * 8 + 4 && slots[1] == (int64_t)tables[6] * 8 + 4);
     CHECK(tables[3] == -1 && tables[7] == -1);
     CHECK(pa_bm_allocate(bm, 3, 1000) == PA_ERR_NO_FREE_BLOCK);
+    /* the same step with the copy reported per sequence, for pa_decode_cow */
+    CHECK(pa_bm_fork(bm, 1, 4) == PA_OK);
+    const int64_t ids2[2] = {4, 1};
+    int32_t cow[2 * 3];
+    int ncopies = -1;
+    CHECK(pa_bm_append_slots_cow(bm, ids2, 2, slots, cow, &ncopies) == PA_OK);
+    CHECK(ncopies == 1);                    /* sequence 4 copies the block it shared */
+    CHECK(cow[0] == tables[2] && cow[1] == 2 && cow[2] == 5);  /* 21 tokens: 5 rows of block 2 */
+    CHECK(cow[3] == -1 && cow[4] == 0 && cow[5] == 0);
+    CHECK(slots[1] == (int64_t)tables[2] * 8 + 5);           /* sequence 1 keeps its block */
     pa_bm_destroy(bm);
 
     /* refusals before any launch (no GPU is touched) */

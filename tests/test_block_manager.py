@@ -178,6 +178,69 @@ def test_parallel_sampling_copy_on_write_counts():
     assert pairs2.shape == (0, 2)
 
 
+@pytest.mark.parametrize("seed,window", [(0, 0), (1, 0), (2, 0), (3, 6), (4, 20)])
+def test_append_slots_cow_reports_the_same_copies_per_sequence(seed, window):
+    """Two managers driven by the same operations, one appending with pairs and one with
+    the per-sequence copy list: the same slots and the same copies; each listed copy names
+    the sequence's last block, the rows filled before the token, and the source the pair
+    names; the token's row is the first one not copied."""
+    rng = np.random.default_rng(seed)
+    nb, bs = int(rng.integers(16, 64)), int(rng.choice([2, 4, 8, 16]))
+    a, b = pa.BlockManager(nb, bs), pa.BlockManager(nb, bs)
+    a.set_sliding_window(window)
+    b.set_sliding_window(window)
+    live, next_id, copies = [], 0, 0
+    for step in range(400):
+        op = rng.choice(["alloc", "fork", "free", "append"], p=[0.2, 0.25, 0.1, 0.45])
+        if op == "alloc":
+            n = int(rng.integers(1, 3 * bs + 2))
+            try:
+                a.allocate(next_id, n)
+            except pa.PAError:
+                with pytest.raises(pa.PAError):
+                    b.allocate(next_id, n)
+            else:
+                b.allocate(next_id, n)
+                live.append(next_id)
+            next_id += 1
+        elif op == "fork" and live:
+            p = int(rng.choice(live))
+            a.fork(p, next_id)
+            b.fork(p, next_id)
+            live.append(next_id)
+            next_id += 1
+        elif op == "free" and live:
+            sid = int(rng.choice(live))
+            a.free(sid)
+            b.free(sid)
+            live.remove(sid)
+        elif op == "append" and live:
+            ids = [int(x) for x in rng.permutation(live)[: int(rng.integers(1, len(live) + 1))]]
+            try:
+                slots, pairs = a.append_slots(ids)
+            except pa.PAError:
+                with pytest.raises(pa.PAError):
+                    b.append_slots_cow(ids)
+                continue
+            slots2, cow = b.append_slots_cow(ids)
+            assert slots2.tolist() == slots.tolist()
+            assert cow.shape == (len(ids), 3) and cow.dtype == np.int32
+            width = max(b.seq_len(i) for i in ids) // bs + 1
+            bt, cl = b.block_tables(ids, width)
+            named = []
+            for i, (src, lb, rows) in enumerate(cow.tolist()):
+                if src < 0:
+                    assert (lb, rows) == (0, 0)
+                    continue
+                L = int(cl[i])
+                assert lb == (L - 1) // bs and rows == (L - 1) % bs and rows > 0
+                assert int(slots[i]) == int(bt[i, lb]) * bs + rows  # the row past the copy
+                named.append((src, int(bt[i, lb])))
+            assert named == [tuple(x) for x in pairs.tolist()]
+            copies += len(named)
+    assert copies > 0
+
+
 @pytest.mark.parametrize("window", [0, 5, 8])
 def test_logical_token_streams_through_tables(window):
     """Drive the oracle's cache write / block copy with the manager through prompts,
