@@ -1,7 +1,9 @@
 """A small serving loop on the GPU driven by the host block manager: prompts, parallel
 samples (forks), decode steps with copy-on-write and cache writes, frees and new
 arrivals.  Every step's attention is compared with the oracle on a host mirror of the
-caches; the device caches must equal the mirror bit for bit."""
+caches; the device caches must equal the mirror bit for bit.  With cow=True the step is
+one call: the manager's per-sequence copy list and the new tokens go to pa_decode_cow,
+which copies, writes and attends."""
 import math
 
 import numpy as np
@@ -44,13 +46,13 @@ def test_swap_blocks_device_and_pinned_host():
     assert pa.device_error(0) == pa.DEVERR["pair"]
 
 
-@pytest.mark.parametrize("hq,hkv,bs,fused,preempt,window", [(16, 4, 16, False, False, 0),
-                                                            (8, 8, 32, True, False, 0),
-                                                            (32, 4, 16, True, False, 0),
-                                                            (16, 2, 16, True, True, 0),
-                                                            (8, 8, 32, False, False, 37),
-                                                            (16, 4, 16, True, True, 100)])
-def test_block_manager_serving_loop(hq, hkv, bs, fused, preempt, window):
+@pytest.mark.parametrize("hq,hkv,bs,fused,preempt,window,cow",
+                         [(16, 4, 16, False, False, 0, False), (8, 8, 32, True, False, 0, False),
+                          (32, 4, 16, True, False, 0, False), (16, 2, 16, True, True, 0, False),
+                          (8, 8, 32, False, False, 37, False),
+                          (16, 4, 16, True, True, 100, False),
+                          (16, 4, 16, True, False, 0, True), (8, 8, 32, True, True, 37, True)])
+def test_block_manager_serving_loop(hq, hkv, bs, fused, preempt, window, cow):
     rng = np.random.default_rng(hq * 100 + bs + window)
     nb, d, width, ncpu = 700, 128, 64, 300
     scale = 1 / math.sqrt(d)
@@ -111,17 +113,34 @@ def test_block_manager_serving_loop(hq, hkv, bs, fused, preempt, window):
         if step % 4 == 3:  # one request ends, one arrives
             bm.free(live.pop(int(rng.integers(0, len(live)))))
             new_prompt()
-        slots, pairs = bm.append_slots(live)
+        if cow:
+            slots, cowl = bm.append_slots_cow(live)
+            pairs = np.zeros((0, 2), np.int64)
+        else:
+            slots, pairs = bm.append_slots(live)
         if pairs.shape[0]:
             oracle.copy_blocks(kc_h, vc_h, pairs)
             pa.copy_blocks(kc, vc, dev(pairs))
         key = _rand_bits(rng, (len(live), hkv, d))
         val = _rand_bits(rng, (len(live), hkv, d))
-        oracle.kv_write(key, val, slots, kc_h, vc_h)
         bt, cl = bm.block_tables(live, width)
+        if cow:  # the mirror: the oracle's block copy of the listed rows, then the write
+            for i, (src, lb, nrows) in enumerate(cowl.tolist()):
+                if src >= 0:
+                    dst = int(bt[i, lb])
+                    k2, v2 = kc_h.copy(), vc_h.copy()
+                    oracle.copy_blocks(k2, v2, np.array([[src, dst]], np.int64))
+                    kc_h[dst, :, :nrows], vc_h[dst, :, :nrows] = (k2[dst, :, :nrows],
+                                                                  v2[dst, :, :nrows])
+        oracle.kv_write(key, val, slots, kc_h, vc_h)
         q = _rand_bits(rng, (len(live), hq, d))
         out = torch.empty(len(live), hq, d, dtype=torch.bfloat16, device="cuda")
-        if fused:  # cache write fused into the decode
+        if cow:  # copies, cache write and attention in one call
+            pa.decode_cow(out, dev16(q, "bf16"), kc, vc, dev(bt), dev(cl), dev(cowl), scale,
+                          key=dev16(key, "bf16"), value=dev16(val, "bf16"),
+                          max_context_len=int(cl.max()), partition_size=128,
+                          sliding_window=window)
+        elif fused:  # cache write fused into the decode
             pa.decode_append(out, dev16(q, "bf16"), dev16(key, "bf16"), dev16(val, "bf16"), kc,
                              vc, dev(bt), dev(cl), scale, max_context_len=int(cl.max()),
                              sliding_window=window)
