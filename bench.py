@@ -2,7 +2,9 @@
 
 A step = (copy-on-write block copies when the workload has them) + the cache write
 of the step's new tokens + paged decode attention, on seeded synthetic inputs that
-are resident in HBM.  Default workload: the Llama-2-7B-shaped decode step (64
+are resident in HBM.  The copies are done by the decode's own CTAs (pa_decode_cow;
+`--cow separate`: a pa_copy_blocks launch before the step), and such workloads' lines
+carry `cow_compare`, both forms timed alternately in the same run.  Default workload: the Llama-2-7B-shaped decode step (64
 sequences, 32 q heads = 32 kv heads, head_dim 128, block size 16, bf16, context
 lengths uniform in [128, 2048], shuffled physical blocks).
 
