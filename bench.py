@@ -2,7 +2,9 @@
 
 A step = (copy-on-write block copies when the workload has them) + the cache write
 of the step's new tokens + paged decode attention, on seeded synthetic inputs that
-are resident in HBM.  The copies are done by the decode's own CTAs (pa_decode_cow;
+are resident in HBM.  The decode is launched over the (sequence, partition) units that
+exist, planned from the host's copy of the lengths (pa_decode_planned; `--no-plan`: the
+full grid).  The copies are done by the decode's own CTAs (pa_decode_cow;
 `--cow separate`: a pa_copy_blocks launch before the step), and such workloads' lines
 carry `cow_compare`, both forms timed alternately in the same run.  Default workload: the Llama-2-7B-shaped decode step (64
 sequences, 32 q heads = 32 kv heads, head_dim 128, block size 16, bf16, context
@@ -337,7 +339,7 @@ class DecodeStep:
     copied; copies are done by the decode's own CTAs (pa_decode_cow, cow="folded") or by
     a pa_copy_blocks launch before the write (cow="separate")."""
 
-    def __init__(self, torch, pa, case, device, partition_size, cow="folded"):
+    def __init__(self, torch, pa, case, device, partition_size, cow="folded", plan=True):
         self.case, self.pa = case, pa
         dt = case.dtype
 
@@ -370,6 +372,9 @@ class DecodeStep:
         self.cow = di(case.cow) if self.cow_folded else None
         self.fused = ((not self.has_pairs) and case.key.shape[0] == case.num_seqs
                       and partition_size >= 0)
+        # launch planned from the host's copy of the lengths (fixed split, no window)
+        self.plan = plan and partition_size >= 0 and case.window == 0 and not self.cow_folded
+        self.host_lens = np.ascontiguousarray(case.context_lens, np.int32)
         decode_launches = 1 if nparts == 1 else 2
         self.launches_per_step = decode_launches + (
             0 if self.fused else 1 + (1 if self.has_pairs and not self.cow_folded else 0))
@@ -377,7 +382,12 @@ class DecodeStep:
                       "dynamic: persistent CTAs claim 32-token chunks + LSE merge"
                       if partition_size == -2 else
                       "balanced over persistent warps (stream-K) + LSE merge")
-        self.kind = ("pa_decode_append (cache write fused into decode)" if self.fused
+        self.kind = ("pa_decode_planned (cache write fused into decode; units planned from "
+                     "the host lengths when that leaves out >= 30% of the grid)"
+                     if self.plan and self.fused
+                     else "pa_kv_write + pa_decode_planned" if self.plan and not self.has_pairs
+                     else "pa_copy_blocks + pa_kv_write + pa_decode_planned" if self.plan
+                     else "pa_decode_append (cache write fused into decode)" if self.fused
                      else "pa_kv_write + pa_decode_cow (copy-on-write rows copied by the "
                           "partition pass)" if self.cow_folded
                      else "pa_copy_blocks + pa_kv_write + pa_decode" if self.has_pairs
@@ -392,7 +402,13 @@ class DecodeStep:
         b = b or {}
         out, q = b.get("out", self.out), b.get("q", self.q)
         bt, cl = b.get("bt", self.bt), b.get("cl", self.cl)
-        if self.fused:
+        if self.plan:
+            kv = (dict(key=b.get("key", self.key), value=b.get("val", self.val)) if self.fused
+                  else {})
+            pa.decode_planned(out, q, self.kc, self.vc, bt, cl, self.host_lens, c.scale,
+                              max_context_len=c.max_context_len, partition_size=self.ps,
+                              workspace=self.workspace, **kv)
+        elif self.fused:
             pa.decode_append(out, q, b.get("key", self.key), b.get("val", self.val), self.kc,
                              self.vc, bt, cl, c.scale, max_context_len=c.max_context_len,
                              partition_size=self.ps, workspace=self.workspace,
@@ -469,7 +485,7 @@ def measure_config(torch, pa, name, device, stream, args, peak, flush):
     wname, kw, desc = WORKLOADS[name]
     from workloads import make_config
     case = make_config(wname, poison=False, **kw)
-    ds = DecodeStep(torch, pa, case, device, args.partition_size)
+    ds = DecodeStep(torch, pa, case, device, args.partition_size, plan=not args.no_plan)
     for _ in range(args.warmup):
         ds.step()
     torch.cuda.synchronize()
@@ -524,7 +540,8 @@ def run_ours(args):
         desc = f"{desc} [profiling subset: first {args.seqs} seqs' distribution]"
     case = make_config(name, poison=False, **kw)
     dt = case.dtype
-    ds = DecodeStep(torch, pa, case, device, args.partition_size, cow=args.cow)
+    ds = DecodeStep(torch, pa, case, device, args.partition_size, cow=args.cow,
+                    plan=not args.no_plan)
     q, out = ds.q, ds.out
     stream = torch.cuda.current_stream()
 
@@ -747,7 +764,10 @@ def run_ours(args):
                          "peak_kind": f"{peak_kind} HBM copy GB/s (burst)",
                          "unit": "GB/s", "frac": round(achieved / peak, 4),
                          "frac_l2_flushed": round(achieved_flushed / peak, 4),
-                         "kernel": ("pa_decode_append (cache write fused into the partition "
+                         "kernel": ("pa_decode_planned (the partition pass over the planned "
+                                    "units, cache write fused in) + LSE merge"
+                                    if ds.plan and ds.fused else
+                                    "pa_decode_append (cache write fused into the partition "
                                     "pass) + LSE merge" if ds.fused else
                                     "pa_decode (partition pass + LSE merge when split)"),
                          "achieved_how": (f"algorithmic bytes / median per-call CUDA-event time "
@@ -1329,6 +1349,9 @@ def main(argv=None):
     ap.add_argument("--cow", choices=["folded", "separate"], default="folded",
                     help="workloads with copy-on-write: copies done by the decode's own CTAs "
                          "(pa_decode_cow) or by a pa_copy_blocks launch before the step")
+    ap.add_argument("--no-plan", action="store_true",
+                    help="launch the full (sequence, partition) grid instead of the units "
+                         "planned from the host's copy of the context lengths")
     ap.add_argument("--swap-seqs", type=int, default=8,
                     help="swap: number of sequences preempted and restored per step")
     args = ap.parse_args(argv)

@@ -234,6 +234,36 @@ pa_status pa_decode_append(void *out, const void *q, const void *key, const void
                            size_t workspace_bytes, pa_dtype dtype, void *stream);
 
 /*
+ * pa_decode (with key and value: pa_decode_append) for a caller that also holds the
+ * context lengths on the host, as a serving engine's scheduler does.  The launch is
+ * planned from them: only the (sequence, partition) units that exist are launched --
+ * under the fixed split a context of L tokens has ceil(L / partition) of them, where the
+ * full grid holds the longest context's count for every sequence -- and they are taken
+ * longest first: every full partition, then the shorter last partitions by decreasing
+ * length.  The results are bit-identical to pa_decode / pa_decode_append.
+ *
+ * host_context_lens : int32 [num_seqs], host memory, read during the call only; it must
+ *                     hold the values of context_lens.  A context whose device length
+ *                     needs another partition count than the plan sets
+ *                     PA_DEVERR_CONTEXT (a partition the plan left out is not computed).
+ * key, value        : both NULL (no cache write) or both given, as pa_decode_append.
+ * The plan applies to the fixed split without a sliding window, with at most
+ * 4096 units and 255 partitions per context, when it leaves out at least 30% of the full
+ * grid's (sequence, partition) rows (with fewer empty rows the full grid's own order was
+ * faster on B200); other calls run as pa_decode / pa_decode_append.  Other arguments,
+ * errors and the workspace as pa_decode.
+ */
+pa_status pa_decode_planned(void *out, const void *q, const void *key, const void *value,
+                            int64_t key_token_stride, int64_t value_token_stride,
+                            void *k_cache, void *v_cache, const int32_t *block_tables,
+                            const int32_t *context_lens, const int32_t *host_context_lens,
+                            int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                            int block_size, int num_blocks, int max_blocks_per_seq, float scale,
+                            int max_context_len, int sliding_window, int partition_size,
+                            void *workspace, size_t workspace_bytes, pa_dtype dtype,
+                            void *stream);
+
+/*
  * One decode step with the copy-on-write of a shared block folded into the attention
  * pass (the pages let several requests share KV blocks -- "PagedAttention" summary,
  * features 2 -- so a sequence that appends into a shared, partially filled block

@@ -13,6 +13,8 @@ The compute lives in ``libpa.so`` (CUDA kernels behind the C ABI in
   write fused into the decode;
 * ``decode_cow(out, q, k_cache, v_cache, block_tables, context_lens, cow, scale, ...)``
   -- each sequence's copy-on-write of a shared block folded into the decode;
+* ``decode_planned(..., host_context_lens, scale, key=None, value=None, ...)`` -- decode
+  launched from a host-side plan of the partitions that exist, longest first;
 * ``prefill(out, q, k_cache, v_cache, block_tables, context_lens, query_start_loc,
   scale)`` -- causal multi-query attention for prompts and prompt chunks (tcgen05);
 * ``swap_blocks(...)`` -- block copies between the GPU cache and a pinned host pool;
@@ -33,6 +35,7 @@ from ._lib import (  # noqa: F401
     decode,
     decode_append,
     decode_cow,
+    decode_planned,
     decode_static_scratch,
     decode_partition_tokens,
     decode_workspace_bytes,

@@ -12,6 +12,8 @@ from __future__ import annotations
 import ctypes
 import os
 
+import numpy as np
+
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libpa.so")
 
@@ -20,7 +22,8 @@ DEVERR = {"block_id": 0x1, "slot": 0x2, "pair": 0x4, "context": 0x8, "timeout": 
           "workspace": 0x20}
 EXPORTS = ("pa_kv_write", "pa_copy_blocks", "pa_decode", "pa_decode_workspace_bytes",
            "pa_decode_partition_tokens", "pa_get_device_error", "pa_status_str", "pa_version",
-           "pa_decode_static_scratch", "pa_decode_append", "pa_decode_cow", "pa_swap_blocks",
+           "pa_decode_static_scratch", "pa_decode_append", "pa_decode_cow", "pa_decode_planned",
+           "pa_swap_blocks",
            "pa_prefill",
            # host block manager (include/pa_block_manager.h)
            "pa_bm_create", "pa_bm_destroy", "pa_bm_blocks_needed", "pa_bm_num_free_blocks",
@@ -75,6 +78,9 @@ def load(path: str = LIB_PATH):
     lib.pa_decode_cow.argtypes = [P, P, P, P, i64, i64, P, P, P, P, P, i32, i32, i32, i32, i32,
                                   i32, i32, f32, i32, i32, i32, P, sz, i32, P]
     lib.pa_decode_cow.restype = i32
+    lib.pa_decode_planned.argtypes = [P, P, P, P, i64, i64, P, P, P, P, P, i32, i32, i32, i32,
+                                      i32, i32, i32, f32, i32, i32, i32, P, sz, i32, P]
+    lib.pa_decode_planned.restype = i32
     lib.pa_prefill.argtypes = [P, P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, i32, i32, f32,
                                i32, i32, P]
     lib.pa_prefill.restype = i32
@@ -381,6 +387,47 @@ def decode_cow(out, q, k_cache, v_cache, block_tables, context_lens, cow, scale,
             _ptr(out), _ptr(q), _ptr(key), _ptr(value), key.stride(0) if key is not None else 0, value.stride(0) if value is not None else 0,
             _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), _ptr(context_lens), _ptr(cow), B,
             hq, hkv, d, bs, nb, W, float(scale), int(max_context_len), int(sliding_window),
+            int(partition_size), wptr, wbytes, _dtype(q), _stream(stream, dev)), what)
+
+
+def decode_planned(out, q, k_cache, v_cache, block_tables, context_lens, host_context_lens,
+                   scale, key=None, value=None, max_context_len=0, partition_size=0,
+                   workspace=None, stream=None, sliding_window=0) -> None:
+    """``decode`` (with key/value: ``decode_append``) launched from a host-side plan:
+    host_context_lens, an int32 host array (numpy or CPU tensor) with the values of
+    context_lens, gives the units that exist, taken longest first."""
+    import torch
+    what = "pa_decode_planned"
+    B, hq, d, nb, hkv, bs, W = _decode_shapes(what, out, q, k_cache, v_cache, block_tables,
+                                              context_lens, None)
+    if (key is None) != (value is None):
+        _fail(what, "key and value must be given together")
+    hl = host_context_lens
+    if isinstance(hl, torch.Tensor):
+        if hl.device.type != "cpu":
+            _fail(what, "host_context_lens must be in host memory")
+        hl = hl.numpy()
+    hl = np.ascontiguousarray(hl)
+    if hl.dtype != np.int32 or hl.shape != (B,):
+        _fail(what, f"host_context_lens must be int32 [{B}], got {hl.dtype} {hl.shape}")
+    rows = {}
+    if key is not None:
+        if not (tuple(key.shape) == (B, hkv, d) and tuple(value.shape) == (B, hkv, d)):
+            _fail(what, f"key {tuple(key.shape)} and value {tuple(value.shape)} must both be "
+                  f"[{B}, {hkv}, {d}]")
+        rows = {"key": key, "value": value}
+    dev = _args(what, {"q": q, "out": out, "k_cache": k_cache, "v_cache": v_cache}, rows=rows,
+                ints={"block_tables": (block_tables, torch.int32),
+                      "context_lens": (context_lens, torch.int32)})
+    with _on(dev):
+        need = decode_workspace_bytes(B, hq, hkv, d, bs, W, max_context_len, partition_size,
+                                      sliding_window)
+        wptr, wbytes = _workspace(what, workspace, need, dev)
+        _check(load().pa_decode_planned(
+            _ptr(out), _ptr(q), _ptr(key), _ptr(value), key.stride(0) if key is not None else 0,
+            value.stride(0) if value is not None else 0, _ptr(k_cache), _ptr(v_cache),
+            _ptr(block_tables), _ptr(context_lens), hl.ctypes.data_as(ctypes.c_void_p), B, hq,
+            hkv, d, bs, nb, W, float(scale), int(max_context_len), int(sliding_window),
             int(partition_size), wptr, wbytes, _dtype(q), _stream(stream, dev)), what)
 
 

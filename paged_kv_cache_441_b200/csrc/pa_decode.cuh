@@ -35,6 +35,8 @@
 // (m is kept in the log2 domain: scores are pre-multiplied by scale * log2(e)).
 #pragma once
 
+#include <type_traits>
+
 #include "pa_common.cuh"
 
 namespace pa {
@@ -89,6 +91,20 @@ struct DecodeParams {
     // Source < 0: no copy for that sequence.  nullptr = no copies at all.
     const int32_t *cow;
 };
+
+// A launch planned on the host (pa_decode_planned): the (sequence, partition) units that
+// exist, in the order the CTAs should take them, carried in the kernel's parameter space.
+// Unit = sequence << 16 | partition << 8 | the sequence's partition count.
+constexpr int kPlanMaxUnits = 4096;
+constexpr int kPlanMaxParts = 255;
+struct PlannedParams {
+    DecodeParams base;
+    uint32_t units[kPlanMaxUnits];
+};
+__device__ __forceinline__ const DecodeParams &param_base(const DecodeParams &p) { return p; }
+__device__ __forceinline__ const DecodeParams &param_base(const PlannedParams &p) {
+    return p.base;
+}
 
 template <int D>
 struct Geom {
@@ -600,9 +616,13 @@ __device__ __forceinline__ void cow_rows(const DecodeParams &p, int src, int dst
 // WIN: compiled with sliding-window support (p.sliding_window > 0); the instances
 // without it keep the whole-context path free of the window's bookkeeping.  COW: compiled
 // with the copy-on-write of p.cow, so that calls without copies run code without it.
-template <typename T, int D, int G, int BOXR, bool WIN, bool COW = false>
+// PLAN: the grid is (kv head, unit) over a host-planned unit list (PlannedParams).
+template <typename T, int D, int G, int BOXR, bool WIN, bool COW = false, bool PLAN = false>
 __global__ void __launch_bounds__(kWarps * 32)
-    pa_decode_partition_kernel(const __grid_constant__ DecodeParams p) {
+    pa_decode_partition_kernel(
+        const __grid_constant__ typename std::conditional<PLAN, PlannedParams, DecodeParams>::type
+            pp) {
+    const DecodeParams &p = param_base(pp);
     pdl_wait_and_release();
     using Gm = Geom<D>;
     extern __shared__ uint8_t smem_raw[];
@@ -617,11 +637,19 @@ __global__ void __launch_bounds__(kWarps * 32)
     // CTAs scheduled together read neighbouring heads of the same physical blocks.  With
     // p.sort_second the second partitions are moreover taken longest first.
     const int g = blockIdx.x;
-    int s = blockIdx.y;
-    const int part = blockIdx.z;
-    if (p.sort_second && part == 1) {
-        s = second_partition_seq<WIN>(p, (int)blockIdx.y, (int)gridDim.y);
-        if (s < 0) return;
+    int s, part, planned_parts = 0;
+    if constexpr (PLAN) {
+        const uint32_t u = pp.units[blockIdx.y];
+        s = (int)(u >> 16);
+        part = (int)((u >> 8) & 0xffu);
+        planned_parts = (int)(u & 0xffu);
+    } else {
+        s = blockIdx.y;
+        part = blockIdx.z;
+        if (p.sort_second && part == 1) {
+            s = second_partition_seq<WIN>(p, (int)blockIdx.y, (int)gridDim.y);
+            if (s < 0) return;
+        }
     }
     const int Hq = p.num_q_heads;
 
@@ -657,6 +685,10 @@ __global__ void __launch_bounds__(kWarps * 32)
     const int wlo = WIN ? window_lo(L, W) : 0, span0 = WIN ? span_begin(L, W) : 0;
     const int nparts = (L - span0 + P - 1) / P;
     if (nparts > p.num_parts && tid == 0 && part == 0) raise_error(PA_DEVERR_CONTEXT);
+    // a plan made from host lengths that disagree with the device's: flagged (a partition
+    // the plan left out is not computed)
+    if (PLAN && part == 0 && tid == 0 && max(nparts, 1) != planned_parts)
+        raise_error(PA_DEVERR_CONTEXT);
     // Copy-on-write: every row of the copied block goes to the CTA whose partition holds
     // its position (rows before the first partition to the first, rows past the last to
     // the last), so the CTA that reads a row copies it.  This CTA's share: rows [cr0, cr1).

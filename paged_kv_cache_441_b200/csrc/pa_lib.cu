@@ -2,6 +2,7 @@
 // include/pa.h.  One translation unit, so the device error word has one definition.
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 #include <cstring>
@@ -261,6 +262,83 @@ cudaError_t launch_partition(const DecodeParams &p, dim3 grid, cudaStream_t st, 
     cudaError_t e = ensure_smem(kernel, Geom<D>::kSmem, flags, dev);
     if (e != cudaSuccess) return e;
     return launch_pdl(kernel, grid, dim3(kWarps * 32), Geom<D>::kSmem, st, p);
+}
+
+// A host-planned launch: grid (kv heads, units), the unit list in the parameters.
+template <typename T, int D, int G, int BOXR>
+cudaError_t launch_planned(const PlannedParams &pp, int units, cudaStream_t st, int dev) {
+    static std::atomic<bool> flags[kMaxDevices];
+    auto kernel = pa_decode_partition_kernel<T, D, G, BOXR, false, false, true>;
+    cudaError_t e = ensure_smem(kernel, Geom<D>::kSmem, flags, dev);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(kernel, dim3((unsigned)pp.base.num_kv_heads, (unsigned)units),
+                      dim3(kWarps * 32), Geom<D>::kSmem, st, pp);
+}
+
+template <typename T, int D>
+cudaError_t planned_group(const PlannedParams &pp, int units, cudaStream_t st, int dev, int G,
+                          int boxr) {
+    switch (G) {
+        case 1: return boxr == 8 ? launch_planned<T, D, 1, 8>(pp, units, st, dev)
+                                 : launch_planned<T, D, 1, 16>(pp, units, st, dev);
+        case 2: return boxr == 8 ? launch_planned<T, D, 2, 8>(pp, units, st, dev)
+                                 : launch_planned<T, D, 2, 16>(pp, units, st, dev);
+        case 4: return boxr == 8 ? launch_planned<T, D, 4, 8>(pp, units, st, dev)
+                                 : launch_planned<T, D, 4, 16>(pp, units, st, dev);
+        case 8: return boxr == 8 ? launch_planned<T, D, 8, 8>(pp, units, st, dev)
+                                 : launch_planned<T, D, 8, 16>(pp, units, st, dev);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+template <typename T>
+cudaError_t planned_dispatch(const PlannedParams &pp, int units, cudaStream_t st, int dev, int D,
+                             int G, int boxr) {
+    return D == 64 ? planned_group<T, 64>(pp, units, st, dev, G, boxr)
+                   : planned_group<T, 128>(pp, units, st, dev, G, boxr);
+}
+
+// The (sequence, partition) units of a fixed-split launch from host copies of the context
+// lengths, longest first: every full partition (partition-major, so CTAs scheduled together
+// read neighbouring heads of the same blocks), then the shorter last partitions by
+// decreasing length.  Returns the unit count, or -1 when the plan does not fit (the caller
+// then launches the full grid).
+int plan_units(const int32_t *lens, int num_seqs, long long cap, int P, int num_parts,
+               uint32_t *units) {
+    if (num_parts > kPlanMaxParts || num_seqs > 65535) return -1;
+    long long total = 0;
+    for (int s = 0; s < num_seqs; ++s) {
+        long long L = lens[s] < 0 ? 0 : (lens[s] > cap ? cap : lens[s]);
+        long long n = L == 0 ? 1 : (L + P - 1) / P;
+        total += n < num_parts ? n : num_parts;
+    }
+    if (total > kPlanMaxUnits) return -1;
+    int k = 0;
+    for (int part = 0; part < num_parts; ++part)
+        for (int s = 0; s < num_seqs; ++s) {
+            const long long L = lens[s] < 0 ? 0 : (lens[s] > cap ? cap : lens[s]);
+            const long long n = L == 0 ? 1 : (L + P - 1) / P;
+            const int np = (int)(n < num_parts ? n : num_parts);
+            if (part < np && (long long)(part + 1) * P <= L)
+                units[k++] = ((uint32_t)s << 16) | ((uint32_t)part << 8) | (uint32_t)np;
+        }
+    const int full = k;
+    for (int s = 0; s < num_seqs; ++s) {  // the last, shorter partition of each context
+        const long long L = lens[s] < 0 ? 0 : (lens[s] > cap ? cap : lens[s]);
+        const long long n = L == 0 ? 1 : (L + P - 1) / P;
+        const int np = (int)(n < num_parts ? n : num_parts);
+        const int last = np - 1;
+        if ((long long)(last + 1) * P > L)
+            units[k++] = ((uint32_t)s << 16) | ((uint32_t)last << 8) | (uint32_t)np;
+    }
+    auto rem = [&](uint32_t u) {
+        const int s = (int)(u >> 16);
+        const long long L = lens[s] < 0 ? 0 : (lens[s] > cap ? cap : lens[s]);
+        return L - (long long)((u >> 8) & 0xffu) * P;
+    };
+    std::stable_sort(units + full, units + k,
+                     [&](uint32_t a, uint32_t b) { return rem(a) > rem(b); });
+    return k;
 }
 
 template <typename T, int D>
@@ -653,7 +731,7 @@ pa_status decode_impl(void *out, const void *q, const void *k_cache, const void 
                       int sliding_window, int partition_size, void *workspace,
                       size_t workspace_bytes, pa_dtype dtype, void *stream, const void *new_k,
                       const void *new_v, long long new_k_stride, long long new_v_stride,
-                      const int32_t *cow = nullptr) {
+                      const int32_t *cow = nullptr, const int32_t *host_lens = nullptr) {
     if (dtype != PA_FP16 && dtype != PA_BF16) return PA_ERR_INVALID_ARG;
     pa_status st = check_decode_shape(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
                                       num_blocks, max_blocks_per_seq, max_context_len,
@@ -822,10 +900,31 @@ pa_status decode_impl(void *out, const void *q, const void *k_cache, const void 
     p.cow = cow;
 
     if (pl.num_parts > 65535) return PA_ERR_UNSUPPORTED;  // use a larger partition_size
-    dim3 grid((unsigned)num_kv_heads, (unsigned)num_seqs, (unsigned)pl.num_parts);
-    cudaError_t e = dtype == PA_BF16
-                        ? dispatch_dim<__nv_bfloat16>(p, grid, st_, dev, head_dim, G, boxr)
-                        : dispatch_dim<__half>(p, grid, st_, dev, head_dim, G, boxr);
+    cudaError_t e = cudaSuccess;
+    bool launched = false;
+    if (host_lens != nullptr && sliding_window == 0 && cow == nullptr) {
+        // the units that exist, longest first, from the host's copy of the lengths
+        PlannedParams pp;
+        const int units =
+            plan_units(host_lens, num_seqs, (long long)max_blocks_per_seq * block_size,
+                       pl.partition_tokens, pl.num_parts, pp.units);
+        // planned only when it leaves out at least 30% of the full grid's rows (A/B on
+        // B200: GQA, 20% of the rows real, -5%; long 8/1, 61%, -1 to -2%; Llama-2, 75%,
+        // +2% -- there the full grid's own order, second partitions longest first, wins)
+        if (units > 0 && (long long)units * 10 <= 7LL * num_seqs * pl.num_parts) {
+            pp.base = p;
+            pp.base.sort_second = 0;
+            e = dtype == PA_BF16
+                    ? planned_dispatch<__nv_bfloat16>(pp, units, st_, dev, head_dim, G, boxr)
+                    : planned_dispatch<__half>(pp, units, st_, dev, head_dim, G, boxr);
+            launched = true;
+        }
+    }
+    if (!launched) {
+        dim3 grid((unsigned)num_kv_heads, (unsigned)num_seqs, (unsigned)pl.num_parts);
+        e = dtype == PA_BF16 ? dispatch_dim<__nv_bfloat16>(p, grid, st_, dev, head_dim, G, boxr)
+                             : dispatch_dim<__half>(p, grid, st_, dev, head_dim, G, boxr);
+    }
     if (e != cudaSuccess) return PA_ERR_CUDA;
     if (pl.num_parts > 1) {
         MergeParams mp;
@@ -888,6 +987,34 @@ pa_status pa_decode_append(void *out, const void *q, const void *key, const void
                        max_blocks_per_seq, scale, max_context_len, sliding_window,
                        partition_size, workspace, workspace_bytes, dtype, stream, key, value,
                        key_token_stride, value_token_stride);
+}
+
+pa_status pa_decode_planned(void *out, const void *q, const void *key, const void *value,
+                            int64_t key_token_stride, int64_t value_token_stride,
+                            void *k_cache, void *v_cache, const int32_t *block_tables,
+                            const int32_t *context_lens, const int32_t *host_context_lens,
+                            int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                            int block_size, int num_blocks, int max_blocks_per_seq, float scale,
+                            int max_context_len, int sliding_window, int partition_size,
+                            void *workspace, size_t workspace_bytes, pa_dtype dtype,
+                            void *stream) {
+    if (num_seqs > 0) {
+        if (!host_context_lens) return PA_ERR_INVALID_ARG;
+        if ((key == nullptr) != (value == nullptr)) return PA_ERR_INVALID_ARG;
+        if (key != nullptr) {
+            if (!aligned(key, 16) || !aligned(value, 16)) return PA_ERR_INVALID_ARG;
+            if (key_token_stride % 8 != 0 || value_token_stride % 8 != 0 ||
+                key_token_stride < (int64_t)num_kv_heads * head_dim ||
+                value_token_stride < (int64_t)num_kv_heads * head_dim)
+                return PA_ERR_INVALID_ARG;
+        }
+    }
+    return decode_impl(out, q, k_cache, v_cache, block_tables, context_lens, num_seqs,
+                       num_q_heads, num_kv_heads, head_dim, block_size, num_blocks,
+                       max_blocks_per_seq, scale, max_context_len, sliding_window,
+                       partition_size, workspace, workspace_bytes, dtype, stream, key, value,
+                       key != nullptr ? key_token_stride : 0,
+                       value != nullptr ? value_token_stride : 0, nullptr, host_context_lens);
 }
 
 pa_status pa_decode_cow(void *out, const void *q, const void *key, const void *value,

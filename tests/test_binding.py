@@ -9,6 +9,7 @@ from __future__ import annotations
 
 import types
 
+import numpy as np
 import pytest
 import torch
 
@@ -149,6 +150,28 @@ def test_decode_cow_marshalling(fake):
     with pytest.raises(_lib.PAError, match="int32"):
         _lib.decode_cow(a["out"], a["q"], a["k_cache"], a["v_cache"], a["block_tables"],
                         a["context_lens"], cow.long(), 0.2, stream=STREAM)
+
+
+def test_decode_planned_marshalling(fake):
+    a = _decode_args()
+    hl = np.array([3, 40, 17], np.int32)
+    _lib.decode_planned(a["out"], a["q"], a["k_cache"], a["v_cache"], a["block_tables"],
+                        a["context_lens"], hl, 0.2, stream=STREAM)
+    args = [_v(x) for x in fake.last("pa_decode_planned")]
+    assert args[2] is None and args[3] is None and args[4:6] == [0, 0]
+    assert args[10] == hl.ctypes.data and args[11:18] == [3, 8, 2, 64, 16, 10, 5]
+    key = torch.zeros(3, 2, 64, dtype=torch.bfloat16)
+    _lib.decode_planned(a["out"], a["q"], a["k_cache"], a["v_cache"], a["block_tables"],
+                        a["context_lens"], torch.from_numpy(hl), 0.2, key=key,
+                        value=torch.zeros_like(key), stream=STREAM)
+    args = [_v(x) for x in fake.last("pa_decode_planned")]
+    assert args[2] == key.data_ptr() and args[4:6] == [2 * 64, 2 * 64]
+    with pytest.raises(_lib.PAError, match="int32"):
+        _lib.decode_planned(a["out"], a["q"], a["k_cache"], a["v_cache"], a["block_tables"],
+                            a["context_lens"], hl.astype(np.int64), 0.2, stream=STREAM)
+    with pytest.raises(_lib.PAError, match="together"):
+        _lib.decode_planned(a["out"], a["q"], a["k_cache"], a["v_cache"], a["block_tables"],
+                            a["context_lens"], hl, 0.2, value=key, stream=STREAM)
 
 
 def test_swap_blocks_host_and_device_pools(fake):

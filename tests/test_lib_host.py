@@ -145,6 +145,28 @@ def test_decode_cow_rejects_before_launch(lib, over, extra, code):
     assert _call_decode_cow(lib, _decode_args(**over), **extra) == code
 
 
+def test_decode_planned_rejects_before_launch(lib):
+    a = _decode_args()
+    P = ctypes.c_void_p
+    host = (ctypes.c_int32 * 2)(10, 20)
+
+    def call(key=None, value=None, hl=host, ks=256, vs=256, **over):
+        b = dict(a, **over)
+        return lib.pa_decode_planned(P(b["out"]), P(b["q"]), P(key) if key else None,
+                                     P(value) if value else None, ks, vs, P(b["kc"]),
+                                     P(b["vc"]), P(b["bt"]), P(b["cl"]),
+                                     ctypes.cast(hl, P) if hl is not None else None, b["B"],
+                                     b["hq"], b["hkv"], b["d"], b["bs"], b["nb"], b["W"],
+                                     b["scale"], b["mcl"], b["win"], b["ps"], b["ws"], b["wsb"],
+                                     b["dt"], b["stream"])
+    assert call(hl=None) == 1              # no host lengths
+    assert call(key=16) == 1               # key without value
+    assert call(key=8, value=16) == 1      # misaligned key
+    assert call(key=16, value=16, ks=100) == 1
+    assert call(d=96) == 2                 # the checks of pa_decode apply too
+    assert call(hl=None, B=0, out=0, q=0) == 0  # nothing to do
+
+
 def test_zero_sized_calls_are_noops(lib):
     P = ctypes.c_void_p
     assert _call_decode(lib, _decode_args(B=0, out=0, q=0)) == 0
