@@ -264,6 +264,20 @@ pa_status pa_decode_planned(void *out, const void *q, const void *key, const voi
                             void *stream);
 
 /*
+ * The launch pa_decode_planned would make for these arguments, host-side (no device
+ * work; the SM count is read as pa_decode_workspace_bytes reads it): returns the number
+ * of (sequence, partition) units it launches -- 0 when it launches the full grid -- and
+ * writes the first min(that, max_units) of them to units in launch order, each
+ * sequence << 16 | partition << 8 | the sequence's partition count.  -1 for invalid
+ * arguments (those pa_decode rejects, a NULL host_context_lens with num_seqs > 0, or
+ * units NULL with max_units > 0).
+ */
+int pa_decode_planned_units(const int32_t *host_context_lens, int num_seqs, int num_q_heads,
+                            int num_kv_heads, int head_dim, int block_size,
+                            int max_blocks_per_seq, int max_context_len, int sliding_window,
+                            int partition_size, uint32_t *units, int max_units);
+
+/*
  * One decode step with the copy-on-write of a shared block folded into the attention
  * pass (the pages let several requests share KV blocks -- "PagedAttention" summary,
  * features 2 -- so a sequence that appends into a shared, partially filled block

@@ -36,6 +36,7 @@ from ._lib import (  # noqa: F401
     decode_append,
     decode_cow,
     decode_planned,
+    decode_planned_units,
     decode_static_scratch,
     decode_partition_tokens,
     decode_workspace_bytes,

@@ -23,6 +23,7 @@ DEVERR = {"block_id": 0x1, "slot": 0x2, "pair": 0x4, "context": 0x8, "timeout": 
 EXPORTS = ("pa_kv_write", "pa_copy_blocks", "pa_decode", "pa_decode_workspace_bytes",
            "pa_decode_partition_tokens", "pa_get_device_error", "pa_status_str", "pa_version",
            "pa_decode_static_scratch", "pa_decode_append", "pa_decode_cow", "pa_decode_planned",
+           "pa_decode_planned_units",
            "pa_swap_blocks",
            "pa_prefill",
            # host block manager (include/pa_block_manager.h)
@@ -81,6 +82,8 @@ def load(path: str = LIB_PATH):
     lib.pa_decode_planned.argtypes = [P, P, P, P, i64, i64, P, P, P, P, P, i32, i32, i32, i32,
                                       i32, i32, i32, f32, i32, i32, i32, P, sz, i32, P]
     lib.pa_decode_planned.restype = i32
+    lib.pa_decode_planned_units.argtypes = [P] + [i32] * 9 + [P, i32]
+    lib.pa_decode_planned_units.restype = i32
     lib.pa_prefill.argtypes = [P, P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, i32, i32, f32,
                                i32, i32, P]
     lib.pa_prefill.restype = i32
@@ -429,6 +432,24 @@ def decode_planned(out, q, k_cache, v_cache, block_tables, context_lens, host_co
             _ptr(block_tables), _ptr(context_lens), hl.ctypes.data_as(ctypes.c_void_p), B, hq,
             hkv, d, bs, nb, W, float(scale), int(max_context_len), int(sliding_window),
             int(partition_size), wptr, wbytes, _dtype(q), _stream(stream, dev)), what)
+
+
+def decode_planned_units(host_context_lens, num_q_heads, num_kv_heads, head_dim, block_size,
+                         max_blocks_per_seq, max_context_len=0, sliding_window=0,
+                         partition_size=0):
+    """The units decode_planned launches for these arguments (host-side): uint32 array,
+    each sequence << 16 | partition << 8 | partition count, in launch order; empty when
+    it launches the full grid."""
+    hl = np.ascontiguousarray(host_context_lens, np.int32)
+    out = np.zeros(4096, np.uint32)
+    n = load().pa_decode_planned_units(
+        hl.ctypes.data_as(ctypes.c_void_p), int(hl.shape[0]), int(num_q_heads),
+        int(num_kv_heads), int(head_dim), int(block_size), int(max_blocks_per_seq),
+        int(max_context_len), int(sliding_window), int(partition_size),
+        out.ctypes.data_as(ctypes.c_void_p), out.shape[0])
+    if n < 0:
+        _fail("pa_decode_planned_units", "invalid arguments")
+    return out[:n].copy()
 
 
 def decode_static_scratch(out, q, k_cache, v_cache, block_tables, context_lens, scale,

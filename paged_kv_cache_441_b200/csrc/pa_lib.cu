@@ -341,6 +341,18 @@ int plan_units(const int32_t *lens, int num_seqs, long long cap, int P, int num_
     return k;
 }
 
+// The units pa_decode_planned launches for a fixed split, or 0 for the full grid: planned
+// only without a window and when the plan leaves out at least 30% of the grid's rows (A/B
+// on B200: GQA, 20% of the rows real, -5%; long 8/1, 61%, -1 to -2%; Llama-2, 75%, +2% --
+// there the full grid's own order, second partitions longest first, wins).
+int planned_units(const int32_t *lens, int num_seqs, int max_blocks_per_seq, int block_size,
+                  int sliding_window, const Plan &pl, uint32_t *units) {
+    if (sliding_window > 0 || pl.streamk || pl.dynamic || pl.partition_tokens <= 0) return 0;
+    const int n = plan_units(lens, num_seqs, (long long)max_blocks_per_seq * block_size,
+                             pl.partition_tokens, pl.num_parts, units);
+    return n > 0 && (long long)n * 10 <= 7LL * num_seqs * pl.num_parts ? n : 0;
+}
+
 template <typename T, int D>
 cudaError_t launch_merge(const MergeParams &p, dim3 grid, cudaStream_t st) {
     if (p.num_parts <= kMergeFew)
@@ -902,16 +914,12 @@ pa_status decode_impl(void *out, const void *q, const void *k_cache, const void 
     if (pl.num_parts > 65535) return PA_ERR_UNSUPPORTED;  // use a larger partition_size
     cudaError_t e = cudaSuccess;
     bool launched = false;
-    if (host_lens != nullptr && sliding_window == 0 && cow == nullptr) {
+    if (host_lens != nullptr && cow == nullptr) {
         // the units that exist, longest first, from the host's copy of the lengths
         PlannedParams pp;
-        const int units =
-            plan_units(host_lens, num_seqs, (long long)max_blocks_per_seq * block_size,
-                       pl.partition_tokens, pl.num_parts, pp.units);
-        // planned only when it leaves out at least 30% of the full grid's rows (A/B on
-        // B200: GQA, 20% of the rows real, -5%; long 8/1, 61%, -1 to -2%; Llama-2, 75%,
-        // +2% -- there the full grid's own order, second partitions longest first, wins)
-        if (units > 0 && (long long)units * 10 <= 7LL * num_seqs * pl.num_parts) {
+        const int units = planned_units(host_lens, num_seqs, max_blocks_per_seq, block_size,
+                                        sliding_window, pl, pp.units);
+        if (units > 0) {
             pp.base = p;
             pp.base.sort_second = 0;
             e = dtype == PA_BF16
@@ -1015,6 +1023,26 @@ pa_status pa_decode_planned(void *out, const void *q, const void *key, const voi
                        partition_size, workspace, workspace_bytes, dtype, stream, key, value,
                        key != nullptr ? key_token_stride : 0,
                        value != nullptr ? value_token_stride : 0, nullptr, host_context_lens);
+}
+
+int pa_decode_planned_units(const int32_t *host_context_lens, int num_seqs, int num_q_heads,
+                            int num_kv_heads, int head_dim, int block_size,
+                            int max_blocks_per_seq, int max_context_len, int sliding_window,
+                            int partition_size, uint32_t *units, int max_units) {
+    if (check_decode_shape(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, 1,
+                           max_blocks_per_seq, max_context_len, sliding_window,
+                           partition_size) != PA_OK ||
+        (num_seqs > 0 && !host_context_lens) || max_units < 0 || (max_units > 0 && !units))
+        return -1;
+    if (num_seqs == 0) return 0;
+    const Plan pl = make_plan(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
+                              max_blocks_per_seq, max_context_len, sliding_window,
+                              partition_size, device_sms(current_device_or_zero()));
+    static thread_local uint32_t buf[kPlanMaxUnits];
+    const int n = planned_units(host_context_lens, num_seqs, max_blocks_per_seq, block_size,
+                                sliding_window, pl, buf);
+    for (int i = 0; i < n && i < max_units; ++i) units[i] = buf[i];
+    return n;
 }
 
 pa_status pa_decode_cow(void *out, const void *q, const void *key, const void *value,

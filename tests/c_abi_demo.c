@@ -27,7 +27,7 @@ int main(void) {
     const any_fn fns[] = {
         (any_fn)pa_kv_write, (any_fn)pa_copy_blocks, (any_fn)pa_swap_blocks,
         (any_fn)pa_decode, (any_fn)pa_decode_append, (any_fn)pa_decode_cow,
-        (any_fn)pa_decode_planned,
+        (any_fn)pa_decode_planned, (any_fn)pa_decode_planned_units,
         (any_fn)pa_decode_workspace_bytes,
         (any_fn)pa_decode_partition_tokens, (any_fn)pa_decode_static_scratch,
         (any_fn)pa_prefill, (any_fn)pa_get_device_error, (any_fn)pa_status_str,

@@ -4,6 +4,7 @@ import ctypes
 import os
 import re
 
+import numpy as np
 import pytest
 from hypothesis import given, settings
 from hypothesis import strategies as st
@@ -251,3 +252,64 @@ def test_workspace_plan_invariants(lib, B, G, hkv, d, bs, W, mcl, win, ps):
             assert ws <= pa.decode_workspace_bytes(B, hq, hkv, d, bs, W, mcl + 4096, ps, win)
         if win > 0:
             assert ws <= pa.decode_workspace_bytes(B, hq, hkv, d, bs, W, mcl, ps, win + 4096)
+
+
+@settings(max_examples=300, derandomize=True, deadline=None)
+@given(B=st.integers(1, 300), G=st.sampled_from([1, 2, 4, 8]), hkv=st.integers(1, 8),
+       bs=st.sampled_from([8, 16, 64, 512]), W=st.integers(1, 600),
+       ps=st.sampled_from([0, 64, 256, 1024]), win=st.sampled_from([0, 0, 0, 300]),
+       mcl_extra=st.integers(-1, 200), seed=st.integers(0, 2**31 - 1))
+def test_planned_units(lib, B, G, hkv, bs, W, ps, win, mcl_extra, seed):
+    """The host plan of pa_decode_planned: when it is used, every (sequence, partition)
+    unit a context needs appears exactly once with its partition count, full partitions
+    first in partition-major order, then the last partitions by decreasing length; it is
+    used only without a window and when it leaves out at least 30% of the grid."""
+    rng = np.random.default_rng(seed)
+    cap = W * bs
+    lens = np.minimum(rng.integers(0, cap + 1, size=B), cap).astype(np.int32)
+    if rng.random() < 0.3:
+        lens[rng.integers(0, B)] = 0
+    mcl = 0 if mcl_extra < 0 else int(lens.max()) + mcl_extra
+    hq = G * hkv
+    units = pa.decode_planned_units(lens, hq, hkv, 128, bs, W, mcl, win, ps)
+    P = pa.decode_partition_tokens(B, hq, hkv, 128, bs, W, mcl, ps, win)
+    bound = _attend_bound(W, bs, mcl, win)
+    parts = -(-bound // P)
+    need = [max(1, -(-min(int(L), bound) // P)) for L in lens]
+    need = [min(n, parts) for n in need]
+    fits = parts <= 255 and sum(need) <= 4096
+    if win > 0 or not fits or 10 * sum(need) > 7 * B * parts:
+        assert units.size == 0
+        return
+    assert units.size == sum(need)
+    su, pu, nu = units >> 16, (units >> 8) & 0xFF, units & 0xFF
+    seen = sorted(zip(su.tolist(), pu.tolist()))
+    assert seen == sorted((s, p) for s in range(B) for p in range(need[s]))
+    assert all(int(nu[i]) == need[int(su[i])] for i in range(units.size))
+    size = np.array([min(P, int(lens[s]) - int(p) * P) for s, p in zip(su, pu)])
+    full = size == P
+    k = int(full.sum())
+    assert full[:k].all() and not full[k:].any()  # full partitions first
+    fp = list(zip(pu[:k].tolist(), su[:k].tolist()))
+    assert fp == sorted(fp)                       # partition-major, then sequence
+    assert np.all(np.diff(size[k:]) <= 0)         # the rest by decreasing length
+
+
+def test_planned_units_on_the_benchmark_workloads(lib):
+    """GQA (lognormal lengths) and the long contexts are planned; the Llama-2 step (75% of
+    its grid rows real) and any windowed call keep the full grid."""
+    from workloads import make_config
+    for name, kw, planned in (("gqa_llama3_8b", {"block_size": 16}, True),
+                              ("long_8_1", {"block_size": 512}, True),
+                              ("llama2_7b", {}, False)):
+        c = make_config(name, poison=False, **kw)
+        u = pa.decode_planned_units(c.context_lens, c.num_q_heads, c.num_kv_heads, c.head_dim,
+                                    c.block_size, c.max_blocks_per_seq, c.max_context_len)
+        assert (u.size > 0) == planned, name
+        w = pa.decode_planned_units(c.context_lens, c.num_q_heads, c.num_kv_heads, c.head_dim,
+                                    c.block_size, c.max_blocks_per_seq, c.max_context_len,
+                                    sliding_window=4096)
+        assert w.size == 0
+    assert pa.decode_planned_units(np.zeros(0, np.int32), 8, 2, 128, 16, 4).size == 0
+    with pytest.raises(pa.PAError):
+        pa.decode_planned_units(np.ones(3, np.int32), 6, 2, 128, 16, 4)  # group 3
