@@ -382,8 +382,8 @@ class DecodeStep:
                       "dynamic: persistent CTAs claim 32-token chunks + LSE merge"
                       if partition_size == -2 else
                       "balanced over persistent warps (stream-K) + LSE merge")
-        self.kind = ("pa_decode_planned (cache write fused into decode; units planned from "
-                     "the host lengths when that leaves out >= 30% of the grid)"
+        self.kind = ("pa_decode_planned (cache write fused into decode; the (sequence, "
+                     "partition) units that exist, planned from the host lengths)"
                      if self.plan and self.fused
                      else "pa_kv_write + pa_decode_planned" if self.plan and not self.has_pairs
                      else "pa_copy_blocks + pa_kv_write + pa_decode_planned" if self.plan

@@ -238,9 +238,12 @@ pa_status pa_decode_append(void *out, const void *q, const void *key, const void
  * context lengths on the host, as a serving engine's scheduler does.  The launch is
  * planned from them: only the (sequence, partition) units that exist are launched --
  * under the fixed split a context of L tokens has ceil(L / partition) of them, where the
- * full grid holds the longest context's count for every sequence -- and they are taken
- * longest first: every full partition, then the shorter last partitions by decreasing
- * length.  The results are bit-identical to pa_decode / pa_decode_append.
+ * full grid holds the longest context's count for every sequence.  When that leaves out
+ * at least 30% of the grid's rows they are taken longest first (every full partition,
+ * then the shorter last partitions by decreasing length); otherwise in the full grid's
+ * own order without its empty rows (partition 0 of every sequence, then each later
+ * partition index longest first).  The results are bit-identical to pa_decode /
+ * pa_decode_append.
  *
  * host_context_lens : int32 [num_seqs], host memory, read during the call only; it must
  *                     hold the values of context_lens.  A context whose device length
@@ -248,10 +251,9 @@ pa_status pa_decode_append(void *out, const void *q, const void *key, const void
  *                     PA_DEVERR_CONTEXT (a partition the plan left out is not computed).
  * key, value        : both NULL (no cache write) or both given, as pa_decode_append.
  * The plan applies to the fixed split without a sliding window, with at most
- * 4096 units and 255 partitions per context, when it leaves out at least 30% of the full
- * grid's (sequence, partition) rows (with fewer empty rows the full grid's own order was
- * faster on B200); other calls run as pa_decode / pa_decode_append.  Other arguments,
- * errors and the workspace as pa_decode.
+ * 4096 units and 255 partitions per context, when the full grid has an empty row; other
+ * calls run as pa_decode / pa_decode_append.  Other arguments, errors and the workspace
+ * as pa_decode.
  */
 pa_status pa_decode_planned(void *out, const void *q, const void *key, const void *value,
                             int64_t key_token_stride, int64_t value_token_stride,

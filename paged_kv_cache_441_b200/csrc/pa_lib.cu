@@ -341,16 +341,36 @@ int plan_units(const int32_t *lens, int num_seqs, long long cap, int P, int num_
     return k;
 }
 
-// The units pa_decode_planned launches for a fixed split, or 0 for the full grid: planned
-// only without a window and when the plan leaves out at least 30% of the grid's rows (A/B
-// on B200: GQA, 20% of the rows real, -5%; long 8/1, 61%, -1 to -2%; Llama-2, 75%, +2% --
-// there the full grid's own order, second partitions longest first, wins).
+// The units pa_decode_planned launches for a fixed split, or 0 for the full grid (a
+// window, or no empty row to leave out).  Where the plan leaves out at least 30% of the
+// grid's rows the units go longest first; otherwise in the full grid's own order without
+// its empty rows: partition 0 of every sequence in order, then each later partition index
+// longest first.  A/B on B200 against the full grid: GQA (20% of the rows real) -5% and
+// long 8/1 (61%) -1 to -2% longest first, where the full grid's order gained nothing;
+// Llama-2 (75%) +2% longest first but -2% in the grid's order.
 int planned_units(const int32_t *lens, int num_seqs, int max_blocks_per_seq, int block_size,
                   int sliding_window, const Plan &pl, uint32_t *units) {
     if (sliding_window > 0 || pl.streamk || pl.dynamic || pl.partition_tokens <= 0) return 0;
     const int n = plan_units(lens, num_seqs, (long long)max_blocks_per_seq * block_size,
                              pl.partition_tokens, pl.num_parts, units);
-    return n > 0 && (long long)n * 10 <= 7LL * num_seqs * pl.num_parts ? n : 0;
+    if (n <= 0) return 0;
+    if ((long long)n * 10 <= 7LL * num_seqs * pl.num_parts) return n;  // longest first
+    if ((long long)n >= (long long)num_seqs * pl.num_parts) return 0;  // no empty row
+    const long long cap = (long long)max_blocks_per_seq * block_size;
+    const int P = pl.partition_tokens;
+    auto size = [&](uint32_t u) {
+        const int s = (int)(u >> 16);
+        const long long L = lens[s] < 0 ? 0 : (lens[s] > cap ? cap : lens[s]);
+        const long long r = L - (long long)((u >> 8) & 0xffu) * P;
+        return r < P ? r : (long long)P;
+    };
+    std::stable_sort(units, units + n, [&](uint32_t a, uint32_t b) {
+        const uint32_t pa_ = (a >> 8) & 0xffu, pb = (b >> 8) & 0xffu;
+        if (pa_ != pb) return pa_ < pb;
+        if (pa_ == 0) return (a >> 16) < (b >> 16);
+        return size(a) > size(b);
+    });
+    return n;
 }
 
 template <typename T, int D>

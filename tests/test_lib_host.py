@@ -261,9 +261,11 @@ def test_workspace_plan_invariants(lib, B, G, hkv, d, bs, W, mcl, win, ps):
        mcl_extra=st.integers(-1, 200), seed=st.integers(0, 2**31 - 1))
 def test_planned_units(lib, B, G, hkv, bs, W, ps, win, mcl_extra, seed):
     """The host plan of pa_decode_planned: when it is used, every (sequence, partition)
-    unit a context needs appears exactly once with its partition count, full partitions
-    first in partition-major order, then the last partitions by decreasing length; it is
-    used only without a window and when it leaves out at least 30% of the grid."""
+    unit a context needs appears exactly once with its partition count.  Leaving out at
+    least 30% of the grid: full partitions first in partition-major order, then the last
+    partitions by decreasing length; leaving out less: partition 0 of every sequence in
+    order, then each later partition index by decreasing length.  Not used under a window
+    or when the grid has no empty row."""
     rng = np.random.default_rng(seed)
     cap = W * bs
     lens = np.minimum(rng.integers(0, cap + 1, size=B), cap).astype(np.int32)
@@ -278,7 +280,7 @@ def test_planned_units(lib, B, G, hkv, bs, W, ps, win, mcl_extra, seed):
     need = [max(1, -(-min(int(L), bound) // P)) for L in lens]
     need = [min(n, parts) for n in need]
     fits = parts <= 255 and sum(need) <= 4096
-    if win > 0 or not fits or 10 * sum(need) > 7 * B * parts:
+    if win > 0 or not fits or sum(need) == B * parts:
         assert units.size == 0
         return
     assert units.size == sum(need)
@@ -287,21 +289,28 @@ def test_planned_units(lib, B, G, hkv, bs, W, ps, win, mcl_extra, seed):
     assert seen == sorted((s, p) for s in range(B) for p in range(need[s]))
     assert all(int(nu[i]) == need[int(su[i])] for i in range(units.size))
     size = np.array([min(P, int(lens[s]) - int(p) * P) for s, p in zip(su, pu)])
-    full = size == P
-    k = int(full.sum())
-    assert full[:k].all() and not full[k:].any()  # full partitions first
-    fp = list(zip(pu[:k].tolist(), su[:k].tolist()))
-    assert fp == sorted(fp)                       # partition-major, then sequence
-    assert np.all(np.diff(size[k:]) <= 0)         # the rest by decreasing length
+    if 10 * sum(need) <= 7 * B * parts:  # longest first
+        full = size == P
+        k = int(full.sum())
+        assert full[:k].all() and not full[k:].any()  # full partitions first
+        fp = list(zip(pu[:k].tolist(), su[:k].tolist()))
+        assert fp == sorted(fp)                       # partition-major, then sequence
+        assert np.all(np.diff(size[k:]) <= 0)         # the rest by decreasing length
+    else:  # the full grid's order without its empty rows
+        assert np.all(np.diff(pu.astype(np.int64)) >= 0)
+        assert su[pu == 0].tolist() == list(range(B))
+        for p in range(1, parts):
+            assert np.all(np.diff(size[pu == p]) <= 0)
 
 
 def test_planned_units_on_the_benchmark_workloads(lib):
-    """GQA (lognormal lengths) and the long contexts are planned; the Llama-2 step (75% of
-    its grid rows real) and any windowed call keep the full grid."""
+    """GQA (lognormal lengths) and the long contexts are planned longest first, the
+    Llama-2 step (75% of its grid rows real) in the grid's order; windowed calls and
+    one-partition contexts keep the full grid."""
     from workloads import make_config
     for name, kw, planned in (("gqa_llama3_8b", {"block_size": 16}, True),
                               ("long_8_1", {"block_size": 512}, True),
-                              ("llama2_7b", {}, False)):
+                              ("llama2_7b", {}, True), ("prefix_cow", {}, False)):
         c = make_config(name, poison=False, **kw)
         u = pa.decode_planned_units(c.context_lens, c.num_q_heads, c.num_kv_heads, c.head_dim,
                                     c.block_size, c.max_blocks_per_seq, c.max_context_len)
