@@ -49,6 +49,8 @@ def _declare(lib):
     lib.orc_kv_write.restype = i32
     lib.orc_copy_blocks.argtypes = [P, P, P, i32, i32, i32, i32, i32]
     lib.orc_copy_blocks.restype = i32
+    lib.orc_copy_rows.argtypes = [P, P, P, i32, i32, i32, i32, i32]
+    lib.orc_copy_rows.restype = i32
     lib.orc_decode.argtypes = [P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, i32, dbl, i32, P,
                                i32, i32]
     lib.orc_decode.restype = i32
@@ -84,6 +86,16 @@ def copy_blocks(k_cache, v_cache, pairs, lib=None) -> int:
     pairs = np.ascontiguousarray(pairs, np.int64).reshape(-1, 2)
     nb, hkv, bs, d = k_cache.shape
     return lib.orc_copy_blocks(_p(k_cache), _p(v_cache), _p(pairs), pairs.shape[0], hkv, bs, d, nb)
+
+
+def copy_rows(k_cache, v_cache, triples, lib=None) -> int:
+    """In place: for each (src, dst, rows), the first ``rows`` slots of every kv head of block
+    dst := block src's (the copy-on-write of a block's filled rows); returns #bad triples."""
+    lib = lib or load()
+    triples = np.ascontiguousarray(triples, np.int64).reshape(-1, 3)
+    nb, hkv, bs, d = k_cache.shape
+    return lib.orc_copy_rows(_p(k_cache), _p(v_cache), _p(triples), triples.shape[0], hkv, bs,
+                             d, nb)
 
 
 def decode(q, k_cache, v_cache, block_tables, context_lens, scale, dtype, num_q_heads=None,

@@ -122,3 +122,11 @@ def copy_blocks(k_cache, v_cache, pairs) -> None:
     for src, dst in np.asarray(pairs, dtype=np.int64).reshape(-1, 2):
         k_cache[dst] = k_cache[src]
         v_cache[dst] = v_cache[src]
+
+
+def copy_rows(k_cache, v_cache, triples) -> None:
+    """Copy-on-write of the filled rows: block dst's first ``rows`` slots of every kv head
+    take block src's; its other slots keep their values."""
+    for src, dst, rows in np.asarray(triples, dtype=np.int64).reshape(-1, 3):
+        k_cache[dst, :, :rows] = k_cache[src, :, :rows]
+        v_cache[dst, :, :rows] = v_cache[src, :, :rows]

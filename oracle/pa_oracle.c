@@ -111,6 +111,33 @@ int orc_copy_blocks(uint16_t *k_cache, uint16_t *v_cache, const int64_t *pairs, 
     return bad;
 }
 
+/* Copy-on-write of the filled rows of a block: for each (src, dst, rows) triple in order,
+ * rows r < rows of every kv head h of block dst := the same rows of block src, in both
+ * caches; the other rows of dst keep their values.  Returns the number of triples with a
+ * block id outside [0, num_blocks) or rows outside [0, block_size] (skipped). */
+int orc_copy_rows(uint16_t *k_cache, uint16_t *v_cache, const int64_t *triples, int n,
+                  int num_kv_heads, int block_size, int head_dim, int num_blocks) {
+    int bad = 0;
+    for (int c = 0; c < n; ++c) {
+        int64_t src = triples[3 * c], dst = triples[3 * c + 1], rows = triples[3 * c + 2];
+        if (src < 0 || src >= num_blocks || dst < 0 || dst >= num_blocks || rows < 0 ||
+            rows > block_size) {
+            ++bad;
+            continue;
+        }
+        for (int h = 0; h < num_kv_heads; ++h)
+            for (int64_t r = 0; r < rows; ++r) {
+                size_t from = (((size_t)src * num_kv_heads + h) * block_size + r) * head_dim;
+                size_t to = (((size_t)dst * num_kv_heads + h) * block_size + r) * head_dim;
+                for (int i = 0; i < head_dim; ++i) {
+                    k_cache[to + i] = k_cache[from + i];
+                    v_cache[to + i] = v_cache[from + i];
+                }
+            }
+    }
+    return bad;
+}
+
 /* Attention for one (sequence, q head), written as the definition:
  *   K_s = concat of the sequence's pages in table order (first L rows),
  *   z_t = scale * <q, K_s[t]>,  out = sum_t softmax(z)_t V_s[t],

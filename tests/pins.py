@@ -382,6 +382,34 @@ def pin_copy_blocks(lib):
         assert np.array_equal(kc_c[b], kc[b]) and np.array_equal(vc_c[b], vc[b])
 
 
+def pin_copy_rows(lib):
+    """The filled-rows copy: the listed rows of every head come from the source, the rest
+    of the destination and every other block keep their values, bad triples are skipped
+    and counted; a whole block's rows equal the block copy; the C and numpy statements
+    agree."""
+    rng = np.random.default_rng(21)
+    nb, hkv, bs, d = 10, 3, 4, 8
+    kc = _rand_bits(rng, (nb, hkv, bs, d))
+    vc = _rand_bits(rng, (nb, hkv, bs, d))
+    triples = np.array([[1, 4, 3], [2, 7, 0], [5, 9, 4], [3, 99, 1], [3, 6, 5]], np.int64)
+    kc_c, vc_c = kc.copy(), vc.copy()
+    assert oracle.copy_rows(kc_c, vc_c, triples, lib=lib) == 2
+    for h in range(hkv):
+        for r in range(bs):
+            src = kc[1] if r < 3 else kc[4]
+            assert np.array_equal(kc_c[4, h, r], src[h, r])
+            assert np.array_equal(vc_c[4, h, r], (vc[1] if r < 3 else vc[4])[h, r])
+    assert np.array_equal(kc_c[9], kc[5]) and np.array_equal(vc_c[9], vc[5])
+    for b in (0, 1, 2, 3, 5, 6, 7, 8):
+        assert np.array_equal(kc_c[b], kc[b]) and np.array_equal(vc_c[b], vc[b])
+    kb, vb = kc.copy(), vc.copy()
+    oracle.copy_blocks(kb, vb, np.array([[5, 9]], np.int64), lib=lib)
+    assert np.array_equal(kb[9], kc_c[9]) and np.array_equal(vb[9], vc_c[9])
+    kn, vn = kc.copy(), vc.copy()
+    oracle_np.copy_rows(kn, vn, triples[[0, 1, 2]])
+    assert np.array_equal(kn, kc_c) and np.array_equal(vn, vc_c)
+
+
 # ------------------------------------------------------------------ sliding window
 
 def _recycle_before(tables, lens, bs, window):
@@ -532,7 +560,8 @@ def pin_prefill_one_token_is_decode(lib):
 
 ALL_PINS = [pin_two_token, pin_len1_exact, pin_identical_keys, pin_zero_len, pin_paged_vs_sdpa,
             pin_block_size_and_permutation, pin_shared_prefix, pin_golden_examples,
-            pin_widening, pin_c_vs_numpy, pin_kv_write, pin_copy_blocks, pin_window_last_token,
+            pin_widening, pin_c_vs_numpy, pin_kv_write, pin_copy_blocks, pin_copy_rows,
+            pin_window_last_token,
             pin_window_vs_sdpa, pin_prefill_vs_sdpa, pin_prefill_one_token_is_decode]
 
 

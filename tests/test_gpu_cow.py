@@ -1,6 +1,6 @@
 """Copy-on-write folded into the decode (pa_decode_cow) against the oracle.
 
-Bar: both caches bit-exact against the oracle's block copy (rows [0, rows) of the
+Bar: both caches bit-exact against the oracle's filled-rows copy (rows [0, rows) of the
 named source into the sequence's own block), its cache write and nothing else; the
 output within max-abs 2e-3 (fp16) / 1e-2 (bf16) of the oracle's attention over those
 caches, and bit-identical to pa_decode run on them.
@@ -27,17 +27,13 @@ def _clean_error_word():
 
 
 def _copy_rows(kc, vc, cow, tables):
-    """The copies a cow list asks for, on host caches: rows [0, rows) of every kv head
-    of the source block into the sequence's block at the logical index (the oracle's
-    whole-block copy, restricted to those rows)."""
-    for s, (src, lb, rows) in enumerate(cow):
-        if src < 0:
-            continue
-        dst = int(tables[s, lb])
-        k2, v2 = kc.copy(), vc.copy()
-        oracle.copy_blocks(k2, v2, np.array([[src, dst]], np.int64))
-        kc[dst, :, :rows] = k2[dst, :, :rows]
-        vc[dst, :, :rows] = v2[dst, :, :rows]
+    """The copies a cow list asks for, on host caches: the oracle's filled-rows copy of
+    rows [0, rows) of every kv head of the source block into the sequence's block at the
+    logical index."""
+    triples = [(int(src), int(tables[s, lb]), int(rows)) for s, (src, lb, rows) in enumerate(cow)
+               if src >= 0]
+    if triples:
+        assert oracle.copy_rows(kc, vc, np.array(triples, np.int64)) == 0
 
 
 def _cow_list(case, rng, frac=0.7):

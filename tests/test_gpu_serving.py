@@ -124,14 +124,11 @@ def test_block_manager_serving_loop(hq, hkv, bs, fused, preempt, window, cow):
         key = _rand_bits(rng, (len(live), hkv, d))
         val = _rand_bits(rng, (len(live), hkv, d))
         bt, cl = bm.block_tables(live, width)
-        if cow:  # the mirror: the oracle's block copy of the listed rows, then the write
-            for i, (src, lb, nrows) in enumerate(cowl.tolist()):
-                if src >= 0:
-                    dst = int(bt[i, lb])
-                    k2, v2 = kc_h.copy(), vc_h.copy()
-                    oracle.copy_blocks(k2, v2, np.array([[src, dst]], np.int64))
-                    kc_h[dst, :, :nrows], vc_h[dst, :, :nrows] = (k2[dst, :, :nrows],
-                                                                  v2[dst, :, :nrows])
+        if cow:  # the mirror: the oracle's copy of the listed rows, then the write
+            triples = [(src, int(bt[i, lb]), nrows)
+                       for i, (src, lb, nrows) in enumerate(cowl.tolist()) if src >= 0]
+            if triples:
+                assert oracle.copy_rows(kc_h, vc_h, np.array(triples, np.int64)) == 0
         oracle.kv_write(key, val, slots, kc_h, vc_h)
         q = _rand_bits(rng, (len(live), hq, d))
         out = torch.empty(len(live), hq, d, dtype=torch.bfloat16, device="cuda")

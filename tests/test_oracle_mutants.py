@@ -50,6 +50,10 @@ MUTANTS = [
     ("copy_v_from_k", "v_cache[(size_t)dst * blk + i] = v_cache[(size_t)src * blk + i];",
      "v_cache[(size_t)dst * blk + i] = k_cache[(size_t)src * blk + i];"),
     ("write_v_from_key", "v_cache[dst + i] = vs[i];", "v_cache[dst + i] = ks[i];"),
+    ("copy_rows_whole_block", "for (int64_t r = 0; r < rows; ++r) {",
+     "for (int64_t r = 0; r < block_size; ++r) {"),
+    ("copy_rows_head0", "size_t from = (((size_t)src * num_kv_heads + h) * block_size + r)",
+     "size_t from = (((size_t)src * num_kv_heads + 0) * block_size + r)"),
 ]
 
 
