@@ -79,6 +79,18 @@ int main(void) {
     CHECK(slots[1] == (int64_t)tables[2] * 8 + 5);           /* sequence 1 keeps its block */
     pa_bm_destroy(bm);
 
+    /* the plan of a planned launch, host-side: 3 contexts at 256-token partitions in a
+     * 4-partition grid (12 rows) need 1 + 3 + 1 = 5 units; full partitions first, then the
+     * last ones by decreasing length: (1,0) (1,1) then (1,2: 188 tokens) (0,0: 5) (2,0: 0) */
+    const int32_t plan_lens[3] = {5, 700, 0};
+    uint32_t plan[16];
+    CHECK(pa_decode_planned_units(plan_lens, 3, 8, 2, 128, 16, 64, 1000, 0, 256, plan, 16) == 5);
+    CHECK(plan[0] == ((1u << 16) | (0u << 8) | 3u) && plan[1] == ((1u << 16) | (1u << 8) | 3u));
+    CHECK(plan[2] == ((1u << 16) | (2u << 8) | 3u) && plan[3] == ((0u << 16) | 1u));
+    CHECK(plan[4] == ((2u << 16) | 1u));
+    CHECK(pa_decode_planned_units(plan_lens, 3, 8, 2, 128, 16, 64, 1000, 300, 256, plan, 16) == 0);
+    CHECK(pa_decode_planned_units(NULL, 3, 8, 2, 128, 16, 64, 1000, 0, 256, plan, 16) == -1);
+
     /* refusals before any launch (no GPU is touched) */
     char buf[64];
     CHECK(pa_decode(buf, buf, buf, buf, (const int32_t *)buf, (const int32_t *)buf, 1, 8, 2, 96,
